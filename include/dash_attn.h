@@ -1,0 +1,178 @@
+/*
+ * dash_attn.h -- C ABI of the B200 (sm_100a) DashAttention forward library.
+ *
+ * DashAttention is defined in "DashAttention: Differentiable and Adaptive
+ * Sparse Hierarchical Attention" (arXiv 2605.18753), cited here as [Dash].
+ * The forward pass has three stages:
+ *   Stage 0  chunk summaries  k̄_c = mean of the chunk's keys
+ *            ([Dash] §3.1 Eq. 3 with the summary query at its zero
+ *            initialisation, which the paper notes is exactly mean pooling)
+ *   Stage 1  entmax routing: zbar_{i,c} = <q_i, k̄_c>/sqrt(d) over the chunks
+ *            visible to row i, w^(h) = alpha-entmax(gamma * zbar) per head,
+ *            averaged over the GQA group, support = union of the heads'
+ *            supports ([Dash] §3.2 Eq. 4; §2 Eq. 2)
+ *   Stage 2  softmax attention over the routed chunks plus the diagonal
+ *            chunk, with the routing distribution folded in as the bias
+ *            d = (log w - mu)/sigma ([Dash] §3.3 Eq. 7, §3.4 Prop. 1)
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are [batch, seq, heads, dim] with dim contiguous (stride[3] = 1);
+ *     other strides are free (elements).  Q and O: [b, nq, hq, d];
+ *     K and V: [b, nk, hkv, d].  hq = gqa_groups * hkv.
+ *   - All data pointers are DEVICE pointers on the current CUDA device, owned
+ *     by the caller; the library never frees caller memory.
+ *   - Causal alignment is bottom-right: query row i sits at key position
+ *     p_i = i + nk - nq.  Its chunk is c_i = floor(p_i / B).  It routes over the
+ *     complete chunks c < min(c_i, floor(nk / B)) and always attends its
+ *     diagonal tokens c_i*B .. p_i (bias 0) ([Dash] App. G Algs. 2-3).
+ *     Non-causal: every chunk, a trailing partial chunk included, is routed,
+ *     and there is no diagonal branch.
+ *   - n_chunks (routing chunks) = floor(nk/B) if causal else ceil(nk/B).
+ *   - Calls are asynchronous on the given stream; the return value reports
+ *     argument validation and launch errors.  Errors found on the device
+ *     (a bounded wait that ran out) are reported by dash_sync_status().
+ *   - Supported: dtype f32 or bf16 (q, k, v, out all the same), d in {64, 128},
+ *     block_size in {16, 32, 64, 128}, alpha > 1, 1 <= gqa_groups <= 16.
+ *   - Base pointers must be 16-byte aligned and every stride but the last a
+ *     multiple of 16 bytes, otherwise DASH_ERR_ALIGNMENT.
+ */
+#ifndef DASH_ATTN_H
+#define DASH_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DASH_API __attribute__((visibility("default")))
+
+typedef enum {
+    DASH_OK = 0,
+    DASH_ERR_INVALID_ARG = -1,    /* bad shape, value or null pointer */
+    DASH_ERR_UNSUPPORTED = -2,    /* valid but outside the supported set above */
+    DASH_ERR_ALIGNMENT = -3,      /* base pointer or stride not 16-byte aligned */
+    DASH_ERR_WORKSPACE = -4,      /* caller workspace too small */
+    DASH_ERR_CUDA = -5,           /* a CUDA runtime call failed */
+    DASH_ERR_DEVICE_TIMEOUT = -6  /* a device-side bounded wait ran out */
+} dash_status_t;
+
+typedef enum { DASH_F32 = 0, DASH_BF16 = 1 } dash_dtype_t;
+
+/* A strided 4-D device tensor [batch, seq, heads, dim]. */
+typedef struct {
+    void *data;
+    dash_dtype_t dtype;
+    int64_t shape[4];
+    int64_t stride[4]; /* in elements; stride[3] must be 1 */
+} dash_tensor_t;
+
+/* Stage-2 work lists: for each (batch, kv head, query tile of tile_rows
+ * consecutive query rows) the union of the chunks any row of the tile attends
+ * (its routed chunks and its diagonal chunk), and a per-row additive bias.
+ * Layout (all device memory, caller-owned, contiguous):
+ *   count [b][hkv][n_tiles]                    int32   entries in the list
+ *   ids   [b][hkv][n_tiles][cap]               int32   chunk ids; diagonal chunks first
+ *   bias  [b][hkv][n_tiles][cap][tile_rows]    float32 bias of that chunk for
+ *         that row: (log w_c - mu)/sigma if the row routed it, 0 if it is the
+ *         row's diagonal chunk, -inf if the row does not attend it.
+ * n_tiles = ceil(nq / tile_rows); cap = ceil(nk / block_size); tile_rows =
+ * 128 / gqa_groups (the tensor-core tile is tile_rows positions x gqa_groups
+ * heads = 128 rows).  Stage 2 also masks key j > p_i when causal. */
+typedef struct {
+    int32_t *count;
+    int32_t *ids;
+    float *bias;
+    int64_t n_tiles;
+    int32_t cap;
+    int32_t tile_rows;
+} dash_lists_t;
+
+#define DASH_FLAG_FORCE_SIMT 0x1      /* Stage 2 on the CUDA-core path (testing) */
+#define DASH_FLAG_TEST_TIMEOUT 0x100  /* testing only: Stage 2 waits on a barrier nothing
+                                         arrives at, gives up after a short bound and
+                                         reports DASH_ERR_DEVICE_TIMEOUT */
+
+/* Optional settings.  Fill with dash_opts_init(). */
+typedef struct {
+    float sigma;            /* prior strength sigma > 0; default 1e8 ([Dash] App. F.5 picks 1e8) */
+    float gamma;            /* Stage-1 logit scale gamma > 0 ([Dash] Eq. 4); default 1 */
+    void *stream;           /* cudaStream_t; NULL = the legacy default stream */
+    void *workspace;        /* device scratch; NULL = library-managed (cached per device) */
+    size_t workspace_bytes; /* size of workspace; see dash_workspace_bytes() */
+    const float *kbar;      /* optional precomputed chunk summaries [b][n_chunks][hkv][d] fp32
+                               contiguous (from dash_pool_keys, e.g. a decode cache) */
+    int flags;              /* DASH_FLAG_* */
+} dash_opts_t;
+
+/* Fill *opts with the defaults above.  Returns DASH_OK or DASH_ERR_INVALID_ARG (NULL). */
+DASH_API int dash_opts_init(dash_opts_t *opts);
+
+/* Full forward pass, Stages 0-2 ([Dash] §3, App. G Algs. 1-3).
+ *   q, out [b, nq, hq, d]; k, v [b, nk, hkv, d]; same dtype.
+ *   block_size B, alpha > 1, causal 0/1, gqa_groups = hq / hkv.
+ * Uses the default options (sigma 1e8, gamma 1, default stream, library
+ * workspace).  Returns a dash_status_t. */
+DASH_API int dash_attn_fwd(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v,
+                           dash_tensor_t *out, int block_size, float alpha, int causal, int gqa_groups);
+
+/* As dash_attn_fwd with explicit options (opts may be NULL for defaults). */
+DASH_API int dash_attn_fwd_ex(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v,
+                              dash_tensor_t *out, int block_size, float alpha, int causal, int gqa_groups,
+                              const dash_opts_t *opts);
+
+/* Stage 0 alone ([Dash] §3.1 Eq. 3, App. G Alg. 1): kbar [b][n_chunks][hkv][d]
+ * fp32 contiguous, n_chunks = floor(nk/B) if causal else ceil(nk/B) (a partial
+ * chunk is the mean of its real keys).  stream may be NULL. */
+DASH_API int dash_pool_keys(const dash_tensor_t *k, int block_size, int causal, float *kbar, void *stream);
+
+/* Stage 1 alone ([Dash] §3.2 Eq. 4; App. G Alg. 2).  Every output is optional
+ * (NULL to skip):
+ *   tau   [b][nq][hq]             fp32 threshold in the (alpha-1)*gamma*zbar domain;
+ *                                 NaN for a row with no visible chunk
+ *   w     [b][nq][hkv][n_chunks]  fp32 group distribution, 0 outside the support
+ *   mask  [b][nq][hkv][ceil(n_chunks/32)] uint32 routed-chunk bits (bit c%32 of
+ *                                 word c/32), the bit-packed mask of [Dash] §3.5
+ *   lists Stage-2 work lists (see dash_lists_t), built with opts->sigma
+ * Returns a dash_status_t. */
+DASH_API int dash_block_select(const dash_tensor_t *q, const dash_tensor_t *k, int block_size, float alpha,
+                               int causal, int gqa_groups, float *tau, float *w, uint32_t *mask,
+                               const dash_lists_t *lists, const dash_opts_t *opts);
+
+/* Stage 2 alone ([Dash] §3.3 Eq. 7 in the bias form of Prop. 1; App. G Alg. 3)
+ * on caller-supplied lists (for example from dash_block_select, or a random
+ * mask).  Returns a dash_status_t. */
+DASH_API int dash_sparse_attn_fwd(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v,
+                                  dash_tensor_t *out, const dash_lists_t *lists, int block_size, int causal,
+                                  int gqa_groups, const dash_opts_t *opts);
+
+/* Sizes of the lists buffers for a problem: *count_bytes, *ids_bytes,
+ * *bias_bytes (any may be NULL) and the geometry (*n_tiles, *cap, *tile_rows). */
+DASH_API int dash_lists_geometry(int64_t batch, int64_t nq, int64_t nk, int hkv, int block_size, int gqa_groups,
+                                 int64_t *n_tiles, int32_t *cap, int32_t *tile_rows, size_t *count_bytes,
+                                 size_t *ids_bytes, size_t *bias_bytes);
+
+/* Device workspace dash_attn_fwd_ex needs for a problem (bytes). */
+DASH_API size_t dash_workspace_bytes(int64_t batch, int64_t nq, int64_t nk, int hq, int hkv, int d,
+                                     int block_size, int causal);
+
+/* Thread-local message describing the last error returned on this thread. */
+DASH_API const char *dash_last_error(void);
+
+/* Synchronise the stream (NULL = default) and report device-side errors:
+ * DASH_ERR_DEVICE_TIMEOUT if a kernel's bounded wait ran out since the last
+ * call (the flag is then cleared), DASH_ERR_CUDA on a CUDA error, else DASH_OK. */
+DASH_API int dash_sync_status(void *stream);
+
+/* Free the library-managed workspace of the current device. */
+DASH_API int dash_release(void);
+
+/* Library version string. */
+DASH_API const char *dash_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DASH_ATTN_H */

@@ -1,0 +1,402 @@
+// api.cu -- the C ABI (include/dash_attn.h): argument validation, workspace,
+// stage orchestration on the caller's stream.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+#include <string>
+
+#include "dash_common.cuh"
+#include "kernels.h"
+
+namespace dash {
+int take_device_error_tc();
+int take_device_error_decode();
+}  // namespace dash
+
+using namespace dash;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char *what) {
+    return fail(DASH_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+size_t esize(dash_dtype_t dt) { return dt == DASH_BF16 ? 2 : 4; }
+
+int check_tensor(const dash_tensor_t *t, const char *name) {
+    if (!t) return fail(DASH_ERR_INVALID_ARG, "%s is NULL", name);
+    if (t->dtype != DASH_F32 && t->dtype != DASH_BF16) return fail(DASH_ERR_UNSUPPORTED, "%s: unknown dtype", name);
+    for (int a = 0; a < 4; ++a)
+        if (t->shape[a] < 0) return fail(DASH_ERR_INVALID_ARG, "%s: negative extent", name);
+    if (t->stride[3] != 1) return fail(DASH_ERR_UNSUPPORTED, "%s: the last dimension must be contiguous", name);
+    int64_t n = t->shape[0] * t->shape[1] * t->shape[2] * t->shape[3];
+    if (n > 0 && !t->data) return fail(DASH_ERR_INVALID_ARG, "%s: data is NULL", name);
+    if (reinterpret_cast<uintptr_t>(t->data) % 16) return fail(DASH_ERR_ALIGNMENT, "%s: base not 16-byte aligned", name);
+    for (int a = 0; a < 3; ++a)
+        if ((t->stride[a] * (int64_t)esize(t->dtype)) % 16)
+            return fail(DASH_ERR_ALIGNMENT, "%s: stride %d is not a multiple of 16 bytes", name, a);
+    return DASH_OK;
+}
+
+TView view(const dash_tensor_t *t) { return TView{t->data, t->stride[0], t->stride[1], t->stride[2]}; }
+
+int make_geom(const dash_tensor_t *q, const dash_tensor_t *k, int B, int causal, int gqa, Geom *G) {
+    const int64_t b = q->shape[0], nq = q->shape[1], hq = q->shape[2], d = q->shape[3];
+    const int64_t nk = k->shape[1], hkv = k->shape[2];
+    if (k->shape[0] != b) return fail(DASH_ERR_INVALID_ARG, "q and k batch differ");
+    if (k->shape[3] != d) return fail(DASH_ERR_INVALID_ARG, "q and k head dim differ");
+    if (hkv <= 0 || hq % hkv) return fail(DASH_ERR_INVALID_ARG, "q heads (%lld) not a multiple of kv heads (%lld)",
+                                          (long long)hq, (long long)hkv);
+    if (gqa != hq / hkv) return fail(DASH_ERR_INVALID_ARG, "gqa_groups %d != hq/hkv = %lld", gqa,
+                                     (long long)(hq / hkv));
+    if (gqa < 1 || gqa > 16) return fail(DASH_ERR_UNSUPPORTED, "gqa_groups must be in [1, 16]");
+    if (d != 64 && d != 128) return fail(DASH_ERR_UNSUPPORTED, "head dim %lld not in {64, 128}", (long long)d);
+    if (B != 16 && B != 32 && B != 64 && B != 128)
+        return fail(DASH_ERR_UNSUPPORTED, "block_size %d not in {16, 32, 64, 128}", B);
+    if (causal != 0 && causal != 1) return fail(DASH_ERR_INVALID_ARG, "causal must be 0 or 1");
+    if (nk <= 0) return fail(DASH_ERR_INVALID_ARG, "empty key sequence");
+    if (causal && nq > nk) return fail(DASH_ERR_INVALID_ARG, "causal attention needs nq <= nk");
+    if (nk > (int64_t)1 << 30 || nq > (int64_t)1 << 30) return fail(DASH_ERR_UNSUPPORTED, "sequence too long");
+    G->b = b;
+    G->nq = nq;
+    G->nk = nk;
+    G->hq = (int)hq;
+    G->hkv = (int)hkv;
+    G->g = gqa;
+    G->d = (int)d;
+    G->B = B;
+    G->causal = causal;
+    G->n_chunks = (int)(causal ? nk / B : (nk + B - 1) / B);
+    G->n_blk = (int)((nk + B - 1) / B);
+    G->tile_rows = 128 / gqa;
+    G->n_tiles = (nq + G->tile_rows - 1) / G->tile_rows;
+    G->words = (G->n_chunks + 31) / 32;
+    return DASH_OK;
+}
+
+dash_opts_t default_opts() {
+    dash_opts_t o;
+    memset(&o, 0, sizeof o);
+    o.sigma = 1e8f;
+    o.gamma = 1.0f;
+    return o;
+}
+
+int check_opts(const dash_opts_t &o) {
+    if (!(o.sigma > 0.f) || !isfinite(o.sigma)) return fail(DASH_ERR_INVALID_ARG, "sigma must be > 0");
+    if (!(o.gamma > 0.f) || !isfinite(o.gamma)) return fail(DASH_ERR_INVALID_ARG, "gamma must be > 0");
+    if (o.workspace && reinterpret_cast<uintptr_t>(o.workspace) % 256)
+        return fail(DASH_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+    return DASH_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct WsLayout {
+    size_t kbar, mask, dvals, count, ids, bias, decode, total;
+};
+
+WsLayout ws_layout(const Geom &G, bool need_kbar, bool need_lists, bool need_decode) {
+    WsLayout L{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off += align256(bytes);
+        return o;
+    };
+    L.kbar = need_kbar ? take((size_t)G.b * G.n_chunks * G.hkv * G.d * 4) : 0;
+    L.mask = take((size_t)G.b * G.nq * G.hkv * (size_t)G.words * 4);
+    L.dvals = need_lists ? take((size_t)G.b * G.nq * G.hkv * (size_t)G.n_chunks * 4) : 0;
+    L.count = need_lists ? take((size_t)G.b * G.hkv * G.n_tiles * 4) : 0;
+    L.ids = need_lists ? take((size_t)G.b * G.hkv * G.n_tiles * G.n_blk * 4) : 0;
+    L.bias = need_lists ? take((size_t)G.b * G.hkv * G.n_tiles * G.n_blk * G.tile_rows * 4) : 0;
+    L.decode = need_decode ? take(attn_decode_workspace(G)) : 0;
+    L.total = off;
+    return L;
+}
+
+// Library-managed workspace, one cached allocation per device.
+std::mutex g_ws_mu;
+struct DevWs {
+    void *p = nullptr;
+    size_t bytes = 0;
+};
+DevWs g_ws[128];
+
+int get_workspace(const dash_opts_t &o, size_t need, char **base) {
+    if (o.workspace) {
+        if (o.workspace_bytes < need)
+            return fail(DASH_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", o.workspace_bytes, need);
+        *base = static_cast<char *>(o.workspace);
+        return DASH_OK;
+    }
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 128) return fail(DASH_ERR_UNSUPPORTED, "device index out of range");
+    std::lock_guard<std::mutex> lk(g_ws_mu);
+    DevWs &w = g_ws[dev];
+    if (w.bytes < need) {
+        if (w.p) {
+            // the old buffer may still be in use by queued work
+            e = cudaDeviceSynchronize();
+            if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+            cudaFree(w.p);
+            w.p = nullptr;
+            w.bytes = 0;
+        }
+        size_t want = need + need / 4;
+        e = cudaMalloc(&w.p, want);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(workspace)");
+        w.bytes = want;
+    }
+    *base = static_cast<char *>(w.p);
+    return DASH_OK;
+}
+
+int check_lists(const dash_lists_t *l, const Geom &G) {
+    if (!l->count || !l->ids || !l->bias) return fail(DASH_ERR_INVALID_ARG, "lists: NULL buffer");
+    if (l->n_tiles != G.n_tiles || l->cap != G.n_blk || l->tile_rows != G.tile_rows)
+        return fail(DASH_ERR_INVALID_ARG, "lists geometry (n_tiles %lld, cap %d, tile_rows %d) does not match the "
+                                          "problem (%lld, %d, %d)",
+                    (long long)l->n_tiles, l->cap, l->tile_rows, (long long)G.n_tiles, G.n_blk, G.tile_rows);
+    return DASH_OK;
+}
+
+ListsView lists_view(const dash_lists_t *l) {
+    return ListsView{l->count, l->ids, l->bias, l->n_tiles, l->cap, l->tile_rows};
+}
+
+int run_stage2(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v, dash_tensor_t *out,
+               const Geom &G, const ListsView &LV, const dash_opts_t &o, char *decode_ws, cudaStream_t st) {
+    cudaError_t e;
+    const dash_dtype_t dt = q->dtype;
+    const bool simt = (o.flags & DASH_FLAG_FORCE_SIMT) != 0;
+    if (!simt && decode_ws && attn_decode_supported(G, dt)) {
+        e = launch_attn_decode(view(q), view(k), view(v), view(out), G, LV, decode_ws, st);
+        if (e != cudaSuccess) return cuda_fail(e, "stage 2 (decode)");
+    } else if (!simt && attn_tc_supported(G, dt)) {
+        e = launch_attn_tc(view(q), view(k), view(v), view(out), G, LV, o.flags, st);
+        if (e != cudaSuccess) return cuda_fail(e, "stage 2 (tensor cores)");
+    } else {
+        e = launch_attn_simt(view(q), view(k), view(v), view(out), dt, G, LV, st);
+        if (e != cudaSuccess) return cuda_fail(e, "stage 2 (CUDA cores)");
+    }
+    return DASH_OK;
+}
+
+int validate_qkvo(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v,
+                  const dash_tensor_t *out) {
+    int rc;
+    if ((rc = check_tensor(q, "q")) || (rc = check_tensor(k, "k")) || (rc = check_tensor(v, "v")) ||
+        (rc = check_tensor(out, "out")))
+        return rc;
+    if (q->dtype != k->dtype || q->dtype != v->dtype || q->dtype != out->dtype)
+        return fail(DASH_ERR_INVALID_ARG, "q, k, v and out must share a dtype");
+    for (int a = 0; a < 4; ++a) {
+        if (q->shape[a] != out->shape[a]) return fail(DASH_ERR_INVALID_ARG, "q and out shapes differ");
+        if (k->shape[a] != v->shape[a]) return fail(DASH_ERR_INVALID_ARG, "k and v shapes differ");
+    }
+    return DASH_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+DASH_API const char *dash_version(void) { return "dash-attn-b200 0.1 (sm_100a)"; }
+
+DASH_API const char *dash_last_error(void) { return g_last_error.c_str(); }
+
+DASH_API int dash_opts_init(dash_opts_t *opts) {
+    if (!opts) return fail(DASH_ERR_INVALID_ARG, "opts is NULL");
+    *opts = default_opts();
+    return DASH_OK;
+}
+
+DASH_API int dash_lists_geometry(int64_t batch, int64_t nq, int64_t nk, int hkv, int block_size, int gqa_groups,
+                                 int64_t *n_tiles, int32_t *cap, int32_t *tile_rows, size_t *count_bytes,
+                                 size_t *ids_bytes, size_t *bias_bytes) {
+    if (batch < 0 || nq < 0 || nk <= 0 || hkv <= 0 || block_size <= 0 || gqa_groups < 1 || gqa_groups > 16)
+        return fail(DASH_ERR_INVALID_ARG, "bad lists geometry arguments");
+    const int64_t tr = 128 / gqa_groups;
+    const int64_t nt = (nq + tr - 1) / tr;
+    const int64_t cp = (nk + block_size - 1) / block_size;
+    if (n_tiles) *n_tiles = nt;
+    if (cap) *cap = (int32_t)cp;
+    if (tile_rows) *tile_rows = (int32_t)tr;
+    if (count_bytes) *count_bytes = (size_t)batch * hkv * nt * 4;
+    if (ids_bytes) *ids_bytes = (size_t)batch * hkv * nt * cp * 4;
+    if (bias_bytes) *bias_bytes = (size_t)batch * hkv * nt * cp * tr * 4;
+    return DASH_OK;
+}
+
+DASH_API size_t dash_workspace_bytes(int64_t batch, int64_t nq, int64_t nk, int hq, int hkv, int d, int block_size,
+                                     int causal) {
+    if (hkv <= 0 || hq % hkv || block_size <= 0 || nk <= 0) return 0;
+    Geom G{};
+    G.b = batch;
+    G.nq = nq;
+    G.nk = nk;
+    G.hq = hq;
+    G.hkv = hkv;
+    G.g = hq / hkv;
+    G.d = d;
+    G.B = block_size;
+    G.causal = causal;
+    G.n_chunks = (int)(causal ? nk / block_size : (nk + block_size - 1) / block_size);
+    G.n_blk = (int)((nk + block_size - 1) / block_size);
+    G.tile_rows = 128 / G.g;
+    G.n_tiles = (nq + G.tile_rows - 1) / G.tile_rows;
+    G.words = (G.n_chunks + 31) / 32;
+    return ws_layout(G, true, true, true).total;
+}
+
+DASH_API int dash_pool_keys(const dash_tensor_t *k, int block_size, int causal, float *kbar, void *stream) {
+    int rc = check_tensor(k, "k");
+    if (rc) return rc;
+    if (!kbar) return fail(DASH_ERR_INVALID_ARG, "kbar is NULL");
+    if (reinterpret_cast<uintptr_t>(kbar) % 16) return fail(DASH_ERR_ALIGNMENT, "kbar not 16-byte aligned");
+    // Stage 0 only needs the key geometry: use k as its own (empty) query
+    dash_tensor_t q0 = *k;
+    q0.shape[1] = 0;
+    Geom G;
+    if ((rc = make_geom(&q0, k, block_size, causal, 1, &G))) return rc;
+    cudaError_t e = launch_pool_keys(view(k), k->dtype, G, kbar, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "pool_keys");
+    return DASH_OK;
+}
+
+DASH_API int dash_block_select(const dash_tensor_t *q, const dash_tensor_t *k, int block_size, float alpha,
+                               int causal, int gqa_groups, float *tau, float *w, uint32_t *mask,
+                               const dash_lists_t *lists, const dash_opts_t *opts) {
+    dash_opts_t o = opts ? *opts : default_opts();
+    int rc;
+    if ((rc = check_opts(o))) return rc;
+    if ((rc = check_tensor(q, "q")) || (rc = check_tensor(k, "k"))) return rc;
+    if (q->dtype != k->dtype) return fail(DASH_ERR_INVALID_ARG, "q and k must share a dtype");
+    if (!(alpha > 1.f) || !isfinite(alpha)) return fail(DASH_ERR_INVALID_ARG, "alpha must be > 1");
+    Geom G;
+    if ((rc = make_geom(q, k, block_size, causal, gqa_groups, &G))) return rc;
+    if (lists && (rc = check_lists(lists, G))) return rc;
+    for (const void *p : {(const void *)tau, (const void *)w, (const void *)mask})
+        if (reinterpret_cast<uintptr_t>(p) % 16) return fail(DASH_ERR_ALIGNMENT, "outputs must be 16-byte aligned");
+    if (G.b == 0 || G.nq == 0) return DASH_OK;
+    const bool need_kbar = o.kbar == nullptr;
+    WsLayout WL = ws_layout(G, need_kbar, lists != nullptr, false);
+    char *ws = nullptr;
+    if ((rc = get_workspace(o, WL.total, &ws))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(o.stream);
+    const float *kbar = o.kbar;
+    cudaError_t e;
+    if (need_kbar) {
+        float *kb = reinterpret_cast<float *>(ws + WL.kbar);
+        if ((e = launch_pool_keys(view(k), k->dtype, G, kb, st)) != cudaSuccess) return cuda_fail(e, "pool_keys");
+        kbar = kb;
+    }
+    SelectOut so{tau, w, mask ? mask : reinterpret_cast<uint32_t *>(ws + WL.mask),
+                 lists ? reinterpret_cast<float *>(ws + WL.dvals) : nullptr};
+    if ((e = launch_select_rows(view(q), q->dtype, kbar, G, alpha, o.gamma, o.sigma, so, st)) != cudaSuccess)
+        return cuda_fail(e, "select_rows");
+    if (lists) {
+        if ((e = launch_compact(G, so.mask, so.dvals, lists_view(lists), st)) != cudaSuccess)
+            return cuda_fail(e, "compact");
+    }
+    return DASH_OK;
+}
+
+DASH_API int dash_sparse_attn_fwd(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v,
+                                  dash_tensor_t *out, const dash_lists_t *lists, int block_size, int causal,
+                                  int gqa_groups, const dash_opts_t *opts) {
+    dash_opts_t o = opts ? *opts : default_opts();
+    int rc;
+    if ((rc = check_opts(o))) return rc;
+    if ((rc = validate_qkvo(q, k, v, out))) return rc;
+    if (!lists) return fail(DASH_ERR_INVALID_ARG, "lists is NULL");
+    Geom G;
+    if ((rc = make_geom(q, k, block_size, causal, gqa_groups, &G))) return rc;
+    if ((rc = check_lists(lists, G))) return rc;
+    if (G.b == 0 || G.nq == 0) return DASH_OK;
+    char *ws = nullptr;
+    const size_t dec = attn_decode_supported(G, q->dtype) ? attn_decode_workspace(G) : 0;
+    if (dec && (rc = get_workspace(o, dec, &ws))) return rc;
+    return run_stage2(q, k, v, out, G, lists_view(lists), o, ws, static_cast<cudaStream_t>(o.stream));
+}
+
+DASH_API int dash_attn_fwd_ex(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v,
+                              dash_tensor_t *out, int block_size, float alpha, int causal, int gqa_groups,
+                              const dash_opts_t *opts) {
+    dash_opts_t o = opts ? *opts : default_opts();
+    int rc;
+    if ((rc = check_opts(o))) return rc;
+    if ((rc = validate_qkvo(q, k, v, out))) return rc;
+    if (!(alpha > 1.f) || !isfinite(alpha)) return fail(DASH_ERR_INVALID_ARG, "alpha must be > 1");
+    Geom G;
+    if ((rc = make_geom(q, k, block_size, causal, gqa_groups, &G))) return rc;
+    if (o.kbar && reinterpret_cast<uintptr_t>(o.kbar) % 16) return fail(DASH_ERR_ALIGNMENT, "kbar not aligned");
+    if (G.b == 0 || G.nq == 0) return DASH_OK;
+    const bool need_kbar = o.kbar == nullptr;
+    const bool dec = attn_decode_supported(G, q->dtype) && !(o.flags & DASH_FLAG_FORCE_SIMT);
+    WsLayout WL = ws_layout(G, need_kbar, true, dec);
+    char *ws = nullptr;
+    if ((rc = get_workspace(o, WL.total, &ws))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(o.stream);
+    cudaError_t e;
+    const float *kbar = o.kbar;
+    if (need_kbar) {
+        float *kb = reinterpret_cast<float *>(ws + WL.kbar);
+        if ((e = launch_pool_keys(view(k), k->dtype, G, kb, st)) != cudaSuccess) return cuda_fail(e, "pool_keys");
+        kbar = kb;
+    }
+    SelectOut so{nullptr, nullptr, reinterpret_cast<uint32_t *>(ws + WL.mask), reinterpret_cast<float *>(ws + WL.dvals)};
+    if ((e = launch_select_rows(view(q), q->dtype, kbar, G, alpha, o.gamma, o.sigma, so, st)) != cudaSuccess)
+        return cuda_fail(e, "select_rows");
+    ListsView LV{reinterpret_cast<int32_t *>(ws + WL.count), reinterpret_cast<int32_t *>(ws + WL.ids),
+                 reinterpret_cast<float *>(ws + WL.bias), G.n_tiles, G.n_blk, G.tile_rows};
+    if ((e = launch_compact(G, so.mask, so.dvals, LV, st)) != cudaSuccess) return cuda_fail(e, "compact");
+    return run_stage2(q, k, v, out, G, LV, o, dec ? ws + WL.decode : nullptr, st);
+}
+
+DASH_API int dash_attn_fwd(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v,
+                           dash_tensor_t *out, int block_size, float alpha, int causal, int gqa_groups) {
+    return dash_attn_fwd_ex(q, k, v, out, block_size, alpha, causal, gqa_groups, nullptr);
+}
+
+DASH_API int dash_sync_status(void *stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    int dev_err = take_device_error_tc() | take_device_error_decode();
+    if (dev_err) return fail(DASH_ERR_DEVICE_TIMEOUT, "a device-side bounded wait ran out");
+    return DASH_OK;
+}
+
+DASH_API int dash_release(void) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    std::lock_guard<std::mutex> lk(g_ws_mu);
+    if (dev >= 0 && dev < 128 && g_ws[dev].p) {
+        e = cudaDeviceSynchronize();
+        if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+        cudaFree(g_ws[dev].p);
+        g_ws[dev] = DevWs{};
+    }
+    return DASH_OK;
+}
+
+}  // extern "C"

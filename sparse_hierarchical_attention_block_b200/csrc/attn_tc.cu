@@ -1,0 +1,461 @@
+// attn_tc.cu -- Stage 2 on the 5th-generation tensor cores (tcgen05 + TMEM + TMA), bf16.
+//
+// Prior-induced sparse softmax in the bias form of "DashAttention" §3.4 Prop. 1
+// (App. G Alg. 3): for every row of a query tile
+//   o = sum_j exp(z_j + d_j) v_j / sum_t exp(z_t + d_t),   z_j = <q, k_j>/sqrt(d),
+// over the keys of the chunks in the tile's work list, d_j the list's per-row
+// bias (-inf where the row does not attend the chunk), keys j > p_i masked when
+// causal.  Online softmax in the exp2 domain with fp32 statistics.
+//
+// One CTA per (batch, kv head, query tile of 128/g positions x g heads = 128 rows),
+// the heaviest tiles (latest, causal) first.  Warp roles (192 threads):
+//   warp 0     TMA producer: Q tile once; per step of 128 keys the listed K and V
+//              blocks (one TMA box per chunk and 64-column half, 128-byte swizzle)
+//              and the step's bias rows (bulk copy) into a ring of stages;
+//   warp 1     TMEM allocator and MMA issuer (one thread):
+//              S_j = Q K_j^T  (SS, M=128 N=128 K=d) into one of two TMEM S buffers,
+//              O  += P_j V_j  (TS: P read from TMEM, V from smem as an MN-major operand);
+//   warps 2-5  softmax: thread = TMEM lane = tile row; reads S_j, adds bias, masks,
+//              online max/sum, writes P_j (bf16) over S_j in TMEM, rescales O only
+//              when the running max grows by more than 2^8; epilogue O / l -> bf16.
+// Every mbarrier wait is bounded (globaltimer); on expiry the kernel records a
+// device error, drains what it issued, frees TMEM and returns.
+#include <math.h>
+
+#include "dash_common.cuh"
+#include "kernels.h"
+
+namespace dash {
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kRows = 128;    // MMA M
+constexpr int kStepKeys = 128;  // keys per step = MMA N of S and K of PV
+constexpr int kNS = 2;        // K / V stages
+constexpr int kNM = 4;        // bias / id stages
+constexpr uint32_t kTmemCols = 512;
+constexpr uint64_t kWaitNs = 2000000000ull;      // 2 s
+constexpr uint64_t kWaitNsTest = 20000000ull;    // 20 ms under DASH_FLAG_TEST_TIMEOUT
+
+struct TcParams {
+    CUtensorMap tmQ, tmK, tmV;
+};
+
+__device__ __forceinline__ uint64_t gtimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+template <int D, int BLK>
+struct Smem {
+    static constexpr int kRegion = kRows * 128;                 // bytes of one 64-column, 128-row swizzled region
+    static constexpr int kDh = D / 64;                          // regions per operand
+    static constexpr int kE = kStepKeys / BLK;                  // list entries per step
+    static constexpr int kQ = 0;
+    static constexpr int kK = kQ + kDh * kRegion;
+    static constexpr int kV = kK + kNS * kDh * kRegion;
+    static constexpr int kBias = kV + kNS * kDh * kRegion;       // [kNM][kE * 128] floats (tile_rows <= 128)
+    static constexpr int kIds = kBias + kNM * kE * 128 * 4;     // [kNM][kE] int
+    static constexpr int kBars = (kIds + kNM * kE * 4 + 7) & ~7;
+    // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], m_full[NM], m_empty[NM],
+    //           s_full[2], p_full[2], pv_done[2], fin
+    static constexpr int kNumBars = 1 + 4 * kNS + 2 * kNM + 6 + 1;
+    static constexpr int kMisc = kBars + kNumBars * 8;          // tmem base, abort flag
+    static constexpr int kTotal = kMisc + 16;
+};
+
+struct Bars {
+    uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *m_full, *m_empty, *s_full, *p_full, *pv_done, *fin;
+};
+
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, uint64_t limit_ns, volatile int *abort) {
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 255u) == 0) {
+            const uint64_t now = gtimer();
+            if (it == 0) t0 = now;
+            else if (now - t0 > limit_ns) {
+                report_timeout();
+                *abort = 1;
+                return false;
+            }
+            if (*abort) return false;
+        }
+    }
+}
+
+template <int D, int BLK>
+__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ TcParams tp, TView O, Geom G,
+                                                              ListsView L, int flags) {
+    using S = Smem<D, BLK>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int64_t t = (int64_t)L.n_tiles - 1 - blockIdx.x;  // heaviest (latest) tiles first
+    const int r = blockIdx.y;
+    const int64_t b = blockIdx.z;
+    const int g = G.g, T = L.tile_rows;
+    const size_t tile_idx = ((size_t)b * G.hkv + r) * L.n_tiles + t;
+    const int count = L.count[tile_idx];
+    const int nsteps = (count + S::kE - 1) / S::kE;
+    const bool test_timeout = (flags & DASH_FLAG_TEST_TIMEOUT) != 0;
+    const uint64_t limit_ns = test_timeout ? kWaitNsTest : kWaitNs;
+
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + S::kBars);
+    Bars B;
+    B.q_full = bars;
+    B.k_full = B.q_full + 1;
+    B.k_empty = B.k_full + kNS;
+    B.v_full = B.k_empty + kNS;
+    B.v_empty = B.v_full + kNS;
+    B.m_full = B.v_empty + kNS;
+    B.m_empty = B.m_full + kNM;
+    B.s_full = B.m_empty + kNM;
+    B.p_full = B.s_full + 2;
+    B.pv_done = B.p_full + 2;
+    B.fin = B.pv_done + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + S::kMisc);
+    volatile int *abort = reinterpret_cast<volatile int *>(sm + S::kMisc + 4);
+    float *bias_s = reinterpret_cast<float *>(sm + S::kBias);
+    int *ids_s = reinterpret_cast<int *>(sm + S::kIds);
+
+    if (threadIdx.x == 0) {
+        mbar_init(B.q_full, 1);
+        for (int s = 0; s < kNS; ++s) {
+            mbar_init(B.k_full + s, 1);
+            mbar_init(B.k_empty + s, 1);
+            mbar_init(B.v_full + s, 1);
+            mbar_init(B.v_empty + s, 1);
+        }
+        for (int s = 0; s < kNM; ++s) {
+            mbar_init(B.m_full + s, 1);
+            mbar_init(B.m_empty + s, 128);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(B.s_full + s, 1);
+            mbar_init(B.p_full + s, 128);
+            mbar_init(B.pv_done + s, 1);
+        }
+        mbar_init(B.fin, 1);
+        *abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tO = tmem + 256;  // O accumulator; S / P buffers at tmem + 0 and tmem + 128
+
+    if (warp == 0) {
+        // ------------------------------------------------------------- producer
+        if (lane == 0 && !test_timeout && nsteps > 0) {
+            tma_prefetch_desc(&tp.tmQ);
+            tma_prefetch_desc(&tp.tmK);
+            tma_prefetch_desc(&tp.tmV);
+            mbar_arrive_expect_tx(B.q_full, kRows * D * 2);
+            for (int dh = 0; dh < S::kDh; ++dh)
+                tma_load_4d(sm + S::kQ + dh * S::kRegion, &tp.tmQ, B.q_full, dh * 64, r * g, (int)(t * T), (int)b);
+            const int32_t *ids_g = L.ids + tile_idx * L.cap;
+            const float *bias_g = L.bias + tile_idx * (size_t)L.cap * T;
+            int issued = 0;
+            for (int j = 0; j < nsteps; ++j) {
+                const int e0 = j * S::kE;
+                const int ne = min(S::kE, count - e0);
+                const int ms = j % kNM, ks = j % kNS;
+                if (!wait_bar(B.m_empty + ms, ((j / kNM) & 1) ^ 1, limit_ns, abort)) break;
+                int *ids_st = ids_s + ms * S::kE;
+                for (int e = 0; e < ne; ++e) ids_st[e] = ids_g[e0 + e];
+                mbar_arrive_expect_tx(B.m_full + ms, (uint32_t)(ne * T * 4));
+                bulk_load(bias_s + ms * S::kE * 128, bias_g + (size_t)e0 * T, (uint32_t)(ne * T * 4), B.m_full + ms);
+                if (!wait_bar(B.k_empty + ks, ((j / kNS) & 1) ^ 1, limit_ns, abort)) break;
+                mbar_arrive_expect_tx(B.k_full + ks, (uint32_t)(ne * S::kDh * BLK * 128));
+                for (int e = 0; e < ne; ++e)
+                    for (int dh = 0; dh < S::kDh; ++dh)
+                        tma_load_4d(sm + S::kK + (ks * S::kDh + dh) * S::kRegion + e * BLK * 128, &tp.tmK,
+                                    B.k_full + ks, dh * 64, r, ids_st[e] * BLK, (int)b);
+                if (!wait_bar(B.v_empty + ks, ((j / kNS) & 1) ^ 1, limit_ns, abort)) break;
+                mbar_arrive_expect_tx(B.v_full + ks, (uint32_t)(ne * S::kDh * BLK * 128));
+                for (int e = 0; e < ne; ++e)
+                    for (int dh = 0; dh < S::kDh; ++dh)
+                        tma_load_4d(sm + S::kV + (ks * S::kDh + dh) * S::kRegion + e * BLK * 128, &tp.tmV,
+                                    B.v_full + ks, dh * 64, r, ids_st[e] * BLK, (int)b);
+                issued = j + 1;
+            }
+            if (*abort) {
+                // drain: every copy issued must land before the CTA's smem goes away
+                for (int j = max(0, issued - kNS); j < issued; ++j) {
+                    wait_bar(B.k_full + j % kNS, (j / kNS) & 1, kWaitNsTest, abort);
+                    wait_bar(B.v_full + j % kNS, (j / kNS) & 1, kWaitNsTest, abort);
+                }
+                for (int j = max(0, issued - kNM); j < issued; ++j)
+                    wait_bar(B.m_full + j % kNM, (j / kNM) & 1, kWaitNsTest, abort);
+                wait_bar(B.q_full, 0, kWaitNsTest, abort);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_bf16_f32(kRows, kStepKeys, 0, 0);
+            constexpr uint32_t idPV = idesc_bf16_f32(kRows, D, 0, 1);
+            const uint32_t q_base = smem_u32(sm + S::kQ);
+            const uint32_t k_base = smem_u32(sm + S::kK);
+            const uint32_t v_base = smem_u32(sm + S::kV);
+            bool ok = nsteps == 0 || wait_bar(B.q_full, 0, limit_ns, abort);
+            for (int j = 0; ok && j <= nsteps; ++j) {
+                if (j < nsteps) {
+                    const int ks = j % kNS;
+                    if (!(ok = wait_bar(B.k_full + ks, (j / kNS) & 1, limit_ns, abort))) break;
+                    if (j >= 2 && !(ok = wait_bar(B.pv_done + (j & 1), ((j - 2) >> 1) & 1, limit_ns, abort))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t qa = q_base + (kk / 4) * S::kRegion + (kk % 4) * 32;
+                        const uint32_t kb = k_base + (ks * S::kDh + kk / 4) * S::kRegion + (kk % 4) * 32;
+                        mma_ss((tmem + (uint32_t)(j & 1) * 128u), smem_desc_sw128(qa, 16, 1024), smem_desc_sw128(kb, 16, 1024), idS,
+                               kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(B.s_full + (j & 1));
+                    mma_commit(B.k_empty + ks);
+                }
+                if (j >= 1) {
+                    const int jj = j - 1, vs = jj % kNS;
+                    const int ne = min(S::kE, count - jj * S::kE);
+                    if (!(ok = wait_bar(B.p_full + (jj & 1), (jj >> 1) & 1, limit_ns, abort))) break;
+                    if (!(ok = wait_bar(B.v_full + vs, (jj / kNS) & 1, limit_ns, abort))) break;
+                    tc_fence_after();
+                    const int nks = ne * BLK / 16;
+                    for (int kk = 0; kk < nks; ++kk) {
+                        const uint32_t vb = v_base + (vs * S::kDh) * S::kRegion + kk * 2048;
+                        mma_ts(tO, (tmem + (uint32_t)(jj & 1) * 128u) + kk * 8, smem_desc_sw128(vb, S::kRegion, 1024), idPV,
+                               (jj > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(B.v_empty + vs);
+                    mma_commit(B.pv_done + (jj & 1));
+                }
+            }
+            // every MMA this thread issued has completed before TMEM is freed
+            mma_commit(B.fin);
+            wait_bar(B.fin, 0, kWaitNsTest * 50, abort);
+        }
+    } else {
+        // ------------------------------------------------------------- softmax warpgroup
+        const int quad = warp & 3;
+        const int m = quad * 32 + lane;  // TMEM lane == tile row
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const int pos = m / g;
+        const int hh = m % g;
+        const int64_t i = t * T + pos;
+        const bool row_ok = i < G.nq;
+        const int64_t p_row = row_pos(G, i);
+        const float sl2 = rsqrtf((float)D) * 1.4426950408889634f;
+        float m_run = -INFINITY, l_run = 0.f;
+        bool ok = true;
+        for (int j = 0; j < nsteps; ++j) {
+            const int ms = j % kNM;
+            const int ne = min(S::kE, count - j * S::kE);
+            if (!(ok = wait_bar(B.m_full + ms, (j / kNM) & 1, limit_ns, abort))) break;
+            int idv[S::kE];
+            float bl2[S::kE];
+#pragma unroll
+            for (int e = 0; e < S::kE; ++e) {
+                idv[e] = e < ne ? ids_s[ms * S::kE + e] : -1;
+                bl2[e] = e < ne ? bias_s[ms * S::kE * 128 + e * T + pos] * 1.4426950408889634f : -INFINITY;
+            }
+            mbar_arrive(B.m_empty + ms);
+            if (!(ok = wait_bar(B.s_full + (j & 1), (j >> 1) & 1, limit_ns, abort))) break;
+            tc_fence_after();
+            float s[kStepKeys];
+#pragma unroll
+            for (int c = 0; c < kStepKeys / 32; ++c) {
+                uint32_t u[32];
+                tmem_ld32((tmem + (uint32_t)(j & 1) * 128u) + lane_off + c * 32, u);
+                tmem_wait_ld();
+#pragma unroll
+                for (int x = 0; x < 32; ++x) s[c * 32 + x] = __uint_as_float(u[x]);
+            }
+            float mx = -INFINITY;
+#pragma unroll
+            for (int kc = 0; kc < kStepKeys; ++kc) {
+                const int e = kc / BLK;
+                const int64_t key = (int64_t)idv[e] * BLK + (kc % BLK);
+                const bool vis = idv[e] >= 0 && key < G.nk && !(G.causal && key > p_row) && row_ok;
+                const float v = vis ? fmaf(s[kc], sl2, bl2[e]) : -INFINITY;
+                s[kc] = v;
+                mx = fmaxf(mx, v);
+            }
+            float m_use = m_run;
+            if (mx > -INFINITY) {
+                if (m_run == -INFINITY) {
+                    m_use = mx;
+                } else if (mx > m_run + 8.f) {
+                    // rescale O and l to the new maximum (O holds every PV up to step j-1)
+                    m_use = mx;
+                    const float f = ex2(m_run - mx);
+                    l_run *= f;
+                    if (j > 0) {
+                        if (!(ok = wait_bar(B.pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, limit_ns, abort))) break;
+                        tc_fence_after();
+#pragma unroll
+                        for (int c = 0; c < D / 32; ++c) {
+                            uint32_t u[32];
+                            tmem_ld32(tO + lane_off + c * 32, u);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int x = 0; x < 32; ++x) u[x] = __float_as_uint(__uint_as_float(u[x]) * f);
+                            tmem_st32(tO + lane_off + c * 32, u);
+                        }
+                    }
+                }
+                m_run = m_use;
+            }
+            float psum = 0.f;
+#pragma unroll
+            for (int c = 0; c < kStepKeys / 64; ++c) {
+                uint32_t u[32];
+#pragma unroll
+                for (int x = 0; x < 32; ++x) {
+                    const float p0 = (m_use == -INFINITY) ? 0.f : ex2(s[c * 64 + 2 * x] - m_use);
+                    const float p1 = (m_use == -INFINITY) ? 0.f : ex2(s[c * 64 + 2 * x + 1] - m_use);
+                    psum += p0 + p1;
+                    u[x] = pack_bf16x2(p0, p1);
+                }
+                tmem_st32((tmem + (uint32_t)(j & 1) * 128u) + lane_off + c * 32, u);
+            }
+            l_run += psum;
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(B.p_full + (j & 1));
+        }
+        // epilogue: O / l -> bf16
+        if (ok && !*abort) {
+            bool have = nsteps > 0;
+            if (have) have = wait_bar(B.pv_done + ((nsteps - 1) & 1), ((nsteps - 1) >> 1) & 1, limit_ns, abort);
+            tc_fence_after();
+            if (row_ok && (have || nsteps == 0)) {
+                __nv_bfloat16 *op = reinterpret_cast<__nv_bfloat16 *>(const_cast<void *>(O.p)) + b * O.s0 +
+                                    i * O.s1 + (int64_t)(r * g + hh) * O.s2;
+                const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t u[32];
+                    if (nsteps > 0) {
+                        tmem_ld32(tO + lane_off + c * 32, u);
+                        tmem_wait_ld();
+                    } else {
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) u[x] = 0u;
+                    }
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int x = 0; x < 16; ++x)
+                        pk[x] = pack_bf16x2(__uint_as_float(u[2 * x]) * inv, __uint_as_float(u[2 * x + 1]) * inv);
+                    uint4 *dst = reinterpret_cast<uint4 *>(op + c * 32);
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 4-D bf16 map over [b][seq][heads][d] (dims innermost first), box {64, box_h, box_s, 1}, 128-byte swizzle.
+bool make_map(CUtensorMap *m, const TView &v, int64_t b, int64_t seq, int64_t heads, int d, int box_h, int box_s) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)seq, (cuuint64_t)b};
+    cuuint64_t strides[3] = {(cuuint64_t)v.s2 * 2, (cuuint64_t)v.s1 * 2, (cuuint64_t)v.s0 * 2};
+    if (b == 1) strides[2] = (cuuint64_t)seq * v.s1 * 2;  // unused dimension: any valid stride
+    cuuint32_t box[4] = {64, (cuuint32_t)box_h, (cuuint32_t)box_s, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(v.p), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int D, int BLK>
+cudaError_t launch_t(const TcParams &tp, const TView &O, const Geom &G, const ListsView &L, int flags,
+                     cudaStream_t st) {
+    using S = Smem<D, BLK>;
+    const size_t smem = S::kTotal + 1024;
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)L.n_tiles, (unsigned)G.hkv, (unsigned)G.b);
+    attn_tc_kernel<D, BLK><<<grid, kThreads, smem, st>>>(tp, O, G, L, flags);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool attn_tc_supported(const Geom &G, dash_dtype_t dt) {
+    if (dt != DASH_BF16) return false;
+    if (G.d != 64 && G.d != 128) return false;
+    if (G.g & (G.g - 1)) return false;  // tile_rows * g must be exactly 128
+    if (G.tile_rows * G.g != kRows) return false;
+    if (G.nq > 0x7fffffff || G.nk > 0x7fffffff) return false;
+    return encode_fn() != nullptr;
+}
+
+cudaError_t launch_attn_tc(const TView &Q, const TView &K, const TView &V, const TView &O, const Geom &G,
+                           const ListsView &L, int flags, cudaStream_t st) {
+    if (G.nq == 0 || G.b == 0) return cudaSuccess;
+    TcParams tp;
+    if (!make_map(&tp.tmQ, Q, G.b, G.nq, G.hq, G.d, G.g, G.tile_rows)) return cudaErrorInvalidValue;
+    if (!make_map(&tp.tmK, K, G.b, G.nk, G.hkv, G.d, 1, G.B)) return cudaErrorInvalidValue;
+    if (!make_map(&tp.tmV, V, G.b, G.nk, G.hkv, G.d, 1, G.B)) return cudaErrorInvalidValue;
+#define DASH_TC_CASE(DD, BB) \
+    if (G.d == DD && G.B == BB) return launch_t<DD, BB>(tp, O, G, L, flags, st);
+    DASH_TC_CASE(128, 64)
+    DASH_TC_CASE(128, 128)
+    DASH_TC_CASE(128, 32)
+    DASH_TC_CASE(128, 16)
+    DASH_TC_CASE(64, 64)
+    DASH_TC_CASE(64, 128)
+    DASH_TC_CASE(64, 32)
+    DASH_TC_CASE(64, 16)
+#undef DASH_TC_CASE
+    return cudaErrorNotSupported;
+}
+
+int take_device_error_tc() { return take_device_error_local(); }
+
+}  // namespace dash

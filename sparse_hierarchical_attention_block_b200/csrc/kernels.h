@@ -1,0 +1,34 @@
+// kernels.h -- host-side launchers of the DashAttention kernels (internal).
+#pragma once
+
+#include "dash_common.cuh"
+
+namespace dash {
+
+// Stage 0 (pool_keys.cu)
+cudaError_t launch_pool_keys(const TView &K, dash_dtype_t dt, const Geom &G, float *kbar, cudaStream_t st);
+
+// Stage 1 (block_select.cu)
+struct SelectOut {
+    float *tau;        // [b][nq][hq] or null
+    float *w;          // [b][nq][hkv][n_chunks] or null
+    uint32_t *mask;    // [b][nq][hkv][words] (required)
+    float *dvals;      // [b][nq][hkv][n_chunks] bias of routed chunks (required when lists are built)
+};
+cudaError_t launch_select_rows(const TView &Q, dash_dtype_t dt, const float *kbar, const Geom &G, float alpha,
+                               float gamma, float sigma, const SelectOut &o, cudaStream_t st);
+cudaError_t launch_compact(const Geom &G, const uint32_t *mask, const float *dvals, const ListsView &L,
+                           cudaStream_t st);
+
+// Stage 2 (attn_simt.cu, attn_tc.cu, attn_decode.cu)
+cudaError_t launch_attn_simt(const TView &Q, const TView &K, const TView &V, const TView &O, dash_dtype_t dt,
+                             const Geom &G, const ListsView &L, cudaStream_t st);
+bool attn_tc_supported(const Geom &G, dash_dtype_t dt);
+cudaError_t launch_attn_tc(const TView &Q, const TView &K, const TView &V, const TView &O, const Geom &G,
+                           const ListsView &L, int flags, cudaStream_t st);
+bool attn_decode_supported(const Geom &G, dash_dtype_t dt);
+size_t attn_decode_workspace(const Geom &G);
+cudaError_t launch_attn_decode(const TView &Q, const TView &K, const TView &V, const TView &O, const Geom &G,
+                               const ListsView &L, void *work, cudaStream_t st);
+
+}  // namespace dash

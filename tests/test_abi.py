@@ -1,0 +1,124 @@
+"""The C-ABI library on the CPU: it builds, loads, exports every entry point
+that include/dash_attn.h declares, and its host-side validation rejects bad
+arguments before touching a GPU."""
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+import sparse_hierarchical_attention_block_b200 as dash
+from sparse_hierarchical_attention_block_b200 import _Opts, _Tensor, build
+
+ROOT = Path(__file__).resolve().parents[1]
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return dash.load_library()
+
+
+def _declared_symbols():
+    text = (ROOT / "include" / "dash_attn.h").read_text()
+    return sorted(set(re.findall(r"DASH_API\s+[\w\s\*]+?\b(dash_\w+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared_symbols()
+    assert len(declared) >= 12
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(declared) == set(dash.EXPORTS)
+    assert b"sm_100a" in lib.dash_version()
+
+
+def test_library_is_sm100a_only():
+    """The shared object carries sm_100a device code (and is self-contained)."""
+    data = (ROOT / "sparse_hierarchical_attention_block_b200" / "libdash_attn.so").read_bytes()
+    assert b"sm_100a" in data
+
+
+def test_lists_geometry(lib):
+    nt, cap, tr = dash.lists_geometry(2, 1000, 1000, 4, 64, 4)
+    assert (tr, nt, cap) == (32, -(-1000 // 32), -(-1000 // 64))
+    nt, cap, tr = dash.lists_geometry(1, 1, 131072, 8, 64, 4)
+    assert (nt, cap, tr) == (1, 2048, 32)
+    cb, ib, bb = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    rc = lib.dash_lists_geometry(2, 1000, 1000, 4, 64, 4, None, None, None, ctypes.byref(cb), ctypes.byref(ib),
+                                 ctypes.byref(bb))
+    assert rc == 0
+    assert cb.value == 2 * 4 * 32 * 4 and ib.value == 2 * 4 * 32 * 16 * 4 and bb.value == ib.value * 32
+    assert dash.dash_workspace_bytes(1, 8192, 8192, 32, 8, 128, 64) > 0
+
+
+def _t(data, dtype, shape, stride=None):
+    t = _Tensor()
+    t.data = data
+    t.dtype = dtype
+    if stride is None:
+        stride = [shape[1] * shape[2] * shape[3], shape[2] * shape[3], shape[3], 1]
+    for a in range(4):
+        t.shape[a] = shape[a]
+        t.stride[a] = stride[a]
+    return t
+
+
+FAKE = 1 << 20  # never dereferenced: validation fails first
+
+
+@pytest.mark.parametrize("case,code", [
+    ("dtype_mix", dash.DASH_ERR_INVALID_ARG),
+    ("shape_mismatch", dash.DASH_ERR_INVALID_ARG),
+    ("gqa_wrong", dash.DASH_ERR_INVALID_ARG),
+    ("head_dim", dash.DASH_ERR_UNSUPPORTED),
+    ("block", dash.DASH_ERR_UNSUPPORTED),
+    ("alpha", dash.DASH_ERR_INVALID_ARG),
+    ("misaligned", dash.DASH_ERR_ALIGNMENT),
+    ("stride", dash.DASH_ERR_ALIGNMENT),
+    ("causal_long_q", dash.DASH_ERR_INVALID_ARG),
+    ("null", dash.DASH_ERR_INVALID_ARG),
+    ("sigma", dash.DASH_ERR_INVALID_ARG),
+])
+def test_validation_rejects(lib, case, code):
+    B, alpha, gqa, causal = 64, 1.5, 4, 1
+    q = _t(FAKE, dash.DASH_BF16, [1, 256, 8, 128])
+    k = _t(FAKE, dash.DASH_BF16, [1, 256, 2, 128])
+    v = _t(FAKE, dash.DASH_BF16, [1, 256, 2, 128])
+    o = _t(FAKE, dash.DASH_BF16, [1, 256, 8, 128])
+    opts = _Opts()
+    lib.dash_opts_init(ctypes.byref(opts))
+    if case == "dtype_mix":
+        v.dtype = dash.DASH_F32
+    elif case == "shape_mismatch":
+        o.shape[2] = 4
+    elif case == "gqa_wrong":
+        gqa = 2
+    elif case == "head_dim":
+        for t in (q, k, v, o):
+            t.shape[3] = 96
+    elif case == "block":
+        B = 48
+    elif case == "alpha":
+        alpha = 1.0
+    elif case == "misaligned":
+        q.data = FAKE + 2
+    elif case == "stride":
+        k.stride[1] = 2 * 128 + 4
+    elif case == "causal_long_q":
+        q.shape[1] = o.shape[1] = 300
+    elif case == "null":
+        q.data = None
+    elif case == "sigma":
+        opts.sigma = 0.0
+    rc = lib.dash_attn_fwd_ex(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), ctypes.byref(o), B, alpha, causal,
+                              gqa, ctypes.byref(opts))
+    assert rc == code, lib.dash_last_error()
+    assert lib.dash_last_error()
+
+
+def test_opts_defaults(lib):
+    o = _Opts()
+    assert lib.dash_opts_init(ctypes.byref(o)) == 0
+    assert o.sigma == pytest.approx(1e8) and o.gamma == 1.0 and o.flags == 0 and not o.workspace
+    assert lib.dash_opts_init(None) == dash.DASH_ERR_INVALID_ARG

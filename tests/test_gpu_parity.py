@@ -1,0 +1,147 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs.  Small cases run every row; the large workloads run every
+row where the oracle finishes in seconds (8K prefill, decode) and stratified
+row samples otherwise (32K, 128K)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_hierarchical_attention_block_b200 as dash
+import synthetic
+from parity import check_forward, sample_rows, to_np32
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.fail("the gpu tests need a CUDA device")
+    dash.load_library()
+    oracle.set_threads(oracle.max_threads())
+    yield
+    dash.dash_release()
+
+
+def _run(q, k, v, block, alpha, causal, **opts):
+    out = torch.empty_like(q)
+    dash.dash_attn_fwd(q, k, v, out, block, alpha, causal, q.shape[2] // k.shape[2], **opts)
+    assert dash.dash_sync_status() == 0
+    return out
+
+
+def _planted(b, nq, nk, hq, hkv, d, block, dtype, seed, causal=True, planted=True):
+    w = synthetic.Workload("case", b, nq, nk, hq, hkv, d, block, 1.5, causal, dtype, seed, planted,
+                           amax_key="b64")
+    q, k, v = synthetic.make_inputs(w, "cuda")
+    return q, k, v
+
+
+@pytest.mark.parametrize("sigma", [1e8, 1.0])
+def test_tiny_full(sigma):
+    w = synthetic.WORKLOADS["tiny"]
+    q, k, v = synthetic.make_inputs(w, "cuda")
+    out = _run(q, k, v, w.block, w.alpha, True, sigma=sigma)
+    check_forward(q, k, v, out, w.block, w.alpha, True, sigma=sigma, label=f"tiny sigma={sigma:g}")
+
+
+CASES = [
+    # b, nq, nk, hq, hkv, d, B, dtype, alpha, causal, sigma
+    (2, 512, 512, 8, 2, 128, 64, "bf16", 1.5, True, 1.0),
+    (1, 512, 512, 8, 2, 128, 64, "bf16", 1.25, True, 1.0),
+    (1, 512, 512, 8, 2, 128, 64, "bf16", 2.0, True, 1e8),
+    (1, 1000, 1000, 8, 2, 128, 64, "bf16", 1.5, True, 1.0),      # ragged: nk % B != 0
+    (1, 130, 1000, 8, 2, 128, 64, "bf16", 1.5, True, 1.0),       # nq < nk, bottom-right alignment
+    (1, 700, 700, 4, 4, 64, 32, "bf16", 1.5, True, 3.0),         # hq == hkv, d = 64
+    (1, 600, 600, 16, 2, 128, 16, "bf16", 1.5, True, 1.0),       # g = 8, B = 16
+    (1, 1024, 1024, 8, 2, 128, 128, "bf16", 1.5, True, 1.0),     # B = 128
+    (1, 300, 1000, 4, 2, 64, 64, "bf16", 1.5, False, 1.0),       # non-causal, partial chunk routed
+    (1, 777, 777, 2, 1, 64, 64, "f32", 1.5, True, 1.0),          # fp32, g = 2
+    (1, 40, 40, 4, 2, 64, 64, "bf16", 1.5, True, 1.0),           # no visible chunk at all
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[f"c{i}" for i in range(len(CASES))])
+def test_small_cases(case):
+    b, nq, nk, hq, hkv, d, B, dt, alpha, causal, sigma = case
+    q, k, v = _planted(b, nq, nk, hq, hkv, d, B, dt, seed=100 + nq, causal=causal)
+    out = _run(q, k, v, B, alpha, causal, sigma=sigma)
+    check_forward(q, k, v, out, B, alpha, causal, sigma=sigma, label=f"case {case}")
+
+
+@pytest.mark.parametrize("case", CASES[:3] + CASES[9:10], ids=["c0", "c1", "c2", "c9"])
+def test_simt_path_matches_oracle(case):
+    """The CUDA-core Stage 2 (forced) also meets the bar."""
+    b, nq, nk, hq, hkv, d, B, dt, alpha, causal, sigma = case
+    q, k, v = _planted(b, nq, nk, hq, hkv, d, B, dt, seed=100 + nq, causal=causal)
+    out = _run(q, k, v, B, alpha, causal, sigma=sigma, flags=dash.DASH_FLAG_FORCE_SIMT)
+    check_forward(q, k, v, out, B, alpha, causal, sigma=sigma, label=f"simt {case}")
+
+
+@pytest.mark.parametrize("dt,causal", [("bf16", True), ("bf16", False), ("f32", True)])
+def test_uniform_all_chunk_prior_is_dense_attention(dt, causal):
+    """Stage 2 alone on lists that route every visible chunk with bias 0 equals
+    dense softmax attention (the paper's KL-to-uniform statement, Eq. 5)."""
+    b, nq, nk, hq, hkv, d, B = 1, 300, 520, 8, 2, 128, 64
+    q, k, v = _planted(b, nq, nk, hq, hkv, d, B, dt, seed=7, causal=causal, planted=False)
+    g = hq // hkv
+    L = dash.make_lists(q, k, B, g)
+    nblk = -(-nk // B)
+    for t in range(L.n_tiles):
+        i0 = t * L.tile_rows
+        last = min(i0 + L.tile_rows, nq) - 1
+        hi = min((last + nk - nq) // B, nblk - 1) if causal else nblk - 1
+        L.count[:, :, t] = hi + 1
+        L.ids[:, :, t, :hi + 1] = torch.arange(hi + 1, dtype=torch.int32, device="cuda")
+    L.bias.zero_()
+    out = torch.empty_like(q)
+    dash.dash_sparse_attn_fwd(q, k, v, out, L, B, causal, g)
+    assert dash.dash_sync_status() == 0
+    ref = oracle.dense_attention(to_np32(q[0]), to_np32(k[0]), to_np32(v[0]), causal=causal)
+    err = np.abs(to_np32(out[0]) - ref)
+    tol = (2e-2, 2e-3) if dt == "bf16" else (1e-4, 1e-5)
+    assert err.max() <= tol[0] and err.mean() <= tol[1], (err.max(), err.mean())
+
+
+def test_deterministic():
+    q, k, v = _planted(1, 512, 512, 8, 2, 128, 64, "bf16", seed=5)
+    a = _run(q, k, v, 64, 1.5, True, sigma=1.0)
+    b = _run(q, k, v, 64, 1.5, True, sigma=1.0)
+    assert torch.equal(a, b)
+
+
+def test_prefill8k_full():
+    w = synthetic.WORKLOADS["prefill8k"]
+    q, k, v = synthetic.make_inputs(w, "cuda")
+    for sigma in (1e8, 1.0):
+        out = _run(q, k, v, w.block, w.alpha, True, sigma=sigma)
+        check_forward(q, k, v, out, w.block, w.alpha, True, sigma=sigma, label=f"prefill8k sigma={sigma:g}")
+
+
+def test_prefill32k_sampled():
+    w = synthetic.WORKLOADS["prefill32k"]
+    q, k, v = synthetic.make_inputs(w, "cuda")
+    rows = sample_rows(w.nq, w.block, 1024, seed=32)
+    for sigma in (1e8, 1.0):
+        out = _run(q, k, v, w.block, w.alpha, True, sigma=sigma)
+        st = check_forward(q, k, v, out, w.block, w.alpha, True, sigma=sigma, rows=rows,
+                           label=f"prefill32k sigma={sigma:g}")
+    assert 0.6 < st["sparsity"] < 0.9
+
+
+def test_decode_full():
+    w = synthetic.WORKLOADS["decode"]
+    q, k, v = synthetic.make_inputs(w, "cuda")
+    for sigma in (1e8, 1.0):
+        out = _run(q, k, v, w.block, w.alpha, True, sigma=sigma)
+        check_forward(q, k, v, out, w.block, w.alpha, True, sigma=sigma, label=f"decode sigma={sigma:g}")
+
+
+@pytest.mark.parametrize("alpha", [1.25, 1.5, 2.0])
+def test_prefill128k_sampled(alpha):
+    w = synthetic.WORKLOADS["prefill128k"]
+    q, k, v = synthetic.make_inputs(w, "cuda")
+    rows = sample_rows(w.nq, w.block, 512, seed=128)
+    out = _run(q, k, v, w.block, alpha, True, sigma=1.0)
+    check_forward(q, k, v, out, w.block, alpha, True, sigma=1.0, rows=rows, label=f"prefill128k alpha={alpha}")
