@@ -1,0 +1,401 @@
+"""Benchmark of the DashAttention forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill8k|prefill32k|prefill128k|decode]
+                    [--impl ours|reference] [--no-cpu-baseline]
+
+One step = one full forward (Stage 0 pooling, Stage 1 routing + work lists,
+Stage 2 sparse attention) of the workload on synthetic seeded inputs resident
+in HBM.  Prints ONE JSON line (rank 0).
+
+Metric: selected-block Stage-2 FLOPs per second for prefill (TFLOP/s), selected
+K/V bytes per second for decode (GB/s) -- the algorithmic work the method must
+do, not the dense work it avoids:
+  F2 = sum_{b,i,h} 4 d (B |R_i| + (p_i mod B) + 1)     (routed chunks + diagonal keys)
+  Y  = sum_{b,r} (B |R^(r)| + diagonal keys) d * 2 tensors * 2 bytes
+Timing: CUDA events on the launching stream, L2 flushed (a 256 MiB write)
+before every timed step, outside the event pair; warm-up steps untimed.
+Multi-GPU (torchrun): every rank runs an independent replica of the workload
+(the method's (batch, kv-head) units share nothing: no collective); value is
+the work of all ranks over the max-over-ranks time ("scaling": "weak").
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+import torch  # noqa: E402
+
+import synthetic  # noqa: E402
+
+METRIC = "DashAttention fwd ms & TFLOP/s (prefill) / GB/s (decode), % of B200 roofline"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# work accounting (bench-side, from the routing mask the library exports)
+# ---------------------------------------------------------------------------
+
+def routed_counts(dash, q, k, w, alpha, sigma):
+    """|R_i^(r)| per (b, i, r) from dash_block_select's bit-packed mask."""
+    nch = dash.n_chunks(w.nk, w.block, True)
+    words = max((nch + 31) // 32, 1)
+    mask = torch.zeros(w.batch, w.nq, w.hkv, words, dtype=torch.int32, device=q.device)
+    dash.dash_block_select(q, k, w.block, alpha, True, mask=mask, sigma=sigma)
+    m = mask.to(torch.int64) & 0xFFFFFFFF
+    cnt = torch.zeros(w.batch, w.nq, w.hkv, dtype=torch.int64, device=q.device)
+    for bit in range(32):
+        cnt += (m >> bit).bitwise_and(1).sum(-1)
+    return cnt
+
+
+def work_of(w, cnt, lists):
+    """Selected FLOPs F2, selected K/V bytes Y, sparsity, and the tile-union FLOPs the kernel executes."""
+    i = torch.arange(w.nq, device=cnt.device, dtype=torch.int64)
+    p = i + w.nk - w.nq
+    diag = (p % w.block + 1).view(1, -1, 1)                        # keys of the diagonal branch
+    keys = w.block * cnt + diag                                      # [b, nq, hkv]
+    f2 = float((4 * w.d * keys.sum()).item()) * w.g                  # every head of the group
+    y = float((keys.sum() * w.d * 2 * 2).item())                     # K and V, bf16, per kv head
+    vis = torch.clamp(p // w.block, max=w.nk // w.block).view(1, -1, 1).expand_as(cnt)
+    sparsity = 1.0 - float(cnt.sum().item()) / max(float(vis.sum().item()), 1.0)
+    exec_f = None
+    if lists is not None:
+        exec_f = float((lists.count.to(torch.int64).sum() * w.block * 128 * 4 * w.d).item())
+    return f2, y, sparsity, exec_f
+
+
+# ---------------------------------------------------------------------------
+# our implementation
+# ---------------------------------------------------------------------------
+
+def run_ours(args, rank, world, device):
+    import sparse_hierarchical_attention_block_b200 as dash
+
+    dash.load_library()
+    w = synthetic.WORKLOADS[args.workload]
+    alpha = args.alpha or w.alpha
+    sigma = args.sigma
+    decode = w.nq == 1  # one new query token per sequence
+    torch.manual_seed(0)
+    q, k, v = synthetic.make_inputs(w, device)
+    out = torch.empty_like(q)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+
+    kbar = None
+    if decode:
+        # the chunk-summary cache persists across decode steps: pooled once, outside the step
+        nch = dash.n_chunks(w.nk, w.block, True)
+        kbar = torch.empty(w.batch, nch, w.hkv, w.d, dtype=torch.float32, device=device)
+        dash.dash_pool_keys(k, w.block, True, kbar)
+    opts = dict(sigma=sigma)
+    if kbar is not None:
+        opts["kbar"] = kbar
+
+    def step():
+        dash.dash_attn_fwd(q, k, v, out, w.block, alpha, True, w.g, **opts)
+
+    lists = dash.make_lists(q, k, w.block, w.g)
+    dash.dash_block_select(q, k, w.block, alpha, True, lists=lists, **opts)
+    cnt = routed_counts(dash, q, k, w, alpha, sigma)
+    f2, y, sparsity, exec_f = work_of(w, cnt, lists)
+    torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    rc = dash.dash_sync_status()
+    if rc != 0:
+        raise RuntimeError(f"warm-up failed with status {rc}")
+
+    def timed(fn, n):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        for a, b in ev:
+            flush.fill_(1.0)  # evict L2 (outside the timed pair)
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in ev]
+
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    smi_id = vis.split(",")[torch.cuda.current_device()] if vis else str(torch.cuda.current_device())
+    with ClockSampler(smi_id) as cs:
+        times = timed(step, args.steps)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+    rc = dash.dash_sync_status()
+    if rc != 0:
+        raise RuntimeError(f"timed steps failed with status {rc}")
+    ms = sum(times) / len(times)
+
+    # dominant kernel alone (Stage 2 on the same lists), and Stages 0-1 alone
+    n_k = max(3, args.steps)
+    t_stage2 = timed(lambda: dash.dash_sparse_attn_fwd(q, k, v, out, lists, w.block, True, w.g, **opts), n_k)
+    t_stage01 = timed(lambda: dash.dash_block_select(q, k, w.block, alpha, True, lists=lists, **opts), n_k)
+    ms2 = sum(t_stage2) / len(t_stage2)
+    ms01 = sum(t_stage01) / len(t_stage01)
+
+    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    qh, kh, vh = q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory()
+    oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def e2e_step():
+        q.copy_(qh, non_blocking=True)
+        k.copy_(kh, non_blocking=True)
+        v.copy_(vh, non_blocking=True)
+        if decode:
+            pass  # the chunk-summary cache stays on the device across decode steps
+        step()
+        oh.copy_(out, non_blocking=True)
+
+    e2e_times = timed(e2e_step, max(2, min(args.steps, 5)))
+    ms_e2e = sum(e2e_times) / len(e2e_times)
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = oh.numel() * oh.element_size()
+
+    # max over ranks
+    t = torch.tensor([ms, ms2, ms01, ms_e2e], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms, ms2, ms01, ms_e2e = t.tolist()
+
+    peaks = load_peaks()
+    if decode:
+        unit, work = "GB/s", y
+        per = lambda msx: work * world / (msx * 1e-3) / 1e9  # noqa: E731
+        achieved = work / (ms2 * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                "kernel": "attn_decode (+ combine)", "peak_source": peaks["source"] + " hbm_gbs"}
+    else:
+        unit, work = "TFLOP/s", f2
+        per = lambda msx: work * world / (msx * 1e-3) / 1e12  # noqa: E731
+        achieved = work / (ms2 * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": None,
+                "kernel": "attn_tc (Stage 2)", "peak_source": peaks["source"] + " bf16_tflops (burst)"}
+    res = {
+        "metric": METRIC,
+        "value": round(per(ms), 3),
+        "unit": unit,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded planted-block generator)",
+        "config": {"workload": w.name, "batch": w.batch, "nq": w.nq, "nk": w.nk, "hq": w.hq, "hkv": w.hkv,
+                   "d": w.d, "block": w.block, "alpha": alpha, "sigma": sigma, "gamma": 1.0, "causal": True,
+                   "a_max": synthetic.amax_for(w), "sparsity": round(sparsity, 4),
+                   "l2": "flushed (256 MiB write) before every timed step", "parallelism": f"replicas x{world}"},
+        "stages_ms": {"total": round(ms, 4), "stage0_1_select": round(ms01, 4), "stage2": round(ms2, 4)},
+        "work": {"selected_flops": f2, "selected_kv_bytes": y,
+                 "executed_tile_flops": exec_f, "union_waste": (round(exec_f / f2, 3) if exec_f else None)},
+        "roofline": roof,
+        "e2e": {"value": round(per(ms_e2e), 3), "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(ms_e2e, 4)},
+        "gpu_launches": args.steps * (4 if not decode else 5),
+        "clocks": cs.summary(),
+    }
+    return res, (q, k, v, w, alpha, sigma)
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host cores (CPU baseline / reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(w, alpha, sigma, q, k, v, budget_s=15.0, max_rows=None):
+    """Time the fp64 oracle on a bounded row sample of the workload; returns (rows, seconds, flops, bytes, cores)."""
+    import numpy as np
+
+    import oracle
+
+    cores = os.cpu_count() or 1
+    oracle.set_threads(cores)
+    rng = np.random.default_rng(0)
+    b = 0
+    K = k[b].float().cpu().numpy()
+    V = v[b].float().cpu().numpy()
+    rows = np.arange(w.nq) if w.nq <= 16 else np.sort(rng.choice(np.arange(w.nq), min(w.nq, 64), replace=False))
+    t0 = time.perf_counter()
+    done = []
+    while True:
+        Qr = q[b, torch.from_numpy(rows).to(q.device)].float().cpu().numpy()
+        res = oracle.fwd_rows(Qr, rows, w.nq, K, V, w.block, alpha, sigma=sigma, want=("out", "routed"))
+        done.append((rows, res["routed"]))
+        el = time.perf_counter() - t0
+        if el > budget_s or (max_rows and sum(len(r) for r, _ in done) >= max_rows) or w.nq <= 16:
+            break
+        rows = np.sort(rng.choice(np.arange(w.nq), min(w.nq, 256), replace=False))
+    el = time.perf_counter() - t0
+    f2 = 0.0
+    y = 0.0
+    nrows = 0
+    for rws, routed in done:
+        p = rws + w.nk - w.nq
+        keys = w.block * routed.sum(-1) + (p % w.block + 1)[:, None]  # [rows, hkv]
+        f2 += float(4 * w.d * keys.sum()) * w.g
+        y += float(keys.sum() * w.d * 4)
+        nrows += len(rws)
+    return nrows, el, f2, y, cores
+
+
+def run_reference(args, device):
+    w = synthetic.WORKLOADS[args.workload]
+    alpha = args.alpha or w.alpha
+    q, k, v = synthetic.make_inputs(w, device)
+    decode = w.nq == 1
+    per_step = []
+    flops = byts = 0.0
+    rows = 0
+    cores = os.cpu_count() or 1
+    for s in range(args.warmup + args.steps):
+        n, el, f2, y, cores = oracle_sample(w, alpha, args.sigma, q, k, v, budget_s=args.ref_budget)
+        if s >= args.warmup:
+            per_step.append(el)
+            flops += f2
+            byts += y
+            rows += n
+    secs = sum(per_step)
+    unit = "GB/s" if decode else "TFLOP/s"
+    value = (byts / secs / 1e9) if decode else (flops / secs / 1e12)
+    sample = f"{rows} query rows x all heads of batch 0 over {args.steps} steps (fp64 oracle, dense masked Stage 2)"
+    return {
+        "metric": METRIC, "impl": "reference", "value": value, "unit": unit, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * secs / max(args.steps, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded planted-block generator)",
+        "config": {"workload": w.name, "batch": w.batch, "nq": w.nq, "nk": w.nk, "hq": w.hq, "hkv": w.hkv, "d": w.d,
+                   "block": w.block, "alpha": alpha, "sigma": args.sigma},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="prefill8k", choices=sorted(synthetic.WORKLOADS))
+    ap.add_argument("--alpha", type=float, default=None)
+    ap.add_argument("--sigma", type=float, default=1e8)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-budget", type=float, default=10.0, help="seconds of oracle work per reference step")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.warmup < 3:
+        args.warmup = 3
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        device = "cuda" if torch.cuda.is_available() else "cpu"
+        print(json.dumps(run_reference(args, device)))
+        return 0
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    try:
+        res, (q, k, v, w, alpha, sigma) = run_ours(args, rank, world, device)
+        if rank == 0:
+            if not args.no_cpu_baseline and world == 1:
+                n, el, f2, y, cores = oracle_sample(w, alpha, sigma, q, k, v, budget_s=15.0)
+                decode = res["unit"] == "GB/s"
+                val = (y / el / 1e9) if decode else (f2 / el / 1e12)
+                res["cpu_baseline"] = {"value": val, "unit": res["unit"], "cores": cores, "kind": "oracle",
+                                       "sample": f"{n} query rows x all heads of batch 0, {el:.1f} s "
+                                                 f"(fp64 oracle, dense masked Stage 2)"}
+            print(json.dumps(res))
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -24,6 +24,7 @@
 
 #include "dash_common.cuh"
 #include "kernels.h"
+#include "tma_host.h"
 
 namespace dash {
 
@@ -76,7 +77,11 @@ struct Bars {
     uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *m_full, *m_empty, *s_full, *p_full, *pv_done, *fin;
 };
 
-__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, uint64_t limit_ns, volatile int *abort) {
+// Bounded wait.  Gives up after limit_ns (recording a device error and raising
+// the CTA's abort flag) or, when honor_abort is set, as soon as another role
+// has raised it.  Drain waits (copies or MMAs in flight) pass honor_abort = false.
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, uint64_t limit_ns, volatile int *abort,
+                                         bool honor_abort = true) {
     uint64_t t0 = 0;
     for (uint32_t it = 0;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
@@ -88,7 +93,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, uint64_
                 *abort = 1;
                 return false;
             }
-            if (*abort) return false;
+            if (honor_abort && *abort) return false;
         }
     }
 }
@@ -171,7 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 tma_load_4d(sm + S::kQ + dh * S::kRegion, &tp.tmQ, B.q_full, dh * 64, r * g, (int)(t * T), (int)b);
             const int32_t *ids_g = L.ids + tile_idx * L.cap;
             const float *bias_g = L.bias + tile_idx * (size_t)L.cap * T;
-            int issued = 0;
+            int issued_m = 0, issued_k = 0, issued_v = 0;  // steps whose copies were issued
             for (int j = 0; j < nsteps; ++j) {
                 const int e0 = j * S::kE;
                 const int ne = min(S::kE, count - e0);
@@ -181,29 +186,31 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 for (int e = 0; e < ne; ++e) ids_st[e] = ids_g[e0 + e];
                 mbar_arrive_expect_tx(B.m_full + ms, (uint32_t)(ne * T * 4));
                 bulk_load(bias_s + ms * S::kE * 128, bias_g + (size_t)e0 * T, (uint32_t)(ne * T * 4), B.m_full + ms);
+                issued_m = j + 1;
                 if (!wait_bar(B.k_empty + ks, ((j / kNS) & 1) ^ 1, limit_ns, abort)) break;
                 mbar_arrive_expect_tx(B.k_full + ks, (uint32_t)(ne * S::kDh * BLK * 128));
                 for (int e = 0; e < ne; ++e)
                     for (int dh = 0; dh < S::kDh; ++dh)
                         tma_load_4d(sm + S::kK + (ks * S::kDh + dh) * S::kRegion + e * BLK * 128, &tp.tmK,
                                     B.k_full + ks, dh * 64, r, ids_st[e] * BLK, (int)b);
+                issued_k = j + 1;
                 if (!wait_bar(B.v_empty + ks, ((j / kNS) & 1) ^ 1, limit_ns, abort)) break;
                 mbar_arrive_expect_tx(B.v_full + ks, (uint32_t)(ne * S::kDh * BLK * 128));
                 for (int e = 0; e < ne; ++e)
                     for (int dh = 0; dh < S::kDh; ++dh)
                         tma_load_4d(sm + S::kV + (ks * S::kDh + dh) * S::kRegion + e * BLK * 128, &tp.tmV,
                                     B.v_full + ks, dh * 64, r, ids_st[e] * BLK, (int)b);
-                issued = j + 1;
+                issued_v = j + 1;
             }
             if (*abort) {
                 // drain: every copy issued must land before the CTA's smem goes away
-                for (int j = max(0, issued - kNS); j < issued; ++j) {
-                    wait_bar(B.k_full + j % kNS, (j / kNS) & 1, kWaitNsTest, abort);
-                    wait_bar(B.v_full + j % kNS, (j / kNS) & 1, kWaitNsTest, abort);
-                }
-                for (int j = max(0, issued - kNM); j < issued; ++j)
-                    wait_bar(B.m_full + j % kNM, (j / kNM) & 1, kWaitNsTest, abort);
-                wait_bar(B.q_full, 0, kWaitNsTest, abort);
+                for (int j = max(0, issued_k - kNS); j < issued_k; ++j)
+                    wait_bar(B.k_full + j % kNS, (j / kNS) & 1, kWaitNsTest, abort, false);
+                for (int j = max(0, issued_v - kNS); j < issued_v; ++j)
+                    wait_bar(B.v_full + j % kNS, (j / kNS) & 1, kWaitNsTest, abort, false);
+                for (int j = max(0, issued_m - kNM); j < issued_m; ++j)
+                    wait_bar(B.m_full + j % kNM, (j / kNM) & 1, kWaitNsTest, abort, false);
+                wait_bar(B.q_full, 0, kWaitNsTest, abort, false);
             }
         }
     } else if (warp == 1) {
@@ -249,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             }
             // every MMA this thread issued has completed before TMEM is freed
             mma_commit(B.fin);
-            wait_bar(B.fin, 0, kWaitNsTest * 50, abort);
+            wait_bar(B.fin, 0, kWaitNsTest * 50, abort, false);
         }
     } else {
         // ------------------------------------------------------------- softmax warpgroup
@@ -264,10 +271,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         const float sl2 = rsqrtf((float)D) * 1.4426950408889634f;
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
+        // tcgen05.ld / st are warp-collective: every decision that guards one is
+        // made uniform across the warp (__any_sync / __all_sync).
         for (int j = 0; j < nsteps; ++j) {
             const int ms = j % kNM;
             const int ne = min(S::kE, count - j * S::kE);
-            if (!(ok = wait_bar(B.m_full + ms, (j / kNM) & 1, limit_ns, abort))) break;
+            ok = __all_sync(0xffffffffu, wait_bar(B.m_full + ms, (j / kNM) & 1, limit_ns, abort));
+            if (!ok) break;
             int idv[S::kE];
             float bl2[S::kE];
 #pragma unroll
@@ -276,13 +286,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 bl2[e] = e < ne ? bias_s[ms * S::kE * 128 + e * T + pos] * 1.4426950408889634f : -INFINITY;
             }
             mbar_arrive(B.m_empty + ms);
-            if (!(ok = wait_bar(B.s_full + (j & 1), (j >> 1) & 1, limit_ns, abort))) break;
+            ok = __all_sync(0xffffffffu, wait_bar(B.s_full + (j & 1), (j >> 1) & 1, limit_ns, abort));
+            if (!ok) break;
             tc_fence_after();
+            const uint32_t tSj = tmem + (uint32_t)(j & 1) * 128u;
             float s[kStepKeys];
 #pragma unroll
             for (int c = 0; c < kStepKeys / 32; ++c) {
                 uint32_t u[32];
-                tmem_ld32((tmem + (uint32_t)(j & 1) * 128u) + lane_off + c * 32, u);
+                tmem_ld32(tSj + lane_off + c * 32, u);
                 tmem_wait_ld();
 #pragma unroll
                 for (int x = 0; x < 32; ++x) s[c * 32 + x] = __uint_as_float(u[x]);
@@ -297,31 +309,35 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 s[kc] = v;
                 mx = fmaxf(mx, v);
             }
-            float m_use = m_run;
+            // running maximum: keep it unless the step's maximum exceeds it by more than 2^8
+            float f = 1.f;
+            const bool rescale = mx > -INFINITY && m_run > -INFINITY && mx > m_run + 8.f;
             if (mx > -INFINITY) {
                 if (m_run == -INFINITY) {
-                    m_use = mx;
-                } else if (mx > m_run + 8.f) {
-                    // rescale O and l to the new maximum (O holds every PV up to step j-1)
-                    m_use = mx;
-                    const float f = ex2(m_run - mx);
+                    m_run = mx;  // nothing accumulated for this row yet: O holds zeros
+                } else if (rescale) {
+                    f = ex2(m_run - mx);
                     l_run *= f;
-                    if (j > 0) {
-                        if (!(ok = wait_bar(B.pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, limit_ns, abort))) break;
-                        tc_fence_after();
-#pragma unroll
-                        for (int c = 0; c < D / 32; ++c) {
-                            uint32_t u[32];
-                            tmem_ld32(tO + lane_off + c * 32, u);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int x = 0; x < 32; ++x) u[x] = __float_as_uint(__uint_as_float(u[x]) * f);
-                            tmem_st32(tO + lane_off + c * 32, u);
-                        }
-                    }
+                    m_run = mx;
                 }
-                m_run = m_use;
             }
+            if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+                // O must hold every PV up to step j-1 before it is rescaled
+                ok = __all_sync(0xffffffffu,
+                                wait_bar(B.pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, limit_ns, abort));
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t u[32];
+                    tmem_ld32(tO + lane_off + c * 32, u);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) u[x] = __float_as_uint(__uint_as_float(u[x]) * f);
+                    tmem_st32(tO + lane_off + c * 32, u);
+                }
+            }
+            const float m_use = m_run;
             float psum = 0.f;
 #pragma unroll
             for (int c = 0; c < kStepKeys / 64; ++c) {
@@ -333,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     psum += p0 + p1;
                     u[x] = pack_bf16x2(p0, p1);
                 }
-                tmem_st32((tmem + (uint32_t)(j & 1) * 128u) + lane_off + c * 32, u);
+                tmem_st32(tSj + lane_off + c * 32, u);
             }
             l_run += psum;
             tmem_wait_st();
@@ -342,30 +358,35 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
         // epilogue: O / l -> bf16
         if (ok && !*abort) {
-            bool have = nsteps > 0;
-            if (have) have = wait_bar(B.pv_done + ((nsteps - 1) & 1), ((nsteps - 1) >> 1) & 1, limit_ns, abort);
+            bool have = true;
+            if (nsteps > 0)
+                have = __all_sync(0xffffffffu, wait_bar(B.pv_done + ((nsteps - 1) & 1), ((nsteps - 1) >> 1) & 1,
+                                                        limit_ns, abort));
             tc_fence_after();
-            if (row_ok && (have || nsteps == 0)) {
+            if (have) {
                 __nv_bfloat16 *op = reinterpret_cast<__nv_bfloat16 *>(const_cast<void *>(O.p)) + b * O.s0 +
                                     i * O.s1 + (int64_t)(r * g + hh) * O.s2;
                 const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t u[32];
-                    if (nsteps > 0) {
+                    if (nsteps > 0) {  // uniform across the CTA
                         tmem_ld32(tO + lane_off + c * 32, u);
                         tmem_wait_ld();
                     } else {
 #pragma unroll
                         for (int x = 0; x < 32; ++x) u[x] = 0u;
                     }
-                    uint32_t pk[16];
+                    if (row_ok) {
+                        uint32_t pk[16];
 #pragma unroll
-                    for (int x = 0; x < 16; ++x)
-                        pk[x] = pack_bf16x2(__uint_as_float(u[2 * x]) * inv, __uint_as_float(u[2 * x + 1]) * inv);
-                    uint4 *dst = reinterpret_cast<uint4 *>(op + c * 32);
+                        for (int x = 0; x < 16; ++x)
+                            pk[x] = pack_bf16x2(__uint_as_float(u[2 * x]) * inv, __uint_as_float(u[2 * x + 1]) * inv);
+                        uint4 *dst = reinterpret_cast<uint4 *>(op + c * 32);
 #pragma unroll
-                    for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+                        for (int x = 0; x < 4; ++x)
+                            dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+                    }
                 }
             }
         }
@@ -379,37 +400,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 }
 
 // ------------------------------------------------------------------ host side
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
-// 4-D bf16 map over [b][seq][heads][d] (dims innermost first), box {64, box_h, box_s, 1}, 128-byte swizzle.
-bool make_map(CUtensorMap *m, const TView &v, int64_t b, int64_t seq, int64_t heads, int d, int box_h, int box_s) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)seq, (cuuint64_t)b};
-    cuuint64_t strides[3] = {(cuuint64_t)v.s2 * 2, (cuuint64_t)v.s1 * 2, (cuuint64_t)v.s0 * 2};
-    if (b == 1) strides[2] = (cuuint64_t)seq * v.s1 * 2;  // unused dimension: any valid stride
-    cuuint32_t box[4] = {64, (cuuint32_t)box_h, (cuuint32_t)box_s, 1};
-    cuuint32_t es[4] = {1, 1, 1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(v.p), dims, strides, box, es,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
 
 template <int D, int BLK>
 cudaError_t launch_t(const TcParams &tp, const TView &O, const Geom &G, const ListsView &L, int flags,
@@ -432,16 +422,16 @@ bool attn_tc_supported(const Geom &G, dash_dtype_t dt) {
     if (G.g & (G.g - 1)) return false;  // tile_rows * g must be exactly 128
     if (G.tile_rows * G.g != kRows) return false;
     if (G.nq > 0x7fffffff || G.nk > 0x7fffffff) return false;
-    return encode_fn() != nullptr;
+    return tma_encode_fn() != nullptr;
 }
 
 cudaError_t launch_attn_tc(const TView &Q, const TView &K, const TView &V, const TView &O, const Geom &G,
                            const ListsView &L, int flags, cudaStream_t st) {
     if (G.nq == 0 || G.b == 0) return cudaSuccess;
     TcParams tp;
-    if (!make_map(&tp.tmQ, Q, G.b, G.nq, G.hq, G.d, G.g, G.tile_rows)) return cudaErrorInvalidValue;
-    if (!make_map(&tp.tmK, K, G.b, G.nk, G.hkv, G.d, 1, G.B)) return cudaErrorInvalidValue;
-    if (!make_map(&tp.tmV, V, G.b, G.nk, G.hkv, G.d, 1, G.B)) return cudaErrorInvalidValue;
+    if (!make_map_bf16(&tp.tmQ, Q, G.b, G.nq, G.hq, G.d, G.g, G.tile_rows)) return cudaErrorInvalidValue;
+    if (!make_map_bf16(&tp.tmK, K, G.b, G.nk, G.hkv, G.d, 1, G.B)) return cudaErrorInvalidValue;
+    if (!make_map_bf16(&tp.tmV, V, G.b, G.nk, G.hkv, G.d, 1, G.B)) return cudaErrorInvalidValue;
 #define DASH_TC_CASE(DD, BB) \
     if (G.d == DD && G.B == BB) return launch_t<DD, BB>(tp, O, G, L, flags, st);
     DASH_TC_CASE(128, 64)

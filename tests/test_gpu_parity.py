@@ -104,6 +104,35 @@ def test_uniform_all_chunk_prior_is_dense_attention(dt, causal):
     assert err.max() <= tol[0] and err.mean() <= tol[1], (err.max(), err.mean())
 
 
+DECODE_CASES = [
+    # b, nq, nk, hq, hkv, d, B, alpha, sigma
+    (3, 1, 1000, 8, 2, 128, 64, 1.5, 1.0),     # ragged cache length
+    (2, 2, 3000, 8, 2, 128, 64, 1.5, 1e8),     # two new tokens per sequence
+    (2, 1, 2048, 16, 1, 128, 128, 2.0, 1.0),   # g = 16 fills the 16-row tile, B = 128
+    (2, 1, 1500, 4, 2, 64, 16, 1.25, 1.0),     # d = 64, B = 16
+    (1, 1, 50, 4, 1, 128, 64, 1.5, 1.0),       # cache shorter than one chunk
+]
+
+
+@pytest.mark.parametrize("case", DECODE_CASES, ids=[f"d{i}" for i in range(len(DECODE_CASES))])
+def test_decode_cases(case):
+    b, nq, nk, hq, hkv, d, B, alpha, sigma = case
+    q, k, v = _planted(b, nq, nk, hq, hkv, d, B, "bf16", seed=200 + nk)
+    out = _run(q, k, v, B, alpha, True, sigma=sigma)
+    check_forward(q, k, v, out, B, alpha, True, sigma=sigma, label=f"decode case {case}")
+
+
+def test_decode_with_cached_summaries():
+    """A chunk-summary cache from dash_pool_keys (kept across decode steps) gives the same result."""
+    b, nq, nk, hq, hkv, d, B = 2, 1, 4096, 8, 2, 128, 64
+    q, k, v = _planted(b, nq, nk, hq, hkv, d, B, "bf16", seed=77)
+    kbar = torch.empty(b, nk // B, hkv, d, dtype=torch.float32, device="cuda")
+    dash.dash_pool_keys(k, B, True, kbar)
+    a = _run(q, k, v, B, 1.5, True, sigma=1.0)
+    c = _run(q, k, v, B, 1.5, True, sigma=1.0, kbar=kbar)
+    assert torch.equal(a, c)
+
+
 def test_deterministic():
     q, k, v = _planted(1, 512, 512, 8, 2, 128, 64, "bf16", seed=5)
     a = _run(q, k, v, 64, 1.5, True, sigma=1.0)
