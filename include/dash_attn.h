@@ -68,28 +68,35 @@ typedef struct {
     int64_t stride[4]; /* in elements; stride[3] must be 1 */
 } dash_tensor_t;
 
-/* Stage-2 work lists: for each (batch, kv head, query tile of tile_rows
- * consecutive query rows) the union of the chunks any row of the tile attends
- * (its routed chunks and its diagonal chunk), and a per-row additive bias.
+/* Stage-2 work lists.  The query rows of a (batch, kv head) are grouped into
+ * tiles of tile_rows rows (x gqa_groups heads = 128 rows of the tensor-core
+ * tile).  For each tile the list holds the union of the chunks any of its rows
+ * attends (routed chunks and each row's diagonal chunk), and a per-row bias.
  * Layout (all device memory, caller-owned, contiguous):
  *   count [b][hkv][n_tiles]                    int32   entries in the list
- *   ids   [b][hkv][n_tiles][cap]               int32   chunk ids; diagonal chunks first
+ *   ids   [b][hkv][n_tiles][cap]               int32   chunk ids (any order)
  *   bias  [b][hkv][n_tiles][cap][tile_rows]    float32 bias of that chunk for
- *         that row: (log w_c - mu)/sigma if the row routed it, 0 if it is the
+ *         that tile row: (log w_c - mu)/sigma if the row routed it, 0 if it is the
  *         row's diagonal chunk, -inf if the row does not attend it.
+ *   rows  [b][hkv][n_tiles][tile_rows]         int32   query index of each tile
+ *         row, -1 for an unused row; rows may come in any order (Stage 1 groups
+ *         rows with similar routed sets into the same tile).  NULL means tile t
+ *         holds the consecutive rows t*tile_rows .. t*tile_rows + tile_rows - 1.
  * n_tiles = ceil(nq / tile_rows); cap = ceil(nk / block_size); tile_rows =
- * 128 / gqa_groups (the tensor-core tile is tile_rows positions x gqa_groups
- * heads = 128 rows).  Stage 2 also masks key j > p_i when causal. */
+ * 128 / gqa_groups.  Stage 2 also masks key j > p_i when causal and keys >= nk. */
 typedef struct {
     int32_t *count;
     int32_t *ids;
     float *bias;
+    int32_t *rows;
     int64_t n_tiles;
     int32_t cap;
     int32_t tile_rows;
 } dash_lists_t;
 
 #define DASH_FLAG_FORCE_SIMT 0x1      /* Stage 2 on the CUDA-core path (testing) */
+#define DASH_FLAG_NO_REGROUP 0x2      /* keep consecutive query rows in each tile (no regrouping
+                                         of rows by routed-set size) */
 #define DASH_FLAG_TEST_TIMEOUT 0x100  /* testing only: Stage 2 waits on a barrier nothing
                                          arrives at, gives up after a short bound and
                                          reports DASH_ERR_DEVICE_TIMEOUT */
@@ -148,10 +155,11 @@ DASH_API int dash_sparse_attn_fwd(const dash_tensor_t *q, const dash_tensor_t *k
                                   int gqa_groups, const dash_opts_t *opts);
 
 /* Sizes of the lists buffers for a problem: *count_bytes, *ids_bytes,
- * *bias_bytes (any may be NULL) and the geometry (*n_tiles, *cap, *tile_rows). */
+ * *bias_bytes, *rows_bytes (any may be NULL) and the geometry (*n_tiles, *cap,
+ * *tile_rows).  Returns DASH_OK or DASH_ERR_INVALID_ARG. */
 DASH_API int dash_lists_geometry(int64_t batch, int64_t nq, int64_t nk, int hkv, int block_size, int gqa_groups,
                                  int64_t *n_tiles, int32_t *cap, int32_t *tile_rows, size_t *count_bytes,
-                                 size_t *ids_bytes, size_t *bias_bytes);
+                                 size_t *ids_bytes, size_t *bias_bytes, size_t *rows_bytes);
 
 /* Device workspace dash_attn_fwd_ex needs for a problem (bytes). */
 DASH_API size_t dash_workspace_bytes(int64_t batch, int64_t nq, int64_t nk, int hq, int hkv, int d,

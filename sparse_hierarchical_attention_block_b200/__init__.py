@@ -36,6 +36,7 @@ DASH_F32 = 0
 DASH_BF16 = 1
 
 DASH_FLAG_FORCE_SIMT = 0x1
+DASH_FLAG_NO_REGROUP = 0x2
 DASH_FLAG_TEST_TIMEOUT = 0x100
 
 
@@ -52,7 +53,8 @@ class _Tensor(ctypes.Structure):
 
 class _Lists(ctypes.Structure):
     _fields_ = [("count", ctypes.c_void_p), ("ids", ctypes.c_void_p), ("bias", ctypes.c_void_p),
-                ("n_tiles", ctypes.c_int64), ("cap", ctypes.c_int32), ("tile_rows", ctypes.c_int32)]
+                ("rows", ctypes.c_void_p), ("n_tiles", ctypes.c_int64), ("cap", ctypes.c_int32),
+                ("tile_rows", ctypes.c_int32)]
 
 
 class _Opts(ctypes.Structure):
@@ -89,7 +91,7 @@ def load_library():
     lib.dash_sparse_attn_fwd.argtypes = [T, T, T, T, ctypes.POINTER(_Lists), i32, i32, i32, ctypes.POINTER(_Opts)]
     lib.dash_lists_geometry.argtypes = [i64, i64, i64, i32, i32, i32, ctypes.POINTER(i64), ctypes.POINTER(ctypes.c_int32),
                                         ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(sz), ctypes.POINTER(sz),
-                                        ctypes.POINTER(sz)]
+                                        ctypes.POINTER(sz), ctypes.POINTER(sz)]
     lib.dash_workspace_bytes.argtypes = [i64, i64, i64, i32, i32, i32, i32, i32]
     lib.dash_workspace_bytes.restype = sz
     lib.dash_last_error.restype = ctypes.c_char_p
@@ -157,29 +159,36 @@ def lists_geometry(batch, nq, nk, hkv, block_size, gqa_groups):
     """(n_tiles, cap, tile_rows) of the Stage-2 work lists."""
     nt, cap, tr = ctypes.c_int64(), ctypes.c_int32(), ctypes.c_int32()
     _check(load_library().dash_lists_geometry(batch, nq, nk, hkv, block_size, gqa_groups, ctypes.byref(nt),
-                                              ctypes.byref(cap), ctypes.byref(tr), None, None, None))
+                                              ctypes.byref(cap), ctypes.byref(tr), None, None, None, None))
     return nt.value, cap.value, tr.value
 
 
 class Lists:
-    """Device buffers of the Stage-2 work lists (see dash_lists_t)."""
+    """Device buffers of the Stage-2 work lists (see dash_lists_t).
 
-    def __init__(self, batch, nq, nk, hkv, block_size, gqa_groups, device="cuda"):
+    with_rows: allocate the row-permutation buffer, so that Stage 1 may regroup
+    rows across tiles; without it every tile holds consecutive query rows."""
+
+    def __init__(self, batch, nq, nk, hkv, block_size, gqa_groups, device="cuda", with_rows=True):
         self.n_tiles, self.cap, self.tile_rows = lists_geometry(batch, nq, nk, hkv, block_size, gqa_groups)
         self.count = torch.zeros(batch, hkv, self.n_tiles, dtype=torch.int32, device=device)
         self.ids = torch.zeros(batch, hkv, self.n_tiles, self.cap, dtype=torch.int32, device=device)
         self.bias = torch.zeros(batch, hkv, self.n_tiles, self.cap, self.tile_rows, dtype=torch.float32,
                                 device=device)
+        self.rows = (torch.full((batch, hkv, self.n_tiles, self.tile_rows), -1, dtype=torch.int32, device=device)
+                     if with_rows else None)
 
     def c(self) -> _Lists:
         l = _Lists()
         l.count, l.ids, l.bias = self.count.data_ptr(), self.ids.data_ptr(), self.bias.data_ptr()
+        l.rows = self.rows.data_ptr() if self.rows is not None else None
         l.n_tiles, l.cap, l.tile_rows = self.n_tiles, self.cap, self.tile_rows
         return l
 
 
-def make_lists(q, k, block_size, gqa_groups) -> Lists:
-    return Lists(q.shape[0], q.shape[1], k.shape[1], k.shape[2], block_size, gqa_groups, device=q.device)
+def make_lists(q, k, block_size, gqa_groups, with_rows=True) -> Lists:
+    return Lists(q.shape[0], q.shape[1], k.shape[1], k.shape[2], block_size, gqa_groups, device=q.device,
+                 with_rows=with_rows)
 
 
 def dash_attn_fwd(q, k, v, out, block_size, alpha, causal=True, gqa_groups=None, **opts):

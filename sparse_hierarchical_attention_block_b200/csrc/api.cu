@@ -14,6 +14,7 @@
 namespace dash {
 int take_device_error_tc();
 int take_device_error_decode();
+int take_device_error_select();
 }  // namespace dash
 
 using namespace dash;
@@ -108,7 +109,7 @@ int check_opts(const dash_opts_t &o) {
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct WsLayout {
-    size_t kbar, mask, dvals, count, ids, bias, decode, total;
+    size_t kbar, mask, dvals, count, ids, bias, rows, decode, split, total;
 };
 
 WsLayout ws_layout(const Geom &G, bool need_kbar, bool need_lists, bool need_decode) {
@@ -125,7 +126,9 @@ WsLayout ws_layout(const Geom &G, bool need_kbar, bool need_lists, bool need_dec
     L.count = need_lists ? take((size_t)G.b * G.hkv * G.n_tiles * 4) : 0;
     L.ids = need_lists ? take((size_t)G.b * G.hkv * G.n_tiles * G.n_blk * 4) : 0;
     L.bias = need_lists ? take((size_t)G.b * G.hkv * G.n_tiles * G.n_blk * G.tile_rows * 4) : 0;
+    L.rows = need_lists ? take((size_t)G.b * G.hkv * G.n_tiles * G.tile_rows * 4) : 0;
     L.decode = need_decode ? take(attn_decode_workspace(G)) : 0;
+    L.split = select_tile_supported(G, DASH_BF16) ? take(select_tile_workspace(G)) : 0;
     L.total = off;
     return L;
 }
@@ -179,7 +182,46 @@ int check_lists(const dash_lists_t *l, const Geom &G) {
 }
 
 ListsView lists_view(const dash_lists_t *l) {
-    return ListsView{l->count, l->ids, l->bias, l->n_tiles, l->cap, l->tile_rows};
+    return ListsView{l->count, l->ids, l->bias, l->rows, l->n_tiles, l->cap, l->tile_rows};
+}
+
+ListsView ws_lists(const Geom &G, char *ws, const WsLayout &WL, bool with_rows) {
+    return ListsView{reinterpret_cast<int32_t *>(ws + WL.count), reinterpret_cast<int32_t *>(ws + WL.ids),
+                     reinterpret_cast<float *>(ws + WL.bias),
+                     with_rows ? reinterpret_cast<int32_t *>(ws + WL.rows) : nullptr, G.n_tiles, G.n_blk,
+                     G.tile_rows};
+}
+
+// Stage 1 (after Stage 0): routing of every (row, head) and, when LV is given, the
+// Stage-2 work lists.  With regroup (LV->rows required) the rows of each window of
+// tiles are regrouped by routed-set size; otherwise tile t holds consecutive rows
+// (and LV->rows, if given, is filled accordingly).
+int run_stage1(const dash_tensor_t *q, const Geom &G, float alpha, const dash_opts_t &o, const float *kbar,
+               float *tau, float *w, uint32_t *mask_out, const ListsView *LV, bool regroup, char *ws,
+               const WsLayout &WL, cudaStream_t st) {
+    cudaError_t e;
+    const bool tile = select_tile_supported(G, q->dtype);
+    regroup = regroup && LV && LV->rows;
+    uint32_t *mask = mask_out ? mask_out : reinterpret_cast<uint32_t *>(ws + WL.mask);
+    float *dv = LV ? reinterpret_cast<float *>(ws + WL.dvals) : nullptr;
+    if (tile && LV && !regroup) {
+        e = launch_select_tile(view(q), kbar, G, alpha, o.gamma, o.sigma, tau, w, mask_out, nullptr, *LV,
+                               ws + WL.split, st);
+        return e == cudaSuccess ? DASH_OK : cuda_fail(e, "select_tile");
+    }
+    if (tile) {
+        const ListsView geom_only{nullptr, nullptr, nullptr, nullptr, G.n_tiles, G.n_blk, G.tile_rows};
+        e = launch_select_tile(view(q), kbar, G, alpha, o.gamma, o.sigma, tau, w, mask, dv, geom_only,
+                               ws + WL.split, st);
+        if (e != cudaSuccess) return cuda_fail(e, "select_tile");
+    } else {
+        SelectOut so{tau, w, mask, dv};
+        e = launch_select_rows(view(q), q->dtype, kbar, G, alpha, o.gamma, o.sigma, so, st);
+        if (e != cudaSuccess) return cuda_fail(e, "select_rows");
+    }
+    if (!LV) return DASH_OK;
+    e = regroup ? launch_regroup_compact(G, mask, dv, *LV, st) : launch_compact(G, mask, dv, *LV, st);
+    return e == cudaSuccess ? DASH_OK : cuda_fail(e, "work-list compaction");
 }
 
 int run_stage2(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v, dash_tensor_t *out,
@@ -231,7 +273,7 @@ DASH_API int dash_opts_init(dash_opts_t *opts) {
 
 DASH_API int dash_lists_geometry(int64_t batch, int64_t nq, int64_t nk, int hkv, int block_size, int gqa_groups,
                                  int64_t *n_tiles, int32_t *cap, int32_t *tile_rows, size_t *count_bytes,
-                                 size_t *ids_bytes, size_t *bias_bytes) {
+                                 size_t *ids_bytes, size_t *bias_bytes, size_t *rows_bytes) {
     if (batch < 0 || nq < 0 || nk <= 0 || hkv <= 0 || block_size <= 0 || gqa_groups < 1 || gqa_groups > 16)
         return fail(DASH_ERR_INVALID_ARG, "bad lists geometry arguments");
     const int64_t tr = 128 / gqa_groups;
@@ -243,6 +285,7 @@ DASH_API int dash_lists_geometry(int64_t batch, int64_t nq, int64_t nk, int hkv,
     if (count_bytes) *count_bytes = (size_t)batch * hkv * nt * 4;
     if (ids_bytes) *ids_bytes = (size_t)batch * hkv * nt * cp * 4;
     if (bias_bytes) *bias_bytes = (size_t)batch * hkv * nt * cp * tr * 4;
+    if (rows_bytes) *rows_bytes = (size_t)batch * hkv * nt * tr * 4;
     return DASH_OK;
 }
 
@@ -298,26 +341,21 @@ DASH_API int dash_block_select(const dash_tensor_t *q, const dash_tensor_t *k, i
         if (reinterpret_cast<uintptr_t>(p) % 16) return fail(DASH_ERR_ALIGNMENT, "outputs must be 16-byte aligned");
     if (G.b == 0 || G.nq == 0) return DASH_OK;
     const bool need_kbar = o.kbar == nullptr;
-    WsLayout WL = ws_layout(G, need_kbar, lists != nullptr, false);
+    WsLayout WL = ws_layout(G, need_kbar, true, false);
     char *ws = nullptr;
     if ((rc = get_workspace(o, WL.total, &ws))) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(o.stream);
     const float *kbar = o.kbar;
-    cudaError_t e;
     if (need_kbar) {
         float *kb = reinterpret_cast<float *>(ws + WL.kbar);
-        if ((e = launch_pool_keys(view(k), k->dtype, G, kb, st)) != cudaSuccess) return cuda_fail(e, "pool_keys");
+        cudaError_t e = launch_pool_keys(view(k), k->dtype, G, kb, st);
+        if (e != cudaSuccess) return cuda_fail(e, "pool_keys");
         kbar = kb;
     }
-    SelectOut so{tau, w, mask ? mask : reinterpret_cast<uint32_t *>(ws + WL.mask),
-                 lists ? reinterpret_cast<float *>(ws + WL.dvals) : nullptr};
-    if ((e = launch_select_rows(view(q), q->dtype, kbar, G, alpha, o.gamma, o.sigma, so, st)) != cudaSuccess)
-        return cuda_fail(e, "select_rows");
-    if (lists) {
-        if ((e = launch_compact(G, so.mask, so.dvals, lists_view(lists), st)) != cudaSuccess)
-            return cuda_fail(e, "compact");
-    }
-    return DASH_OK;
+    ListsView LV;
+    if (lists) LV = lists_view(lists);
+    const bool regroup = lists && lists->rows && !(o.flags & DASH_FLAG_NO_REGROUP) && G.n_tiles > 1;
+    return run_stage1(q, G, alpha, o, kbar, tau, w, mask, lists ? &LV : nullptr, regroup, ws, WL, st);
 }
 
 DASH_API int dash_sparse_attn_fwd(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v,
@@ -363,12 +401,9 @@ DASH_API int dash_attn_fwd_ex(const dash_tensor_t *q, const dash_tensor_t *k, co
         if ((e = launch_pool_keys(view(k), k->dtype, G, kb, st)) != cudaSuccess) return cuda_fail(e, "pool_keys");
         kbar = kb;
     }
-    SelectOut so{nullptr, nullptr, reinterpret_cast<uint32_t *>(ws + WL.mask), reinterpret_cast<float *>(ws + WL.dvals)};
-    if ((e = launch_select_rows(view(q), q->dtype, kbar, G, alpha, o.gamma, o.sigma, so, st)) != cudaSuccess)
-        return cuda_fail(e, "select_rows");
-    ListsView LV{reinterpret_cast<int32_t *>(ws + WL.count), reinterpret_cast<int32_t *>(ws + WL.ids),
-                 reinterpret_cast<float *>(ws + WL.bias), G.n_tiles, G.n_blk, G.tile_rows};
-    if ((e = launch_compact(G, so.mask, so.dvals, LV, st)) != cudaSuccess) return cuda_fail(e, "compact");
+    const bool regroup = !(o.flags & DASH_FLAG_NO_REGROUP) && G.n_tiles > 1;
+    const ListsView LV = ws_lists(G, ws, WL, regroup);
+    if ((rc = run_stage1(q, G, alpha, o, kbar, nullptr, nullptr, nullptr, &LV, regroup, ws, WL, st))) return rc;
     return run_stage2(q, k, v, out, G, LV, o, dec ? ws + WL.decode : nullptr, st);
 }
 
@@ -380,7 +415,7 @@ DASH_API int dash_attn_fwd(const dash_tensor_t *q, const dash_tensor_t *k, const
 DASH_API int dash_sync_status(void *stream) {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
-    int dev_err = take_device_error_tc() | take_device_error_decode();
+    int dev_err = take_device_error_tc() | take_device_error_decode() | take_device_error_select();
     if (dev_err) return fail(DASH_ERR_DEVICE_TIMEOUT, "a device-side bounded wait ran out");
     return DASH_OK;
 }

@@ -149,7 +149,7 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(const __grid_c
     {
         const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(Q.p) + b * Q.s0;
         auto qrow = [&](int m) -> const __nv_bfloat16 * {
-            return qb + (int64_t)(m / g) * Q.s1 + (int64_t)(r * g + m % g) * Q.s2;
+            return qb + tile_row(L, G, tile_idx, 0, m / g) * Q.s1 + (int64_t)(r * g + m % g) * Q.s2;
         };
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -162,8 +162,8 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(const __grid_c
         }
     }
     const int row0 = gr, row1 = gr + 8;
-    const int64_t p0 = row0 < M ? row_pos(G, row0 / g) : -1;
-    const int64_t p1 = row1 < M ? row_pos(G, row1 / g) : -1;
+    const int64_t p0 = row0 < M ? row_pos(G, tile_row(L, G, tile_idx, 0, row0 / g)) : -1;
+    const int64_t p1 = row1 < M ? row_pos(G, tile_row(L, G, tile_idx, 0, row1 / g)) : -1;
     const float sl2 = rsqrtf((float)D) * 1.4426950408889634f;
 
     float o[D / 8][4];
@@ -336,7 +336,8 @@ __global__ void __launch_bounds__(128) combine_kernel(TView O, Geom G, ListsView
             num += f * p[2 + col];
         }
         __nv_bfloat16 *op = reinterpret_cast<__nv_bfloat16 *>(const_cast<void *>(O.p)) + b * O.s0 +
-                            (int64_t)(row / g) * O.s1 + (int64_t)(r * g + row % g) * O.s2;
+                            tile_row(L, G, ((size_t)b * G.hkv + r) * L.n_tiles, 0, row / g) * O.s1 +
+                            (int64_t)(r * g + row % g) * O.s2;
         op[col] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
     }
 }

@@ -39,8 +39,9 @@ __global__ void __launch_bounds__(kSimtRows) attn_simt_kernel(TView Q, TView K, 
     const int M = TR * g;
     const int m = threadIdx.x;
     const int pos = m / g, hh = m % g;
-    const int64_t i = t * TR + pos;
-    const bool valid = (m < M) && (i < G.nq);
+    const size_t tile_idx = ((size_t)b * G.hkv + r) * L.n_tiles + t;
+    const int64_t i = m < M ? tile_row(L, G, tile_idx, t, pos) : -1;
+    const bool valid = i >= 0;
     const int64_t p_i = row_pos(G, i);
 
     const T *qb = reinterpret_cast<const T *>(Q.p) + b * Q.s0;
@@ -54,7 +55,6 @@ __global__ void __launch_bounds__(kSimtRows) attn_simt_kernel(TView Q, TView K, 
     const float sl2 = rsqrtf((float)d) * 1.4426950408889634f;  // 1/sqrt(d) * log2(e)
     float mrun = -INFINITY, lrun = 0.f;
 
-    const size_t tile_idx = ((size_t)b * G.hkv + r) * L.n_tiles + t;
     const int count = L.count[tile_idx];
     const int32_t *ids = L.ids + tile_idx * L.cap;
     const float *bias = L.bias + tile_idx * (size_t)L.cap * TR;

@@ -8,16 +8,19 @@
 // causal.  Online softmax in the exp2 domain with fp32 statistics.
 //
 // One CTA per (batch, kv head, query tile of 128/g positions x g heads = 128 rows),
-// the heaviest tiles (latest, causal) first.  Warp roles (192 threads):
+// the heaviest tiles (latest, causal) first, two CTAs resident per SM so that one
+// CTA's MMAs overlap the other's softmax.  Warp roles (192 threads):
 //   warp 0     TMA producer: Q tile once; per step of 128 keys the listed K and V
 //              blocks (one TMA box per chunk and 64-column half, 128-byte swizzle)
-//              and the step's bias rows (bulk copy) into a ring of stages;
-//   warp 1     TMEM allocator and MMA issuer (one thread):
-//              S_j = Q K_j^T  (SS, M=128 N=128 K=d) into one of two TMEM S buffers,
+//              and the step's bias rows (bulk copy);
+//   warp 1     TMEM allocator (256 columns: S/P and O) and MMA issuer (one thread):
+//              S_j = Q K_j^T  (SS, M=128 N=128 K=d) into TMEM,
 //              O  += P_j V_j  (TS: P read from TMEM, V from smem as an MN-major operand);
-//   warps 2-5  softmax: thread = TMEM lane = tile row; reads S_j, adds bias, masks,
-//              online max/sum, writes P_j (bf16) over S_j in TMEM, rescales O only
-//              when the running max grows by more than 2^8; epilogue O / l -> bf16.
+//   warps 2-5  softmax: thread = TMEM lane = tile row; two passes over S_j in TMEM
+//              (row max, then exp2 / sum / bf16 P written over S_j), bias added and
+//              keys masked only on steps that hold a diagonal or partial chunk; O is
+//              rescaled only when the running max grows by more than 2^8; epilogue
+//              O / l -> bf16.
 // Every mbarrier wait is bounded (globaltimer); on expiry the kernel records a
 // device error, drains what it issued, frees TMEM and returns.
 #include <math.h>
@@ -31,11 +34,11 @@ namespace dash {
 namespace {
 
 constexpr int kThreads = 192;
-constexpr int kRows = 128;    // MMA M
+constexpr int kRows = 128;      // MMA M
 constexpr int kStepKeys = 128;  // keys per step = MMA N of S and K of PV
-constexpr int kNS = 2;        // K / V stages
-constexpr int kNM = 4;        // bias / id stages
-constexpr uint32_t kTmemCols = 512;
+constexpr int kNS = 1;          // K / V stages (two CTAs per SM share the SM's shared memory)
+constexpr int kNM = 2;          // bias / id stages
+constexpr uint32_t kTmemCols = 256;
 constexpr uint64_t kWaitNs = 2000000000ull;      // 2 s
 constexpr uint64_t kWaitNsTest = 20000000ull;    // 20 ms under DASH_FLAG_TEST_TIMEOUT
 
@@ -63,14 +66,14 @@ struct Smem {
     static constexpr int kQ = 0;
     static constexpr int kK = kQ + kDh * kRegion;
     static constexpr int kV = kK + kNS * kDh * kRegion;
-    static constexpr int kBias = kV + kNS * kDh * kRegion;       // [kNM][kE * 128] floats (tile_rows <= 128)
+    static constexpr int kBias = kV + kNS * kDh * kRegion;      // [kNM][kE * 128] floats (tile_rows <= 128)
     static constexpr int kIds = kBias + kNM * kE * 128 * 4;     // [kNM][kE] int
     static constexpr int kBars = (kIds + kNM * kE * 4 + 7) & ~7;
     // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], m_full[NM], m_empty[NM],
-    //           s_full[2], p_full[2], pv_done[2], fin
-    static constexpr int kNumBars = 1 + 4 * kNS + 2 * kNM + 6 + 1;
-    static constexpr int kMisc = kBars + kNumBars * 8;          // tmem base, abort flag
-    static constexpr int kTotal = kMisc + 16;
+    //           s_full, p_full, pv_done, fin
+    static constexpr int kNumBars = 1 + 4 * kNS + 2 * kNM + 3 + 1;
+    static constexpr int kMisc = kBars + kNumBars * 8;          // tmem base, abort flag, p_min
+    static constexpr int kTotal = kMisc + 16 + 8;
 };
 
 struct Bars {
@@ -99,8 +102,8 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, uint64_
 }
 
 template <int D, int BLK>
-__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ TcParams tp, TView O, Geom G,
-                                                              ListsView L, int flags) {
+__global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_constant__ TcParams tp, TView Qv, TView O,
+                                                              Geom G, ListsView L, int flags) {
     using S = Smem<D, BLK>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -126,16 +129,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     B.m_full = B.v_empty + kNS;
     B.m_empty = B.m_full + kNM;
     B.s_full = B.m_empty + kNM;
-    B.p_full = B.s_full + 2;
-    B.pv_done = B.p_full + 2;
-    B.fin = B.pv_done + 2;
+    B.p_full = B.s_full + 1;
+    B.pv_done = B.p_full + 1;
+    B.fin = B.pv_done + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + S::kMisc);
     volatile int *abort = reinterpret_cast<volatile int *>(sm + S::kMisc + 4);
+    long long *p_min_s = reinterpret_cast<long long *>(sm + S::kMisc + 8);
     float *bias_s = reinterpret_cast<float *>(sm + S::kBias);
     int *ids_s = reinterpret_cast<int *>(sm + S::kIds);
 
+    const bool gather_q = L.rows != nullptr;  // rows regrouped: Q rows are gathered by the softmax threads
     if (threadIdx.x == 0) {
-        mbar_init(B.q_full, 1);
+        mbar_init(B.q_full, gather_q ? 128 : 1);
+        *p_min_s = 0x7fffffffffffffffll;
         for (int s = 0; s < kNS; ++s) {
             mbar_init(B.k_full + s, 1);
             mbar_init(B.k_empty + s, 1);
@@ -146,11 +152,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             mbar_init(B.m_full + s, 1);
             mbar_init(B.m_empty + s, 128);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(B.s_full + s, 1);
-            mbar_init(B.p_full + s, 128);
-            mbar_init(B.pv_done + s, 1);
-        }
+        mbar_init(B.s_full, 1);
+        mbar_init(B.p_full, 128);
+        mbar_init(B.pv_done, 1);
         mbar_init(B.fin, 1);
         *abort = 0;
         fence_mbar_init();
@@ -163,17 +167,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tO = tmem + 256;  // O accumulator; S / P buffers at tmem + 0 and tmem + 128
+    const uint32_t tS = tmem;        // S_j, then P_j (bf16) over its first 64 columns
+    const uint32_t tO = tmem + 128;  // O accumulator (D columns)
 
     if (warp == 0) {
         // ------------------------------------------------------------- producer
         if (lane == 0 && !test_timeout && nsteps > 0) {
-            tma_prefetch_desc(&tp.tmQ);
             tma_prefetch_desc(&tp.tmK);
             tma_prefetch_desc(&tp.tmV);
-            mbar_arrive_expect_tx(B.q_full, kRows * D * 2);
-            for (int dh = 0; dh < S::kDh; ++dh)
-                tma_load_4d(sm + S::kQ + dh * S::kRegion, &tp.tmQ, B.q_full, dh * 64, r * g, (int)(t * T), (int)b);
+            if (!gather_q) {
+                mbar_arrive_expect_tx(B.q_full, kRows * D * 2);
+                for (int dh = 0; dh < S::kDh; ++dh)
+                    tma_load_4d(sm + S::kQ + dh * S::kRegion, &tp.tmQ, B.q_full, dh * 64, r * g, (int)(t * T),
+                                (int)b);
+            }
             const int32_t *ids_g = L.ids + tile_idx * L.cap;
             const float *bias_g = L.bias + tile_idx * (size_t)L.cap * T;
             int issued_m = 0, issued_k = 0, issued_v = 0;  // steps whose copies were issued
@@ -210,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     wait_bar(B.v_full + j % kNS, (j / kNS) & 1, kWaitNsTest, abort, false);
                 for (int j = max(0, issued_m - kNM); j < issued_m; ++j)
                     wait_bar(B.m_full + j % kNM, (j / kNM) & 1, kWaitNsTest, abort, false);
-                wait_bar(B.q_full, 0, kWaitNsTest, abort, false);
+                if (!gather_q) wait_bar(B.q_full, 0, kWaitNsTest, abort, false);
             }
         }
     } else if (warp == 1) {
@@ -222,37 +229,31 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const uint32_t k_base = smem_u32(sm + S::kK);
             const uint32_t v_base = smem_u32(sm + S::kV);
             bool ok = nsteps == 0 || wait_bar(B.q_full, 0, limit_ns, abort);
-            for (int j = 0; ok && j <= nsteps; ++j) {
-                if (j < nsteps) {
-                    const int ks = j % kNS;
-                    if (!(ok = wait_bar(B.k_full + ks, (j / kNS) & 1, limit_ns, abort))) break;
-                    if (j >= 2 && !(ok = wait_bar(B.pv_done + (j & 1), ((j - 2) >> 1) & 1, limit_ns, abort))) break;
-                    tc_fence_after();
+            for (int j = 0; ok && j < nsteps; ++j) {
+                const int ks = j % kNS;
+                const int ne = min(S::kE, count - j * S::kE);
+                if (!(ok = wait_bar(B.k_full + ks, (j / kNS) & 1, limit_ns, abort))) break;
+                // the S / P buffer is free once PV_{j-1} has read P_{j-1}
+                if (j > 0 && !(ok = wait_bar(B.pv_done, (j - 1) & 1, limit_ns, abort))) break;
+                tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t qa = q_base + (kk / 4) * S::kRegion + (kk % 4) * 32;
-                        const uint32_t kb = k_base + (ks * S::kDh + kk / 4) * S::kRegion + (kk % 4) * 32;
-                        mma_ss((tmem + (uint32_t)(j & 1) * 128u), smem_desc_sw128(qa, 16, 1024), smem_desc_sw128(kb, 16, 1024), idS,
-                               kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(B.s_full + (j & 1));
-                    mma_commit(B.k_empty + ks);
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t qa = q_base + (kk / 4) * S::kRegion + (kk % 4) * 32;
+                    const uint32_t kb = k_base + (ks * S::kDh + kk / 4) * S::kRegion + (kk % 4) * 32;
+                    mma_ss(tS, smem_desc_sw128(qa, 16, 1024), smem_desc_sw128(kb, 16, 1024), idS, kk > 0 ? 1u : 0u);
                 }
-                if (j >= 1) {
-                    const int jj = j - 1, vs = jj % kNS;
-                    const int ne = min(S::kE, count - jj * S::kE);
-                    if (!(ok = wait_bar(B.p_full + (jj & 1), (jj >> 1) & 1, limit_ns, abort))) break;
-                    if (!(ok = wait_bar(B.v_full + vs, (jj / kNS) & 1, limit_ns, abort))) break;
-                    tc_fence_after();
-                    const int nks = ne * BLK / 16;
-                    for (int kk = 0; kk < nks; ++kk) {
-                        const uint32_t vb = v_base + (vs * S::kDh) * S::kRegion + kk * 2048;
-                        mma_ts(tO, (tmem + (uint32_t)(jj & 1) * 128u) + kk * 8, smem_desc_sw128(vb, S::kRegion, 1024), idPV,
-                               (jj > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    mma_commit(B.v_empty + vs);
-                    mma_commit(B.pv_done + (jj & 1));
+                mma_commit(B.s_full);
+                mma_commit(B.k_empty + ks);
+                if (!(ok = wait_bar(B.p_full, j & 1, limit_ns, abort))) break;
+                if (!(ok = wait_bar(B.v_full + ks, (j / kNS) & 1, limit_ns, abort))) break;
+                tc_fence_after();
+                const int nks = ne * BLK / 16;
+                for (int kk = 0; kk < nks; ++kk) {
+                    const uint32_t vb = v_base + (ks * S::kDh) * S::kRegion + kk * 2048;
+                    mma_ts(tO, tS + kk * 8, smem_desc_sw128(vb, S::kRegion, 1024), idPV, (j > 0 || kk > 0) ? 1u : 0u);
                 }
+                mma_commit(B.v_empty + ks);
+                mma_commit(B.pv_done);
             }
             // every MMA this thread issued has completed before TMEM is freed
             mma_commit(B.fin);
@@ -265,9 +266,26 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const int pos = m / g;
         const int hh = m % g;
-        const int64_t i = t * T + pos;
-        const bool row_ok = i < G.nq;
+        const int64_t i = tile_row(L, G, tile_idx, t, pos);
+        const bool row_ok = i >= 0;
         const int64_t p_row = row_pos(G, i);
+        if (gather_q && nsteps > 0) {
+            // this thread's Q row into the 128-byte-swizzled K-major layout the MMA reads
+            const __nv_bfloat16 *src = reinterpret_cast<const __nv_bfloat16 *>(Qv.p) + b * Qv.s0 +
+                                       (row_ok ? i : 0) * Qv.s1 + (int64_t)(r * g + hh) * Qv.s2;
+#pragma unroll
+            for (int cc = 0; cc < D / 8; ++cc) {
+                const uint4 val = row_ok ? *reinterpret_cast<const uint4 *>(src + cc * 8) : make_uint4(0u, 0u, 0u, 0u);
+                *reinterpret_cast<uint4 *>(sm + S::kQ + (cc / 8) * S::kRegion + m * 128 + (((cc % 8) ^ (m & 7)) << 4)) =
+                    val;
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(B.q_full);
+        }
+        // keys of a chunk up to the smallest row position are visible to every row of the tile
+        if (row_ok) atomicMin(p_min_s, (long long)p_row);
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        const int64_t p_min = *p_min_s;
         const float sl2 = rsqrtf((float)D) * 1.4426950408889634f;
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
@@ -278,38 +296,50 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const int ne = min(S::kE, count - j * S::kE);
             ok = __all_sync(0xffffffffu, wait_bar(B.m_full + ms, (j / kNM) & 1, limit_ns, abort));
             if (!ok) break;
-            int idv[S::kE];
+            // per-entry constants of this step: bias (exp2 domain) and, for masking, the
+            // number of leading keys of the entry this row may see
             float bl2[S::kE];
+            int lim[S::kE];
+            bool need_mask = ne < S::kE;
+            const int vis_end = (int)((G.causal && row_ok) ? min((int64_t)G.nk, p_row + 1) : G.nk);
 #pragma unroll
             for (int e = 0; e < S::kE; ++e) {
-                idv[e] = e < ne ? ids_s[ms * S::kE + e] : -1;
+                const int id = e < ne ? ids_s[ms * S::kE + e] : 0;
                 bl2[e] = e < ne ? bias_s[ms * S::kE * 128 + e * T + pos] * 1.4426950408889634f : -INFINITY;
+                lim[e] = e < ne ? max(0, min(BLK, vis_end - id * BLK)) : 0;
+                // a chunk needs per-key masks if it reaches past the sequence or past the
+                // smallest row position of the tile (it is some row's diagonal chunk)
+                if (e < ne) {
+                    const int64_t last_key = (int64_t)id * BLK + BLK - 1;
+                    need_mask |= last_key >= G.nk || (G.causal && last_key > p_min);
+                }
             }
             mbar_arrive(B.m_empty + ms);
-            ok = __all_sync(0xffffffffu, wait_bar(B.s_full + (j & 1), (j >> 1) & 1, limit_ns, abort));
+            ok = __all_sync(0xffffffffu, wait_bar(B.s_full, j & 1, limit_ns, abort));
             if (!ok) break;
             tc_fence_after();
-            const uint32_t tSj = tmem + (uint32_t)(j & 1) * 128u;
-            float s[kStepKeys];
-#pragma unroll
-            for (int c = 0; c < kStepKeys / 32; ++c) {
-                uint32_t u[32];
-                tmem_ld32(tSj + lane_off + c * 32, u);
-                tmem_wait_ld();
-#pragma unroll
-                for (int x = 0; x < 32; ++x) s[c * 32 + x] = __uint_as_float(u[x]);
-            }
+            // pass 1: row maximum of the biased, masked logits (exp2 domain)
             float mx = -INFINITY;
 #pragma unroll
-            for (int kc = 0; kc < kStepKeys; ++kc) {
-                const int e = kc / BLK;
-                const int64_t key = (int64_t)idv[e] * BLK + (kc % BLK);
-                const bool vis = idv[e] >= 0 && key < G.nk && !(G.causal && key > p_row) && row_ok;
-                const float v = vis ? fmaf(s[kc], sl2, bl2[e]) : -INFINITY;
-                s[kc] = v;
-                mx = fmaxf(mx, v);
+            for (int half = 0; half < 2; ++half) {
+                uint32_t u[64];
+                tmem_ld32(tS + lane_off + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+                tmem_ld32(tS + lane_off + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+                tmem_wait_ld();
+                if (!need_mask) {
+#pragma unroll
+                    for (int x = 0; x < 64; ++x) mx = fmaxf(mx, fmaf(__uint_as_float(u[x]), sl2, bl2[(half * 64 + x) / BLK]));
+                } else {
+#pragma unroll
+                    for (int x = 0; x < 64; ++x) {
+                        const int kc = half * 64 + x;
+                        const float v = fmaf(__uint_as_float(u[x]), sl2, bl2[kc / BLK]);
+                        mx = fmaxf(mx, (kc % BLK) < lim[kc / BLK] ? v : -INFINITY);
+                    }
+                }
             }
-            // running maximum: keep it unless the step's maximum exceeds it by more than 2^8
+            if (!row_ok) mx = -INFINITY;
+            // running maximum: kept unless the step's maximum exceeds it by more than 2^8
             float f = 1.f;
             const bool rescale = mx > -INFINITY && m_run > -INFINITY && mx > m_run + 8.f;
             if (mx > -INFINITY) {
@@ -323,8 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             }
             if (j > 0 && __any_sync(0xffffffffu, rescale)) {
                 // O must hold every PV up to step j-1 before it is rescaled
-                ok = __all_sync(0xffffffffu,
-                                wait_bar(B.pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, limit_ns, abort));
+                ok = __all_sync(0xffffffffu, wait_bar(B.pv_done, (j - 1) & 1, limit_ns, abort));
                 if (!ok) break;
                 tc_fence_after();
 #pragma unroll
@@ -337,31 +366,53 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     tmem_st32(tO + lane_off + c * 32, u);
                 }
             }
-            const float m_use = m_run;
+            // pass 2: p = 2^(s * scale + bias - m), row sum, bf16 P over the first 64 columns of S.
+            // A dead row (padding, or nothing visible yet) gets p = 0 through its constants.
+            const bool live = row_ok && m_run > -INFINITY;
+            float cbm[S::kE];
+#pragma unroll
+            for (int e = 0; e < S::kE; ++e) cbm[e] = live ? bl2[e] - m_run : -INFINITY;
             float psum = 0.f;
 #pragma unroll
-            for (int c = 0; c < kStepKeys / 64; ++c) {
-                uint32_t u[32];
+            for (int half = 0; half < 2; ++half) {
+                uint32_t u[64];
+                tmem_ld32(tS + lane_off + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+                tmem_ld32(tS + lane_off + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+                tmem_wait_ld();
+                uint32_t pk[32];
+                if (!need_mask) {
 #pragma unroll
-                for (int x = 0; x < 32; ++x) {
-                    const float p0 = (m_use == -INFINITY) ? 0.f : ex2(s[c * 64 + 2 * x] - m_use);
-                    const float p1 = (m_use == -INFINITY) ? 0.f : ex2(s[c * 64 + 2 * x + 1] - m_use);
-                    psum += p0 + p1;
-                    u[x] = pack_bf16x2(p0, p1);
+                    for (int x = 0; x < 32; ++x) {
+                        const int kc = half * 64 + 2 * x;
+                        const float p0 = ex2(fmaf(__uint_as_float(u[2 * x]), sl2, cbm[kc / BLK]));
+                        const float p1 = ex2(fmaf(__uint_as_float(u[2 * x + 1]), sl2, cbm[(kc + 1) / BLK]));
+                        psum += p0 + p1;
+                        pk[x] = pack_bf16x2(p0, p1);
+                    }
+                } else {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) {
+                        const int kc = half * 64 + 2 * x;
+                        const float a0 = (kc % BLK) < lim[kc / BLK] ? cbm[kc / BLK] : -INFINITY;
+                        const float a1 = ((kc + 1) % BLK) < lim[(kc + 1) / BLK] ? cbm[(kc + 1) / BLK] : -INFINITY;
+                        const float p0 = ex2(fmaf(__uint_as_float(u[2 * x]), sl2, a0));
+                        const float p1 = ex2(fmaf(__uint_as_float(u[2 * x + 1]), sl2, a1));
+                        psum += p0 + p1;
+                        pk[x] = pack_bf16x2(p0, p1);
+                    }
                 }
-                tmem_st32(tSj + lane_off + c * 32, u);
+                tmem_st32(tS + lane_off + half * 32, pk);
             }
             l_run += psum;
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(B.p_full + (j & 1));
+            mbar_arrive(B.p_full);
         }
         // epilogue: O / l -> bf16
         if (ok && !*abort) {
             bool have = true;
             if (nsteps > 0)
-                have = __all_sync(0xffffffffu, wait_bar(B.pv_done + ((nsteps - 1) & 1), ((nsteps - 1) >> 1) & 1,
-                                                        limit_ns, abort));
+                have = __all_sync(0xffffffffu, wait_bar(B.pv_done, (nsteps - 1) & 1, limit_ns, abort));
             tc_fence_after();
             if (have) {
                 __nv_bfloat16 *op = reinterpret_cast<__nv_bfloat16 *>(const_cast<void *>(O.p)) + b * O.s0 +
@@ -402,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 // ------------------------------------------------------------------ host side
 
 template <int D, int BLK>
-cudaError_t launch_t(const TcParams &tp, const TView &O, const Geom &G, const ListsView &L, int flags,
+cudaError_t launch_t(const TcParams &tp, const TView &Q, const TView &O, const Geom &G, const ListsView &L, int flags,
                      cudaStream_t st) {
     using S = Smem<D, BLK>;
     const size_t smem = S::kTotal + 1024;
@@ -410,7 +461,7 @@ cudaError_t launch_t(const TcParams &tp, const TView &O, const Geom &G, const Li
                                          (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)L.n_tiles, (unsigned)G.hkv, (unsigned)G.b);
-    attn_tc_kernel<D, BLK><<<grid, kThreads, smem, st>>>(tp, O, G, L, flags);
+    attn_tc_kernel<D, BLK><<<grid, kThreads, smem, st>>>(tp, Q, O, G, L, flags);
     return cudaGetLastError();
 }
 
@@ -433,7 +484,7 @@ cudaError_t launch_attn_tc(const TView &Q, const TView &K, const TView &V, const
     if (!make_map_bf16(&tp.tmK, K, G.b, G.nk, G.hkv, G.d, 1, G.B)) return cudaErrorInvalidValue;
     if (!make_map_bf16(&tp.tmV, V, G.b, G.nk, G.hkv, G.d, 1, G.B)) return cudaErrorInvalidValue;
 #define DASH_TC_CASE(DD, BB) \
-    if (G.d == DD && G.B == BB) return launch_t<DD, BB>(tp, O, G, L, flags, st);
+    if (G.d == DD && G.B == BB) return launch_t<DD, BB>(tp, Q, O, G, L, flags, st);
     DASH_TC_CASE(128, 64)
     DASH_TC_CASE(128, 128)
     DASH_TC_CASE(128, 32)

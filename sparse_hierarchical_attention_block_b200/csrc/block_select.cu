@@ -65,114 +65,124 @@ __device__ __forceinline__ float relu_pow_m1(float t, const SelParams &P) {
     }
 }
 
-// f(tau) and f'(tau) over x = (alpha-1) * X[0..n) read from shared memory.
-__device__ __forceinline__ void residual(const float *X, int n, float am1, float tau, const SelParams &P,
-                                         float &f, float &df) {
-    float a = 0.f, b = 0.f;
-    for (int c = threadIdx.x % 32; c < n; c += 32) {
-        float t = am1 * X[c] - tau;
-        a += relu_pow(t, P);
-        b += relu_pow_m1(t, P);
-    }
-    f = warp_sum(a) - 1.f;
-    df = -P.kexp * warp_sum(b);
-}
-
-// Solve the entmax threshold of one (row, head) pair; the whole warp calls it.
+// Solve the entmax threshold of one (row, head) pair over x = (alpha-1) * X[0..n)
+// in shared memory; the whole warp calls it.
+//   bracket  f(mx - 1) >= 0 (the largest term alone is 1), f(mx - n^{1-alpha}) <= 0
+//            (every term is at most 1/n);
+//   start    a 32-bin histogram of x over [mx - 1, mx) estimates f at the bin edges
+//            (mass at the bin centres): the highest edge still estimated >= 0;
+//   iterate  alpha = 2 / 1.5: the exact closed form on the current support
+//            {x > tau}, until the support no longer changes; other alpha: Newton.
+//            Steps leaving the bracket fall back to bisection.
 __device__ float solve_tau(const float *X, int n, const SelParams &P, int *hist) {
     const int lane = threadIdx.x % 32;
     const float am1 = P.alpha - 1.f;
     float mx = -INFINITY;
     for (int c = lane; c < n; c += 32) mx = fmaxf(mx, am1 * X[c]);
     mx = warp_max(mx);
-    // Bracket: f(mx - 1) >= 0 (the largest term alone is 1) and
-    //          f(mx - n^{1-alpha}) <= 0 (every term is at most 1/n).
     float lo = mx - 1.f;
     float hi = mx - powf((float)n, 1.f - P.alpha);
     if (n == 1) return lo;
 
-    // Histogram initialisation: 32 bins over [mx - 1, mx); estimate f at each
-    // bin's lower edge from the bin counts (mass at bin centres), start from
-    // the highest edge whose estimate is still >= 0.
     hist[lane] = 0;
     __syncwarp();
     for (int c = lane; c < n; c += 32) {
-        float y = am1 * X[c] - lo;  // in [.., 1]
-        if (y >= 0.f) {
-            int bin = min(31, (int)(y * 32.f));
-            atomicAdd(&hist[bin], 1);
-        }
+        const float y = am1 * X[c] - lo;
+        if (y >= 0.f) atomicAdd(&hist[min(31, (int)(y * 32.f))], 1);
     }
     __syncwarp();
+    float tau = lo;
     {
         const float edge = (float)lane * (1.f / 32.f);
-        float fe = 0.f;
+        float fe = -1.f;
         for (int j = lane; j < 32; ++j) fe += (float)hist[j] * relu_pow(((float)j + 0.5f) * (1.f / 32.f) - edge, P);
-        fe -= 1.f;
-        unsigned ok = __ballot_sync(0xffffffffu, fe >= 0.f);
-        int jstar = 31 - __clz(ok | 1u);
-        float t0 = lo + (float)jstar * (1.f / 32.f);
-        if (t0 > lo && t0 < hi) {
-            float f, df;
-            residual(X, n, am1, t0, P, f, df);
-            if (f >= 0.f) lo = t0;
-            else hi = t0;
-        }
+        const unsigned okb = __ballot_sync(0xffffffffu, fe >= 0.f);
+        const float t0 = lo + (float)(31 - __clz(okb | 1u)) * (1.f / 32.f);
+        if (t0 > lo && t0 < hi) tau = t0;
     }
     __syncwarp();
 
-    // Safeguarded Newton: f is decreasing; Newton steps that leave (lo, hi)
-    // are replaced by bisection.
-    float tau = lo;
-    for (int it = 0; it < 60; ++it) {
-        float f, df;
-        residual(X, n, am1, tau, P, f, df);
-        if (f == 0.f) break;
-        if (f > 0.f) lo = tau;
+    int prev_cnt = -1;
+    for (int it = 0; it < 40; ++it) {
+        float f = 0.f, df = 0.f, s1 = 0.f, s2 = 0.f;
+        int cnt = 0;
+        for (int c = lane; c < n; c += 32) {
+            const float xv = am1 * X[c];
+            const float t = xv - tau;
+            if (t > 0.f) {
+                f += relu_pow(t, P);
+                df += relu_pow_m1(t, P);
+                const float y = xv - mx;
+                s1 += y;
+                s2 += y * y;
+                ++cnt;
+            }
+        }
+        f = warp_sum(f) - 1.f;
+        df = -P.kexp * warp_sum(df);
+        s1 = warp_sum(s1);
+        s2 = warp_sum(s2);
+        cnt = warp_sum_i(cnt);
+        if (f >= 0.f) lo = tau;
         else hi = tau;
-        float nt = (df < 0.f) ? tau - f / df : 0.5f * (lo + hi);
-        if (!(nt > lo && nt < hi)) nt = 0.5f * (lo + hi);
-        if (fabsf(nt - tau) <= 1e-7f * fmaxf(1.f, fabsf(tau)) || hi - lo <= 1e-7f * fmaxf(1.f, fabsf(tau))) {
-            tau = nt;
-            break;
+        float nt;
+        if ((P.kint == 1 || P.kint == 2) && cnt > 0) {
+            // the previous step was the exact closed form on this same support
+            // (supports {x > tau} are nested, so equal counts mean equal sets): done
+            if (cnt == prev_cnt) break;
+            prev_cnt = cnt;
+            const float m1 = s1 / (float)cnt;
+            if (P.kint == 1) {
+                nt = mx + (s1 - 1.f) / (float)cnt;
+            } else {
+                const float var = fmaxf(s2 / (float)cnt - m1 * m1, 0.f);
+                nt = mx + m1 - sqrtf(fmaxf(1.f / (float)cnt - var, 0.f));
+            }
+            if (!(nt >= lo && nt <= hi)) {
+                nt = 0.5f * (lo + hi);  // a bisection step: the next count proves nothing
+                prev_cnt = -1;
+            }
+        } else {
+            nt = df < 0.f ? tau - f / df : 0.5f * (lo + hi);
+            if (!(nt > lo && nt < hi)) nt = 0.5f * (lo + hi);
+            if (fabsf(nt - tau) <= 1e-7f * fmaxf(1.f, fabsf(tau)) || hi - lo <= 1e-7f * fmaxf(1.f, fabsf(tau))) {
+                tau = nt;
+                break;
+            }
         }
         tau = nt;
     }
+    return tau;
+}
 
-    // Exact polish on the support for alpha = 2 and alpha = 1.5.
-    if (P.kint == 1 || P.kint == 2) {
-        for (int pass = 0; pass < 4; ++pass) {
-            float s1 = 0.f;
-            int k = 0;
-            for (int c = lane; c < n; c += 32) {
-                float x = am1 * X[c];
-                if (x > tau) { s1 += x; ++k; }
-            }
-            s1 = warp_sum(s1);
-            k = warp_sum_i(k);
-            if (k == 0) break;
-            float nt;
-            if (P.kint == 1) {
-                nt = (s1 - 1.f) / (float)k;
-            } else {
-                const float m = s1 / (float)k;
-                float v = 0.f;
-                for (int c = lane; c < n; c += 32) {
-                    float x = am1 * X[c];
-                    if (x > tau) v += (x - m) * (x - m);
-                }
-                v = warp_sum(v) / (float)k;
-                nt = m - sqrtf(fmaxf(1.f / (float)k - v, 0.f));
-            }
-            // same support under the new threshold?
-            int k2 = 0;
-            for (int c = lane; c < n; c += 32) k2 += (am1 * X[c] > nt);
-            k2 = warp_sum_i(k2);
-            tau = nt;
-            if (k2 == k) break;
+// log w_c of one row and chunk: w_c = (1/g) sum_h [x_c^(h) - tau_h]_+^{1/(alpha-1)}.
+// Returns -inf when no head routes the chunk.  The direct power sum is used
+// unless it underflows, then the log-sum-exp form of the same sum.
+__device__ __forceinline__ float group_logw(const float *X, int ldx, const float *taus, int g, int c,
+                                            const SelParams &P, float log_g) {
+    const float am1 = P.alpha - 1.f;
+    float v = 0.f;
+    bool sel = false;
+    for (int hh = 0; hh < g; ++hh) {
+        const float t = am1 * X[(size_t)hh * ldx + c] - taus[hh];
+        if (t > 0.f) {
+            sel = true;
+            v += relu_pow(t, P);
         }
     }
-    return tau;
+    if (!sel) return -INFINITY;
+    if (v > 0.f) return logf(v) - log_g;
+    float mlog = -INFINITY;
+    for (int hh = 0; hh < g; ++hh) {
+        const float t = am1 * X[(size_t)hh * ldx + c] - taus[hh];
+        if (t > 0.f) mlog = fmaxf(mlog, P.kexp * logf(t));
+    }
+    float acc = 0.f;
+    for (int hh = 0; hh < g; ++hh) {
+        const float t = am1 * X[(size_t)hh * ldx + c] - taus[hh];
+        if (t > 0.f) acc += expf(P.kexp * logf(t) - mlog);
+    }
+    return mlog + logf(acc) - log_g;
 }
 
 // Logits of P pairs against chunks [0, nvis) -> X[p][c] (scaled by gamma/sqrt(d)).
@@ -276,61 +286,55 @@ __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(TView Q, const
     }
     __syncthreads();
 
-    // (3) group prior, routed set, bias and mask, one warp per row
-    const float am1 = P.alpha - 1.f;
+    // (3) group prior, routed set, bias and mask; every warp works on each row
     const float log_g = logf((float)g);
-    for (int s = warp; s < nrows; s += kSelWarps) {
+    float *red = taus + P.S * g;   // [2 * warps] block reduction scratch (after the histogram)
+    red += kSelWarps * 32;
+    for (int s = 0; s < nrows; ++s) {
         const int64_t i = i0 + s;
         const int n = row_nvis(G, i);
         const size_t rowoff = ((size_t)(b * G.nq + i) * G.hkv + r);
+        const float *Xs = X + (size_t)(s * g) * P.ldx;
+        const float *ts = taus + s * g;
+        // sweep 1: log w per chunk into the first head's logits row (no longer needed), mu
+        float *lw = X + (size_t)(s * g) * P.ldx;
         float lsum = 0.f;
         int cnt = 0;
-        // first sweep: mu
-        for (int c = lane; c < n; c += 32) {
-            float mlog = -INFINITY;
-            for (int hh = 0; hh < g; ++hh) {
-                float t = am1 * X[(size_t)(s * g + hh) * P.ldx + c] - taus[s * g + hh];
-                if (t > 0.f) mlog = fmaxf(mlog, P.kexp * logf(t));
-            }
-            if (mlog > -INFINITY) {
-                float acc = 0.f;
-                for (int hh = 0; hh < g; ++hh) {
-                    float t = am1 * X[(size_t)(s * g + hh) * P.ldx + c] - taus[s * g + hh];
-                    if (t > 0.f) acc += expf(P.kexp * logf(t) - mlog);
-                }
-                lsum += mlog + logf(acc) - log_g;
+        // each column is read and then overwritten by the one thread that owns it
+        for (int c = threadIdx.x; c < n; c += kSelThreads) {
+            const float v = group_logw(Xs, P.ldx, ts, g, c, P, log_g);
+            if (v > -INFINITY) {
+                lsum += v;
                 ++cnt;
             }
+            lw[c] = v;
         }
+        __syncthreads();
         lsum = warp_sum(lsum);
         cnt = warp_sum_i(cnt);
-        const float mu = cnt ? lsum / (float)cnt : 0.f;
-        // second sweep: bias, mask bits, optional w
-        for (int c0 = 0; c0 < G.words * 32; c0 += 32) {
-            const int c = c0 + lane;
-            bool sel = false;
-            float lw = -INFINITY;
-            if (c < n) {
-                float mlog = -INFINITY;
-                for (int hh = 0; hh < g; ++hh) {
-                    float t = am1 * X[(size_t)(s * g + hh) * P.ldx + c] - taus[s * g + hh];
-                    if (t > 0.f) mlog = fmaxf(mlog, P.kexp * logf(t));
-                }
-                if (mlog > -INFINITY) {
-                    float acc = 0.f;
-                    for (int hh = 0; hh < g; ++hh) {
-                        float t = am1 * X[(size_t)(s * g + hh) * P.ldx + c] - taus[s * g + hh];
-                        if (t > 0.f) acc += expf(P.kexp * logf(t) - mlog);
-                    }
-                    lw = mlog + logf(acc) - log_g;
-                    sel = true;
-                }
-            }
-            const unsigned bits = __ballot_sync(0xffffffffu, sel);
-            if (lane == 0) out.mask[rowoff * G.words + c0 / 32] = bits;
-            if (sel && out.dvals) out.dvals[rowoff * G.n_chunks + c] = (lw - mu) / P.sigma;
-            if (out.w && c < G.n_chunks) out.w[rowoff * G.n_chunks + c] = sel ? expf(lw) : 0.f;
+        if (lane == 0) {
+            red[warp] = lsum;
+            reinterpret_cast<int *>(red)[kSelWarps + warp] = cnt;
         }
+        __syncthreads();
+        float tl = 0.f;
+        int tc = 0;
+        for (int w = 0; w < kSelWarps; ++w) {
+            tl += red[w];
+            tc += reinterpret_cast<int *>(red)[kSelWarps + w];
+        }
+        const float mu = tc ? tl / (float)tc : 0.f;
+        // sweep 2: bias, mask bits, optional w (a warp per 32-chunk word)
+        for (int wd = warp; wd < G.words; wd += kSelWarps) {
+            const int c = wd * 32 + lane;
+            const float v = c < n ? lw[c] : -INFINITY;
+            const bool sel = v > -INFINITY;
+            const unsigned bits = __ballot_sync(0xffffffffu, sel);
+            if (lane == 0) out.mask[rowoff * G.words + wd] = bits;
+            if (sel && out.dvals) out.dvals[rowoff * G.n_chunks + c] = (v - mu) / P.sigma;
+            if (out.w && c < G.n_chunks) out.w[rowoff * G.n_chunks + c] = sel ? expf(v) : 0.f;
+        }
+        __syncthreads();
     }
 }
 
@@ -347,6 +351,8 @@ __global__ void __launch_bounds__(128) compact_kernel(Geom G, const uint32_t *__
     const int64_t i0 = t * T;
     const int nrows = (int)min((int64_t)T, G.nq - i0);
     const size_t tile_idx = ((size_t)b * G.hkv + r) * L.n_tiles + t;
+    if (L.rows)
+        for (int s = threadIdx.x; s < T; s += blockDim.x) L.rows[tile_idx * T + s] = s < nrows ? (int)(i0 + s) : -1;
 
     // diagonal chunk range of the tile's rows (causal)
     int dlo = 0, dhi = -1;
@@ -408,6 +414,144 @@ __global__ void __launch_bounds__(128) compact_kernel(Geom G, const uint32_t *__
     }
 }
 
+// Regroup + compact: one CTA per (window of kTilesPerWindow tiles, kv head, batch),
+// one warp per output tile.  The window's query rows are sorted by the size of
+// their routed set (stable), consecutive runs of tile_rows rows form the tiles,
+// and each tile's list is built as in compact_kernel: the rows' diagonal chunks
+// first (ascending), then the union of their routed chunks (ascending), and the
+// per-row bias table.  Rows with similar routed sets share a tile, so the union a
+// tile streams through Stage 2 is smaller than for consecutive rows.
+constexpr int kTilesPerWindow = 4;
+
+__global__ void __launch_bounds__(32 * kTilesPerWindow) regroup_compact_kernel(Geom G, const uint32_t *__restrict__ mask,
+                                                                               const float *__restrict__ dvals,
+                                                                               ListsView L, int wpow2) {
+    extern __shared__ __align__(16) uint32_t rsm[];
+    const int T = L.tile_rows;
+    const int W = T * kTilesPerWindow;
+    uint32_t *key = rsm;                              // [wpow2] sort keys
+    int *rowi = reinterpret_cast<int *>(key + wpow2);  // [W] query index per window slot
+    const int64_t win = blockIdx.x;
+    const int r = blockIdx.y;
+    const int64_t b = blockIdx.z;
+    const int64_t i0 = win * W;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+    for (int j = threadIdx.x; j < wpow2; j += blockDim.x) {
+        const int64_t i = i0 + j;
+        uint32_t k = 0xffffffffu;
+        if (j < W && i < G.nq) {
+            const uint32_t *mw = mask + ((size_t)(b * G.nq + i) * G.hkv + r) * G.words;
+            int cnt = 0;
+            for (int w = 0; w < G.words; ++w) cnt += __popc(mw[w]);
+            k = ((uint32_t)cnt << 16) | (uint32_t)j;
+        }
+        key[j] = k;
+    }
+    __syncthreads();
+    // bitonic sort, ascending
+    for (int k2 = 2; k2 <= wpow2; k2 <<= 1) {
+        for (int jj = k2 >> 1; jj > 0; jj >>= 1) {
+            for (int idx = threadIdx.x; idx < wpow2; idx += blockDim.x) {
+                const int ixj = idx ^ jj;
+                if (ixj > idx) {
+                    const bool asc = (idx & k2) == 0;
+                    const uint32_t a = key[idx], c = key[ixj];
+                    if ((a > c) == asc) {
+                        key[idx] = c;
+                        key[ixj] = a;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    for (int j = threadIdx.x; j < W; j += blockDim.x) {
+        const uint32_t k = key[j];
+        rowi[j] = k == 0xffffffffu ? -1 : (int)(i0 + (k & 0xffffu));
+    }
+    __syncthreads();
+
+    const int64_t tile = win * kTilesPerWindow + warp;
+    if (tile >= L.n_tiles) return;
+    const size_t tile_idx = ((size_t)b * G.hkv + r) * L.n_tiles + tile;
+    const int *tr = rowi + warp * T;
+    for (int j = lane; j < T; j += 32) L.rows[tile_idx * T + j] = tr[j];
+
+    // diagonal chunks of the tile's rows, relative to the window's first chunk
+    uint64_t dmask = 0;
+    const int dbase = G.causal ? (int)(row_pos(G, i0) / G.B) : 0;
+    if (G.causal)
+        for (int j = lane; j < T; j += 32)
+            if (tr[j] >= 0) dmask |= 1ull << ((int)(row_pos(G, tr[j]) / G.B) - dbase);
+    const uint32_t dlo32 = __reduce_or_sync(0xffffffffu, (uint32_t)dmask);
+    const uint32_t dhi32 = __reduce_or_sync(0xffffffffu, (uint32_t)(dmask >> 32));
+    dmask = ((uint64_t)dhi32 << 32) | dlo32;
+    const int nd = __popcll(dmask);
+
+    // union of routed chunks, diagonal ones removed; lane l owns the contiguous words
+    // [l*wpl, (l+1)*wpl) so that the lane-order prefix is the chunk order
+    uint32_t *uw = reinterpret_cast<uint32_t *>(rowi + W) + (size_t)warp * G.words;
+    const int wpl = (G.words + 31) / 32;
+    int cnt = 0;
+    for (int wd = lane * wpl; wd < min(G.words, (lane + 1) * wpl); ++wd) {
+        uint32_t acc = 0;
+        for (int j = 0; j < T; ++j)
+            if (tr[j] >= 0) acc |= mask[((size_t)(b * G.nq + tr[j]) * G.hkv + r) * G.words + wd];
+        for (int c = wd * 32; c < wd * 32 + 32; ++c) {
+            const int rel = c - dbase;
+            if (rel >= 0 && rel < 64 && ((dmask >> rel) & 1ull)) acc &= ~(1u << (c - wd * 32));
+        }
+        uw[wd] = acc;
+        cnt += __popc(acc);
+    }
+    // exclusive prefix of the per-lane counts
+    int incl = cnt;
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    int pos = nd + incl - cnt;
+    int32_t *ids = L.ids + tile_idx * L.cap;
+    float *bias = L.bias + tile_idx * (size_t)L.cap * T;
+    if (lane == 0) {
+        int e = 0;
+        uint64_t dm = dmask;
+        while (dm) {
+            const int bit = __ffsll((long long)dm) - 1;
+            dm &= dm - 1;
+            ids[e++] = dbase + bit;
+        }
+        L.count[tile_idx] = nd + total;
+    }
+    for (int wd = lane * wpl; wd < min(G.words, (lane + 1) * wpl); ++wd) {
+        uint32_t acc = uw[wd];
+        while (acc) {
+            const int bit = __ffs(acc) - 1;
+            acc &= acc - 1;
+            ids[pos++] = wd * 32 + bit;
+        }
+    }
+    __syncwarp();
+    const int count = nd + total;
+    for (int idx = lane; idx < count * T; idx += 32) {
+        const int e = idx / T, j = idx % T;
+        const int c = ids[e];
+        const int i = tr[j];
+        float v = -INFINITY;
+        if (i < 0) {
+            v = 0.f;  // unused row: never stored
+        } else {
+            const size_t rowoff = (size_t)(b * G.nq + i) * G.hkv + r;
+            if (G.causal && c == (int)(row_pos(G, i) / G.B)) v = 0.f;
+            else if (c < row_nvis(G, i) && ((mask[rowoff * G.words + c / 32] >> (c % 32)) & 1u))
+                v = dvals[rowoff * G.n_chunks + c];
+        }
+        bias[(size_t)e * T + j] = v;
+    }
+}
+
 }  // namespace
 
 static int pick_rows_per_cta(const Geom &G, int dpad, int ldx, size_t *smem_out) {
@@ -416,7 +560,7 @@ static int pick_rows_per_cta(const Geom &G, int dpad, int ldx, size_t *smem_out)
     for (int S = 1; S <= 32; S *= 2) {
         if (S * G.g > 128 && S > 1) break;
         size_t sm = ((size_t)S * G.g * dpad + (size_t)kTileChunks * dpad + (size_t)S * G.g * ldx + S * G.g) * 4 +
-                    kSelWarps * 32 * 4;
+                    kSelWarps * 32 * 4 + 2 * kSelWarps * 4;
         if (sm > 200 * 1024 && S > 1) break;
         best = S;
         best_smem = sm;
@@ -452,6 +596,19 @@ cudaError_t launch_select_rows(const TView &Q, dash_dtype_t dt, const float *kba
         if (e != cudaSuccess) return e;
         select_rows_kernel<float><<<grid, kSelThreads, smem, st>>>(Q, kbar, G, P, o);
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_regroup_compact(const Geom &G, const uint32_t *mask, const float *dvals, const ListsView &L,
+                                   cudaStream_t st) {
+    if (G.nq == 0 || G.b == 0) return cudaSuccess;
+    const int W = L.tile_rows * kTilesPerWindow;
+    int wp = 1;
+    while (wp < W) wp *= 2;
+    const int64_t nwin = (L.n_tiles + kTilesPerWindow - 1) / kTilesPerWindow;
+    const size_t smem = (size_t)wp * 4 + (size_t)W * 4 + (size_t)kTilesPerWindow * G.words * 4;
+    regroup_compact_kernel<<<dim3((unsigned)nwin, (unsigned)G.hkv, (unsigned)G.b), 32 * kTilesPerWindow, smem, st>>>(
+        G, mask, dvals, L, wp);
     return cudaGetLastError();
 }
 

@@ -35,10 +35,19 @@ struct ListsView {
     int32_t *count;
     int32_t *ids;
     float *bias;
+    int32_t *rows;  // query index of each tile row (-1 unused); null = consecutive rows
     int64_t n_tiles;
     int cap;
     int tile_rows;
 };
+
+// Query index held by row `pos` of tile `tile_idx` (flattened [b][hkv][tile]) whose
+// tile number is t; -1 if the row is unused.
+__host__ __device__ inline int64_t tile_row(const ListsView &L, const Geom &G, size_t tile_idx, int64_t t, int pos) {
+    if (L.rows) return L.rows[tile_idx * L.tile_rows + pos];
+    const int64_t i = t * L.tile_rows + pos;
+    return i < G.nq ? i : -1;
+}
 
 // Causal geometry of query row i: key position, own chunk, visible chunks.
 __host__ __device__ inline int64_t row_pos(const Geom &G, int64_t i) { return i + G.nk - G.nq; }
@@ -150,6 +159,29 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32
         if (mbar_try_wait(bar, parity)) return true;
     report_timeout();
     return false;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for phase `parity` of `bar`, giving up after limit_ns of wall time
+// (global timer); on expiry the device error word is set and false returned.
+__device__ __forceinline__ bool mbar_wait_ns(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 255u) == 0) {
+            const uint64_t now = global_ns();
+            if (it == 0) t0 = now;
+            else if (now - t0 > limit_ns) {
+                report_timeout();
+                return false;
+            }
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------

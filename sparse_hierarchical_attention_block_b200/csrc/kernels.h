@@ -17,6 +17,15 @@ struct SelectOut {
 };
 cudaError_t launch_select_rows(const TView &Q, dash_dtype_t dt, const float *kbar, const Geom &G, float alpha,
                                float gamma, float sigma, const SelectOut &o, cudaStream_t st);
+bool select_tile_supported(const Geom &G, dash_dtype_t dt);
+size_t select_tile_workspace(const Geom &G);
+cudaError_t launch_select_tile(const TView &Q, const float *kbar, const Geom &G, float alpha, float gamma,
+                               float sigma, float *tau, float *w, uint32_t *mask, float *dvals, const ListsView &L,
+                               void *work, cudaStream_t st);
+// Regroup the query rows of each window of tiles by routed-set size and build the
+// tiles' work lists (with the row permutation) from the per-row masks and biases.
+cudaError_t launch_regroup_compact(const Geom &G, const uint32_t *mask, const float *dvals, const ListsView &L,
+                                   cudaStream_t st);
 cudaError_t launch_compact(const Geom &G, const uint32_t *mask, const float *dvals, const ListsView &L,
                            cudaStream_t st);
 

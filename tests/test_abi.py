@@ -44,11 +44,12 @@ def test_lists_geometry(lib):
     assert (tr, nt, cap) == (32, -(-1000 // 32), -(-1000 // 64))
     nt, cap, tr = dash.lists_geometry(1, 1, 131072, 8, 64, 4)
     assert (nt, cap, tr) == (1, 2048, 32)
-    cb, ib, bb = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    cb, ib, bb, rb = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
     rc = lib.dash_lists_geometry(2, 1000, 1000, 4, 64, 4, None, None, None, ctypes.byref(cb), ctypes.byref(ib),
-                                 ctypes.byref(bb))
+                                 ctypes.byref(bb), ctypes.byref(rb))
     assert rc == 0
     assert cb.value == 2 * 4 * 32 * 4 and ib.value == 2 * 4 * 32 * 16 * 4 and bb.value == ib.value * 32
+    assert rb.value == 2 * 4 * 32 * 32 * 4
     assert dash.dash_workspace_bytes(1, 8192, 8192, 32, 8, 128, 64) > 0
 
 

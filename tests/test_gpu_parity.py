@@ -86,7 +86,7 @@ def test_uniform_all_chunk_prior_is_dense_attention(dt, causal):
     b, nq, nk, hq, hkv, d, B = 1, 300, 520, 8, 2, 128, 64
     q, k, v = _planted(b, nq, nk, hq, hkv, d, B, dt, seed=7, causal=causal, planted=False)
     g = hq // hkv
-    L = dash.make_lists(q, k, B, g)
+    L = dash.make_lists(q, k, B, g, with_rows=False)
     nblk = -(-nk // B)
     for t in range(L.n_tiles):
         i0 = t * L.tile_rows
@@ -131,6 +131,52 @@ def test_decode_with_cached_summaries():
     a = _run(q, k, v, B, 1.5, True, sigma=1.0)
     c = _run(q, k, v, B, 1.5, True, sigma=1.0, kbar=kbar)
     assert torch.equal(a, c)
+
+
+@pytest.mark.parametrize("case", [CASES[0], CASES[3], CASES[5], CASES[9]], ids=["c0", "c3", "c5", "c9"])
+def test_consecutive_tiles_match_oracle(case):
+    """Without regrouping rows by routed-set size (every tile holds consecutive rows)."""
+    b, nq, nk, hq, hkv, d, B, dt, alpha, causal, sigma = case
+    q, k, v = _planted(b, nq, nk, hq, hkv, d, B, dt, seed=100 + nq, causal=causal)
+    out = _run(q, k, v, B, alpha, causal, sigma=sigma, flags=dash.DASH_FLAG_NO_REGROUP)
+    check_forward(q, k, v, out, B, alpha, causal, sigma=sigma, label=f"consecutive {case}")
+
+
+def test_regrouped_rows_are_a_permutation():
+    """Regrouping permutes the query rows within windows of 4 tiles: every row appears
+    once, tiles are filled before padding, and a tile's rows come from its window."""
+    b, nq, nk, hq, hkv, d, B = 2, 1000, 1000, 8, 2, 128, 64
+    q, k, v = _planted(b, nq, nk, hq, hkv, d, B, "bf16", seed=3)
+    L = dash.make_lists(q, k, B, hq // hkv)
+    dash.dash_block_select(q, k, B, 1.5, True, lists=L, sigma=1.0)
+    torch.cuda.synchronize()
+    rows = L.rows.cpu().numpy()          # [b, hkv, n_tiles, T]
+    T, nt = L.tile_rows, L.n_tiles
+    for bi in range(b):
+        for r in range(hkv):
+            flat = rows[bi, r].reshape(-1)
+            valid = np.sort(flat[flat >= 0])
+            assert np.array_equal(valid, np.arange(nq))
+            for t in range(nt):
+                tile = rows[bi, r, t]
+                w0 = (t // 4) * 4 * T
+                assert ((tile < 0) | ((tile >= w0) & (tile < w0 + 4 * T))).all()
+    counts = L.count.cpu().numpy()
+    assert (counts >= 1).all() and (counts <= L.cap).all()
+
+
+def test_regrouping_shrinks_the_union():
+    """On the planted workload, regrouped tiles stream fewer chunk entries than consecutive ones."""
+    w = synthetic.WORKLOADS["prefill8k"]
+    q, k, v = synthetic.make_inputs(w, "cuda")
+    La = dash.make_lists(q, k, w.block, w.g)
+    Lb = dash.make_lists(q, k, w.block, w.g, with_rows=False)
+    dash.dash_block_select(q, k, w.block, w.alpha, True, lists=La)
+    dash.dash_block_select(q, k, w.block, w.alpha, True, lists=Lb)
+    torch.cuda.synchronize()
+    ea, eb = int(La.count.sum()), int(Lb.count.sum())
+    print(f"[regroup] list entries regrouped {ea} vs consecutive {eb} ({ea / eb:.3f})")
+    assert ea < 0.85 * eb
 
 
 def test_deterministic():
