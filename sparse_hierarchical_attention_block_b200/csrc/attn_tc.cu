@@ -325,7 +325,6 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
                 uint32_t u[64];
                 tmem_ld32(tS + lane_off + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
                 tmem_ld32(tS + lane_off + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
-                tmem_wait_ld();
                 if (!need_mask) {
 #pragma unroll
                     for (int x = 0; x < 64; ++x) mx = fmaxf(mx, fmaf(__uint_as_float(u[x]), sl2, bl2[(half * 64 + x) / BLK]));
@@ -360,8 +359,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t u[32];
                     tmem_ld32(tO + lane_off + c * 32, u);
-                    tmem_wait_ld();
-#pragma unroll
+    #pragma unroll
                     for (int x = 0; x < 32; ++x) u[x] = __float_as_uint(__uint_as_float(u[x]) * f);
                     tmem_st32(tO + lane_off + c * 32, u);
                 }
@@ -378,7 +376,6 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
                 uint32_t u[64];
                 tmem_ld32(tS + lane_off + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
                 tmem_ld32(tS + lane_off + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
-                tmem_wait_ld();
                 uint32_t pk[32];
                 if (!need_mask) {
 #pragma unroll
@@ -393,10 +390,11 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
 #pragma unroll
                     for (int x = 0; x < 32; ++x) {
                         const int kc = half * 64 + 2 * x;
-                        const float a0 = (kc % BLK) < lim[kc / BLK] ? cbm[kc / BLK] : -INFINITY;
-                        const float a1 = ((kc + 1) % BLK) < lim[(kc + 1) / BLK] ? cbm[(kc + 1) / BLK] : -INFINITY;
-                        const float p0 = ex2(fmaf(__uint_as_float(u[2 * x]), sl2, a0));
-                        const float p1 = ex2(fmaf(__uint_as_float(u[2 * x + 1]), sl2, a1));
+                        // select after exp2: S of a key outside the list may be any bit pattern
+                        const float e0 = ex2(fmaf(__uint_as_float(u[2 * x]), sl2, cbm[kc / BLK]));
+                        const float e1 = ex2(fmaf(__uint_as_float(u[2 * x + 1]), sl2, cbm[(kc + 1) / BLK]));
+                        const float p0 = (kc % BLK) < lim[kc / BLK] ? e0 : 0.f;
+                        const float p1 = ((kc + 1) % BLK) < lim[(kc + 1) / BLK] ? e1 : 0.f;
                         psum += p0 + p1;
                         pk[x] = pack_bf16x2(p0, p1);
                     }
@@ -423,8 +421,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
                     uint32_t u[32];
                     if (nsteps > 0) {  // uniform across the CTA
                         tmem_ld32(tO + lane_off + c * 32, u);
-                        tmem_wait_ld();
-                    } else {
+                            } else {
 #pragma unroll
                         for (int x = 0; x < 32; ++x) u[x] = 0u;
                     }

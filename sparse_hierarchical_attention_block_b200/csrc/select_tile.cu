@@ -29,7 +29,7 @@ namespace dash {
 
 namespace {
 
-constexpr int kTileThreads = 128;
+constexpr int kTileThreads = 256;  // two threads per (row, head) pair
 constexpr int kChunkTile = 128;  // chunks per logits MMA (N)
 constexpr int kMaxTileChunks = 512;
 constexpr uint64_t kTileWaitNs = 2000000000ull;
@@ -74,13 +74,19 @@ template <int D>
 struct TSmem {
     static constexpr int kRegion = 128 * 128;              // 128 rows x 128 bytes
     static constexpr int kDh = D / 64;
+    // MMA phase: Q tile and one chunk tile of k̄ hi / lo operands
     static constexpr int kQ = 0;
     static constexpr int kHi = kQ + kDh * kRegion;
     static constexpr int kLo = kHi + kDh * kRegion;
-    static constexpr int kHist = kLo + kDh * kRegion;       // [32][128] int
-    static constexpr int kUnion = kHist + 32 * 128 * 4;     // [16] uint32
-    static constexpr int kWofs = kUnion + 16 * 4;           // [17] int
-    static constexpr int kBars = (kWofs + 17 * 4 + 7) & ~7; // q_full, mma_done, k_full
+    static constexpr int kMmaEnd = kLo + kDh * kRegion;
+    // solve phase (reuses the MMA region once the logits are in TMEM)
+    static constexpr int kHist = 0;                          // [2 halves][32 bins][128 pairs] uint16
+    static constexpr int kXch = kHist + 2 * 32 * 128 * 2;     // [2 parity][2 halves][128 pairs][8] float
+    static constexpr int kSolveEnd = kXch + 2 * 2 * 128 * 8 * 4;
+    static constexpr int kData = kMmaEnd > kSolveEnd ? kMmaEnd : kSolveEnd;
+    static constexpr int kUnion = kData;                     // [16] uint32
+    static constexpr int kWofs = kUnion + 16 * 4;            // [17] int
+    static constexpr int kBars = (kWofs + 17 * 4 + 7) & ~7;  // q_full, mma_done, k_full
     static constexpr int kSlot = kBars + 3 * 8;
     static constexpr int kTotal = kSlot + 16;
 };
@@ -126,6 +132,32 @@ __global__ void __launch_bounds__(256) kbar_split_kernel(const float *__restrict
     }
 }
 
+// Exchange of per-pass partial sums between the two threads of a pair (warps w and
+// w + 4 share TMEM lanes): each writes its NV values, a named barrier over those two
+// warps, each reads its partner's.  `parity` alternates the buffer so one barrier per
+// pass suffices.
+// Named barrier over the two warps (64 threads) that share TMEM lane quadrant `quad`;
+// constant ids 1..4 (0 is __syncthreads).
+__device__ __forceinline__ void quad_sync(int quad) {
+    switch (quad) {
+        case 0: asm volatile("bar.sync 1, 64;" ::: "memory"); break;
+        case 1: asm volatile("bar.sync 2, 64;" ::: "memory"); break;
+        case 2: asm volatile("bar.sync 3, 64;" ::: "memory"); break;
+        default: asm volatile("bar.sync 4, 64;" ::: "memory"); break;
+    }
+}
+
+template <int NV>
+__device__ __forceinline__ void pair_exchange(float *xch, int parity, int half, int p, int quad, float (&v)[NV]) {
+    float *mine = xch + ((size_t)(parity * 2 + half) * 128 + p) * 8;
+    const float *other = xch + ((size_t)(parity * 2 + (half ^ 1)) * 128 + p) * 8;
+#pragma unroll
+    for (int k = 0; k < NV; ++k) mine[k] = v[k];
+    quad_sync(quad);
+#pragma unroll
+    for (int k = 0; k < NV; ++k) v[k] = other[k];
+}
+
 template <int D, int KINT>
 __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                                       const uint8_t *__restrict__ ksplit, Geom G,
@@ -137,16 +169,18 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
     uint64_t *mma_done = q_full + 1;
     uint64_t *k_full = q_full + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + S::kSlot);
-    int *hist = reinterpret_cast<int *>(sm + S::kHist);
+    uint16_t *hist = reinterpret_cast<uint16_t *>(sm + S::kHist);
+    float *xch = reinterpret_cast<float *>(sm + S::kXch);
     uint32_t *uni = reinterpret_cast<uint32_t *>(sm + S::kUnion);
     int *wofs = reinterpret_cast<int *>(sm + S::kWofs);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int quad = warp & 3, half = warp >> 2;  // TMEM lane quadrant; which 32-column blocks
     const int64_t t = (int64_t)L.n_tiles - 1 - blockIdx.x;
     const int r = blockIdx.y;
     const int64_t b = blockIdx.z;
     const int g = G.g, T = L.tile_rows;
-    const int p = threadIdx.x;  // pair == TMEM lane
+    const int p = quad * 32 + lane;  // pair == TMEM lane
     const int pos = p / g, hh = p % g;
     const int64_t i = t * T + pos;
     const bool row_ok = i < G.nq;
@@ -154,7 +188,7 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
     const int64_t last_row = min(G.nq - 1, t * T + T - 1);
     const int nvis_max = row_nvis(G, last_row);
     const size_t tile_idx = ((size_t)b * G.hkv + r) * L.n_tiles + t;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const bool lead = hh == 0;
 
     if (threadIdx.x == 0) {
@@ -183,14 +217,12 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
     const int n_ct_all = (G.n_chunks + kChunkTile - 1) / kChunkTile;
     const uint8_t *ks = ksplit + (((size_t)b * G.hkv + r) * n_ct_all) * 2 * (size_t)(S::kDh * S::kRegion);
     for (int ct = 0; ct < n_ct; ++ct) {
-        // the chunk tile's hi / lo operands, pre-split and pre-swizzled: two bulk copies
         if (threadIdx.x == 0) {
+            // the chunk tile's hi / lo operands, pre-split and pre-swizzled: two bulk copies
             const uint8_t *src = ks + (size_t)ct * 2 * S::kDh * S::kRegion;
             mbar_arrive_expect_tx(k_full, 2 * S::kDh * S::kRegion);
             bulk_load(sm + S::kHi, src, S::kDh * S::kRegion, k_full);
             bulk_load(sm + S::kLo, src + S::kDh * S::kRegion, S::kDh * S::kRegion, k_full);
-        }
-        if (threadIdx.x == 0) {
             if (ct == 0) mbar_wait_ns(q_full, 0, kTileWaitNs);
             mbar_wait_ns(k_full, ct & 1, kTileWaitNs);
             tc_fence_after();
@@ -214,37 +246,46 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
         mbar_wait_ns(mma_done, ct & 1, kTileWaitNs);  // smem tile free, TMEM columns written
         tc_fence_after();
     }
+    __syncthreads();  // the MMA staging memory is reused below
 
     // ---------------------------------------------------------------- tau per pair
-    // Columns are read 32 at a time; the loop bound is uniform across the warp.
+    // Thread (quad, half) owns the 32-column blocks blk = half, half + 2, ... of its
+    // pair's TMEM row; the loop bound is uniform across each warp (tcgen05.ld is
+    // warp-collective) and the two threads of a pair combine partial sums per pass.
     const int nb = (__reduce_max_sync(0xffffffffu, (unsigned)nvis) + 31) / 32;
-    const float am1 = P.am1;
-    float tau;
+    const float xs = P.am1 * P.scale;  // x = (alpha - 1) * gamma / sqrt(d) * <q, k̄>
+    int parity = 0;
     float mx = -INFINITY;
-    for (int blk = 0; blk < nb; ++blk) {
+    for (int blk = half; blk < nb; blk += 2) {
         uint32_t u[32];
         tmem_ld32(tmem + lane_off + blk * 32, u);
-        tmem_wait_ld();
 #pragma unroll
         for (int x = 0; x < 32; ++x)
-            if (blk * 32 + x < nvis) mx = fmaxf(mx, am1 * P.scale * __uint_as_float(u[x]));
+            if (blk * 32 + x < nvis) mx = fmaxf(mx, xs * __uint_as_float(u[x]));
+    }
+    {
+        float v[1] = {mx};
+        pair_exchange<1>(xch, parity, half, p, quad, v);
+        parity ^= 1;
+        mx = fmaxf(mx, v[0]);
     }
     // bracket: f(mx - 1) >= 0 (the largest term alone is 1), f(mx - n^{1-alpha}) <= 0
     float lo = mx - 1.f;
     float hi = nvis > 0 ? mx - powf((float)nvis, 1.f - P.alpha) : 0.f;
-    // histogram initialisation: per-thread bins [bin][thread] over [mx - 1, mx)
+    // histogram initialisation: bins [half][bin][pair] over [mx - 1, mx)
+    uint16_t *hmine = hist + (size_t)half * 32 * 128;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) hist[j * kTileThreads + p] = 0;
-    for (int blk = 0; blk < nb; ++blk) {
+    for (int j = 0; j < 32; ++j) hmine[j * 128 + p] = 0;
+    for (int blk = half; blk < nb; blk += 2) {
         uint32_t u[32];
         tmem_ld32(tmem + lane_off + blk * 32, u);
-        tmem_wait_ld();
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
-            const float y = am1 * P.scale * __uint_as_float(u[x]) - lo;
-            if (blk * 32 + x < nvis && y >= 0.f) hist[min(31, (int)(y * 32.f)) * kTileThreads + p] += 1;
+            const float y = xs * __uint_as_float(u[x]) - lo;
+            if (blk * 32 + x < nvis && y >= 0.f) hmine[min(31, (int)(y * 32.f)) * 128 + p] += 1;
         }
     }
+    quad_sync(quad);
     float t0 = lo;
     if (nvis > 1) {
         // estimated f at a bin edge (mass at the bin centres) decreases with the edge:
@@ -255,42 +296,49 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
             const float edge = (float)e * (1.f / 32.f);
             float fe = -1.f;
             for (int j = e; j < 32; ++j)
-                fe += (float)hist[j * kTileThreads + p] * rpow<KINT>(((float)j + 0.5f) * (1.f / 32.f) - edge, P);
+                fe += (float)(hist[j * 128 + p] + hist[32 * 128 + j * 128 + p]) *
+                      rpow<KINT>(((float)j + 0.5f) * (1.f / 32.f) - edge, P);
             if (fe >= 0.f) elo = e;
             else ehi = e - 1;
         }
         t0 = lo + (float)elo * (1.f / 32.f);
         if (!(t0 < hi)) t0 = lo;
     }
-    // bracketed iteration; the loop runs while any lane of the warp is unfinished
-    // (tcgen05.ld is warp-collective), finished lanes only read.
-    tau = nvis == 1 ? lo : t0;
+    // bracketed iteration (identical on both threads of the pair: same combined sums)
+    float tau = nvis == 1 ? lo : t0;
     bool done = nvis <= 1;
     int prev_cnt = -1;
     for (int it = 0; it < 40; ++it) {
         if (__all_sync(0xffffffffu, done)) break;
-        float f = -1.f, df = 0.f, s1 = 0.f, s2 = 0.f;
-        int cnt = 0;
-        for (int blk = 0; blk < nb; ++blk) {
+        float acc[5] = {0.f, 0.f, 0.f, 0.f, 0.f};  // f + 1, -f'/k, s1, s2, count
+        for (int blk = half; blk < nb; blk += 2) {
             uint32_t u[32];
             tmem_ld32(tmem + lane_off + blk * 32, u);
-            tmem_wait_ld();
 #pragma unroll
             for (int x = 0; x < 32; ++x) {
-                const float xv = am1 * P.scale * __uint_as_float(u[x]);
+                const float xv = xs * __uint_as_float(u[x]);
                 const float tt = xv - tau;
                 if (blk * 32 + x < nvis && tt > 0.f) {
-                    f += rpow<KINT>(tt, P);
-                    df += rpow_m1<KINT>(tt, P);
+                    acc[0] += rpow<KINT>(tt, P);
+                    acc[1] += rpow_m1<KINT>(tt, P);
                     const float yv = xv - mx;
-                    s1 += yv;
-                    s2 += yv * yv;
-                    ++cnt;
+                    acc[2] += yv;
+                    acc[3] += yv * yv;
+                    acc[4] += 1.f;
                 }
             }
         }
+        {
+            float v[5] = {acc[0], acc[1], acc[2], acc[3], acc[4]};
+            pair_exchange<5>(xch, parity, half, p, quad, v);
+            parity ^= 1;
+            // the same order of additions on both threads of the pair
+#pragma unroll
+            for (int k = 0; k < 5; ++k) acc[k] = half == 0 ? acc[k] + v[k] : v[k] + acc[k];
+        }
         if (done) continue;
-        df *= -P.kexp;
+        const float f = acc[0] - 1.f, df = -P.kexp * acc[1], s1 = acc[2], s2 = acc[3];
+        const int cnt = (int)acc[4];
         if (f >= 0.f) lo = tau;
         else hi = tau;
         float nt;
@@ -322,8 +370,10 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
         tau = nt;
     }
     if (nvis == 0) tau = NAN;
-    if (out.tau && row_ok) out.tau[((size_t)b * G.nq + i) * G.hq + r * g + hh] = tau;
-    if (L.rows && lead) L.rows[tile_idx * T + pos] = row_ok ? (int)i : -1;
+    if (half == 0) {
+        if (out.tau && row_ok) out.tau[((size_t)b * G.nq + i) * G.hq + r * g + hh] = tau;
+        if (L.rows && lead) L.rows[tile_idx * T + pos] = row_ok ? (int)i : -1;
+    }
 
     // ---------------------------------------------------------------- group prior, pass 1: mu, union
     // log w_c replaces x_c in this lane's TMEM row (-inf where the row does not route c),
@@ -332,16 +382,14 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
     const uint32_t gmask = (g == 32) ? 0xffffffffu : ((1u << g) - 1u);
     const float log_g = logf((float)g);
     const float tau_r = nvis > 0 ? tau : INFINITY;  // rows without chunks select nothing
-    float lsum = 0.f;
-    int lcnt = 0;
-    for (int blk = 0; blk < nb; ++blk) {
+    float lsum = 0.f, lcnt = 0.f;
+    for (int blk = half; blk < nb; blk += 2) {
         uint32_t u[32];
         tmem_ld32(tmem + lane_off + blk * 32, u);
-        tmem_wait_ld();
         uint32_t word = 0;
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
-            const float tt = am1 * P.scale * __uint_as_float(u[x]) - tau_r;
+            const float tt = xs * __uint_as_float(u[x]) - tau_r;
             const bool own = (blk * 32 + x < nvis) && tt > 0.f;
             float v = own ? rpow<KINT>(tt, P) : 0.f;
             for (int o = 1; o < g; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -353,7 +401,7 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
                 // keep such a chunk routed with the smallest representable weight
                 lw = v > 0.f ? __logf(v) - log_g : -103.28f - log_g;
                 lsum += lw;
-                ++lcnt;
+                lcnt += 1.f;
                 word |= 1u << x;
             }
             u[x] = __float_as_uint(lw);
@@ -363,7 +411,14 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
         if (lane == 0 && wu) atomicOr(&uni[blk], wu);
     }
     tmem_wait_st();
-    const float mu = lcnt ? lsum / (float)lcnt : 0.f;
+    {
+        float v[2] = {lsum, lcnt};
+        pair_exchange<2>(xch, parity, half, p, quad, v);
+        parity ^= 1;
+        lsum = half == 0 ? lsum + v[0] : v[0] + lsum;
+        lcnt = half == 0 ? lcnt + v[1] : v[1] + lcnt;
+    }
+    const float mu = lcnt > 0.f ? lsum / lcnt : 0.f;
     __syncthreads();
 
     // ---------------------------------------------------------------- the tile's list
@@ -417,10 +472,9 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
     // ---------------------------------------------------------------- pass 2: bias, optional w / mask
     const float inv_sigma = 1.f / P.sigma;
     const size_t rowoff = ((size_t)b * G.nq + i) * G.hkv + r;
-    for (int blk = 0; blk < nb; ++blk) {
+    for (int blk = half; blk < nb; blk += 2) {
         uint32_t u[32];
         tmem_ld32(tmem + lane_off + blk * 32, u);
-        tmem_wait_ld();
         uint32_t word = 0;
         const uint32_t uw = uni[blk];
         const int base = wofs[blk];
@@ -444,7 +498,7 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
         }
         if (out.mask && lead && row_ok && blk < G.words) out.mask[rowoff * G.words + blk] = word;
     }
-    if (lead && row_ok) {
+    if (lead && row_ok && half == 0) {
         if (out.mask)
             for (int blk = nb; blk < G.words; ++blk) out.mask[rowoff * G.words + blk] = 0u;
         if (out.w)
@@ -467,7 +521,7 @@ bool select_tile_supported(const Geom &G, dash_dtype_t dt) {
     if (dt != DASH_BF16) return false;
     if (G.d != 64 && G.d != 128) return false;
     if (G.g & (G.g - 1)) return false;
-    if (G.tile_rows * G.g != kTileThreads) return false;
+    if (G.tile_rows * G.g != 128) return false;
     if (G.n_chunks > kMaxTileChunks) return false;
     return tma_encode_fn() != nullptr;
 }
