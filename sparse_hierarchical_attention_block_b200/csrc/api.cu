@@ -109,7 +109,7 @@ int check_opts(const dash_opts_t &o) {
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct WsLayout {
-    size_t kbar, mask, dvals, count, ids, bias, rows, decode, split, total;
+    size_t kbar, mask, logw, mu, count, ids, bias, rows, decode, split, total;
 };
 
 WsLayout ws_layout(const Geom &G, bool need_kbar, bool need_lists, bool need_decode) {
@@ -122,7 +122,8 @@ WsLayout ws_layout(const Geom &G, bool need_kbar, bool need_lists, bool need_dec
     };
     L.kbar = need_kbar ? take((size_t)G.b * G.n_chunks * G.hkv * G.d * 4) : 0;
     L.mask = take((size_t)G.b * G.nq * G.hkv * (size_t)G.words * 4);
-    L.dvals = need_lists ? take((size_t)G.b * G.nq * G.hkv * (size_t)G.n_chunks * 4) : 0;
+    L.logw = need_lists ? take((size_t)G.b * G.nq * G.hkv * (size_t)G.n_chunks * 4) : 0;
+    L.mu = need_lists ? take((size_t)G.b * G.nq * G.hkv * 4) : 0;
     L.count = need_lists ? take((size_t)G.b * G.hkv * G.n_tiles * 4) : 0;
     L.ids = need_lists ? take((size_t)G.b * G.hkv * G.n_tiles * G.n_blk * 4) : 0;
     L.bias = need_lists ? take((size_t)G.b * G.hkv * G.n_tiles * G.n_blk * G.tile_rows * 4) : 0;
@@ -201,26 +202,28 @@ int run_stage1(const dash_tensor_t *q, const Geom &G, float alpha, const dash_op
                const WsLayout &WL, cudaStream_t st) {
     cudaError_t e;
     const bool tile = select_tile_supported(G, q->dtype);
-    regroup = regroup && LV && LV->rows;
+    regroup = regroup && LV && LV->rows && regroup_supported(G);
     uint32_t *mask = mask_out ? mask_out : reinterpret_cast<uint32_t *>(ws + WL.mask);
-    float *dv = LV ? reinterpret_cast<float *>(ws + WL.dvals) : nullptr;
+    float *logw = reinterpret_cast<float *>(ws + WL.logw);
+    float *mu = reinterpret_cast<float *>(ws + WL.mu);
     if (tile && LV && !regroup) {
-        e = launch_select_tile(view(q), kbar, G, alpha, o.gamma, o.sigma, tau, w, mask_out, nullptr, *LV,
+        e = launch_select_tile(view(q), kbar, G, alpha, o.gamma, o.sigma, tau, w, mask_out, nullptr, nullptr, *LV,
                                ws + WL.split, st);
         return e == cudaSuccess ? DASH_OK : cuda_fail(e, "select_tile");
     }
     if (tile) {
         const ListsView geom_only{nullptr, nullptr, nullptr, nullptr, G.n_tiles, G.n_blk, G.tile_rows};
-        e = launch_select_tile(view(q), kbar, G, alpha, o.gamma, o.sigma, tau, w, mask, dv, geom_only,
+        e = launch_select_tile(view(q), kbar, G, alpha, o.gamma, o.sigma, tau, w, mask, logw, mu, geom_only,
                                ws + WL.split, st);
         if (e != cudaSuccess) return cuda_fail(e, "select_tile");
     } else {
-        SelectOut so{tau, w, mask, dv};
+        SelectOut so{tau, w, mask, LV ? logw : nullptr, LV ? mu : nullptr};
         e = launch_select_rows(view(q), q->dtype, kbar, G, alpha, o.gamma, o.sigma, so, st);
         if (e != cudaSuccess) return cuda_fail(e, "select_rows");
     }
     if (!LV) return DASH_OK;
-    e = regroup ? launch_regroup_compact(G, mask, dv, *LV, st) : launch_compact(G, mask, dv, *LV, st);
+    e = regroup ? launch_regroup_compact(G, mask, logw, mu, o.sigma, *LV, st)
+                : launch_compact(G, mask, logw, mu, o.sigma, *LV, st);
     return e == cudaSuccess ? DASH_OK : cuda_fail(e, "work-list compaction");
 }
 

@@ -324,6 +324,7 @@ __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(TView Q, const
             tc += reinterpret_cast<int *>(red)[kSelWarps + w];
         }
         const float mu = tc ? tl / (float)tc : 0.f;
+        if (out.mu && threadIdx.x == 0) out.mu[rowoff] = mu;
         // sweep 2: bias, mask bits, optional w (a warp per 32-chunk word)
         for (int wd = warp; wd < G.words; wd += kSelWarps) {
             const int c = wd * 32 + lane;
@@ -331,7 +332,7 @@ __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(TView Q, const
             const bool sel = v > -INFINITY;
             const unsigned bits = __ballot_sync(0xffffffffu, sel);
             if (lane == 0) out.mask[rowoff * G.words + wd] = bits;
-            if (sel && out.dvals) out.dvals[rowoff * G.n_chunks + c] = (v - mu) / P.sigma;
+            if (sel && out.logw) out.logw[rowoff * G.n_chunks + c] = v;
             if (out.w && c < G.n_chunks) out.w[rowoff * G.n_chunks + c] = sel ? expf(v) : 0.f;
         }
         __syncthreads();
@@ -340,7 +341,8 @@ __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(TView Q, const
 
 // One CTA per (batch, kv head, query tile).
 __global__ void __launch_bounds__(128) compact_kernel(Geom G, const uint32_t *__restrict__ mask,
-                                                      const float *__restrict__ dvals, ListsView L) {
+                                                      const float *__restrict__ logw, const float *__restrict__ mu,
+                                                      float inv_sigma, ListsView L) {
     extern __shared__ __align__(16) uint32_t csm[];
     uint32_t *uw = csm;                 // [words] union bits (diagonal range removed)
     int *wofs = reinterpret_cast<int *>(uw + G.words);  // [words + 1] exclusive prefix of popcounts
@@ -407,7 +409,7 @@ __global__ void __launch_bounds__(128) compact_kernel(Geom G, const uint32_t *__
             if (G.causal && c == (int)(row_pos(G, i) / G.B)) {
                 v = 0.f;  // diagonal chunk: bias 0, causal mask in Stage 2
             } else if (c < row_nvis(G, i) && ((mask[rowoff * G.words + c / 32] >> (c % 32)) & 1u)) {
-                v = dvals[rowoff * G.n_chunks + c];
+                v = (logw[rowoff * G.n_chunks + c] - mu[rowoff]) * inv_sigma;  // d_c = (log w_c - mu) / sigma
             }
         }
         bias[(size_t)e * T + s] = v;
@@ -424,8 +426,9 @@ __global__ void __launch_bounds__(128) compact_kernel(Geom G, const uint32_t *__
 constexpr int kTilesPerWindow = 4;
 
 __global__ void __launch_bounds__(32 * kTilesPerWindow) regroup_compact_kernel(Geom G, const uint32_t *__restrict__ mask,
-                                                                               const float *__restrict__ dvals,
-                                                                               ListsView L, int wpow2) {
+                                                                               const float *__restrict__ logw,
+                                                                               const float *__restrict__ mu,
+                                                                               float inv_sigma, ListsView L, int wpow2) {
     extern __shared__ __align__(16) uint32_t rsm[];
     const int T = L.tile_rows;
     const int W = T * kTilesPerWindow;
@@ -489,15 +492,25 @@ __global__ void __launch_bounds__(32 * kTilesPerWindow) regroup_compact_kernel(G
     dmask = ((uint64_t)dhi32 << 32) | dlo32;
     const int nd = __popcll(dmask);
 
+    // the tile rows' mask words and mu, cached in shared memory for the bias fill
+    uint32_t *uw = reinterpret_cast<uint32_t *>(rowi + W) + (size_t)warp * G.words;
+    uint32_t *mrow = reinterpret_cast<uint32_t *>(rowi + W) + (size_t)kTilesPerWindow * G.words +
+                     (size_t)warp * T * G.words;
+    float *murow = reinterpret_cast<float *>(reinterpret_cast<uint32_t *>(rowi + W) + (size_t)kTilesPerWindow * G.words +
+                                             (size_t)kTilesPerWindow * T * G.words) + warp * T;
+    for (int idx = lane; idx < T * G.words; idx += 32) {
+        const int j = idx / G.words, wd = idx % G.words;
+        mrow[idx] = tr[j] >= 0 ? mask[((size_t)(b * G.nq + tr[j]) * G.hkv + r) * G.words + wd] : 0u;
+    }
+    for (int j = lane; j < T; j += 32) murow[j] = tr[j] >= 0 ? mu[(size_t)(b * G.nq + tr[j]) * G.hkv + r] : 0.f;
+    __syncwarp();
     // union of routed chunks, diagonal ones removed; lane l owns the contiguous words
     // [l*wpl, (l+1)*wpl) so that the lane-order prefix is the chunk order
-    uint32_t *uw = reinterpret_cast<uint32_t *>(rowi + W) + (size_t)warp * G.words;
     const int wpl = (G.words + 31) / 32;
     int cnt = 0;
     for (int wd = lane * wpl; wd < min(G.words, (lane + 1) * wpl); ++wd) {
         uint32_t acc = 0;
-        for (int j = 0; j < T; ++j)
-            if (tr[j] >= 0) acc |= mask[((size_t)(b * G.nq + tr[j]) * G.hkv + r) * G.words + wd];
+        for (int j = 0; j < T; ++j) acc |= mrow[j * G.words + wd];
         for (int c = wd * 32; c < wd * 32 + 32; ++c) {
             const int rel = c - dbase;
             if (rel >= 0 && rel < 64 && ((dmask >> rel) & 1ull)) acc &= ~(1u << (c - wd * 32));
@@ -535,6 +548,7 @@ __global__ void __launch_bounds__(32 * kTilesPerWindow) regroup_compact_kernel(G
     }
     __syncwarp();
     const int count = nd + total;
+#pragma unroll 4
     for (int idx = lane; idx < count * T; idx += 32) {
         const int e = idx / T, j = idx % T;
         const int c = ids[e];
@@ -542,11 +556,11 @@ __global__ void __launch_bounds__(32 * kTilesPerWindow) regroup_compact_kernel(G
         float v = -INFINITY;
         if (i < 0) {
             v = 0.f;  // unused row: never stored
-        } else {
+        } else if (G.causal && c == (int)(row_pos(G, i) / G.B)) {
+            v = 0.f;
+        } else if (c < row_nvis(G, i) && ((mrow[j * G.words + c / 32] >> (c % 32)) & 1u)) {
             const size_t rowoff = (size_t)(b * G.nq + i) * G.hkv + r;
-            if (G.causal && c == (int)(row_pos(G, i) / G.B)) v = 0.f;
-            else if (c < row_nvis(G, i) && ((mask[rowoff * G.words + c / 32] >> (c % 32)) & 1u))
-                v = dvals[rowoff * G.n_chunks + c];
+            v = (logw[rowoff * G.n_chunks + c] - murow[j]) * inv_sigma;  // d_c = (log w_c - mu) / sigma
         }
         bias[(size_t)e * T + j] = v;
     }
@@ -599,25 +613,40 @@ cudaError_t launch_select_rows(const TView &Q, dash_dtype_t dt, const float *kba
     return cudaGetLastError();
 }
 
-cudaError_t launch_regroup_compact(const Geom &G, const uint32_t *mask, const float *dvals, const ListsView &L,
-                                   cudaStream_t st) {
+static size_t regroup_smem(const Geom &G) {
+    const int W = G.tile_rows * kTilesPerWindow;
+    int wp = 1;
+    while (wp < W) wp *= 2;
+    return (size_t)wp * 4 + (size_t)W * 4 + (size_t)kTilesPerWindow * G.words * 4 +
+           (size_t)kTilesPerWindow * G.tile_rows * G.words * 4 + (size_t)kTilesPerWindow * G.tile_rows * 4;
+}
+
+bool regroup_supported(const Geom &G) { return regroup_smem(G) <= 200 * 1024; }
+
+cudaError_t launch_regroup_compact(const Geom &G, const uint32_t *mask, const float *logw, const float *mu,
+                                   float sigma, const ListsView &L, cudaStream_t st) {
     if (G.nq == 0 || G.b == 0) return cudaSuccess;
     const int W = L.tile_rows * kTilesPerWindow;
     int wp = 1;
     while (wp < W) wp *= 2;
     const int64_t nwin = (L.n_tiles + kTilesPerWindow - 1) / kTilesPerWindow;
-    const size_t smem = (size_t)wp * 4 + (size_t)W * 4 + (size_t)kTilesPerWindow * G.words * 4;
+    const size_t smem = regroup_smem(G);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(regroup_compact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+    }
     regroup_compact_kernel<<<dim3((unsigned)nwin, (unsigned)G.hkv, (unsigned)G.b), 32 * kTilesPerWindow, smem, st>>>(
-        G, mask, dvals, L, wp);
+        G, mask, logw, mu, 1.f / sigma, L, wp);
     return cudaGetLastError();
 }
 
-cudaError_t launch_compact(const Geom &G, const uint32_t *mask, const float *dvals, const ListsView &L,
-                           cudaStream_t st) {
+cudaError_t launch_compact(const Geom &G, const uint32_t *mask, const float *logw, const float *mu, float sigma,
+                           const ListsView &L, cudaStream_t st) {
     if (G.nq == 0 || G.b == 0) return cudaSuccess;
     dim3 grid((unsigned)L.n_tiles, (unsigned)G.hkv, (unsigned)G.b);
     const size_t smem = (size_t)G.words * 4 + (size_t)(G.words + 1) * 4 + 16;
-    compact_kernel<<<grid, 128, smem, st>>>(G, mask, dvals, L);
+    compact_kernel<<<grid, 128, smem, st>>>(G, mask, logw, mu, 1.f / sigma, L);
     return cudaGetLastError();
 }
 

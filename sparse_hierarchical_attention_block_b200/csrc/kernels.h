@@ -13,21 +13,23 @@ struct SelectOut {
     float *tau;        // [b][nq][hq] or null
     float *w;          // [b][nq][hkv][n_chunks] or null
     uint32_t *mask;    // [b][nq][hkv][words] (required)
-    float *dvals;      // [b][nq][hkv][n_chunks] bias of routed chunks (required when lists are built)
+    float *logw;       // [b][nq][hkv][n_chunks] log w of the routed chunks (when lists are built)
+    float *mu;         // [b][nq][hkv] mean log w over the routed chunks (when lists are built)
 };
 cudaError_t launch_select_rows(const TView &Q, dash_dtype_t dt, const float *kbar, const Geom &G, float alpha,
                                float gamma, float sigma, const SelectOut &o, cudaStream_t st);
 bool select_tile_supported(const Geom &G, dash_dtype_t dt);
 size_t select_tile_workspace(const Geom &G);
 cudaError_t launch_select_tile(const TView &Q, const float *kbar, const Geom &G, float alpha, float gamma,
-                               float sigma, float *tau, float *w, uint32_t *mask, float *dvals, const ListsView &L,
-                               void *work, cudaStream_t st);
+                               float sigma, float *tau, float *w, uint32_t *mask, float *logw, float *mu,
+                               const ListsView &L, void *work, cudaStream_t st);
 // Regroup the query rows of each window of tiles by routed-set size and build the
 // tiles' work lists (with the row permutation) from the per-row masks and biases.
-cudaError_t launch_regroup_compact(const Geom &G, const uint32_t *mask, const float *dvals, const ListsView &L,
-                                   cudaStream_t st);
-cudaError_t launch_compact(const Geom &G, const uint32_t *mask, const float *dvals, const ListsView &L,
-                           cudaStream_t st);
+bool regroup_supported(const Geom &G);
+cudaError_t launch_regroup_compact(const Geom &G, const uint32_t *mask, const float *logw, const float *mu,
+                                   float sigma, const ListsView &L, cudaStream_t st);
+cudaError_t launch_compact(const Geom &G, const uint32_t *mask, const float *logw, const float *mu, float sigma,
+                           const ListsView &L, cudaStream_t st);
 
 // Stage 2 (attn_simt.cu, attn_tc.cu, attn_decode.cu)
 cudaError_t launch_attn_simt(const TView &Q, const TView &K, const TView &V, const TView &O, dash_dtype_t dt,

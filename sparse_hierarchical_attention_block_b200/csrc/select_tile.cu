@@ -48,7 +48,8 @@ struct TileOut {
     float *tau;
     float *w;
     uint32_t *mask;   // [b][nq][hkv][words]; required when lists are not built here
-    float *dvals;     // [b][nq][hkv][n_chunks] bias of the routed chunks (regrouped lists)
+    float *logw;      // [b][nq][hkv][n_chunks] log w of the routed chunks (lists built later)
+    float *mu;        // [b][nq][hkv] mean log w over the routed chunks (lists built later)
 };
 
 // [t]_+^{1/(alpha-1)} and [t]_+^{1/(alpha-1) - 1}; KINT is the exponent when it is
@@ -255,14 +256,21 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
     const int nb = (__reduce_max_sync(0xffffffffu, (unsigned)nvis) + 31) / 32;
     const float xs = P.am1 * P.scale;  // x = (alpha - 1) * gamma / sqrt(d) * <q, k̄>
     int parity = 0;
+    // pass 0: x = (alpha-1) gamma/sqrt(d) <q, k̄> written back over the logits (later
+    // passes read x directly), and its maximum over the visible chunks
     float mx = -INFINITY;
     for (int blk = half; blk < nb; blk += 2) {
         uint32_t u[32];
         tmem_ld32(tmem + lane_off + blk * 32, u);
 #pragma unroll
-        for (int x = 0; x < 32; ++x)
-            if (blk * 32 + x < nvis) mx = fmaxf(mx, xs * __uint_as_float(u[x]));
+        for (int x = 0; x < 32; ++x) {
+            const float xv = xs * __uint_as_float(u[x]);
+            if (blk * 32 + x < nvis) mx = fmaxf(mx, xv);
+            u[x] = __float_as_uint(xv);
+        }
+        tmem_st32(tmem + lane_off + blk * 32, u);
     }
+    tmem_wait_st();
     {
         float v[1] = {mx};
         pair_exchange<1>(xch, parity, half, p, quad, v);
@@ -281,25 +289,52 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
         tmem_ld32(tmem + lane_off + blk * 32, u);
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
-            const float y = xs * __uint_as_float(u[x]) - lo;
+            const float y = __uint_as_float(u[x]) - lo;
             if (blk * 32 + x < nvis && y >= 0.f) hmine[min(31, (int)(y * 32.f)) * 128 + p] += 1;
         }
     }
     quad_sync(quad);
     float t0 = lo;
     if (nvis > 1) {
-        // estimated f at a bin edge (mass at the bin centres) decreases with the edge:
-        // binary search for the highest edge still estimated >= 0
-        int elo = 0, ehi = 31;
-        while (elo < ehi) {
-            const int e = (elo + ehi + 1) / 2;
-            const float edge = (float)e * (1.f / 32.f);
-            float fe = -1.f;
-            for (int j = e; j < 32; ++j)
-                fe += (float)(hist[j * 128 + p] + hist[32 * 128 + j * 128 + p]) *
-                      rpow<KINT>(((float)j + 0.5f) * (1.f / 32.f) - edge, P);
-            if (fe >= 0.f) elo = e;
-            else ehi = e - 1;
+        // estimated f at a bin edge e (every element at its bin centre c_j):
+        //   f~(e) = sum_{j >= bin(e)} n_j (c_j - e)^k - 1, decreasing in e;
+        // start from the highest edge still estimated >= 0.  For k = 1, 2, 4 the sum is
+        // expanded in suffix moments A_m = sum_{j >= bin} n_j c_j^m (one sweep from the top).
+        int elo = 0;
+        if (KINT == 1 || KINT == 2 || KINT == 4) {
+            float A0 = 0.f, A1 = 0.f, A2 = 0.f, A3 = 0.f, A4 = 0.f;
+            for (int e = 31; e >= 1; --e) {
+                const float n = (float)(hist[e * 128 + p] + hist[32 * 128 + e * 128 + p]);
+                const float c = ((float)e + 0.5f) * (1.f / 32.f), c2 = c * c;
+                A0 += n;
+                A1 += n * c;
+                A2 += n * c2;
+                if (KINT == 4) {
+                    A3 += n * c2 * c;
+                    A4 += n * c2 * c2;
+                }
+                const float x = (float)e * (1.f / 32.f);
+                float fe;
+                if (KINT == 1) fe = A1 - x * A0;
+                else if (KINT == 2) fe = A2 - 2.f * x * A1 + x * x * A0;
+                else fe = A4 - 4.f * x * A3 + 6.f * x * x * A2 - 4.f * x * x * x * A1 + x * x * x * x * A0;
+                if (fe - 1.f >= 0.f) {
+                    elo = e;
+                    break;
+                }
+            }
+        } else {
+            int ehi = 31;
+            while (elo < ehi) {
+                const int e = (elo + ehi + 1) / 2;
+                const float edge = (float)e * (1.f / 32.f);
+                float fe = -1.f;
+                for (int j = e; j < 32; ++j)
+                    fe += (float)(hist[j * 128 + p] + hist[32 * 128 + j * 128 + p]) *
+                          rpow<KINT>(((float)j + 0.5f) * (1.f / 32.f) - edge, P);
+                if (fe >= 0.f) elo = e;
+                else ehi = e - 1;
+            }
         }
         t0 = lo + (float)elo * (1.f / 32.f);
         if (!(t0 < hi)) t0 = lo;
@@ -310,21 +345,25 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
     int prev_cnt = -1;
     for (int it = 0; it < 40; ++it) {
         if (__all_sync(0xffffffffu, done)) break;
-        float acc[5] = {0.f, 0.f, 0.f, 0.f, 0.f};  // f + 1, -f'/k, s1, s2, count
+        // partial sums over the support {x > tau}: for alpha = 2 / 1.5 only the moments of
+        // y = x - mx (f follows from them), otherwise f + 1 and -f'/k as well
+        float acc[5] = {0.f, 0.f, 0.f, 0.f, 0.f};  // s1, s2, count, f + 1, -f'/k
         for (int blk = half; blk < nb; blk += 2) {
             uint32_t u[32];
             tmem_ld32(tmem + lane_off + blk * 32, u);
 #pragma unroll
             for (int x = 0; x < 32; ++x) {
-                const float xv = xs * __uint_as_float(u[x]);
+                const float xv = __uint_as_float(u[x]);
                 const float tt = xv - tau;
                 if (blk * 32 + x < nvis && tt > 0.f) {
-                    acc[0] += rpow<KINT>(tt, P);
-                    acc[1] += rpow_m1<KINT>(tt, P);
                     const float yv = xv - mx;
-                    acc[2] += yv;
-                    acc[3] += yv * yv;
-                    acc[4] += 1.f;
+                    acc[0] += yv;
+                    acc[1] = fmaf(yv, yv, acc[1]);
+                    acc[2] += 1.f;
+                    if (KINT != 1 && KINT != 2) {
+                        acc[3] += rpow<KINT>(tt, P);
+                        acc[4] += rpow_m1<KINT>(tt, P);
+                    }
                 }
             }
         }
@@ -337,8 +376,20 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
             for (int k = 0; k < 5; ++k) acc[k] = half == 0 ? acc[k] + v[k] : v[k] + acc[k];
         }
         if (done) continue;
-        const float f = acc[0] - 1.f, df = -P.kexp * acc[1], s1 = acc[2], s2 = acc[3];
-        const int cnt = (int)acc[4];
+        const float s1 = acc[0], s2 = acc[1];
+        const int cnt = (int)acc[2];
+        const float tr = tau - mx;  // tau in the y = x - mx frame
+        float f, df;
+        if (KINT == 1) {
+            f = s1 - tr * (float)cnt - 1.f;  // sum (y - tr) - 1
+            df = -(float)cnt;
+        } else if (KINT == 2) {
+            f = s2 - 2.f * tr * s1 + tr * tr * (float)cnt - 1.f;  // sum (y - tr)^2 - 1
+            df = -2.f * (s1 - tr * (float)cnt);
+        } else {
+            f = acc[3] - 1.f;
+            df = -P.kexp * acc[4];
+        }
         if (f >= 0.f) lo = tau;
         else hi = tau;
         float nt;
@@ -376,8 +427,12 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
     }
 
     // ---------------------------------------------------------------- group prior, pass 1: mu, union
-    // log w_c replaces x_c in this lane's TMEM row (-inf where the row does not route c),
-    // so pass 2 reads it back instead of recomputing it.
+    // When this kernel builds the tile's lists itself, log w_c replaces x_c in this lane's
+    // TMEM row (-inf where the row does not route c) and pass 2 writes the bias table once
+    // mu is known.  Otherwise (rows regrouped across tiles) pass 1 writes log w, the mask
+    // and mu, and the regroup kernel forms d = (log w - mu) / sigma.
+    const bool lists_mode = L.count != nullptr;
+    const size_t rowoff = ((size_t)b * G.nq + i) * G.hkv + r;
     const int gshift = (lane / g) * g;
     const uint32_t gmask = (g == 32) ? 0xffffffffu : ((1u << g) - 1u);
     const float log_g = logf((float)g);
@@ -389,7 +444,7 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
         uint32_t word = 0;
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
-            const float tt = xs * __uint_as_float(u[x]) - tau_r;
+            const float tt = __uint_as_float(u[x]) - tau_r;
             const bool own = (blk * 32 + x < nvis) && tt > 0.f;
             float v = own ? rpow<KINT>(tt, P) : 0.f;
             for (int o = 1; o < g; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -405,12 +460,17 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
                 word |= 1u << x;
             }
             u[x] = __float_as_uint(lw);
+            if (!lists_mode && lead && row_ok && blk * 32 + x < nvis) {
+                if (sel) out.logw[rowoff * G.n_chunks + blk * 32 + x] = lw;
+                if (out.w) out.w[rowoff * G.n_chunks + blk * 32 + x] = sel ? expf(lw) : 0.f;
+            }
         }
-        tmem_st32(tmem + lane_off + blk * 32, u);
+        if (lists_mode) tmem_st32(tmem + lane_off + blk * 32, u);
+        else if (lead && row_ok) out.mask[rowoff * G.words + blk] = word;
         const uint32_t wu = __reduce_or_sync(0xffffffffu, word);
         if (lane == 0 && wu) atomicOr(&uni[blk], wu);
     }
-    tmem_wait_st();
+    if (lists_mode) tmem_wait_st();
     {
         float v[2] = {lsum, lcnt};
         pair_exchange<2>(xch, parity, half, p, quad, v);
@@ -419,12 +479,15 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
         lcnt = half == 0 ? lcnt + v[1] : v[1] + lcnt;
     }
     const float mu = lcnt > 0.f ? lsum / lcnt : 0.f;
+    if (!lists_mode && lead && row_ok && half == 0) {
+        out.mu[rowoff] = mu;
+        for (int blk = nb; blk < G.words; ++blk) out.mask[rowoff * G.words + blk] = 0u;
+        if (out.w)
+            for (int c = nvis; c < G.n_chunks; ++c) out.w[rowoff * G.n_chunks + c] = 0.f;
+    }
     __syncthreads();
 
     // ---------------------------------------------------------------- the tile's list
-    // (when rows are regrouped across tiles, a later kernel builds the lists from the
-    // per-row masks and biases written in pass 2 instead)
-    const bool lists_mode = L.count != nullptr;
     int dlo = 0, dhi = -1;
     if (G.causal) {
         dlo = (int)(row_pos(G, t * T) / G.B);
@@ -469,10 +532,9 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
     }
     __syncthreads();
 
-    // ---------------------------------------------------------------- pass 2: bias, optional w / mask
+    // ---------------------------------------------------------------- pass 2 (lists mode): bias, optional w / mask
     const float inv_sigma = 1.f / P.sigma;
-    const size_t rowoff = ((size_t)b * G.nq + i) * G.hkv + r;
-    for (int blk = half; blk < nb; blk += 2) {
+    for (int blk = half; lists_mode && blk < nb; blk += 2) {
         uint32_t u[32];
         tmem_ld32(tmem + lane_off + blk * 32, u);
         uint32_t word = 0;
@@ -485,9 +547,7 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
             const bool sel = lw > -INFINITY;
             if (lead && row_ok && c < nvis) {
                 if (sel) word |= 1u << x;
-                if (!lists_mode) {
-                    if (sel && out.dvals) out.dvals[rowoff * G.n_chunks + c] = (lw - mu) * inv_sigma;
-                } else if ((uw >> x) & 1u) {
+                if ((uw >> x) & 1u) {
                     const int e = base + __popc(uw & ((1u << x) - 1u));
                     bias[(size_t)e * T + pos] = sel ? (lw - mu) * inv_sigma : -INFINITY;
                 } else if (c >= dlo && c <= dhi && sel) {
@@ -498,7 +558,7 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
         }
         if (out.mask && lead && row_ok && blk < G.words) out.mask[rowoff * G.words + blk] = word;
     }
-    if (lead && row_ok && half == 0) {
+    if (lists_mode && lead && row_ok && half == 0) {
         if (out.mask)
             for (int blk = nb; blk < G.words; ++blk) out.mask[rowoff * G.words + blk] = 0u;
         if (out.w)
@@ -532,8 +592,8 @@ size_t select_tile_workspace(const Geom &G) {
 }
 
 cudaError_t launch_select_tile(const TView &Q, const float *kbar, const Geom &G, float alpha, float gamma,
-                               float sigma, float *tau, float *w, uint32_t *mask, float *dvals, const ListsView &L,
-                               void *work, cudaStream_t st) {
+                               float sigma, float *tau, float *w, uint32_t *mask, float *logw, float *mu,
+                               const ListsView &L, void *work, cudaStream_t st) {
     if (G.nq == 0 || G.b == 0) return cudaSuccess;
     uint8_t *ksplit = static_cast<uint8_t *>(work);
     const int n_ct = (G.n_chunks + kChunkTile - 1) / kChunkTile;
@@ -557,7 +617,7 @@ cudaError_t launch_select_tile(const TView &Q, const float *kbar, const Geom &G,
     int ncols = 32;
     while (ncols < nc) ncols *= 2;
     P.ncols = ncols;
-    TileOut o{tau, w, mask, dvals};
+    TileOut o{tau, w, mask, logw, mu};
     dim3 grid((unsigned)L.n_tiles, (unsigned)G.hkv, (unsigned)G.b);
     cudaError_t e = cudaErrorNotSupported;
 #define DASH_SEL_CASE(DD, KK)                                                                              \
