@@ -176,6 +176,33 @@ DASH_API int dash_sync_status(void *stream);
 /* Free the library-managed workspace of the current device. */
 DASH_API int dash_release(void);
 
+/* Size of the static scratch area that dash_attn_fwd_noalloc works in (32 MiB,
+ * reserved on every device that loads the library, until the process exits). */
+#define DASH_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* dash_attn_fwd_ex for callers that cannot let the library allocate device
+ * memory: serving engines that hand nearly all of HBM to their own KV-cache
+ * pool (a run-time cudaMalloc may fail there), multi-stream loops that cannot
+ * take the device-wide synchronisation of cudaFree, hosts that route all device
+ * memory through their own allocator.  It calls no cudaMalloc, cudaFree or other
+ * allocating routine; the intermediates go to a static device array of
+ * DASH_NOALLOC_SCRATCH_BYTES inside the library.  The paper has no counterpart
+ * to this entry point: it is a deployment variant of dash_attn_fwd_ex.
+ *   Arguments and result as dash_attn_fwd_ex; opts may be NULL, and
+ *   opts->workspace must be NULL (DASH_ERR_INVALID_ARG otherwise).
+ *   A problem whose dash_workspace_bytes() exceeds DASH_NOALLOC_SCRATCH_BYTES is
+ *   rejected with DASH_ERR_WORKSPACE before anything is launched.
+ *   The first call on a device (with that device current) looks up the array's
+ *   device address with cudaGetSymbolAddress; make that first call before any
+ *   stream capture.
+ *   All calls share the one array, which keeps the last call's contents (the
+ *   forward pass writes every scratch word before reading it).  Calls whose
+ *   execution overlaps on the GPU (different streams or host threads) race on
+ *   it: serialise them. */
+DASH_API int dash_attn_fwd_noalloc(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v,
+                                   dash_tensor_t *out, int block_size, float alpha, int causal, int gqa_groups,
+                                   const dash_opts_t *opts);
+
 /* Library version string. */
 DASH_API const char *dash_version(void);
 

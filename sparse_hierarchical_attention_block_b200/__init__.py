@@ -68,7 +68,10 @@ _lib = None
 # every entry point include/dash_attn.h declares
 EXPORTS = ("dash_opts_init", "dash_attn_fwd", "dash_attn_fwd_ex", "dash_pool_keys", "dash_block_select",
            "dash_sparse_attn_fwd", "dash_lists_geometry", "dash_workspace_bytes", "dash_last_error",
-           "dash_sync_status", "dash_release", "dash_version")
+           "dash_sync_status", "dash_release", "dash_version", "dash_attn_fwd_noalloc")
+
+# size of the library's static scratch area used by dash_attn_fwd_noalloc
+DASH_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 def load_library():
@@ -85,6 +88,7 @@ def load_library():
     lib.dash_opts_init.argtypes = [ctypes.POINTER(_Opts)]
     lib.dash_attn_fwd.argtypes = [T, T, T, T, i32, f32, i32, i32]
     lib.dash_attn_fwd_ex.argtypes = [T, T, T, T, i32, f32, i32, i32, ctypes.POINTER(_Opts)]
+    lib.dash_attn_fwd_noalloc.argtypes = [T, T, T, T, i32, f32, i32, i32, ctypes.POINTER(_Opts)]
     lib.dash_pool_keys.argtypes = [T, i32, i32, P, P]
     lib.dash_block_select.argtypes = [T, T, i32, f32, i32, i32, P, P, P, ctypes.POINTER(_Lists),
                                       ctypes.POINTER(_Opts)]
@@ -203,6 +207,21 @@ def dash_attn_fwd(q, k, v, out, block_size, alpha, causal=True, gqa_groups=None,
     else:
         _check(lib.dash_attn_fwd(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.byref(od),
                                  int(block_size), float(alpha), int(bool(causal)), int(g)))
+    return out
+
+
+def dash_attn_fwd_noalloc(q, k, v, out, block_size, alpha, causal=True, gqa_groups=None, **opts):
+    """Full forward into ``out`` without any device allocation by the library:
+    the intermediates go to its static scratch area of DASH_NOALLOC_SCRATCH_BYTES
+    (problems that need more raise DashError with DASH_ERR_WORKSPACE).  Calls
+    share that area: do not let two of them run concurrently on the GPU.
+    ``opts`` as for dash_attn_fwd, except ``workspace``."""
+    lib = load_library()
+    g = gqa_groups if gqa_groups is not None else q.shape[2] // k.shape[2]
+    qd, kd, vd, od = _desc(q), _desc(k), _desc(v), _desc(out)
+    o = _opts(**opts)
+    _check(lib.dash_attn_fwd_noalloc(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.byref(od),
+                                     int(block_size), float(alpha), int(bool(causal)), int(g), ctypes.byref(o)))
     return out
 
 

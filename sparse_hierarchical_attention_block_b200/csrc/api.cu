@@ -262,6 +262,12 @@ int validate_qkvo(const dash_tensor_t *q, const dash_tensor_t *k, const dash_ten
 
 }  // namespace
 
+namespace dash {
+// Records msg as this thread's last error (dash_last_error) and returns code;
+// for entry points defined in other translation units.
+int report_error(int code, const char *msg) { return fail(code, "%s", msg); }
+}  // namespace dash
+
 extern "C" {
 
 DASH_API const char *dash_version(void) { return "dash-attn-b200 0.1 (sm_100a)"; }

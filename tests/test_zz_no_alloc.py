@@ -1,0 +1,118 @@
+"""dash_attn_fwd_noalloc: the forward pass on the library's static scratch area.
+
+Host-side checks (no GPU): the entry point is exported, rejects a problem
+larger than its scratch area with DASH_ERR_WORKSPACE and refuses a caller
+workspace, before any CUDA call.  GPU check: consecutive calls through the C
+ABI (a prefill and a split-KV decode problem, alternating, so each call finds
+the other's leftovers in the shared area) agree with dash_attn_fwd within the
+tolerance of the parity tests, and the calls after the first change the
+device's free memory by nothing.
+
+Kept in a file of its own, collected last, so it runs both alone in a fresh
+process and after every other test."""
+import ctypes
+
+import pytest
+import torch
+
+import sparse_hierarchical_attention_block_b200 as dash
+import synthetic
+from sparse_hierarchical_attention_block_b200 import _Opts, _Tensor, build
+
+MAX_ABS, MEAN_ABS = 2e-2, 2e-3  # the bf16 output tolerance of the parity tests
+FAKE = 1 << 20  # never dereferenced: the checks fail first
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return dash.load_library()
+
+
+def _t(dtype, shape):
+    t = _Tensor()
+    t.data = FAKE
+    t.dtype = dtype
+    stride = [shape[1] * shape[2] * shape[3], shape[2] * shape[3], shape[3], 1]
+    for a in range(4):
+        t.shape[a] = shape[a]
+        t.stride[a] = stride[a]
+    return t
+
+
+def test_noalloc_exported(lib):
+    assert hasattr(lib, "dash_attn_fwd_noalloc")
+    assert "dash_attn_fwd_noalloc" in dash.EXPORTS
+
+
+def test_noalloc_rejects_oversize(lib):
+    # 8K-token prefill with 32 heads needs ~68 MiB of scratch, above the 32 MiB area
+    q = _t(dash.DASH_BF16, [1, 8192, 32, 128])
+    k = _t(dash.DASH_BF16, [1, 8192, 8, 128])
+    need = dash.dash_workspace_bytes(1, 8192, 8192, 32, 8, 128, 64, True)
+    assert need > dash.DASH_NOALLOC_SCRATCH_BYTES
+    rc = lib.dash_attn_fwd_noalloc(ctypes.byref(q), ctypes.byref(k), ctypes.byref(k), ctypes.byref(q), 64, 1.5, 1,
+                                   4, None)
+    assert rc == dash.DASH_ERR_WORKSPACE
+    msg = lib.dash_last_error().decode()
+    assert str(need) in msg and str(dash.DASH_NOALLOC_SCRATCH_BYTES) in msg
+
+
+def test_noalloc_rejects_caller_workspace(lib):
+    q = _t(dash.DASH_BF16, [1, 256, 8, 128])
+    k = _t(dash.DASH_BF16, [1, 256, 2, 128])
+    o = _Opts()
+    lib.dash_opts_init(ctypes.byref(o))
+    o.workspace = FAKE
+    o.workspace_bytes = 1 << 20
+    rc = lib.dash_attn_fwd_noalloc(ctypes.byref(q), ctypes.byref(k), ctypes.byref(k), ctypes.byref(q), 64, 1.5, 1,
+                                   4, ctypes.byref(o))
+    assert rc == dash.DASH_ERR_INVALID_ARG
+    assert "workspace" in lib.dash_last_error().decode()
+
+
+# b, nq, nk, hq, hkv, d, B, alpha, causal, sigma
+PROBLEMS = [
+    (1, 1000, 1000, 8, 2, 128, 64, 1.5, True, 1.0),  # prefill, ragged tail, regrouped tiles
+    (2, 1, 3000, 8, 2, 128, 64, 1.5, True, 1e8),  # decode, split-KV partials in the scratch
+]
+
+
+def _inputs(p, seed):
+    b, nq, nk, hq, hkv, d, B, alpha, causal, _ = p
+    w = synthetic.Workload("noalloc", b, nq, nk, hq, hkv, d, B, alpha, causal, "bf16", seed, True, amax_key="b64")
+    return synthetic.make_inputs(w, "cuda")
+
+
+@pytest.mark.gpu
+def test_noalloc_matches_fwd_on_consecutive_calls(lib):
+    if not torch.cuda.is_available():
+        pytest.fail("the gpu tests need a CUDA device")
+    data = []
+    for i, p in enumerate(PROBLEMS):
+        b, nq, nk, hq, hkv, d, B, alpha, causal, sigma = p
+        assert dash.dash_workspace_bytes(b, nq, nk, hq, hkv, d, B, causal) <= dash.DASH_NOALLOC_SCRATCH_BYTES
+        q, k, v = _inputs(p, 40 + i)
+        ref = torch.empty_like(q)
+        dash.dash_attn_fwd(q, k, v, ref, B, alpha, causal, hq // hkv, sigma=sigma)
+        assert dash.dash_sync_status() == 0
+        data.append((p, q, k, v, ref))
+    order = [0, 1, 0, 1]  # each call after the first finds another problem's contents in the scratch
+    outs = [torch.full_like(data[j][1], float("nan")) for j in order]
+    torch.cuda.synchronize()
+    free = []
+    for j, out in zip(order, outs):  # no torch allocation between the calls
+        p, q, k, v, ref = data[j]
+        b, nq, nk, hq, hkv, d, B, alpha, causal, sigma = p
+        dash.dash_attn_fwd_noalloc(q, k, v, out, B, alpha, causal, hq // hkv, sigma=sigma)
+        assert dash.dash_sync_status() == 0, dash.load_library().dash_last_error()
+        free.append(torch.cuda.mem_get_info()[0])
+    # the first call may load the library's device module (which holds the area);
+    # the calls after it allocate nothing
+    assert free[1:] == free[:1] * (len(free) - 1), free
+    for n, (j, out) in enumerate(zip(order, outs)):
+        ref = data[j][4]
+        err = (out.float() - ref.float()).abs()
+        print(f"[noalloc] call {n} problem {j}: max_abs={err.max().item():.3g} mean_abs={err.mean().item():.3g}")
+        assert torch.isfinite(out.float()).all()
+        assert err.max().item() <= MAX_ABS and err.mean().item() <= MEAN_ABS
