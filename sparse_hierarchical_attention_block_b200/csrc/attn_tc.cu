@@ -18,9 +18,10 @@
 //              O  += P_j V_j  (TS: P read from TMEM, V from smem as an MN-major operand);
 //   warps 2-5  softmax: thread = TMEM lane = tile row; two passes over S_j in TMEM
 //              (row max, then exp2 / sum / bf16 P written over S_j), bias added and
-//              keys masked only on steps that hold a diagonal or partial chunk; O is
-//              rescaled only when the running max grows by more than 2^8; epilogue
-//              O / l -> bf16.
+//              keys masked only on steps that hold a diagonal or partial chunk; after
+//              the first step a single pass on the running maximum, redone as two
+//              passes only if a row's maximum grows by more than 2^16 (O is then
+//              rescaled); epilogue O / l -> bf16.
 // Every mbarrier wait is bounded (globaltimer); on expiry the kernel records a
 // device error, drains what it issued, frees TMEM and returns.
 #include <math.h>
@@ -39,6 +40,9 @@ constexpr int kStepKeys = 128;  // keys per step = MMA N of S and K of PV
 constexpr int kNS = 1;          // K / V stages (two CTAs per SM share the SM's shared memory)
 constexpr int kNM = 2;          // bias / id stages
 constexpr uint32_t kTmemCols = 256;
+// The running maximum (exp2 domain) is kept until a step's maximum exceeds it by more
+// than this: p <= 2^16, so P (bf16), l and O (fp32) stay far from overflow.
+constexpr float kRescaleL2 = 16.f;
 constexpr uint64_t kWaitNs = 2000000000ull;      // 2 s
 constexpr uint64_t kWaitNsTest = 20000000ull;    // 20 ms under DASH_FLAG_TEST_TIMEOUT
 
@@ -318,29 +322,65 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
             ok = __all_sync(0xffffffffu, wait_bar(B.s_full, j & 1, limit_ns, abort));
             if (!ok) break;
             tc_fence_after();
-            // pass 1: row maximum of the biased, masked logits (exp2 domain)
-            float mx = -INFINITY;
+            // Single pass on the running maximum of the earlier steps: p = 2^(s * scale +
+            // bias - m_run) straight from S.  It stands unless a row of the warp finds a
+            // logit above m_run + kRescaleL2 (then P is discarded, S is still intact, and
+            // the two-pass path below redoes the step with a new maximum).  P is held in
+            // registers and written over S only once the step is known to stand.
+            bool step_done = false;
+            if (j > 0 && __all_sync(0xffffffffu, !row_ok || m_run > -INFINITY)) {
+                float cbm[S::kE];
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t u[64];
-                tmem_ld32(tS + lane_off + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
-                tmem_ld32(tS + lane_off + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
-                if (!need_mask) {
+                for (int e = 0; e < S::kE; ++e) cbm[e] = row_ok ? bl2[e] - m_run : -INFINITY;
+                uint32_t pk[64];
+                float mr[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int x = 0; x < 64; ++x) mx = fmaxf(mx, fmaf(__uint_as_float(u[x]), sl2, bl2[(half * 64 + x) / BLK]));
-                } else {
+                for (int qc = 0; qc < 4; ++qc) {
+                    uint32_t u[32];
+                    tmem_ld32(tS + lane_off + qc * 32, u);
 #pragma unroll
-                    for (int x = 0; x < 64; ++x) {
-                        const int kc = half * 64 + x;
-                        const float v = fmaf(__uint_as_float(u[x]), sl2, bl2[kc / BLK]);
-                        mx = fmaxf(mx, (kc % BLK) < lim[kc / BLK] ? v : -INFINITY);
+                    for (int x = 0; x < 16; ++x) {
+                        const int kc = qc * 32 + 2 * x;
+                        float v0 = fmaf(__uint_as_float(u[2 * x]), sl2, cbm[kc / BLK]);
+                        float v1 = fmaf(__uint_as_float(u[2 * x + 1]), sl2, cbm[(kc + 1) / BLK]);
+                        if (need_mask) {  // select before exp2: S outside the list may be any bit pattern
+                            v0 = (kc % BLK) < lim[kc / BLK] ? v0 : -INFINITY;
+                            v1 = ((kc + 1) % BLK) < lim[(kc + 1) / BLK] ? v1 : -INFINITY;
+                        }
+                        mr[x & 3] = fmaxf(mr[x & 3], fmaxf(v0, v1));
+                        const float p0 = ex2(v0), p1 = ex2(v1);
+                        ps[x & 3] += p0 + p1;
+                        pk[qc * 16 + x] = pack_bf16x2(p0, p1);
                     }
                 }
+                const float mrel = fmaxf(fmaxf(mr[0], mr[1]), fmaxf(mr[2], mr[3]));
+                if (!__any_sync(0xffffffffu, mrel > kRescaleL2)) {
+                    tmem_st32(tS + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+                    tmem_st32(tS + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+                    l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+                    step_done = true;
+                }
             }
+            if (!step_done) {
+            // pass 1: row maximum of the biased, masked logits (exp2 domain)
+            float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int qc = 0; qc < 4; ++qc) {
+                uint32_t u[32];
+                tmem_ld32(tS + lane_off + qc * 32, u);
+#pragma unroll
+                for (int x = 0; x < 32; ++x) {
+                    const int kc = qc * 32 + x;
+                    const float v = fmaf(__uint_as_float(u[x]), sl2, bl2[kc / BLK]);
+                    mq[x & 3] = fmaxf(mq[x & 3], (!need_mask || (kc % BLK) < lim[kc / BLK]) ? v : -INFINITY);
+                }
+            }
+            float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
             if (!row_ok) mx = -INFINITY;
             // running maximum: kept unless the step's maximum exceeds it by more than 2^8
             float f = 1.f;
-            const bool rescale = mx > -INFINITY && m_run > -INFINITY && mx > m_run + 8.f;
+            const bool rescale = mx > -INFINITY && m_run > -INFINITY && mx > m_run + kRescaleL2;
             if (mx > -INFINITY) {
                 if (m_run == -INFINITY) {
                     m_run = mx;  // nothing accumulated for this row yet: O holds zeros
@@ -370,38 +410,31 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
             float cbm[S::kE];
 #pragma unroll
             for (int e = 0; e < S::kE; ++e) cbm[e] = live ? bl2[e] - m_run : -INFINITY;
-            float psum = 0.f;
+            float pq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t u[64];
-                tmem_ld32(tS + lane_off + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
-                tmem_ld32(tS + lane_off + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
-                uint32_t pk[32];
-                if (!need_mask) {
+            for (int qc = 0; qc < 4; ++qc) {
+                uint32_t u[32];
+                tmem_ld32(tS + lane_off + qc * 32, u);
+                uint32_t pk[16];
 #pragma unroll
-                    for (int x = 0; x < 32; ++x) {
-                        const int kc = half * 64 + 2 * x;
-                        const float p0 = ex2(fmaf(__uint_as_float(u[2 * x]), sl2, cbm[kc / BLK]));
-                        const float p1 = ex2(fmaf(__uint_as_float(u[2 * x + 1]), sl2, cbm[(kc + 1) / BLK]));
-                        psum += p0 + p1;
-                        pk[x] = pack_bf16x2(p0, p1);
+                for (int x = 0; x < 16; ++x) {
+                    const int kc = qc * 32 + 2 * x;
+                    float v0 = fmaf(__uint_as_float(u[2 * x]), sl2, cbm[kc / BLK]);
+                    float v1 = fmaf(__uint_as_float(u[2 * x + 1]), sl2, cbm[(kc + 1) / BLK]);
+                    if (need_mask) {  // select before exp2: S outside the list may be any bit pattern
+                        v0 = (kc % BLK) < lim[kc / BLK] ? v0 : -INFINITY;
+                        v1 = ((kc + 1) % BLK) < lim[(kc + 1) / BLK] ? v1 : -INFINITY;
                     }
-                } else {
-#pragma unroll
-                    for (int x = 0; x < 32; ++x) {
-                        const int kc = half * 64 + 2 * x;
-                        // select after exp2: S of a key outside the list may be any bit pattern
-                        const float e0 = ex2(fmaf(__uint_as_float(u[2 * x]), sl2, cbm[kc / BLK]));
-                        const float e1 = ex2(fmaf(__uint_as_float(u[2 * x + 1]), sl2, cbm[(kc + 1) / BLK]));
-                        const float p0 = (kc % BLK) < lim[kc / BLK] ? e0 : 0.f;
-                        const float p1 = ((kc + 1) % BLK) < lim[(kc + 1) / BLK] ? e1 : 0.f;
-                        psum += p0 + p1;
-                        pk[x] = pack_bf16x2(p0, p1);
-                    }
+                    const float p0 = ex2(v0), p1 = ex2(v1);
+                    pq[x & 3] += p0 + p1;
+                    pk[x] = pack_bf16x2(p0, p1);
                 }
-                tmem_st32(tS + lane_off + half * 32, pk);
+                // P of keys 32qc.. over columns 16qc..: S columns below 32(qc+1) are already read
+                tmem_st16(tS + lane_off + qc * 16, pk);
             }
+            const float psum = (pq[0] + pq[1]) + (pq[2] + pq[3]);
             l_run += psum;
+            }  // two-pass path
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(B.p_full);
