@@ -8,7 +8,7 @@
 // causal.  Online softmax in the exp2 domain with fp32 statistics.
 //
 // One CTA per (batch, kv head, query tile of 128/g positions x g heads = 128 rows),
-// the heaviest tiles (latest, causal) first, two CTAs resident per SM so that one
+// the heaviest tiles (latest, causal) of all heads first, two CTAs resident per SM so that one
 // CTA's MMAs overlap the other's softmax.  Warp roles (192 threads):
 //   warp 0     TMA producer: Q tile once; per step of 128 keys the listed K and V
 //              blocks (one TMA box per chunk and 64-column half, 128-byte swizzle)
@@ -43,6 +43,7 @@ constexpr uint32_t kTmemCols = 256;
 // The running maximum (exp2 domain) is kept until a step's maximum exceeds it by more
 // than this: p <= 2^16, so P (bf16), l and O (fp32) stay far from overflow.
 constexpr float kRescaleL2 = 16.f;
+constexpr float kRescaleP = 65536.f;  // 2^kRescaleL2
 constexpr uint64_t kWaitNs = 2000000000ull;      // 2 s
 constexpr uint64_t kWaitNsTest = 20000000ull;    // 20 ms under DASH_FLAG_TEST_TIMEOUT
 
@@ -113,12 +114,21 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
     uint8_t *sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int64_t t = (int64_t)L.n_tiles - 1 - blockIdx.x;  // heaviest (latest) tiles first
-    const int r = blockIdx.y;
-    const int64_t b = blockIdx.z;
+    // one CTA per (tile, batch, kv head), launched heaviest (latest, causal) tiles first
+    // across all heads, so that the long tiles do not gather at the end of the grid
+    const int64_t bh = G.b * G.hkv;
+    const int64_t t = (int64_t)L.n_tiles - 1 - (int64_t)blockIdx.x / bh;
+    const int r = (int)(((int64_t)blockIdx.x % bh) % G.hkv);
+    const int64_t b = ((int64_t)blockIdx.x % bh) / G.hkv;
     const int g = G.g, T = L.tile_rows;
     const size_t tile_idx = ((size_t)b * G.hkv + r) * L.n_tiles + t;
     const int count = L.count[tile_idx];
+    // the first step's chunk ids, requested before the set-up below (the first K copy waits on them)
+    int ids_pre[Smem<D, BLK>::kE];
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int e = 0; e < Smem<D, BLK>::kE; ++e) ids_pre[e] = e < L.cap ? L.ids[tile_idx * L.cap + e] : 0;
+    }
     const int nsteps = (count + S::kE - 1) / S::kE;
     const bool test_timeout = (flags & DASH_FLAG_TEST_TIMEOUT) != 0;
     const uint64_t limit_ns = test_timeout ? kWaitNsTest : kWaitNs;
@@ -194,7 +204,13 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
                 const int ms = j % kNM, ks = j % kNS;
                 if (!wait_bar(B.m_empty + ms, ((j / kNM) & 1) ^ 1, limit_ns, abort)) break;
                 int *ids_st = ids_s + ms * S::kE;
-                for (int e = 0; e < ne; ++e) ids_st[e] = ids_g[e0 + e];
+                if (j == 0) {
+#pragma unroll
+                    for (int e = 0; e < S::kE; ++e)
+                        if (e < ne) ids_st[e] = ids_pre[e];
+                } else {
+                    for (int e = 0; e < ne; ++e) ids_st[e] = ids_g[e0 + e];
+                }
                 mbar_arrive_expect_tx(B.m_full + ms, (uint32_t)(ne * T * 4));
                 bulk_load(bias_s + ms * S::kE * 128, bias_g + (size_t)e0 * T, (uint32_t)(ne * T * 4), B.m_full + ms);
                 issued_m = j + 1;
@@ -333,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
 #pragma unroll
                 for (int e = 0; e < S::kE; ++e) cbm[e] = row_ok ? bl2[e] - m_run : -INFINITY;
                 uint32_t pk[64];
-                float mr[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                float mr[4] = {0.f, 0.f, 0.f, 0.f};
                 float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int qc = 0; qc < 4; ++qc) {
@@ -348,14 +364,15 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
                             v0 = (kc % BLK) < lim[kc / BLK] ? v0 : -INFINITY;
                             v1 = ((kc + 1) % BLK) < lim[(kc + 1) / BLK] ? v1 : -INFINITY;
                         }
-                        mr[x & 3] = fmaxf(mr[x & 3], fmaxf(v0, v1));
                         const float p0 = ex2(v0), p1 = ex2(v1);
+                        mr[x & 3] = fmaxf(mr[x & 3], fmaxf(p0, p1));
                         ps[x & 3] += p0 + p1;
                         pk[qc * 16 + x] = pack_bf16x2(p0, p1);
                     }
                 }
-                const float mrel = fmaxf(fmaxf(mr[0], mr[1]), fmaxf(mr[2], mr[3]));
-                if (!__any_sync(0xffffffffu, mrel > kRescaleL2)) {
+                // largest p of the row (2^(logit - m_run)); inf if it overflowed
+                const float pmax = fmaxf(fmaxf(mr[0], mr[1]), fmaxf(mr[2], mr[3]));
+                if (!__any_sync(0xffffffffu, pmax > kRescaleP)) {
                     tmem_st32(tS + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
                     tmem_st32(tS + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
                     l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
@@ -490,8 +507,9 @@ cudaError_t launch_t(const TcParams &tp, const TView &Q, const TView &O, const G
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)L.n_tiles, (unsigned)G.hkv, (unsigned)G.b);
-    attn_tc_kernel<D, BLK><<<grid, kThreads, smem, st>>>(tp, Q, O, G, L, flags);
+    const int64_t ctas = L.n_tiles * G.hkv * G.b;
+    if (ctas > 0x7fffffff) return cudaErrorInvalidValue;
+    attn_tc_kernel<D, BLK><<<(unsigned)ctas, kThreads, smem, st>>>(tp, Q, O, G, L, flags);
     return cudaGetLastError();
 }
 
