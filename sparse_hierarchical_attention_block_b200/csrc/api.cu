@@ -206,15 +206,9 @@ int run_stage1(const dash_tensor_t *q, const Geom &G, float alpha, const dash_op
     uint32_t *mask = mask_out ? mask_out : reinterpret_cast<uint32_t *>(ws + WL.mask);
     float *logw = reinterpret_cast<float *>(ws + WL.logw);
     float *mu = reinterpret_cast<float *>(ws + WL.mu);
-    if (tile && LV && !regroup) {
-        e = launch_select_tile(view(q), kbar, G, alpha, o.gamma, o.sigma, tau, w, mask_out, nullptr, nullptr, *LV,
-                               ws + WL.split, st);
-        return e == cudaSuccess ? DASH_OK : cuda_fail(e, "select_tile");
-    }
     if (tile) {
-        const ListsView geom_only{nullptr, nullptr, nullptr, nullptr, G.n_tiles, G.n_blk, G.tile_rows};
-        e = launch_select_tile(view(q), kbar, G, alpha, o.gamma, o.sigma, tau, w, mask, logw, mu, geom_only,
-                               ws + WL.split, st);
+        e = launch_select_tile(view(q), kbar, G, alpha, o.gamma, tau, w, mask, LV ? logw : nullptr,
+                               LV ? mu : nullptr, ws + WL.split, st);
         if (e != cudaSuccess) return cuda_fail(e, "select_tile");
     } else {
         SelectOut so{tau, w, mask, LV ? logw : nullptr, LV ? mu : nullptr};

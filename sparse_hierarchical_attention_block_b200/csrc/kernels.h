@@ -20,9 +20,12 @@ cudaError_t launch_select_rows(const TView &Q, dash_dtype_t dt, const float *kba
                                float gamma, float sigma, const SelectOut &o, cudaStream_t st);
 bool select_tile_supported(const Geom &G, dash_dtype_t dt);
 size_t select_tile_workspace(const Geom &G);
+// Routing of every (row, head) pair on tensor cores (up to 2048 chunks): tau, optional
+// dense w, the bit mask (required), log w of the routed chunks and mu (optional; both
+// are needed to build work lists).  `work` holds select_tile_workspace(G) bytes.
 cudaError_t launch_select_tile(const TView &Q, const float *kbar, const Geom &G, float alpha, float gamma,
-                               float sigma, float *tau, float *w, uint32_t *mask, float *logw, float *mu,
-                               const ListsView &L, void *work, cudaStream_t st);
+                               float *tau, float *w, uint32_t *mask, float *logw, float *mu, void *work,
+                               cudaStream_t st);
 // Regroup the query rows of each window of tiles by routed-set size and build the
 // tiles' work lists (with the row permutation) from the per-row masks and biases.
 bool regroup_supported(const Geom &G);

@@ -1,24 +1,30 @@
-// select_tile.cu -- Stage 1 fused on tensor cores: routing + work-list compaction for
-// one Stage-2 query tile per CTA (bf16 inputs, up to 512 routing chunks).
+// select_tile.cu -- Stage 1 on tensor cores: entmax routing of the (query row, head)
+// pairs of a block of query rows per CTA (bf16 inputs, up to 2048 routing chunks).
 //
-// For the 128 (query row, head) pairs of one (batch, kv head, query tile)
-// ("DashAttention" §3.2 Eq. 4, App. G Alg. 2):
+// For the pairs of one (batch, kv head, block of query rows) ("DashAttention" §3.2
+// Eq. 4, App. G Alg. 2):
 //   logits   X = gamma/sqrt(d) * Q K̄^T on tcgen05 into tensor memory: Q is bf16,
 //            the fp32 chunk summaries are split k̄ = hi + lo into two bf16 operands
 //            and both products accumulate in fp32 (relative error ~2^-17, i.e.
-//            fp32-class logits); one TMEM lane per pair, one column per chunk;
-//   tau      one thread per pair walks its TMEM row: max, a 32-bin shared-memory
-//            histogram over [max x - 1, max x) for the starting point (AdaSplash-2's
-//            initialisation), then a bracketed iteration: for alpha = 2 and 1.5 the
-//            exact closed form on the current support (support shrinks until it is
-//            stable), otherwise Newton, bisection as the safeguard;
+//            fp32-class logits).  TMEM holds 128 lanes x 512 fp32 columns; with LG
+//            lane groups a CTA routes 128/LG pairs over up to 512*LG chunks: lane
+//            group lg holds chunk tiles lg, lg + LG, ... of its pairs.  The logits
+//            MMA of a tile of lane group lg reads Q through a zero-padded A operand
+//            whose only non-zero rows are that group's lanes, so accumulating the
+//            LG groups' products into one column block writes each group's lanes
+//            and adds zero to the others;
+//   tau      4*LG threads per pair walk its TMEM row in 32-column blocks: max, a
+//            32-bin shared-memory histogram over [max x - 1, max x) for the
+//            starting point (AdaSplash-2's initialisation), then a bracketed
+//            iteration: for alpha = 2 and 1.5 the exact closed form on the current
+//            support (until the support is stable), otherwise Newton, with
+//            bisection as the safeguard; partial sums are combined in a fixed order
+//            so every thread of a pair takes the same decisions;
 //   prior    the g heads of a query row sit in g adjacent lanes of one warp:
-//            w_c = (1/g) sum_h [x_c - tau_h]_+^{1/(alpha-1)} by shuffles, membership by
-//            comparison (ballot), mu = mean log w over the routed chunks,
-//            d_c = (log w_c - mu) / sigma (§3.4 Prop. 1);
-//   lists    union of the tile's routed chunks (warp OR + shared atomics), the
-//            diagonal chunks first, then the routed chunks ascending, and the
-//            per-row bias table, written straight into the Stage-2 work lists.
+//            w_c = (1/g) sum_h [x_c - tau_h]_+^{1/(alpha-1)} by shuffles, membership
+//            by comparison (ballot), mu = mean log w over the routed chunks
+//            (§3.4 Prop. 1); outputs the bit mask, log w of the routed chunks and mu
+//            per row, from which the work lists are built (d = (log w - mu)/sigma).
 #include <math.h>
 
 #include "dash_common.cuh"
@@ -29,27 +35,27 @@ namespace dash {
 
 namespace {
 
-constexpr int kTileThreads = 256;  // two threads per (row, head) pair
-constexpr int kChunkTile = 128;  // chunks per logits MMA (N)
-constexpr int kMaxTileChunks = 512;
+constexpr int kSelT = 512;         // 16 warps: 4 TMEM lane quadrants x 4 column parts
+constexpr int kChunkTile = 128;    // chunks per logits MMA (N)
+constexpr int kTmemCols = 512;
+constexpr int kMaxTileChunks = 512 * 4;
+constexpr int kBins = 32;
+constexpr int kXchVals = 5;
 constexpr uint64_t kTileWaitNs = 2000000000ull;
 
 struct TileP {
     float am1;    // alpha - 1
     float kexp;   // 1 / (alpha - 1)
-    int kint;     // 1/(alpha-1) when it is 1, 2 or 4, else 0
     float alpha;
     float scale;  // gamma / sqrt(d)
-    float sigma;
-    int ncols;    // allocated TMEM columns
 };
 
 struct TileOut {
-    float *tau;
-    float *w;
-    uint32_t *mask;   // [b][nq][hkv][words]; required when lists are not built here
-    float *logw;      // [b][nq][hkv][n_chunks] log w of the routed chunks (lists built later)
-    float *mu;        // [b][nq][hkv] mean log w over the routed chunks (lists built later)
+    float *tau;       // [b][nq][hq] or null
+    float *w;         // [b][nq][hkv][n_chunks] or null
+    uint32_t *mask;   // [b][nq][hkv][words] (required)
+    float *logw;      // [b][nq][hkv][n_chunks] log w of the routed chunks, or null
+    float *mu;        // [b][nq][hkv] mean log w over the routed chunks, or null
 };
 
 // [t]_+^{1/(alpha-1)} and [t]_+^{1/(alpha-1) - 1}; KINT is the exponent when it is
@@ -71,24 +77,26 @@ __device__ __forceinline__ float rpow_m1(float t, const TileP &P) {
     return powf(t, P.kexp - 1.f);
 }
 
-template <int D>
+template <int D, int LG>
 struct TSmem {
-    static constexpr int kRegion = 128 * 128;              // 128 rows x 128 bytes
+    static constexpr int kNP = 128 / LG;              // pairs per CTA
     static constexpr int kDh = D / 64;
-    // MMA phase: Q tile and one chunk tile of k̄ hi / lo operands
-    static constexpr int kQ = 0;
-    static constexpr int kHi = kQ + kDh * kRegion;
-    static constexpr int kLo = kHi + kDh * kRegion;
-    static constexpr int kMmaEnd = kLo + kDh * kRegion;
-    // solve phase (reuses the MMA region once the logits are in TMEM)
-    static constexpr int kHist = 0;                          // [2 halves][32 bins][128 pairs] uint16
-    static constexpr int kXch = kHist + 2 * 32 * 128 * 2;     // [2 parity][2 halves][128 pairs][8] float
-    static constexpr int kSolveEnd = kXch + 2 * 2 * 128 * 8 * 4;
+    // A operand: rows [0, 128-NP) zero, [128-NP, 128) the Q pairs, [128, 256-NP) zero;
+    // the MMA of lane group lg starts at row 128 - NP - lg*NP
+    static constexpr int kArows = 256 - kNP;
+    static constexpr int kAregion = kArows * 128;     // one 64-column region
+    static constexpr int kBregion = 128 * 128;
+    static constexpr int kA = 0;
+    static constexpr int kB = kA + kDh * kAregion;    // [stage][hi, lo][kDh regions]
+    static constexpr int kBstage = 2 * kDh * kBregion;
+    static constexpr int kMmaEnd = kB + 2 * kBstage;
+    // solve phase (reuses the MMA region once every logit is in TMEM)
+    static constexpr int kHist = 0;                          // [kBins][NP] uint32
+    static constexpr int kXch = kHist + kBins * kNP * 4;     // [2 parity][kXchVals][512] float
+    static constexpr int kSolveEnd = kXch + 2 * kXchVals * 512 * 4;
     static constexpr int kData = kMmaEnd > kSolveEnd ? kMmaEnd : kSolveEnd;
-    static constexpr int kUnion = kData;                     // [16] uint32
-    static constexpr int kWofs = kUnion + 16 * 4;            // [17] int
-    static constexpr int kBars = (kWofs + 17 * 4 + 7) & ~7;  // q_full, mma_done, k_full
-    static constexpr int kSlot = kBars + 3 * 8;
+    static constexpr int kBars = kData;                      // q_full, k_full[2], mma_done[2], all_done
+    static constexpr int kSlot = kBars + 6 * 8;
     static constexpr int kTotal = kSlot + 16;
 };
 
@@ -133,167 +141,188 @@ __global__ void __launch_bounds__(256) kbar_split_kernel(const float *__restrict
     }
 }
 
-// Exchange of per-pass partial sums between the two threads of a pair (warps w and
-// w + 4 share TMEM lanes): each writes its NV values, a named barrier over those two
-// warps, each reads its partner's.  `parity` alternates the buffer so one barrier per
-// pass suffices.
-// Named barrier over the two warps (64 threads) that share TMEM lane quadrant `quad`;
-// constant ids 1..4 (0 is __syncthreads).
-__device__ __forceinline__ void quad_sync(int quad) {
-    switch (quad) {
-        case 0: asm volatile("bar.sync 1, 64;" ::: "memory"); break;
-        case 1: asm volatile("bar.sync 2, 64;" ::: "memory"); break;
-        case 2: asm volatile("bar.sync 3, 64;" ::: "memory"); break;
-        default: asm volatile("bar.sync 4, 64;" ::: "memory"); break;
+// Sum (or max) of one value over the 4*LG threads of each pair: every thread writes
+// its partial to slot (lg, cp) of its pair, one barrier, every thread reads the
+// pair's slots in the same order (so the threads of a pair hold identical results).
+// `parity` alternates the buffer so one barrier per exchange suffices.
+template <int NV, int LG>
+__device__ __forceinline__ void pair_reduce(float *xch, int parity, int slot, int p, float (&v)[NV], bool is_max) {
+    constexpr int kNP = 128 / LG, kSlots = 4 * LG;
+    float *buf = xch + (size_t)parity * kXchVals * 512;
+#pragma unroll
+    for (int k = 0; k < NV; ++k) buf[k * 512 + slot * kNP + p] = v[k];
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+        float a = buf[k * 512 + p];
+#pragma unroll
+        for (int s = 1; s < kSlots; ++s) {
+            const float o = buf[k * 512 + s * kNP + p];
+            a = is_max ? fmaxf(a, o) : a + o;
+        }
+        v[k] = a;
     }
 }
 
-template <int NV>
-__device__ __forceinline__ void pair_exchange(float *xch, int parity, int half, int p, int quad, float (&v)[NV]) {
-    float *mine = xch + ((size_t)(parity * 2 + half) * 128 + p) * 8;
-    const float *other = xch + ((size_t)(parity * 2 + (half ^ 1)) * 128 + p) * 8;
-#pragma unroll
-    for (int k = 0; k < NV; ++k) mine[k] = v[k];
-    quad_sync(quad);
-#pragma unroll
-    for (int k = 0; k < NV; ++k) v[k] = other[k];
-}
-
-template <int D, int KINT>
-__global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __grid_constant__ CUtensorMap tmQ,
-                                                                      const uint8_t *__restrict__ ksplit, Geom G,
-                                                                      TileP P, TileOut out, ListsView L) {
-    using S = TSmem<D>;
+template <int D, int KINT, int LG>
+__global__ void __launch_bounds__(kSelT, 1) select_tile_kernel(const __grid_constant__ CUtensorMap tmQ,
+                                                               const uint8_t *__restrict__ ksplit, Geom G, TileP P,
+                                                               TileOut out) {
+    using S = TSmem<D, LG>;
+    constexpr int kNP = S::kNP;
     extern __shared__ uint8_t tsm_raw[];
     uint8_t *sm = tsm_raw + ((1024 - (smem_u32(tsm_raw) & 1023)) & 1023);
     uint64_t *q_full = reinterpret_cast<uint64_t *>(sm + S::kBars);
-    uint64_t *mma_done = q_full + 1;
-    uint64_t *k_full = q_full + 2;
+    uint64_t *k_full = q_full + 1;      // [2]
+    uint64_t *mma_done = q_full + 3;    // [2]
+    uint64_t *all_done = q_full + 5;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + S::kSlot);
-    uint16_t *hist = reinterpret_cast<uint16_t *>(sm + S::kHist);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(sm + S::kHist);
     float *xch = reinterpret_cast<float *>(sm + S::kXch);
-    uint32_t *uni = reinterpret_cast<uint32_t *>(sm + S::kUnion);
-    int *wofs = reinterpret_cast<int *>(sm + S::kWofs);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int quad = warp & 3, half = warp >> 2;  // TMEM lane quadrant; which 32-column blocks
-    const int64_t t = (int64_t)L.n_tiles - 1 - blockIdx.x;
+    const int qd = warp & 3, cp = warp >> 2;  // TMEM lane quadrant; column part
+    const int L = qd * 32 + lane;             // TMEM lane
+    const int lg = L / kNP, p = L % kNP;      // lane group; pair
+    const int slot = lg * 4 + cp;
+    const int g = G.g;
+    const int npos = kNP / g;                 // query positions per CTA
+    const int64_t t = (int64_t)gridDim.x - 1 - blockIdx.x;  // latest (longest) rows first
     const int r = blockIdx.y;
     const int64_t b = blockIdx.z;
-    const int g = G.g, T = L.tile_rows;
-    const int p = quad * 32 + lane;  // pair == TMEM lane
     const int pos = p / g, hh = p % g;
-    const int64_t i = t * T + pos;
+    const int64_t i = t * npos + pos;
     const bool row_ok = i < G.nq;
     const int nvis = row_ok ? row_nvis(G, i) : 0;
-    const int64_t last_row = min(G.nq - 1, t * T + T - 1);
+    const int64_t last_row = min(G.nq - 1, t * npos + npos - 1);
     const int nvis_max = row_nvis(G, last_row);
-    const size_t tile_idx = ((size_t)b * G.hkv + r) * L.n_tiles + t;
-    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const int n_ct = (nvis_max + kChunkTile - 1) / kChunkTile;
+    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
     const bool lead = hh == 0;
 
     if (threadIdx.x == 0) {
-        mbar_init(q_full, 1);
-        mbar_init(mma_done, 1);
-        mbar_init(k_full, 1);
+        for (int k = 0; k < 6; ++k) mbar_init(q_full + k, 1);
         fence_mbar_init();
     }
-    if (threadIdx.x < 16) uni[threadIdx.x] = 0u;
-    if (warp == 0) {
-        tmem_alloc(tmem_slot, (uint32_t)P.ncols);
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, (uint32_t)kTmemCols);
         tmem_relinquish();
     }
+    // zero rows of the A operand (generic-proxy stores, made visible to the MMA below)
+    constexpr int kZeroRows = S::kArows - kNP;                   // 0 when LG == 1
+    constexpr int kZeroUnits = (kZeroRows > 0 ? kZeroRows : 1) * 8;  // 16-byte units per region
+    for (int u = threadIdx.x; kZeroRows > 0 && u < S::kDh * kZeroUnits; u += kSelT) {
+        const int dh = u / kZeroUnits, rem = u % kZeroUnits;
+        int row = rem / 8;
+        if (row >= 128 - kNP) row += kNP;  // skip the Q rows
+        *reinterpret_cast<uint4 *>(sm + S::kA + dh * S::kAregion + row * 128 + (rem % 8) * 16) =
+            make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
     // ---------------------------------------------------------------- logits
-    const int n_ct = (nvis_max + kChunkTile - 1) / kChunkTile;
-    if (n_ct > 0 && threadIdx.x == 0) {
-        mbar_arrive_expect_tx(q_full, 128 * D * 2);
-        for (int dh = 0; dh < S::kDh; ++dh)
-            tma_load_4d(sm + S::kQ + dh * S::kRegion, &tmQ, q_full, dh * 64, r * g, (int)(t * T), (int)b);
-    }
-    const int n_ct_all = (G.n_chunks + kChunkTile - 1) / kChunkTile;
-    const uint8_t *ks = ksplit + (((size_t)b * G.hkv + r) * n_ct_all) * 2 * (size_t)(S::kDh * S::kRegion);
-    for (int ct = 0; ct < n_ct; ++ct) {
-        if (threadIdx.x == 0) {
-            // the chunk tile's hi / lo operands, pre-split and pre-swizzled: two bulk copies
-            const uint8_t *src = ks + (size_t)ct * 2 * S::kDh * S::kRegion;
-            mbar_arrive_expect_tx(k_full, 2 * S::kDh * S::kRegion);
-            bulk_load(sm + S::kHi, src, S::kDh * S::kRegion, k_full);
-            bulk_load(sm + S::kLo, src + S::kDh * S::kRegion, S::kDh * S::kRegion, k_full);
-            if (ct == 0) mbar_wait_ns(q_full, 0, kTileWaitNs);
-            mbar_wait_ns(k_full, ct & 1, kTileWaitNs);
-            tc_fence_after();
+    if (warp == 0) {
+        if (lane == 0 && n_ct > 0) {
+            mbar_arrive_expect_tx(q_full, kNP * D * 2);
+            for (int dh = 0; dh < S::kDh; ++dh)
+                tma_load_4d(sm + S::kA + dh * S::kAregion + (128 - kNP) * 128, &tmQ, q_full, dh * 64, r * g,
+                            (int)(t * npos), (int)b);
+            const int n_ct_all = (G.n_chunks + kChunkTile - 1) / kChunkTile;
+            const uint8_t *ks = ksplit + (((size_t)b * G.hkv + r) * n_ct_all) * 2 * (size_t)(S::kDh * S::kBregion);
+            auto load_b = [&](int k, int s) {
+                const uint8_t *src = ks + (size_t)k * 2 * S::kDh * S::kBregion;
+                mbar_arrive_expect_tx(k_full + s, 2 * S::kDh * S::kBregion);
+                bulk_load(sm + S::kB + s * S::kBstage, src, 2 * S::kDh * S::kBregion, k_full + s);
+            };
+            load_b(0, 0);
+            if (n_ct > 1) load_b(1, 1);
+            bool ok = mbar_wait_ns(q_full, 0, kTileWaitNs);
             constexpr uint32_t id = idesc_bf16_f32(128, kChunkTile, 0, 0);
-            const uint32_t qb = smem_u32(sm + S::kQ), hb = smem_u32(sm + S::kHi), lb = smem_u32(sm + S::kLo);
-            const uint32_t dcol = tmem + (uint32_t)(ct * kChunkTile);
+            for (int k = 0; ok && k < n_ct; ++k) {
+                const int s = k & 1;
+                if (!(ok = mbar_wait_ns(k_full + s, (k >> 1) & 1, kTileWaitNs))) break;
+                tc_fence_after();
+                const int klg = k % LG;
+                const uint32_t qb = smem_u32(sm + S::kA) + (uint32_t)((128 - kNP - klg * kNP) * 128);
+                const uint32_t hb = smem_u32(sm + S::kB + s * S::kBstage);
+                const uint32_t lb = hb + S::kDh * S::kBregion;
+                const uint32_t dcol = tmem + (uint32_t)((k / LG) * kChunkTile);
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t qa = qb + (kk / 4) * S::kRegion + (kk % 4) * 32;
-                const uint32_t ka = hb + (kk / 4) * S::kRegion + (kk % 4) * 32;
-                mma_ss(dcol, smem_desc_sw128(qa, 16, 1024), smem_desc_sw128(ka, 16, 1024), id, kk > 0 ? 1u : 0u);
-            }
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t qa = qb + (kk / 4) * S::kAregion + (kk % 4) * 32;
+                    const uint32_t ka = hb + (kk / 4) * S::kBregion + (kk % 4) * 32;
+                    // the first lane group of a column block initialises it (other lanes get 0)
+                    mma_ss(dcol, smem_desc_sw128(qa, 16, 1024), smem_desc_sw128(ka, 16, 1024), id,
+                           (kk > 0 || klg > 0) ? 1u : 0u);
+                }
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t qa = qb + (kk / 4) * S::kRegion + (kk % 4) * 32;
-                const uint32_t ka = lb + (kk / 4) * S::kRegion + (kk % 4) * 32;
-                mma_ss(dcol, smem_desc_sw128(qa, 16, 1024), smem_desc_sw128(ka, 16, 1024), id, 1u);
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t qa = qb + (kk / 4) * S::kAregion + (kk % 4) * 32;
+                    const uint32_t ka = lb + (kk / 4) * S::kBregion + (kk % 4) * 32;
+                    mma_ss(dcol, smem_desc_sw128(qa, 16, 1024), smem_desc_sw128(ka, 16, 1024), id, 1u);
+                }
+                mma_commit(mma_done + s);
+                // the stage of tile k-1 takes tile k+1 once MMA k-1 has read it
+                if (k >= 1 && k + 1 < n_ct) {
+                    if (!(ok = mbar_wait_ns(mma_done + (s ^ 1), ((k - 1) >> 1) & 1, kTileWaitNs))) break;
+                    load_b(k + 1, s ^ 1);
+                }
             }
-            mma_commit(mma_done);
+            mma_commit(all_done);  // arrives when every MMA issued above has completed
         }
-        mbar_wait_ns(mma_done, ct & 1, kTileWaitNs);  // smem tile free, TMEM columns written
-        tc_fence_after();
+        __syncwarp();
     }
+    if (n_ct > 0) mbar_wait_ns(all_done, 0, kTileWaitNs);
+    tc_fence_after();
     __syncthreads();  // the MMA staging memory is reused below
+    for (int u = threadIdx.x; u < kBins * kNP; u += kSelT) hist[u] = 0u;
 
     // ---------------------------------------------------------------- tau per pair
-    // Thread (quad, half) owns the 32-column blocks blk = half, half + 2, ... of its
-    // pair's TMEM row; the loop bound is uniform across each warp (tcgen05.ld is
-    // warp-collective) and the two threads of a pair combine partial sums per pass.
-    const int nb = (__reduce_max_sync(0xffffffffu, (unsigned)nvis) + 31) / 32;
+    // this thread's column blocks: j = 0 .. nj-1 at TMEM columns j*128 + cp*32, chunks
+    // (j*LG + lg)*128 + cp*32 + x; the bound is uniform across the warp
+    const int nj = lg < n_ct ? (n_ct - lg + LG - 1) / LG : 0;
     const float xs = P.am1 * P.scale;  // x = (alpha - 1) * gamma / sqrt(d) * <q, k̄>
     int parity = 0;
-    // pass 0: x = (alpha-1) gamma/sqrt(d) <q, k̄> written back over the logits (later
-    // passes read x directly), and its maximum over the visible chunks
+    // pass 0: x written back over the logits (-inf past the row's visible chunks), max
     float mx = -INFINITY;
-    for (int blk = half; blk < nb; blk += 2) {
+    for (int j = 0; j < nj; ++j) {
         uint32_t u[32];
-        tmem_ld32(tmem + lane_off + blk * 32, u);
+        const uint32_t col = (uint32_t)(j * 128 + cp * 32);
+        tmem_ld32(tmem + lane_off + col, u);
+        const int lim = nvis - ((j * LG + lg) * 128 + cp * 32);
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
-            const float xv = xs * __uint_as_float(u[x]);
-            if (blk * 32 + x < nvis) mx = fmaxf(mx, xv);
+            const float xv = x < lim ? xs * __uint_as_float(u[x]) : -INFINITY;
+            mx = fmaxf(mx, xv);
             u[x] = __float_as_uint(xv);
         }
-        tmem_st32(tmem + lane_off + blk * 32, u);
+        tmem_st32(tmem + lane_off + col, u);
     }
     tmem_wait_st();
     {
         float v[1] = {mx};
-        pair_exchange<1>(xch, parity, half, p, quad, v);
+        pair_reduce<1, LG>(xch, parity, slot, p, v, true);
         parity ^= 1;
-        mx = fmaxf(mx, v[0]);
+        mx = v[0];
     }
     // bracket: f(mx - 1) >= 0 (the largest term alone is 1), f(mx - n^{1-alpha}) <= 0
     float lo = mx - 1.f;
     float hi = nvis > 0 ? mx - powf((float)nvis, 1.f - P.alpha) : 0.f;
-    // histogram initialisation: bins [half][bin][pair] over [mx - 1, mx)
-    uint16_t *hmine = hist + (size_t)half * 32 * 128;
-#pragma unroll
-    for (int j = 0; j < 32; ++j) hmine[j * 128 + p] = 0;
-    for (int blk = half; blk < nb; blk += 2) {
+    // histogram of x over [mx - 1, mx), 32 bins per pair
+    for (int j = 0; j < nj; ++j) {
         uint32_t u[32];
-        tmem_ld32(tmem + lane_off + blk * 32, u);
+        tmem_ld32(tmem + lane_off + (uint32_t)(j * 128 + cp * 32), u);
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
             const float y = __uint_as_float(u[x]) - lo;
-            if (blk * 32 + x < nvis && y >= 0.f) hmine[min(31, (int)(y * 32.f)) * 128 + p] += 1;
+            if (y >= 0.f) atomicAdd(hist + min(kBins - 1, (int)(y * (float)kBins)) * kNP + p, 1u);
         }
     }
-    quad_sync(quad);
+    __syncthreads();
     float t0 = lo;
     if (nvis > 1) {
         // estimated f at a bin edge e (every element at its bin centre c_j):
@@ -303,9 +332,9 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
         int elo = 0;
         if (KINT == 1 || KINT == 2 || KINT == 4) {
             float A0 = 0.f, A1 = 0.f, A2 = 0.f, A3 = 0.f, A4 = 0.f;
-            for (int e = 31; e >= 1; --e) {
-                const float n = (float)(hist[e * 128 + p] + hist[32 * 128 + e * 128 + p]);
-                const float c = ((float)e + 0.5f) * (1.f / 32.f), c2 = c * c;
+            for (int e = kBins - 1; e >= 1; --e) {
+                const float n = (float)hist[e * kNP + p];
+                const float c = ((float)e + 0.5f) * (1.f / kBins), c2 = c * c;
                 A0 += n;
                 A1 += n * c;
                 A2 += n * c2;
@@ -313,7 +342,7 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
                     A3 += n * c2 * c;
                     A4 += n * c2 * c2;
                 }
-                const float x = (float)e * (1.f / 32.f);
+                const float x = (float)e * (1.f / kBins);
                 float fe;
                 if (KINT == 1) fe = A1 - x * A0;
                 else if (KINT == 2) fe = A2 - 2.f * x * A1 + x * x * A0;
@@ -324,38 +353,37 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
                 }
             }
         } else {
-            int ehi = 31;
+            int ehi = kBins - 1;
             while (elo < ehi) {
                 const int e = (elo + ehi + 1) / 2;
-                const float edge = (float)e * (1.f / 32.f);
+                const float edge = (float)e * (1.f / kBins);
                 float fe = -1.f;
-                for (int j = e; j < 32; ++j)
-                    fe += (float)(hist[j * 128 + p] + hist[32 * 128 + j * 128 + p]) *
-                          rpow<KINT>(((float)j + 0.5f) * (1.f / 32.f) - edge, P);
+                for (int jb = e; jb < kBins; ++jb)
+                    fe += (float)hist[jb * kNP + p] * rpow<KINT>(((float)jb + 0.5f) * (1.f / kBins) - edge, P);
                 if (fe >= 0.f) elo = e;
                 else ehi = e - 1;
             }
         }
-        t0 = lo + (float)elo * (1.f / 32.f);
+        t0 = lo + (float)elo * (1.f / kBins);
         if (!(t0 < hi)) t0 = lo;
     }
-    // bracketed iteration (identical on both threads of the pair: same combined sums)
+    // bracketed iteration (identical on every thread of the pair: same combined sums)
     float tau = nvis == 1 ? lo : t0;
     bool done = nvis <= 1;
     int prev_cnt = -1;
     for (int it = 0; it < 40; ++it) {
-        if (__all_sync(0xffffffffu, done)) break;
+        if (!__syncthreads_or(!done)) break;
         // partial sums over the support {x > tau}: for alpha = 2 / 1.5 only the moments of
         // y = x - mx (f follows from them), otherwise f + 1 and -f'/k as well
-        float acc[5] = {0.f, 0.f, 0.f, 0.f, 0.f};  // s1, s2, count, f + 1, -f'/k
-        for (int blk = half; blk < nb; blk += 2) {
+        float acc[kXchVals] = {0.f, 0.f, 0.f, 0.f, 0.f};  // s1, s2, count, f + 1, -f'/k
+        for (int j = 0; j < nj; ++j) {
             uint32_t u[32];
-            tmem_ld32(tmem + lane_off + blk * 32, u);
+            tmem_ld32(tmem + lane_off + (uint32_t)(j * 128 + cp * 32), u);
 #pragma unroll
             for (int x = 0; x < 32; ++x) {
                 const float xv = __uint_as_float(u[x]);
                 const float tt = xv - tau;
-                if (blk * 32 + x < nvis && tt > 0.f) {
+                if (tt > 0.f) {
                     const float yv = xv - mx;
                     acc[0] += yv;
                     acc[1] = fmaf(yv, yv, acc[1]);
@@ -367,14 +395,8 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
                 }
             }
         }
-        {
-            float v[5] = {acc[0], acc[1], acc[2], acc[3], acc[4]};
-            pair_exchange<5>(xch, parity, half, p, quad, v);
-            parity ^= 1;
-            // the same order of additions on both threads of the pair
-#pragma unroll
-            for (int k = 0; k < 5; ++k) acc[k] = half == 0 ? acc[k] + v[k] : v[k] + acc[k];
-        }
+        pair_reduce<kXchVals, LG>(xch, parity, slot, p, acc, false);
+        parity ^= 1;
         if (done) continue;
         const float s1 = acc[0], s2 = acc[1];
         const int cnt = (int)acc[2];
@@ -421,31 +443,25 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
         tau = nt;
     }
     if (nvis == 0) tau = NAN;
-    if (half == 0) {
-        if (out.tau && row_ok) out.tau[((size_t)b * G.nq + i) * G.hq + r * g + hh] = tau;
-        if (L.rows && lead) L.rows[tile_idx * T + pos] = row_ok ? (int)i : -1;
-    }
+    if (slot == 0 && out.tau && row_ok) out.tau[((size_t)b * G.nq + i) * G.hq + r * g + hh] = tau;
 
-    // ---------------------------------------------------------------- group prior, pass 1: mu, union
-    // When this kernel builds the tile's lists itself, log w_c replaces x_c in this lane's
-    // TMEM row (-inf where the row does not route c) and pass 2 writes the bias table once
-    // mu is known.  Otherwise (rows regrouped across tiles) pass 1 writes log w, the mask
-    // and mu, and the regroup kernel forms d = (log w - mu) / sigma.
-    const bool lists_mode = L.count != nullptr;
+    // ---------------------------------------------------------------- group prior
     const size_t rowoff = ((size_t)b * G.nq + i) * G.hkv + r;
     const int gshift = (lane / g) * g;
     const uint32_t gmask = (g == 32) ? 0xffffffffu : ((1u << g) - 1u);
     const float log_g = logf((float)g);
     const float tau_r = nvis > 0 ? tau : INFINITY;  // rows without chunks select nothing
+    const bool writer = lead && row_ok;
     float lsum = 0.f, lcnt = 0.f;
-    for (int blk = half; blk < nb; blk += 2) {
+    for (int j = 0; j < nj; ++j) {
         uint32_t u[32];
-        tmem_ld32(tmem + lane_off + blk * 32, u);
+        tmem_ld32(tmem + lane_off + (uint32_t)(j * 128 + cp * 32), u);
+        const int c0 = (j * LG + lg) * 128 + cp * 32;
         uint32_t word = 0;
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
             const float tt = __uint_as_float(u[x]) - tau_r;
-            const bool own = (blk * 32 + x < nvis) && tt > 0.f;
+            const bool own = tt > 0.f;
             float v = own ? rpow<KINT>(tt, P) : 0.f;
             for (int o = 1; o < g; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
             const uint32_t bal = __ballot_sync(0xffffffffu, own);
@@ -458,119 +474,61 @@ __global__ void __launch_bounds__(kTileThreads, 1) select_tile_kernel(const __gr
                 lsum += lw;
                 lcnt += 1.f;
                 word |= 1u << x;
+                if (writer && out.logw) out.logw[rowoff * G.n_chunks + c0 + x] = lw;
             }
-            u[x] = __float_as_uint(lw);
-            if (!lists_mode && lead && row_ok && blk * 32 + x < nvis) {
-                if (sel) out.logw[rowoff * G.n_chunks + blk * 32 + x] = lw;
-                if (out.w) out.w[rowoff * G.n_chunks + blk * 32 + x] = sel ? expf(lw) : 0.f;
-            }
+            if (out.w && writer && c0 + x < G.n_chunks) out.w[rowoff * G.n_chunks + c0 + x] = sel ? expf(lw) : 0.f;
         }
-        if (lists_mode) tmem_st32(tmem + lane_off + blk * 32, u);
-        else if (lead && row_ok) out.mask[rowoff * G.words + blk] = word;
-        const uint32_t wu = __reduce_or_sync(0xffffffffu, word);
-        if (lane == 0 && wu) atomicOr(&uni[blk], wu);
+        if (writer && c0 / 32 < G.words) out.mask[rowoff * G.words + c0 / 32] = word;
     }
-    if (lists_mode) tmem_wait_st();
     {
         float v[2] = {lsum, lcnt};
-        pair_exchange<2>(xch, parity, half, p, quad, v);
+        pair_reduce<2, LG>(xch, parity, slot, p, v, false);
         parity ^= 1;
-        lsum = half == 0 ? lsum + v[0] : v[0] + lsum;
-        lcnt = half == 0 ? lcnt + v[1] : v[1] + lcnt;
+        lsum = v[0];
+        lcnt = v[1];
     }
-    const float mu = lcnt > 0.f ? lsum / lcnt : 0.f;
-    if (!lists_mode && lead && row_ok && half == 0) {
-        out.mu[rowoff] = mu;
-        for (int blk = nb; blk < G.words; ++blk) out.mask[rowoff * G.words + blk] = 0u;
+    if (writer && slot == 0) {
+        if (out.mu) out.mu[rowoff] = lcnt > 0.f ? lsum / lcnt : 0.f;
+        // words and chunks past the computed column blocks
+        for (int wd = n_ct * 4; wd < G.words; ++wd) out.mask[rowoff * G.words + wd] = 0u;
         if (out.w)
-            for (int c = nvis; c < G.n_chunks; ++c) out.w[rowoff * G.n_chunks + c] = 0.f;
-    }
-    __syncthreads();
-
-    // ---------------------------------------------------------------- the tile's list
-    int dlo = 0, dhi = -1;
-    if (G.causal) {
-        dlo = (int)(row_pos(G, t * T) / G.B);
-        dhi = (int)(row_pos(G, last_row) / G.B);
-        if (dhi > G.n_blk - 1) dhi = G.n_blk - 1;
-    }
-    const int nd = dhi - dlo + 1;
-    const int nwords = (nvis_max + 31) / 32;
-    if (threadIdx.x == 0 && lists_mode) {
-        int acc = nd;
-        for (int w = 0; w < nwords; ++w) {
-            uint32_t uw = uni[w];
-            for (int c = max(dlo, w * 32); c <= min(dhi, w * 32 + 31); ++c) uw &= ~(1u << (c - w * 32));
-            uni[w] = uw;
-            wofs[w] = acc;
-            acc += __popc(uw);
-        }
-        wofs[nwords] = acc;
-        L.count[tile_idx] = acc;
-    }
-    __syncthreads();
-    const int count = lists_mode ? wofs[nwords] : 0;
-    int32_t *ids = lists_mode ? L.ids + tile_idx * L.cap : nullptr;
-    float *bias = lists_mode ? L.bias + tile_idx * (size_t)L.cap * T : nullptr;
-    for (int e = threadIdx.x; lists_mode && e < nd; e += kTileThreads) ids[e] = dlo + e;
-    for (int w = threadIdx.x; lists_mode && w < nwords; w += kTileThreads) {
-        uint32_t uw = uni[w];
-        int q = wofs[w];
-        while (uw) {
-            const int bit = __ffs(uw) - 1;
-            uw &= uw - 1;
-            ids[q++] = w * 32 + bit;
-        }
-    }
-    // default bias: -inf (row does not attend), 0 for padding rows and for each row's own diagonal chunk
-    for (int idx = threadIdx.x; lists_mode && idx < count * T; idx += kTileThreads) {
-        const int e = idx / T, s = idx % T;
-        float v = -INFINITY;
-        if (t * T + s >= G.nq) v = 0.f;
-        else if (e < nd && dlo + e == (int)(row_pos(G, t * T + s) / G.B)) v = 0.f;
-        bias[idx] = v;
-    }
-    __syncthreads();
-
-    // ---------------------------------------------------------------- pass 2 (lists mode): bias, optional w / mask
-    const float inv_sigma = 1.f / P.sigma;
-    for (int blk = half; lists_mode && blk < nb; blk += 2) {
-        uint32_t u[32];
-        tmem_ld32(tmem + lane_off + blk * 32, u);
-        uint32_t word = 0;
-        const uint32_t uw = uni[blk];
-        const int base = wofs[blk];
-#pragma unroll
-        for (int x = 0; x < 32; ++x) {
-            const int c = blk * 32 + x;
-            const float lw = __uint_as_float(u[x]);
-            const bool sel = lw > -INFINITY;
-            if (lead && row_ok && c < nvis) {
-                if (sel) word |= 1u << x;
-                if ((uw >> x) & 1u) {
-                    const int e = base + __popc(uw & ((1u << x) - 1u));
-                    bias[(size_t)e * T + pos] = sel ? (lw - mu) * inv_sigma : -INFINITY;
-                } else if (c >= dlo && c <= dhi && sel) {
-                    bias[(size_t)(c - dlo) * T + pos] = (lw - mu) * inv_sigma;
-                }
-                if (out.w) out.w[rowoff * G.n_chunks + c] = sel ? expf(lw) : 0.f;
-            }
-        }
-        if (out.mask && lead && row_ok && blk < G.words) out.mask[rowoff * G.words + blk] = word;
-    }
-    if (lists_mode && lead && row_ok && half == 0) {
-        if (out.mask)
-            for (int blk = nb; blk < G.words; ++blk) out.mask[rowoff * G.words + blk] = 0u;
-        if (out.w)
-            for (int c = nvis; c < G.n_chunks; ++c) out.w[rowoff * G.n_chunks + c] = 0.f;
+            for (int c = n_ct * 128; c < G.n_chunks; ++c) out.w[rowoff * G.n_chunks + c] = 0.f;
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, (uint32_t)P.ncols);
+        tmem_dealloc(tmem, (uint32_t)kTmemCols);
     }
+}
+
+template <int D, int KINT, int LG>
+cudaError_t launch_sel(const CUtensorMap &tmQ, const uint8_t *ksplit, const Geom &G, const TileP &P,
+                       const TileOut &o, cudaStream_t st) {
+    using S = TSmem<D, LG>;
+    const size_t smem = S::kTotal + 1024;
+    cudaError_t e = cudaFuncSetAttribute(select_tile_kernel<D, KINT, LG>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int npos = (128 / LG) / G.g;
+    const int64_t nblk = (G.nq + npos - 1) / npos;
+    if (nblk > 0x7fffffff) return cudaErrorInvalidValue;
+    dim3 grid((unsigned)nblk, (unsigned)G.hkv, (unsigned)G.b);
+    select_tile_kernel<D, KINT, LG><<<grid, kSelT, smem, st>>>(tmQ, ksplit, G, P, o);
+    return cudaGetLastError();
+}
+
+template <int D, int KINT>
+cudaError_t launch_sel_lg(const TView &Q, const uint8_t *ksplit, const Geom &G, const TileP &P, const TileOut &o,
+                          cudaStream_t st) {
+    const int LG = G.n_chunks <= 512 ? 1 : G.n_chunks <= 1024 ? 2 : 4;
+    const int npos = (128 / LG) / G.g;
+    CUtensorMap tmQ;
+    if (!make_map_bf16(&tmQ, Q, G.b, G.nq, G.hq, G.d, G.g, npos)) return cudaErrorInvalidValue;
+    if (LG == 1) return launch_sel<D, KINT, 1>(tmQ, ksplit, G, P, o, st);
+    if (LG == 2) return launch_sel<D, KINT, 2>(tmQ, ksplit, G, P, o, st);
+    return launch_sel<D, KINT, 4>(tmQ, ksplit, G, P, o, st);
 }
 
 }  // namespace
@@ -581,7 +539,8 @@ bool select_tile_supported(const Geom &G, dash_dtype_t dt) {
     if (dt != DASH_BF16) return false;
     if (G.d != 64 && G.d != 128) return false;
     if (G.g & (G.g - 1)) return false;
-    if (G.tile_rows * G.g != 128) return false;
+    const int LG = G.n_chunks <= 512 ? 1 : G.n_chunks <= 1024 ? 2 : 4;
+    if (G.g > 128 / LG || G.g > 32) return false;  // the heads of a row share one warp and one CTA
     if (G.n_chunks > kMaxTileChunks) return false;
     return tma_encode_fn() != nullptr;
 }
@@ -592,9 +551,10 @@ size_t select_tile_workspace(const Geom &G) {
 }
 
 cudaError_t launch_select_tile(const TView &Q, const float *kbar, const Geom &G, float alpha, float gamma,
-                               float sigma, float *tau, float *w, uint32_t *mask, float *logw, float *mu,
-                               const ListsView &L, void *work, cudaStream_t st) {
+                               float *tau, float *w, uint32_t *mask, float *logw, float *mu, void *work,
+                               cudaStream_t st) {
     if (G.nq == 0 || G.b == 0) return cudaSuccess;
+    if (!mask) return cudaErrorInvalidValue;
     uint8_t *ksplit = static_cast<uint8_t *>(work);
     const int n_ct = (G.n_chunks + kChunkTile - 1) / kChunkTile;
     if (n_ct > 0) {
@@ -604,31 +564,15 @@ cudaError_t launch_select_tile(const TView &Q, const float *kbar, const Geom &G,
         cudaError_t e0 = cudaGetLastError();
         if (e0 != cudaSuccess) return e0;
     }
-    CUtensorMap tmQ;
-    if (!make_map_bf16(&tmQ, Q, G.b, G.nq, G.hq, G.d, G.g, G.tile_rows)) return cudaErrorInvalidValue;
     TileP P;
     P.alpha = alpha;
     P.am1 = alpha - 1.f;
     P.kexp = 1.f / (alpha - 1.f);
-    P.kint = (alpha == 2.f) ? 1 : (alpha == 1.5f) ? 2 : (alpha == 1.25f) ? 4 : 0;
     P.scale = gamma / sqrtf((float)G.d);
-    P.sigma = sigma;
-    int nc = ((G.n_chunks + kChunkTile - 1) / kChunkTile) * kChunkTile;
-    int ncols = 32;
-    while (ncols < nc) ncols *= 2;
-    P.ncols = ncols;
+    const int kint = (alpha == 2.f) ? 1 : (alpha == 1.5f) ? 2 : (alpha == 1.25f) ? 4 : 0;
     TileOut o{tau, w, mask, logw, mu};
-    dim3 grid((unsigned)L.n_tiles, (unsigned)G.hkv, (unsigned)G.b);
-    cudaError_t e = cudaErrorNotSupported;
-#define DASH_SEL_CASE(DD, KK)                                                                              \
-    if (G.d == DD && P.kint == KK) {                                                                       \
-        const size_t smem = TSmem<DD>::kTotal + 1024;                                                      \
-        e = cudaFuncSetAttribute(select_tile_kernel<DD, KK>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                                 (int)smem);                                                               \
-        if (e != cudaSuccess) return e;                                                                    \
-        select_tile_kernel<DD, KK><<<grid, kTileThreads, smem, st>>>(tmQ, ksplit, G, P, o, L);            \
-        return cudaGetLastError();                                                                         \
-    }
+#define DASH_SEL_CASE(DD, KK) \
+    if (G.d == DD && kint == KK) return launch_sel_lg<DD, KK>(Q, ksplit, G, P, o, st);
     DASH_SEL_CASE(128, 2)
     DASH_SEL_CASE(128, 1)
     DASH_SEL_CASE(128, 4)
@@ -638,7 +582,7 @@ cudaError_t launch_select_tile(const TView &Q, const float *kbar, const Geom &G,
     DASH_SEL_CASE(64, 4)
     DASH_SEL_CASE(64, 0)
 #undef DASH_SEL_CASE
-    return e;
+    return cudaErrorNotSupported;
 }
 
 }  // namespace dash
