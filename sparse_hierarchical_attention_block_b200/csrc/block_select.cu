@@ -138,9 +138,18 @@ __device__ float solve_tau(const float *X, int n, const SelParams &P, int *hist)
                 const float var = fmaxf(s2 / (float)cnt - m1 * m1, 0.f);
                 nt = mx + m1 - sqrtf(fmaxf(1.f / (float)cnt - var, 0.f));
             }
-            if (!(nt >= lo && nt <= hi)) {
+            // at the root the closed form can land a rounding error outside the bracket:
+            // a step that close is clamped into it, a farther one is replaced by bisection
+            const float slack = 4e-7f * fmaxf(1.f, fabsf(tau));
+            if (nt >= lo - slack && nt <= hi + slack) {
+                nt = fminf(fmaxf(nt, lo), hi);
+            } else {
                 nt = 0.5f * (lo + hi);  // a bisection step: the next count proves nothing
                 prev_cnt = -1;
+            }
+            if (hi - lo <= slack) {
+                tau = nt;
+                break;
             }
         } else {
             nt = df < 0.f ? tau - f / df : 0.5f * (lo + hi);
@@ -332,7 +341,7 @@ __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(TView Q, const
             const bool sel = v > -INFINITY;
             const unsigned bits = __ballot_sync(0xffffffffu, sel);
             if (lane == 0) out.mask[rowoff * G.words + wd] = bits;
-            if (sel && out.logw) out.logw[rowoff * G.n_chunks + c] = v;
+            if (sel && out.logw) out.logw[logw_index(G, b, r, i, c)] = v;
             if (out.w && c < G.n_chunks) out.w[rowoff * G.n_chunks + c] = sel ? expf(v) : 0.f;
         }
         __syncthreads();
@@ -409,7 +418,7 @@ __global__ void __launch_bounds__(128) compact_kernel(Geom G, const uint32_t *__
             if (G.causal && c == (int)(row_pos(G, i) / G.B)) {
                 v = 0.f;  // diagonal chunk: bias 0, causal mask in Stage 2
             } else if (c < row_nvis(G, i) && ((mask[rowoff * G.words + c / 32] >> (c % 32)) & 1u)) {
-                v = (logw[rowoff * G.n_chunks + c] - mu[rowoff]) * inv_sigma;  // d_c = (log w_c - mu) / sigma
+                v = (logw[logw_index(G, b, r, i, c)] - mu[rowoff]) * inv_sigma;  // d_c = (log w_c - mu) / sigma
             }
         }
         bias[(size_t)e * T + s] = v;
@@ -559,8 +568,7 @@ __global__ void __launch_bounds__(32 * kTilesPerWindow) regroup_compact_kernel(G
         } else if (G.causal && c == (int)(row_pos(G, i) / G.B)) {
             v = 0.f;
         } else if (c < row_nvis(G, i) && ((mrow[j * G.words + c / 32] >> (c % 32)) & 1u)) {
-            const size_t rowoff = (size_t)(b * G.nq + i) * G.hkv + r;
-            v = (logw[rowoff * G.n_chunks + c] - murow[j]) * inv_sigma;  // d_c = (log w_c - mu) / sigma
+            v = (logw[logw_index(G, b, r, i, c)] - murow[j]) * inv_sigma;  // d_c = (log w_c - mu) / sigma
         }
         bias[(size_t)e * T + j] = v;
     }

@@ -49,6 +49,12 @@ __host__ __device__ inline int64_t tile_row(const ListsView &L, const Geom &G, s
     return i < G.nq ? i : -1;
 }
 
+// Index of log w for (batch b, kv head r, query row i, chunk c) in the chunk-major
+// layout [b][hkv][n_chunks][nq]: the rows of a tile that route one chunk sit together.
+__host__ __device__ inline size_t logw_index(const Geom &G, int64_t b, int r, int64_t i, int c) {
+    return (((size_t)b * G.hkv + r) * G.n_chunks + c) * (size_t)G.nq + i;
+}
+
 // Causal geometry of query row i: key position, own chunk, visible chunks.
 __host__ __device__ inline int64_t row_pos(const Geom &G, int64_t i) { return i + G.nk - G.nq; }
 __host__ __device__ inline int row_nvis(const Geom &G, int64_t i) {

@@ -13,7 +13,7 @@ struct SelectOut {
     float *tau;        // [b][nq][hq] or null
     float *w;          // [b][nq][hkv][n_chunks] or null
     uint32_t *mask;    // [b][nq][hkv][words] (required)
-    float *logw;       // [b][nq][hkv][n_chunks] log w of the routed chunks (when lists are built)
+    float *logw;       // [b][hkv][n_chunks][nq] (logw_index) log w of the routed chunks (when lists are built)
     float *mu;         // [b][nq][hkv] mean log w over the routed chunks (when lists are built)
 };
 cudaError_t launch_select_rows(const TView &Q, dash_dtype_t dt, const float *kbar, const Geom &G, float alpha,

@@ -54,7 +54,7 @@ struct TileOut {
     float *tau;       // [b][nq][hq] or null
     float *w;         // [b][nq][hkv][n_chunks] or null
     uint32_t *mask;   // [b][nq][hkv][words] (required)
-    float *logw;      // [b][nq][hkv][n_chunks] log w of the routed chunks, or null
+    float *logw;      // [b][hkv][n_chunks][nq] log w of the routed chunks (logw_index), or null
     float *mu;        // [b][nq][hkv] mean log w over the routed chunks, or null
 };
 
@@ -141,12 +141,14 @@ __global__ void __launch_bounds__(256) kbar_split_kernel(const float *__restrict
     }
 }
 
-// Sum (or max) of one value over the 4*LG threads of each pair: every thread writes
-// its partial to slot (lg, cp) of its pair, one barrier, every thread reads the
-// pair's slots in the same order (so the threads of a pair hold identical results).
-// `parity` alternates the buffer so one barrier per exchange suffices.
+// Sum, max or min of NV values over the 4*LG threads of each pair: every thread writes
+// its partials to slot (lg, cp) of its pair, one barrier, every thread reads the pair's
+// slots in the same order (so the threads of a pair hold identical results).  Bit k of
+// max_bits / min_bits selects max / min for value k (sum otherwise).  `parity`
+// alternates the buffer so one barrier per exchange suffices.
 template <int NV, int LG>
-__device__ __forceinline__ void pair_reduce(float *xch, int parity, int slot, int p, float (&v)[NV], bool is_max) {
+__device__ __forceinline__ void pair_reduce(float *xch, int parity, int slot, int p, float (&v)[NV], int max_bits,
+                                            int min_bits) {
     constexpr int kNP = 128 / LG, kSlots = 4 * LG;
     float *buf = xch + (size_t)parity * kXchVals * 512;
 #pragma unroll
@@ -158,7 +160,7 @@ __device__ __forceinline__ void pair_reduce(float *xch, int parity, int slot, in
 #pragma unroll
         for (int s = 1; s < kSlots; ++s) {
             const float o = buf[k * 512 + s * kNP + p];
-            a = is_max ? fmaxf(a, o) : a + o;
+            a = ((max_bits >> k) & 1) ? fmaxf(a, o) : ((min_bits >> k) & 1) ? fminf(a, o) : a + o;
         }
         v[k] = a;
     }
@@ -305,7 +307,7 @@ __global__ void __launch_bounds__(kSelT, 1) select_tile_kernel(const __grid_cons
     tmem_wait_st();
     {
         float v[1] = {mx};
-        pair_reduce<1, LG>(xch, parity, slot, p, v, true);
+        pair_reduce<1, LG>(xch, parity, slot, p, v, 1, 0);
         parity ^= 1;
         mx = v[0];
     }
@@ -370,71 +372,82 @@ __global__ void __launch_bounds__(kSelT, 1) select_tile_kernel(const __grid_cons
     // bracketed iteration (identical on every thread of the pair: same combined sums)
     float tau = nvis == 1 ? lo : t0;
     bool done = nvis <= 1;
+    constexpr bool kClosed = KINT == 1 || KINT == 2;
     int prev_cnt = -1;
     for (int it = 0; it < 40; ++it) {
         if (!__syncthreads_or(!done)) break;
-        // partial sums over the support {x > tau}: for alpha = 2 / 1.5 only the moments of
-        // y = x - mx (f follows from them), otherwise f + 1 and -f'/k as well
-        float acc[kXchVals] = {0.f, 0.f, 0.f, 0.f, 0.f};  // s1, s2, count, f + 1, -f'/k
-        for (int j = 0; j < nj; ++j) {
-            uint32_t u[32];
-            tmem_ld32(tmem + lane_off + (uint32_t)(j * 128 + cp * 32), u);
+        // alpha = 2 / 1.5: moments of y = x - mx over the support {x > tau}, its count,
+        // the smallest score inside and the largest outside; otherwise f + 1, -f'/k, count
+        float acc[kXchVals] = {0.f, 0.f, 0.f, INFINITY, -INFINITY};
+        // a warp whose pairs are all settled skips the pass (the threads of a pair share
+        // their decisions, so the pair's other warps skip it too)
+        if (!__all_sync(0xffffffffu, done)) {
+            for (int j = 0; j < nj; ++j) {
+                uint32_t u[32];
+                tmem_ld32(tmem + lane_off + (uint32_t)(j * 128 + cp * 32), u);
 #pragma unroll
-            for (int x = 0; x < 32; ++x) {
-                const float xv = __uint_as_float(u[x]);
-                const float tt = xv - tau;
-                if (tt > 0.f) {
-                    const float yv = xv - mx;
-                    acc[0] += yv;
-                    acc[1] = fmaf(yv, yv, acc[1]);
-                    acc[2] += 1.f;
-                    if (KINT != 1 && KINT != 2) {
-                        acc[3] += rpow<KINT>(tt, P);
-                        acc[4] += rpow_m1<KINT>(tt, P);
+                for (int x = 0; x < 32; ++x) {
+                    const float xv = __uint_as_float(u[x]);
+                    const float tt = xv - tau;
+                    if (tt > 0.f) {
+                        if (kClosed) {
+                            const float yv = xv - mx;
+                            acc[0] += yv;
+                            acc[1] = fmaf(yv, yv, acc[1]);
+                            acc[3] = fminf(acc[3], xv);
+                        } else {
+                            acc[0] += rpow<KINT>(tt, P);
+                            acc[1] += rpow_m1<KINT>(tt, P);
+                        }
+                        acc[2] += 1.f;
+                    } else if (kClosed) {
+                        acc[4] = fmaxf(acc[4], xv);
                     }
                 }
             }
         }
-        pair_reduce<kXchVals, LG>(xch, parity, slot, p, acc, false);
+        pair_reduce<kXchVals, LG>(xch, parity, slot, p, acc, 1 << 4, 1 << 3);
         parity ^= 1;
         if (done) continue;
-        const float s1 = acc[0], s2 = acc[1];
         const int cnt = (int)acc[2];
         const float tr = tau - mx;  // tau in the y = x - mx frame
-        float f, df;
-        if (KINT == 1) {
-            f = s1 - tr * (float)cnt - 1.f;  // sum (y - tr) - 1
-            df = -(float)cnt;
-        } else if (KINT == 2) {
-            f = s2 - 2.f * tr * s1 + tr * tr * (float)cnt - 1.f;  // sum (y - tr)^2 - 1
-            df = -2.f * (s1 - tr * (float)cnt);
-        } else {
-            f = acc[3] - 1.f;
-            df = -P.kexp * acc[4];
-        }
+        float f;
+        if (KINT == 1) f = acc[0] - tr * (float)cnt - 1.f;                                    // sum (y - tr) - 1
+        else if (KINT == 2) f = acc[1] - 2.f * tr * acc[0] + tr * tr * (float)cnt - 1.f;     // sum (y - tr)^2 - 1
+        else f = acc[0] - 1.f;
         if (f >= 0.f) lo = tau;
         else hi = tau;
         float nt;
-        if ((KINT == 1 || KINT == 2) && cnt > 0) {
-            // the previous step was the exact closed form on this same support
-            // (supports {x > tau} are nested, so equal counts mean equal sets): done
+        if (kClosed && cnt > 0) {
+            // exact threshold if the support were S = {x > tau}; it is the answer when S is
+            // also {x > nt}: every score of S above nt, every other score at most nt
+            const float m1 = acc[0] / (float)cnt;
+            if (KINT == 1) {
+                nt = mx + (acc[0] - 1.f) / (float)cnt;
+            } else {
+                const float var = fmaxf(acc[1] / (float)cnt - m1 * m1, 0.f);
+                nt = mx + m1 - sqrtf(fmaxf(1.f / (float)cnt - var, 0.f));
+            }
+            // (or, with rounding ties, when two closed-form steps in a row saw the same
+            // support: supports {x > tau} are nested, so equal counts mean equal sets)
             if (cnt == prev_cnt) {
                 done = true;
                 continue;
             }
             prev_cnt = cnt;
-            const float m1 = s1 / (float)cnt;
-            if (KINT == 1) {
-                nt = mx + (s1 - 1.f) / (float)cnt;
+            // at the root the closed form can land a rounding error outside the bracket:
+            // a step that close is clamped into it, a farther one is replaced by bisection
+            const float slack = 4e-7f * fmaxf(1.f, fabsf(tau));
+            if (nt >= lo - slack && nt <= hi + slack) {
+                nt = fminf(fmaxf(nt, lo), hi);
+                if (acc[3] > nt && acc[4] <= nt) done = true;
             } else {
-                const float var = fmaxf(s2 / (float)cnt - m1 * m1, 0.f);
-                nt = mx + m1 - sqrtf(fmaxf(1.f / (float)cnt - var, 0.f));
-            }
-            if (!(nt >= lo && nt <= hi)) {
                 nt = 0.5f * (lo + hi);  // a bisection step: the next count proves nothing
                 prev_cnt = -1;
             }
+            if (hi - lo <= slack) done = true;  // the bracket has collapsed onto the root
         } else {
+            const float df = -P.kexp * acc[1];
             nt = df < 0.f ? tau - f / df : 0.5f * (lo + hi);
             if (!(nt > lo && nt < hi)) nt = 0.5f * (lo + hi);
             if (fabsf(nt - tau) <= 1e-7f * fmaxf(1.f, fabsf(tau)) || hi - lo <= 1e-7f * fmaxf(1.f, fabsf(tau)))
@@ -462,9 +475,13 @@ __global__ void __launch_bounds__(kSelT, 1) select_tile_kernel(const __grid_cons
         for (int x = 0; x < 32; ++x) {
             const float tt = __uint_as_float(u[x]) - tau_r;
             const bool own = tt > 0.f;
+            const uint32_t bal = __ballot_sync(0xffffffffu, own);
+            if (bal == 0u) {  // no head of the warp's rows routes this chunk
+                if (out.w && writer && c0 + x < G.n_chunks) out.w[rowoff * G.n_chunks + c0 + x] = 0.f;
+                continue;
+            }
             float v = own ? rpow<KINT>(tt, P) : 0.f;
             for (int o = 1; o < g; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            const uint32_t bal = __ballot_sync(0xffffffffu, own);
             const bool sel = ((bal >> gshift) & gmask) != 0u;
             float lw = -INFINITY;
             if (sel) {
@@ -474,7 +491,7 @@ __global__ void __launch_bounds__(kSelT, 1) select_tile_kernel(const __grid_cons
                 lsum += lw;
                 lcnt += 1.f;
                 word |= 1u << x;
-                if (writer && out.logw) out.logw[rowoff * G.n_chunks + c0 + x] = lw;
+                if (writer && out.logw) out.logw[logw_index(G, b, r, i, c0 + x)] = lw;
             }
             if (out.w && writer && c0 + x < G.n_chunks) out.w[rowoff * G.n_chunks + c0 + x] = sel ? expf(lw) : 0.f;
         }
@@ -482,7 +499,7 @@ __global__ void __launch_bounds__(kSelT, 1) select_tile_kernel(const __grid_cons
     }
     {
         float v[2] = {lsum, lcnt};
-        pair_reduce<2, LG>(xch, parity, slot, p, v, false);
+        pair_reduce<2, LG>(xch, parity, slot, p, v, 0, 0);
         parity ^= 1;
         lsum = v[0];
         lcnt = v[1];
