@@ -39,6 +39,16 @@ import synthetic  # noqa: E402
 METRIC = "DashAttention fwd ms & TFLOP/s (prefill) / GB/s (decode), % of B200 roofline"
 L2_FLUSH_BYTES = 256 << 20
 
+# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu capture of
+# the current kernel on the workload (the summaries under profiles/ name the command):
+# Stage 2 tensor-core kernel on prefill8k (profiles/attn_tc_prefill8k.md); the decode
+# kernel captured at batch 4 and scaled by the (batch, kv head) units to batch 16
+# (profiles/attn_decode_decode.md).  Workloads without a capture report null.
+TRAFFIC_BYTES = {
+    ("prefill8k", 1): 1.449e8,
+    ("decode", 16): None,
+}
+
 
 def load_peaks():
     p = ROOT / "MEASURED_PEAKS.json"
@@ -156,6 +166,8 @@ def run_ours(args, rank, world, device):
 
     dash.load_library()
     w = synthetic.WORKLOADS[args.workload]
+    if args.batch:
+        w = w.with_(batch=args.batch)
     alpha = args.alpha or w.alpha
     sigma = args.sigma
     decode = w.nq == 1  # one new query token per sequence
@@ -255,14 +267,14 @@ def run_ours(args, rank, world, device):
         per = lambda msx: job_throughput(work, world, msx) / 1e9  # noqa: E731
         achieved = work / (ms2 * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": TRAFFIC_BYTES.get((w.name, w.batch)),
                 "kernel": "attn_decode (+ combine)", "peak_source": peaks["source"] + " hbm_gbs"}
     else:
         unit, work = "TFLOP/s", f2
         per = lambda msx: job_throughput(work, world, msx) / 1e12  # noqa: E731
         achieved = work / (ms2 * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": None,
+                "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": TRAFFIC_BYTES.get((w.name, w.batch)),
                 "kernel": "attn_tc (Stage 2)", "peak_source": peaks["source"] + " bf16_tflops (burst)"}
     res = {
         "metric": METRIC,
@@ -335,6 +347,8 @@ def oracle_sample(w, alpha, sigma, q, k, v, budget_s=15.0, max_rows=None):
 
 def run_reference(args, device):
     w = synthetic.WORKLOADS[args.workload]
+    if args.batch:
+        w = w.with_(batch=args.batch)
     alpha = args.alpha or w.alpha
     q, k, v = synthetic.make_inputs(w, device)
     decode = w.nq == 1
@@ -370,6 +384,7 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="prefill8k", choices=sorted(synthetic.WORKLOADS))
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (smaller profiling cases)")
     ap.add_argument("--alpha", type=float, default=None)
     ap.add_argument("--sigma", type=float, default=1e8)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

@@ -94,7 +94,9 @@ struct DecSmem {
     static constexpr int kMerge = 4 * kDecRows * (D + 2) * 4;  // per-warp states at the end
     static constexpr int kData = kRing > kMerge ? kRing : kMerge;
     static constexpr int kBars = kData;
-    static constexpr int kTotal = kBars + kNS * 8;
+    static constexpr int kIds = kBars + kNS * 8;                      // [kEntriesPerSplit] chunk ids
+    static constexpr int kBias = kIds + kEntriesPerSplit * 4;         // [kEntriesPerSplit][kDecRows] bias (exp2 domain)
+    static constexpr int kTotal = kBias + kEntriesPerSplit * kDecRows * 4;
 };
 
 template <int D, int BLK>
@@ -120,14 +122,23 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(const __grid_c
     const int32_t *ids = L.ids + tile_idx * L.cap;
     const float *bias = L.bias + tile_idx * (size_t)L.cap * T;
 
+    int *ids_s = reinterpret_cast<int *>(sm + S::kIds);
+    float *bias_s = reinterpret_cast<float *>(sm + S::kBias);
     if (threadIdx.x == 0) {
         for (int s = 0; s < S::kNS; ++s) mbar_init(full + s, 1);
         fence_mbar_init();
     }
+    // the split's chunk ids and per-row biases, read once (they would otherwise sit on
+    // the critical path of every chunk)
+    for (int idx = threadIdx.x; idx < n * kDecRows; idx += kDecThreads) {
+        const int e = idx / kDecRows, row = idx % kDecRows;
+        if (row == 0) ids_s[e] = ids[e_begin + e];
+        bias_s[idx] = row < M ? bias[(size_t)(e_begin + e) * T + row / g] * 1.4426950408889634f : -INFINITY;
+    }
     __syncthreads();
     const uint32_t ring = smem_u32(sm);
     auto issue = [&](int e, int st) {
-        const int c = ids[e_begin + e];
+        const int c = ids_s[e];
         uint8_t *kd = sm + st * S::kStage;
         mbar_arrive_expect_tx(full + st, (uint32_t)S::kStage);
         for (int dh = 0; dh < S::kDh; ++dh) {
@@ -175,9 +186,9 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(const __grid_c
 
     for (int e = 0; e < n; ++e) {
         const int st = e % S::kNS;
-        const int c = ids[e_begin + e];
-        const float b0 = row0 < M ? bias[(size_t)(e_begin + e) * T + row0 / g] * 1.4426950408889634f : -INFINITY;
-        const float b1 = row1 < M ? bias[(size_t)(e_begin + e) * T + row1 / g] * 1.4426950408889634f : -INFINITY;
+        const int c = ids_s[e];
+        const float b0 = bias_s[e * kDecRows + row0];
+        const float b1 = bias_s[e * kDecRows + row1];
         ok = __syncthreads_and(wait_full(full + st, (e / S::kNS) & 1)) != 0;
         if (!ok) {
             e_fail = e;
