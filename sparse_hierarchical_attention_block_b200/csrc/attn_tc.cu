@@ -339,9 +339,9 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
             if (!ok) break;
             tc_fence_after();
             // Single pass on the running maximum of the earlier steps: p = 2^(s * scale +
-            // bias - m_run) straight from S.  It stands unless a row of the warp finds a
-            // logit above m_run + kRescaleL2 (then P is discarded, S is still intact, and
-            // the two-pass path below redoes the step with a new maximum).  P is held in
+            // bias - m_run) straight from S.  It stands unless a row of the warp sums p
+            // above 2^kRescaleL2 (then P is discarded, S is still intact, and the two-pass
+            // path below redoes the step with a new maximum).  P is held in
             // registers and written over S only once the step is known to stand.
             bool step_done = false;
             if (j > 0 && __all_sync(0xffffffffu, !row_ok || m_run > -INFINITY)) {
@@ -349,15 +349,14 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
 #pragma unroll
                 for (int e = 0; e < S::kE; ++e) cbm[e] = row_ok ? bl2[e] - m_run : -INFINITY;
                 uint32_t pk[64];
-                float mr[4] = {0.f, 0.f, 0.f, 0.f};
                 float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int qc = 0; qc < 4; ++qc) {
-                    uint32_t u[32];
-                    tmem_ld32(tS + lane_off + qc * 32, u);
+                for (int qc = 0; qc < 8; ++qc) {
+                    uint32_t u[16];
+                    tmem_ld16(tS + lane_off + qc * 16, u);
 #pragma unroll
-                    for (int x = 0; x < 16; ++x) {
-                        const int kc = qc * 32 + 2 * x;
+                    for (int x = 0; x < 8; ++x) {
+                        const int kc = qc * 16 + 2 * x;
                         float v0 = fmaf(__uint_as_float(u[2 * x]), sl2, cbm[kc / BLK]);
                         float v1 = fmaf(__uint_as_float(u[2 * x + 1]), sl2, cbm[(kc + 1) / BLK]);
                         if (need_mask) {  // select before exp2: S outside the list may be any bit pattern
@@ -365,17 +364,17 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
                             v1 = ((kc + 1) % BLK) < lim[(kc + 1) / BLK] ? v1 : -INFINITY;
                         }
                         const float p0 = ex2(v0), p1 = ex2(v1);
-                        mr[x & 3] = fmaxf(mr[x & 3], fmaxf(p0, p1));
                         ps[x & 3] += p0 + p1;
-                        pk[qc * 16 + x] = pack_bf16x2(p0, p1);
+                        pk[qc * 8 + x] = pack_bf16x2(p0, p1);
                     }
                 }
-                // largest p of the row (2^(logit - m_run)); inf if it overflowed
-                const float pmax = fmaxf(fmaxf(mr[0], mr[1]), fmaxf(mr[2], mr[3]));
-                if (!__any_sync(0xffffffffu, pmax > kRescaleP)) {
+                // the step stands while the row's sum of p = 2^(logit - m_run) stays at most
+                // 2^kRescaleL2 (then so does every p); a sum that overflowed is not finite
+                const float psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
+                if (!__any_sync(0xffffffffu, !(psum <= kRescaleP))) {
                     tmem_st32(tS + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
                     tmem_st32(tS + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
-                    l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+                    l_run += psum;
                     step_done = true;
                 }
             }
