@@ -20,9 +20,10 @@
 //            support (until the support is stable), otherwise Newton, with
 //            bisection as the safeguard; partial sums are combined in a fixed order
 //            so every thread of a pair takes the same decisions;
-//   prior    the g heads of a query row sit in g adjacent lanes of one warp:
-//            w_c = (1/g) sum_h [x_c - tau_h]_+^{1/(alpha-1)} by shuffles, membership
-//            by comparison (ballot), mu = mean log w over the routed chunks
+//   prior    the g heads of a query row sit in g adjacent lanes of one warp; a
+//            shared-memory transpose gives each lane the g heads' scores of 32/g
+//            chunks: w_c = (1/g) sum_h [x_c - tau_h]_+^{1/(alpha-1)}, membership by
+//            comparison, mu = mean log w over the routed chunks
 //            (§3.4 Prop. 1); outputs the bit mask, log w of the routed chunks and mu
 //            per row, from which the work lists are built (d = (log w - mu)/sigma).
 #include <math.h>
@@ -93,7 +94,8 @@ struct TSmem {
     // solve phase (reuses the MMA region once every logit is in TMEM)
     static constexpr int kHist = 0;                          // [kBins][NP] uint32
     static constexpr int kXch = kHist + kBins * kNP * 4;     // [2 parity][kXchVals][512] float
-    static constexpr int kSolveEnd = kXch + 2 * kXchVals * 512 * 4;
+    static constexpr int kTr = kXch + 2 * kXchVals * 512 * 4;  // [16 warps][32 lanes][33] float transpose
+    static constexpr int kSolveEnd = kTr + 16 * 32 * 33 * 4;
     static constexpr int kData = kMmaEnd > kSolveEnd ? kMmaEnd : kSolveEnd;
     static constexpr int kBars = kData;                      // q_full, k_full[2], mma_done[2], all_done
     static constexpr int kSlot = kBars + 6 * 8;
@@ -459,30 +461,36 @@ __global__ void __launch_bounds__(kSelT, 1) select_tile_kernel(const __grid_cons
     if (slot == 0 && out.tau && row_ok) out.tau[((size_t)b * G.nq + i) * G.hq + r * g + hh] = tau;
 
     // ---------------------------------------------------------------- group prior
+    // The g heads of a query row sit in g adjacent lanes.  Per 32-column block every lane
+    // puts its t = x - tau into a padded shared-memory row; lane (pos, k) then reads the
+    // g heads' t of the chunks x = k, k + g, ... of its row (32 values, bank-conflict free)
+    // and forms w_c = (1/g) sum_h [t_h]_+^{1/(alpha-1)}, membership (some t_h > 0) and
+    // log w for those chunks alone, so no work is repeated across the group.
     const size_t rowoff = ((size_t)b * G.nq + i) * G.hkv + r;
-    const int gshift = (lane / g) * g;
-    const uint32_t gmask = (g == 32) ? 0xffffffffu : ((1u << g) - 1u);
     const float log_g = logf((float)g);
     const float tau_r = nvis > 0 ? tau : INFINITY;  // rows without chunks select nothing
     const bool writer = lead && row_ok;
+    float *tr = reinterpret_cast<float *>(sm + S::kTr) + warp * 32 * 33;
+    const int gbase = lane - hh;  // lane of the row's first head
     float lsum = 0.f, lcnt = 0.f;
     for (int j = 0; j < nj; ++j) {
         uint32_t u[32];
         tmem_ld32(tmem + lane_off + (uint32_t)(j * 128 + cp * 32), u);
         const int c0 = (j * LG + lg) * 128 + cp * 32;
-        uint32_t word = 0;
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
-            const float tt = __uint_as_float(u[x]) - tau_r;
-            const bool own = tt > 0.f;
-            const uint32_t bal = __ballot_sync(0xffffffffu, own);
-            if (bal == 0u) {  // no head of the warp's rows routes this chunk
-                if (out.w && writer && c0 + x < G.n_chunks) out.w[rowoff * G.n_chunks + c0 + x] = 0.f;
-                continue;
+        for (int x = 0; x < 32; ++x) tr[lane * 33 + x] = __uint_as_float(u[x]) - tau_r;
+        __syncwarp();
+        uint32_t word = 0;  // membership bits of this lane's chunks
+        for (int x = hh; x < 32; x += g) {
+            float v = 0.f;
+            bool sel = false;
+            for (int h = 0; h < g; ++h) {
+                const float tt = tr[(gbase + h) * 33 + x];
+                if (tt > 0.f) {
+                    sel = true;
+                    v += rpow<KINT>(tt, P);
+                }
             }
-            float v = own ? rpow<KINT>(tt, P) : 0.f;
-            for (int o = 1; o < g; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            const bool sel = ((bal >> gshift) & gmask) != 0u;
             float lw = -INFINITY;
             if (sel) {
                 // the power sum underflows only for scores within ~1e-10 of tau at alpha = 1.25;
@@ -491,11 +499,18 @@ __global__ void __launch_bounds__(kSelT, 1) select_tile_kernel(const __grid_cons
                 lsum += lw;
                 lcnt += 1.f;
                 word |= 1u << x;
-                if (writer && out.logw) out.logw[logw_index(G, b, r, i, c0 + x)] = lw;
+                if (row_ok && out.logw) out.logw[logw_index(G, b, r, i, c0 + x)] = lw;
             }
-            if (out.w && writer && c0 + x < G.n_chunks) out.w[rowoff * G.n_chunks + c0 + x] = sel ? expf(lw) : 0.f;
+            if (out.w && row_ok && c0 + x < G.n_chunks) out.w[rowoff * G.n_chunks + c0 + x] = sel ? expf(lw) : 0.f;
         }
+        __syncwarp();  // the transpose rows are rewritten by the next block
+        for (int o = 1; o < g; o <<= 1) word |= __shfl_xor_sync(0xffffffffu, word, o);
         if (writer && c0 / 32 < G.words) out.mask[rowoff * G.words + c0 / 32] = word;
+    }
+    // the row's sums over the chunks its g lanes took (the same totals on every lane)
+    for (int o = 1; o < g; o <<= 1) {
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+        lcnt += __shfl_xor_sync(0xffffffffu, lcnt, o);
     }
     {
         float v[2] = {lsum, lcnt};
