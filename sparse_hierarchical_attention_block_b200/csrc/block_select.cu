@@ -426,45 +426,86 @@ __global__ void __launch_bounds__(128) compact_kernel(Geom G, const uint32_t *__
 }
 
 // Regroup + compact: one CTA per (window of kTilesPerWindow tiles, kv head, batch),
-// one warp per output tile.  The window's query rows are sorted by the size of
-// their routed set (stable), consecutive runs of tile_rows rows form the tiles,
-// and each tile's list is built as in compact_kernel: the rows' diagonal chunks
-// first (ascending), then the union of their routed chunks (ascending), and the
-// per-row bias table.  Rows with similar routed sets share a tile, so the union a
-// tile streams through Stage 2 is smaller than for consecutive rows.
+// kWarpsPerTile warps per output tile.  The window's query rows are sorted by the size
+// of their routed set (stable), consecutive runs of tile_rows rows form the tiles, and
+// each tile's list is built as in compact_kernel: the rows' diagonal chunks first
+// (ascending), then the union of their routed chunks (ascending), and the per-row bias
+// table.  Rows with similar routed sets share a tile, so the union a tile streams
+// through Stage 2 is smaller than for consecutive rows.  The window's mask words are
+// cached in shared memory with an odd row stride (column reads are bank-conflict free)
+// and each tile's list is kept there for the bias fill.
 constexpr int kTilesPerWindow = 4;
+constexpr int kWarpsPerTile = 4;
+constexpr int kRegroupThreads = 32 * kTilesPerWindow * kWarpsPerTile;
 
-__global__ void __launch_bounds__(32 * kTilesPerWindow) regroup_compact_kernel(Geom G, const uint32_t *__restrict__ mask,
-                                                                               const float *__restrict__ logw,
-                                                                               const float *__restrict__ mu,
-                                                                               float inv_sigma, ListsView L, int wpow2) {
-    extern __shared__ __align__(16) uint32_t rsm[];
+struct RegroupSmem {
+    int wpow2, W, ws, words, cap;
+    size_t key, rowi, mrow, murow, uw, wofs, ids, total;
+    __host__ __device__ RegroupSmem(const Geom &G, int tile_rows, int cap_) {
+        W = tile_rows * kTilesPerWindow;
+        wpow2 = 1;
+        while (wpow2 < W) wpow2 *= 2;
+        words = G.words;
+        ws = G.words | 1;
+        cap = cap_;
+        key = 0;
+        rowi = key + (size_t)wpow2 * 4;
+        mrow = rowi + (size_t)W * 4;
+        murow = mrow + (size_t)W * ws * 4;
+        uw = murow + (size_t)W * 4;
+        wofs = uw + (size_t)kTilesPerWindow * words * 4;
+        ids = wofs + (size_t)kTilesPerWindow * (words + 1) * 4;
+        total = ids + (size_t)kTilesPerWindow * cap * 4;
+    }
+};
+
+// named barrier over the kWarpsPerTile warps of output tile tt (ids 1..kTilesPerWindow)
+__device__ __forceinline__ void tile_sync(int tt) {
+    asm volatile("bar.sync %0, %1;" ::"r"(tt + 1), "r"(32 * kWarpsPerTile) : "memory");
+}
+
+__global__ void __launch_bounds__(kRegroupThreads) regroup_compact_kernel(Geom G, const uint32_t *__restrict__ mask,
+                                                                         const float *__restrict__ logw,
+                                                                         const float *__restrict__ mu,
+                                                                         float inv_sigma, ListsView L) {
+    extern __shared__ __align__(16) uint8_t rsm_raw[];
     const int T = L.tile_rows;
-    const int W = T * kTilesPerWindow;
-    uint32_t *key = rsm;                              // [wpow2] sort keys
-    int *rowi = reinterpret_cast<int *>(key + wpow2);  // [W] query index per window slot
+    const RegroupSmem R(G, T, L.cap);
+    uint32_t *key = reinterpret_cast<uint32_t *>(rsm_raw + R.key);   // [wpow2] sort keys
+    int *rowi = reinterpret_cast<int *>(rsm_raw + R.rowi);           // [W] window slot per sorted position
+    uint32_t *mrow = reinterpret_cast<uint32_t *>(rsm_raw + R.mrow);  // [W][ws] mask words per window slot
+    float *murow = reinterpret_cast<float *>(rsm_raw + R.murow);     // [W] mu per window slot
     const int64_t win = blockIdx.x;
     const int r = blockIdx.y;
     const int64_t b = blockIdx.z;
-    const int64_t i0 = win * W;
+    const int64_t i0 = win * R.W;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
-    for (int j = threadIdx.x; j < wpow2; j += blockDim.x) {
+    // the window's rows: mask words (cached), mu, and sort keys (popcount, slot)
+    for (int j = threadIdx.x; j < R.wpow2; j += kRegroupThreads) {
         const int64_t i = i0 + j;
         uint32_t k = 0xffffffffu;
-        if (j < W && i < G.nq) {
+        if (j < R.W && i < G.nq) {
             const uint32_t *mw = mask + ((size_t)(b * G.nq + i) * G.hkv + r) * G.words;
             int cnt = 0;
-            for (int w = 0; w < G.words; ++w) cnt += __popc(mw[w]);
+            for (int w = 0; w < G.words; ++w) {
+                const uint32_t m = mw[w];
+                mrow[j * R.ws + w] = m;
+                cnt += __popc(m);
+            }
+            murow[j] = mu[(size_t)(b * G.nq + i) * G.hkv + r];
             k = ((uint32_t)cnt << 16) | (uint32_t)j;
+        } else if (j < R.W) {
+            for (int w = 0; w < G.words; ++w) mrow[j * R.ws + w] = 0u;
+            murow[j] = 0.f;
         }
         key[j] = k;
     }
     __syncthreads();
     // bitonic sort, ascending
-    for (int k2 = 2; k2 <= wpow2; k2 <<= 1) {
+    for (int k2 = 2; k2 <= R.wpow2; k2 <<= 1) {
         for (int jj = k2 >> 1; jj > 0; jj >>= 1) {
-            for (int idx = threadIdx.x; idx < wpow2; idx += blockDim.x) {
+            for (int idx = threadIdx.x; idx < R.wpow2; idx += kRegroupThreads) {
                 const int ixj = idx ^ jj;
                 if (ixj > idx) {
                     const bool asc = (idx & k2) == 0;
@@ -478,97 +519,105 @@ __global__ void __launch_bounds__(32 * kTilesPerWindow) regroup_compact_kernel(G
             __syncthreads();
         }
     }
-    for (int j = threadIdx.x; j < W; j += blockDim.x) {
+    for (int j = threadIdx.x; j < R.W; j += kRegroupThreads) {
         const uint32_t k = key[j];
-        rowi[j] = k == 0xffffffffu ? -1 : (int)(i0 + (k & 0xffffu));
+        rowi[j] = k == 0xffffffffu ? -1 : (int)(k & 0xffffu);
     }
     __syncthreads();
 
-    const int64_t tile = win * kTilesPerWindow + warp;
-    if (tile >= L.n_tiles) return;
+    const int tt = warp / kWarpsPerTile;           // output tile of this warp
+    const int tq = threadIdx.x % (32 * kWarpsPerTile);  // thread within the tile's group
+    const int64_t tile = win * kTilesPerWindow + tt;
+    if (tile >= L.n_tiles) return;  // whole tile groups leave together
     const size_t tile_idx = ((size_t)b * G.hkv + r) * L.n_tiles + tile;
-    const int *tr = rowi + warp * T;
-    for (int j = lane; j < T; j += 32) L.rows[tile_idx * T + j] = tr[j];
+    const int *slot = rowi + tt * T;                // window slot of each tile row (-1 unused)
+    for (int j = tq; j < T; j += 32 * kWarpsPerTile)
+        L.rows[tile_idx * T + j] = slot[j] >= 0 ? (int)(i0 + slot[j]) : -1;
 
     // diagonal chunks of the tile's rows, relative to the window's first chunk
-    uint64_t dmask = 0;
     const int dbase = G.causal ? (int)(row_pos(G, i0) / G.B) : 0;
+    uint64_t dmask = 0;
     if (G.causal)
         for (int j = lane; j < T; j += 32)
-            if (tr[j] >= 0) dmask |= 1ull << ((int)(row_pos(G, tr[j]) / G.B) - dbase);
-    const uint32_t dlo32 = __reduce_or_sync(0xffffffffu, (uint32_t)dmask);
-    const uint32_t dhi32 = __reduce_or_sync(0xffffffffu, (uint32_t)(dmask >> 32));
-    dmask = ((uint64_t)dhi32 << 32) | dlo32;
+            if (slot[j] >= 0) dmask |= 1ull << ((int)(row_pos(G, i0 + slot[j]) / G.B) - dbase);
+    dmask = ((uint64_t)__reduce_or_sync(0xffffffffu, (uint32_t)(dmask >> 32)) << 32) |
+            __reduce_or_sync(0xffffffffu, (uint32_t)dmask);
     const int nd = __popcll(dmask);
 
-    // the tile rows' mask words and mu, cached in shared memory for the bias fill
-    uint32_t *uw = reinterpret_cast<uint32_t *>(rowi + W) + (size_t)warp * G.words;
-    uint32_t *mrow = reinterpret_cast<uint32_t *>(rowi + W) + (size_t)kTilesPerWindow * G.words +
-                     (size_t)warp * T * G.words;
-    float *murow = reinterpret_cast<float *>(reinterpret_cast<uint32_t *>(rowi + W) + (size_t)kTilesPerWindow * G.words +
-                                             (size_t)kTilesPerWindow * T * G.words) + warp * T;
-    for (int idx = lane; idx < T * G.words; idx += 32) {
-        const int j = idx / G.words, wd = idx % G.words;
-        mrow[idx] = tr[j] >= 0 ? mask[((size_t)(b * G.nq + tr[j]) * G.hkv + r) * G.words + wd] : 0u;
-    }
-    for (int j = lane; j < T; j += 32) murow[j] = tr[j] >= 0 ? mu[(size_t)(b * G.nq + tr[j]) * G.hkv + r] : 0.f;
-    __syncwarp();
-    // union of routed chunks, diagonal ones removed; lane l owns the contiguous words
-    // [l*wpl, (l+1)*wpl) so that the lane-order prefix is the chunk order
-    const int wpl = (G.words + 31) / 32;
-    int cnt = 0;
-    for (int wd = lane * wpl; wd < min(G.words, (lane + 1) * wpl); ++wd) {
+    // union of routed chunks, diagonal ones removed
+    uint32_t *uw = reinterpret_cast<uint32_t *>(rsm_raw + R.uw) + tt * R.words;
+    int *wofs = reinterpret_cast<int *>(rsm_raw + R.wofs) + tt * (R.words + 1);
+    int *ids_s = reinterpret_cast<int *>(rsm_raw + R.ids) + (size_t)tt * R.cap;
+    for (int wd = tq; wd < G.words; wd += 32 * kWarpsPerTile) {
         uint32_t acc = 0;
-        for (int j = 0; j < T; ++j) acc |= mrow[j * G.words + wd];
+        for (int j = 0; j < T; ++j)
+            if (slot[j] >= 0) acc |= mrow[slot[j] * R.ws + wd];
         for (int c = wd * 32; c < wd * 32 + 32; ++c) {
             const int rel = c - dbase;
             if (rel >= 0 && rel < 64 && ((dmask >> rel) & 1ull)) acc &= ~(1u << (c - wd * 32));
         }
         uw[wd] = acc;
-        cnt += __popc(acc);
     }
-    // exclusive prefix of the per-lane counts
-    int incl = cnt;
-    for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-    }
-    const int total = __shfl_sync(0xffffffffu, incl, 31);
-    int pos = nd + incl - cnt;
-    int32_t *ids = L.ids + tile_idx * L.cap;
-    float *bias = L.bias + tile_idx * (size_t)L.cap * T;
-    if (lane == 0) {
-        int e = 0;
-        uint64_t dm = dmask;
-        while (dm) {
-            const int bit = __ffsll((long long)dm) - 1;
-            dm &= dm - 1;
-            ids[e++] = dbase + bit;
+    tile_sync(tt);
+    if (tq < 32) {
+        // exclusive prefix of the words' popcounts (lane l owns words [l*wpl, (l+1)*wpl))
+        const int wpl = (G.words + 31) / 32;
+        int cnt = 0;
+        for (int wd = lane * wpl; wd < min(G.words, (lane + 1) * wpl); ++wd) cnt += __popc(uw[wd]);
+        int incl = cnt;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
         }
-        L.count[tile_idx] = nd + total;
+        int run = nd + incl - cnt;
+        for (int wd = lane * wpl; wd < min(G.words, (lane + 1) * wpl); ++wd) {
+            wofs[wd] = run;
+            run += __popc(uw[wd]);
+        }
+        if (lane == 31) {
+            wofs[G.words] = run;
+            L.count[tile_idx] = run;
+        }
+        if (lane == 0) {
+            int e = 0;
+            uint64_t dm = dmask;
+            while (dm) {
+                const int bit = __ffsll((long long)dm) - 1;
+                dm &= dm - 1;
+                ids_s[e++] = dbase + bit;
+            }
+        }
     }
-    for (int wd = lane * wpl; wd < min(G.words, (lane + 1) * wpl); ++wd) {
+    tile_sync(tt);
+    for (int wd = tq; wd < G.words; wd += 32 * kWarpsPerTile) {
         uint32_t acc = uw[wd];
+        int pos = wofs[wd];
         while (acc) {
             const int bit = __ffs(acc) - 1;
             acc &= acc - 1;
-            ids[pos++] = wd * 32 + bit;
+            ids_s[pos++] = wd * 32 + bit;
         }
     }
-    __syncwarp();
-    const int count = nd + total;
+    tile_sync(tt);
+    const int count = wofs[G.words];
+    int32_t *ids = L.ids + tile_idx * L.cap;
+    for (int e = tq; e < count; e += 32 * kWarpsPerTile) ids[e] = ids_s[e];
+    float *bias = L.bias + tile_idx * (size_t)L.cap * T;
 #pragma unroll 4
-    for (int idx = lane; idx < count * T; idx += 32) {
+    for (int idx = tq; idx < count * T; idx += 32 * kWarpsPerTile) {
         const int e = idx / T, j = idx % T;
-        const int c = ids[e];
-        const int i = tr[j];
+        const int c = ids_s[e];
+        const int sl = slot[j];
         float v = -INFINITY;
-        if (i < 0) {
+        if (sl < 0) {
             v = 0.f;  // unused row: never stored
-        } else if (G.causal && c == (int)(row_pos(G, i) / G.B)) {
-            v = 0.f;
-        } else if (c < row_nvis(G, i) && ((mrow[j * G.words + c / 32] >> (c % 32)) & 1u)) {
-            v = (logw[logw_index(G, b, r, i, c)] - murow[j]) * inv_sigma;  // d_c = (log w_c - mu) / sigma
+        } else {
+            const int64_t i = i0 + sl;
+            if (G.causal && c == (int)(row_pos(G, i) / G.B)) {
+                v = 0.f;
+            } else if (c < row_nvis(G, i) && ((mrow[sl * R.ws + c / 32] >> (c % 32)) & 1u)) {
+                v = (logw[logw_index(G, b, r, i, c)] - murow[sl]) * inv_sigma;  // d_c = (log w_c - mu) / sigma
+            }
         }
         bias[(size_t)e * T + j] = v;
     }
@@ -621,31 +670,26 @@ cudaError_t launch_select_rows(const TView &Q, dash_dtype_t dt, const float *kba
     return cudaGetLastError();
 }
 
-static size_t regroup_smem(const Geom &G) {
-    const int W = G.tile_rows * kTilesPerWindow;
-    int wp = 1;
-    while (wp < W) wp *= 2;
-    return (size_t)wp * 4 + (size_t)W * 4 + (size_t)kTilesPerWindow * G.words * 4 +
-           (size_t)kTilesPerWindow * G.tile_rows * G.words * 4 + (size_t)kTilesPerWindow * G.tile_rows * 4;
-}
+static size_t regroup_smem(const Geom &G) { return RegroupSmem(G, G.tile_rows, G.n_blk).total; }
 
-bool regroup_supported(const Geom &G) { return regroup_smem(G) <= 200 * 1024; }
+bool regroup_supported(const Geom &G) {
+    // the tile_rows of a window must fit the sort key's slot field; shared memory is bounded
+    return G.tile_rows * kTilesPerWindow <= 65536 && regroup_smem(G) <= 200 * 1024;
+}
 
 cudaError_t launch_regroup_compact(const Geom &G, const uint32_t *mask, const float *logw, const float *mu,
                                    float sigma, const ListsView &L, cudaStream_t st) {
     if (G.nq == 0 || G.b == 0) return cudaSuccess;
-    const int W = L.tile_rows * kTilesPerWindow;
-    int wp = 1;
-    while (wp < W) wp *= 2;
+    const RegroupSmem R(G, L.tile_rows, L.cap);
     const int64_t nwin = (L.n_tiles + kTilesPerWindow - 1) / kTilesPerWindow;
-    const size_t smem = regroup_smem(G);
+    const size_t smem = R.total;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(regroup_compact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess) return e;
     }
-    regroup_compact_kernel<<<dim3((unsigned)nwin, (unsigned)G.hkv, (unsigned)G.b), 32 * kTilesPerWindow, smem, st>>>(
-        G, mask, logw, mu, 1.f / sigma, L, wp);
+    regroup_compact_kernel<<<dim3((unsigned)nwin, (unsigned)G.hkv, (unsigned)G.b), kRegroupThreads, smem, st>>>(
+        G, mask, logw, mu, 1.f / sigma, L);
     return cudaGetLastError();
 }
 
