@@ -406,13 +406,13 @@ __global__ void __launch_bounds__(128) compact_kernel(Geom G, const uint32_t *__
     __syncthreads();
     const int count = wofs[G.words];
     float *bias = L.bias + tile_idx * (size_t)L.cap * T;
-    for (int idx = threadIdx.x; idx < count * T; idx += blockDim.x) {
-        const int e = idx / T, s = idx % T;
+    // rows past the query length have no bias entries: Stage 2 never reads them (their
+    // scores are masked before the bias is used), so only the tile's nrows rows are filled
+    for (int idx = threadIdx.x; idx < count * nrows; idx += blockDim.x) {
+        const int e = idx / nrows, s = idx % nrows;
         const int c = ids[e];
         float v = -INFINITY;
-        if (s >= nrows) {
-            v = 0.f;  // padding row: never stored
-        } else {
+        {
             const int64_t i = i0 + s;
             const size_t rowoff = ((size_t)(b * G.nq + i) * G.hkv + r);
             if (G.causal && c == (int)(row_pos(G, i) / G.B)) {
