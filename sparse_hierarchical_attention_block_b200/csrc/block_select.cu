@@ -434,7 +434,7 @@ __global__ void __launch_bounds__(128) compact_kernel(Geom G, const uint32_t *__
 // through Stage 2 is smaller than for consecutive rows.  The window's mask words are
 // cached in shared memory with an odd row stride (column reads are bank-conflict free)
 // and each tile's list is kept there for the bias fill.
-constexpr int kTilesPerWindow = 4;
+constexpr int kTilesPerWindow = 8;
 constexpr int kWarpsPerTile = 4;
 constexpr int kRegroupThreads = 32 * kTilesPerWindow * kWarpsPerTile;
 

@@ -143,7 +143,7 @@ def test_consecutive_tiles_match_oracle(case):
 
 
 def test_regrouped_rows_are_a_permutation():
-    """Regrouping permutes the query rows within windows of 4 tiles: every row appears
+    """Regrouping permutes the query rows within windows of 8 tiles: every row appears
     once, tiles are filled before padding, and a tile's rows come from its window."""
     b, nq, nk, hq, hkv, d, B = 2, 1000, 1000, 8, 2, 128, 64
     q, k, v = _planted(b, nq, nk, hq, hkv, d, B, "bf16", seed=3)
@@ -159,8 +159,8 @@ def test_regrouped_rows_are_a_permutation():
             assert np.array_equal(valid, np.arange(nq))
             for t in range(nt):
                 tile = rows[bi, r, t]
-                w0 = (t // 4) * 4 * T
-                assert ((tile < 0) | ((tile >= w0) & (tile < w0 + 4 * T))).all()
+                w0 = (t // 8) * 8 * T
+                assert ((tile < 0) | ((tile >= w0) & (tile < w0 + 8 * T))).all()
     counts = L.count.cpu().numpy()
     assert (counts >= 1).all() and (counts <= L.cap).all()
 
