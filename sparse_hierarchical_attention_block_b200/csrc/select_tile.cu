@@ -36,9 +36,7 @@ namespace dash {
 
 namespace {
 
-constexpr int kSelT = 512;         // 16 warps: 4 TMEM lane quadrants x 4 column parts
 constexpr int kChunkTile = 128;    // chunks per logits MMA (N)
-constexpr int kTmemCols = 512;
 constexpr int kMaxTileChunks = 512 * 4;
 constexpr int kBins = 32;
 constexpr int kXchVals = 5;
@@ -78,7 +76,9 @@ __device__ __forceinline__ float rpow_m1(float t, const TileP &P) {
     return powf(t, P.kexp - 1.f);
 }
 
-template <int D, int LG>
+// Smem layout for D, LG lane groups, CP column parts (128 * CP threads) and NSB stages
+// of the chunk-summary operands.
+template <int D, int LG, int CP, int NSB>
 struct TSmem {
     static constexpr int kNP = 128 / LG;              // pairs per CTA
     static constexpr int kDh = D / 64;
@@ -90,12 +90,12 @@ struct TSmem {
     static constexpr int kA = 0;
     static constexpr int kB = kA + kDh * kAregion;    // [stage][hi, lo][kDh regions]
     static constexpr int kBstage = 2 * kDh * kBregion;
-    static constexpr int kMmaEnd = kB + 2 * kBstage;
+    static constexpr int kMmaEnd = kB + NSB * kBstage;
     // solve phase (reuses the MMA region once every logit is in TMEM)
     static constexpr int kHist = 0;                          // [kBins][NP] uint32
     static constexpr int kXch = kHist + kBins * kNP * 4;     // [2 parity][kXchVals][512] float
     static constexpr int kTr = kXch + 2 * kXchVals * 512 * 4;  // [16 warps][32 lanes][33] float transpose
-    static constexpr int kSolveEnd = kTr + 16 * 32 * 33 * 4;
+    static constexpr int kSolveEnd = kTr + 4 * CP * 32 * 33 * 4;
     static constexpr int kData = kMmaEnd > kSolveEnd ? kMmaEnd : kSolveEnd;
     static constexpr int kBars = kData;                      // q_full, k_full[2], mma_done[2], all_done
     static constexpr int kSlot = kBars + 6 * 8;
@@ -148,10 +148,10 @@ __global__ void __launch_bounds__(256) kbar_split_kernel(const float *__restrict
 // slots in the same order (so the threads of a pair hold identical results).  Bit k of
 // max_bits / min_bits selects max / min for value k (sum otherwise).  `parity`
 // alternates the buffer so one barrier per exchange suffices.
-template <int NV, int LG>
+template <int NV, int LG, int CP>
 __device__ __forceinline__ void pair_reduce(float *xch, int parity, int slot, int p, float (&v)[NV], int max_bits,
                                             int min_bits) {
-    constexpr int kNP = 128 / LG, kSlots = 4 * LG;
+    constexpr int kNP = 128 / LG, kSlots = CP * LG;
     float *buf = xch + (size_t)parity * kXchVals * 512;
 #pragma unroll
     for (int k = 0; k < NV; ++k) buf[k * 512 + slot * kNP + p] = v[k];
@@ -168,11 +168,13 @@ __device__ __forceinline__ void pair_reduce(float *xch, int parity, int slot, in
     }
 }
 
-template <int D, int KINT, int LG>
-__global__ void __launch_bounds__(kSelT, 1) select_tile_kernel(const __grid_constant__ CUtensorMap tmQ,
-                                                               const uint8_t *__restrict__ ksplit, Geom G, TileP P,
-                                                               TileOut out) {
-    using S = TSmem<D, LG>;
+template <int D, int KINT, int LG, int CP, int NSB>
+__global__ void __launch_bounds__(128 * CP, 4 / CP) select_tile_kernel(const __grid_constant__ CUtensorMap tmQ,
+                                                                      const uint8_t *__restrict__ ksplit, Geom G,
+                                                                      TileP P, TileOut out, uint32_t ncols) {
+    using S = TSmem<D, LG, CP, NSB>;
+    constexpr int kT = 128 * CP;       // 4 TMEM lane quadrants x CP column parts
+    constexpr int kQB = 4 / CP;        // 32-column blocks per chunk tile and thread
     constexpr int kNP = S::kNP;
     extern __shared__ uint8_t tsm_raw[];
     uint8_t *sm = tsm_raw + ((1024 - (smem_u32(tsm_raw) & 1023)) & 1023);
@@ -188,7 +190,7 @@ __global__ void __launch_bounds__(kSelT, 1) select_tile_kernel(const __grid_cons
     const int qd = warp & 3, cp = warp >> 2;  // TMEM lane quadrant; column part
     const int L = qd * 32 + lane;             // TMEM lane
     const int lg = L / kNP, p = L % kNP;      // lane group; pair
-    const int slot = lg * 4 + cp;
+    const int slot = lg * CP + cp;
     const int g = G.g;
     const int npos = kNP / g;                 // query positions per CTA
     const int64_t t = (int64_t)gridDim.x - 1 - blockIdx.x;  // latest (longest) rows first
@@ -209,13 +211,13 @@ __global__ void __launch_bounds__(kSelT, 1) select_tile_kernel(const __grid_cons
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, (uint32_t)kTmemCols);
+        tmem_alloc(tmem_slot, ncols);
         tmem_relinquish();
     }
     // zero rows of the A operand (generic-proxy stores, made visible to the MMA below)
     constexpr int kZeroRows = S::kArows - kNP;                   // 0 when LG == 1
     constexpr int kZeroUnits = (kZeroRows > 0 ? kZeroRows : 1) * 8;  // 16-byte units per region
-    for (int u = threadIdx.x; kZeroRows > 0 && u < S::kDh * kZeroUnits; u += kSelT) {
+    for (int u = threadIdx.x; kZeroRows > 0 && u < S::kDh * kZeroUnits; u += kT) {
         const int dh = u / kZeroUnits, rem = u % kZeroUnits;
         int row = rem / 8;
         if (row >= 128 - kNP) row += kNP;  // skip the Q rows
@@ -243,12 +245,12 @@ __global__ void __launch_bounds__(kSelT, 1) select_tile_kernel(const __grid_cons
                 bulk_load(sm + S::kB + s * S::kBstage, src, 2 * S::kDh * S::kBregion, k_full + s);
             };
             load_b(0, 0);
-            if (n_ct > 1) load_b(1, 1);
+            if (NSB > 1 && n_ct > 1) load_b(1, 1);
             bool ok = mbar_wait_ns(q_full, 0, kTileWaitNs);
             constexpr uint32_t id = idesc_bf16_f32(128, kChunkTile, 0, 0);
             for (int k = 0; ok && k < n_ct; ++k) {
-                const int s = k & 1;
-                if (!(ok = mbar_wait_ns(k_full + s, (k >> 1) & 1, kTileWaitNs))) break;
+                const int s = k % NSB;
+                if (!(ok = mbar_wait_ns(k_full + s, (k / NSB) & 1, kTileWaitNs))) break;
                 tc_fence_after();
                 const int klg = k % LG;
                 const uint32_t qb = smem_u32(sm + S::kA) + (uint32_t)((128 - kNP - klg * kNP) * 128);
@@ -270,10 +272,11 @@ __global__ void __launch_bounds__(kSelT, 1) select_tile_kernel(const __grid_cons
                     mma_ss(dcol, smem_desc_sw128(qa, 16, 1024), smem_desc_sw128(ka, 16, 1024), id, 1u);
                 }
                 mma_commit(mma_done + s);
-                // the stage of tile k-1 takes tile k+1 once MMA k-1 has read it
-                if (k >= 1 && k + 1 < n_ct) {
-                    if (!(ok = mbar_wait_ns(mma_done + (s ^ 1), ((k - 1) >> 1) & 1, kTileWaitNs))) break;
-                    load_b(k + 1, s ^ 1);
+                // the stage of tile k+1-NSB takes tile k+1 once that tile's MMA has read it
+                if (k + 1 < n_ct && k + 1 >= NSB) {
+                    const int kp = k + 1 - NSB, sp = kp % NSB;
+                    if (!(ok = mbar_wait_ns(mma_done + sp, (kp / NSB) & 1, kTileWaitNs))) break;
+                    load_b(k + 1, sp);
                 }
             }
             mma_commit(all_done);  // arrives when every MMA issued above has completed
@@ -283,21 +286,25 @@ __global__ void __launch_bounds__(kSelT, 1) select_tile_kernel(const __grid_cons
     if (n_ct > 0) mbar_wait_ns(all_done, 0, kTileWaitNs);
     tc_fence_after();
     __syncthreads();  // the MMA staging memory is reused below
-    for (int u = threadIdx.x; u < kBins * kNP; u += kSelT) hist[u] = 0u;
+    for (int u = threadIdx.x; u < kBins * kNP; u += kT) hist[u] = 0u;
 
     // ---------------------------------------------------------------- tau per pair
-    // this thread's column blocks: j = 0 .. nj-1 at TMEM columns j*128 + cp*32, chunks
-    // (j*LG + lg)*128 + cp*32 + x; the bound is uniform across the warp
+    // this thread's column blocks: jb = 0 .. nb-1, tile j = jb / kQB and block q = cp + CP (jb %
+    // kQB) at TMEM columns j*128 + q*32, chunks (j*LG + lg)*128 + q*32 + x; the bound is
+    // uniform across the warp
     const int nj = lg < n_ct ? (n_ct - lg + LG - 1) / LG : 0;
+    const int nb = nj * kQB;
+    auto blk_col = [&](int jb) -> uint32_t { return (uint32_t)((jb / kQB) * 128 + (cp + CP * (jb % kQB)) * 32); };
+    auto blk_chunk = [&](int jb) -> int { return ((jb / kQB) * LG + lg) * 128 + (cp + CP * (jb % kQB)) * 32; };
     const float xs = P.am1 * P.scale;  // x = (alpha - 1) * gamma / sqrt(d) * <q, k̄>
     int parity = 0;
     // pass 0: x written back over the logits (-inf past the row's visible chunks), max
     float mx = -INFINITY;
-    for (int j = 0; j < nj; ++j) {
+    for (int jb = 0; jb < nb; ++jb) {
         uint32_t u[32];
-        const uint32_t col = (uint32_t)(j * 128 + cp * 32);
+        const uint32_t col = blk_col(jb);
         tmem_ld32(tmem + lane_off + col, u);
-        const int lim = nvis - ((j * LG + lg) * 128 + cp * 32);
+        const int lim = nvis - blk_chunk(jb);
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
             const float xv = x < lim ? xs * __uint_as_float(u[x]) : -INFINITY;
@@ -309,7 +316,7 @@ __global__ void __launch_bounds__(kSelT, 1) select_tile_kernel(const __grid_cons
     tmem_wait_st();
     {
         float v[1] = {mx};
-        pair_reduce<1, LG>(xch, parity, slot, p, v, 1, 0);
+        pair_reduce<1, LG, CP>(xch, parity, slot, p, v, 1, 0);
         parity ^= 1;
         mx = v[0];
     }
@@ -317,9 +324,9 @@ __global__ void __launch_bounds__(kSelT, 1) select_tile_kernel(const __grid_cons
     float lo = mx - 1.f;
     float hi = nvis > 0 ? mx - powf((float)nvis, 1.f - P.alpha) : 0.f;
     // histogram of x over [mx - 1, mx), 32 bins per pair
-    for (int j = 0; j < nj; ++j) {
+    for (int jb = 0; jb < nb; ++jb) {
         uint32_t u[32];
-        tmem_ld32(tmem + lane_off + (uint32_t)(j * 128 + cp * 32), u);
+        tmem_ld32(tmem + lane_off + blk_col(jb), u);
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
             const float y = __uint_as_float(u[x]) - lo;
@@ -384,9 +391,9 @@ __global__ void __launch_bounds__(kSelT, 1) select_tile_kernel(const __grid_cons
         // a warp whose pairs are all settled skips the pass (the threads of a pair share
         // their decisions, so the pair's other warps skip it too)
         if (!__all_sync(0xffffffffu, done)) {
-            for (int j = 0; j < nj; ++j) {
+            for (int jb = 0; jb < nb; ++jb) {
                 uint32_t u[32];
-                tmem_ld32(tmem + lane_off + (uint32_t)(j * 128 + cp * 32), u);
+                tmem_ld32(tmem + lane_off + blk_col(jb), u);
 #pragma unroll
                 for (int x = 0; x < 32; ++x) {
                     const float xv = __uint_as_float(u[x]);
@@ -408,7 +415,7 @@ __global__ void __launch_bounds__(kSelT, 1) select_tile_kernel(const __grid_cons
                 }
             }
         }
-        pair_reduce<kXchVals, LG>(xch, parity, slot, p, acc, 1 << 4, 1 << 3);
+        pair_reduce<kXchVals, LG, CP>(xch, parity, slot, p, acc, 1 << 4, 1 << 3);
         parity ^= 1;
         if (done) continue;
         const int cnt = (int)acc[2];
@@ -473,10 +480,10 @@ __global__ void __launch_bounds__(kSelT, 1) select_tile_kernel(const __grid_cons
     float *tr = reinterpret_cast<float *>(sm + S::kTr) + warp * 32 * 33;
     const int gbase = lane - hh;  // lane of the row's first head
     float lsum = 0.f, lcnt = 0.f;
-    for (int j = 0; j < nj; ++j) {
+    for (int jb = 0; jb < nb; ++jb) {
         uint32_t u[32];
-        tmem_ld32(tmem + lane_off + (uint32_t)(j * 128 + cp * 32), u);
-        const int c0 = (j * LG + lg) * 128 + cp * 32;
+        tmem_ld32(tmem + lane_off + blk_col(jb), u);
+        const int c0 = blk_chunk(jb);
 #pragma unroll
         for (int x = 0; x < 32; ++x) tr[lane * 33 + x] = __uint_as_float(u[x]) - tau_r;
         __syncwarp();
@@ -514,7 +521,7 @@ __global__ void __launch_bounds__(kSelT, 1) select_tile_kernel(const __grid_cons
     }
     {
         float v[2] = {lsum, lcnt};
-        pair_reduce<2, LG>(xch, parity, slot, p, v, 0, 0);
+        pair_reduce<2, LG, CP>(xch, parity, slot, p, v, 0, 0);
         parity ^= 1;
         lsum = v[0];
         lcnt = v[1];
@@ -531,23 +538,27 @@ __global__ void __launch_bounds__(kSelT, 1) select_tile_kernel(const __grid_cons
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, (uint32_t)kTmemCols);
+        tmem_dealloc(tmem, ncols);
     }
 }
 
-template <int D, int KINT, int LG>
+template <int D, int KINT, int LG, int CP, int NSB>
 cudaError_t launch_sel(const CUtensorMap &tmQ, const uint8_t *ksplit, const Geom &G, const TileP &P,
                        const TileOut &o, cudaStream_t st) {
-    using S = TSmem<D, LG>;
+    using S = TSmem<D, LG, CP, NSB>;
     const size_t smem = S::kTotal + 1024;
-    cudaError_t e = cudaFuncSetAttribute(select_tile_kernel<D, KINT, LG>,
+    cudaError_t e = cudaFuncSetAttribute(select_tile_kernel<D, KINT, LG, CP, NSB>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int npos = (128 / LG) / G.g;
     const int64_t nblk = (G.nq + npos - 1) / npos;
     if (nblk > 0x7fffffff) return cudaErrorInvalidValue;
+    // tensor-memory columns: the chunk tiles of one lane group, 128 each (a power of two)
+    const int n_ct_all = (G.n_chunks + kChunkTile - 1) / kChunkTile;
+    uint32_t ncols = 32;
+    while (ncols < (uint32_t)(((n_ct_all + LG - 1) / LG) * kChunkTile)) ncols *= 2;
     dim3 grid((unsigned)nblk, (unsigned)G.hkv, (unsigned)G.b);
-    select_tile_kernel<D, KINT, LG><<<grid, kSelT, smem, st>>>(tmQ, ksplit, G, P, o);
+    select_tile_kernel<D, KINT, LG, CP, NSB><<<grid, 128 * CP, smem, st>>>(tmQ, ksplit, G, P, o, ncols);
     return cudaGetLastError();
 }
 
@@ -558,9 +569,12 @@ cudaError_t launch_sel_lg(const TView &Q, const uint8_t *ksplit, const Geom &G, 
     const int npos = (128 / LG) / G.g;
     CUtensorMap tmQ;
     if (!make_map_bf16(&tmQ, Q, G.b, G.nq, G.hq, G.d, G.g, npos)) return cudaErrorInvalidValue;
-    if (LG == 1) return launch_sel<D, KINT, 1>(tmQ, ksplit, G, P, o, st);
-    if (LG == 2) return launch_sel<D, KINT, 2>(tmQ, ksplit, G, P, o, st);
-    return launch_sel<D, KINT, 4>(tmQ, ksplit, G, P, o, st);
+    // up to two chunk tiles: half the threads, one operand stage and at most 256 tensor-memory
+    // columns, so that two CTAs share an SM and one's logits overlap the other's passes
+    if (G.n_chunks <= 2 * kChunkTile) return launch_sel<D, KINT, 1, 2, 1>(tmQ, ksplit, G, P, o, st);
+    if (LG == 1) return launch_sel<D, KINT, 1, 4, 2>(tmQ, ksplit, G, P, o, st);
+    if (LG == 2) return launch_sel<D, KINT, 2, 4, 2>(tmQ, ksplit, G, P, o, st);
+    return launch_sel<D, KINT, 4, 4, 2>(tmQ, ksplit, G, P, o, st);
 }
 
 }  // namespace
