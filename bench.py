@@ -300,7 +300,9 @@ def run_ours(args, rank, world, device):
         "roofline": roof,
         "e2e": {"value": round(per(ms_e2e), 3), "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(ms_e2e, 4)},
-        "gpu_launches": args.steps * 4,  # pool|select, compact, stage 2 (+ combine for decode)
+        # per step: prefill pool_keys, kbar_split, select_tile, regroup_compact, attn_tc;
+        # decode (summaries cached) kbar_split, select_tile, compact, attn_decode, combine
+        "gpu_launches": args.steps * 5,
         "clocks": cs.summary(),
     }
     return res, (q, k, v, w, alpha, sigma)
