@@ -8,16 +8,20 @@
 // causal.  Online softmax in the exp2 domain with fp32 statistics.
 //
 // One CTA per (batch, kv head, query tile of 128/g positions x g heads = 128 rows),
-// the heaviest tiles (latest, causal) of all heads first, two CTAs resident per SM so that one
-// CTA's MMAs overlap the other's softmax.  Warp roles (192 threads):
-//   warp 0     TMA producer: Q tile once; per step of 128 keys the listed K and V
-//              blocks (one TMA box per chunk and 64-column half, 128-byte swizzle)
-//              and the step's bias rows (bulk copy);
-//   warp 1     TMEM allocator (256 columns: S/P and O) and MMA issuer (one thread):
-//              S_j = Q K_j^T  (SS, M=128 N=128 K=d) into TMEM,
+// the heaviest tiles (latest, causal) of all heads first, two CTAs resident per SM.  A step
+// covers 64 keys (one or more listed chunks, or half of a 128-key chunk); S is
+// double-buffered in tensor memory, so the MMA of step j+1 runs during the softmax of
+// step j.  Warp roles (192 threads):
+//   warp 0     TMA producer: Q tile once; per step the listed K and V blocks (one TMA
+//              box per chunk, or half chunk, and 64-column half, 128-byte swizzle) into
+//              two-stage rings, and the step's bias rows (bulk copy);
+//   warp 1     TMEM allocator (256 columns: S[0], S[1] of 64 columns each, O) and MMA
+//              issuer (one thread), order S_0, S_1, PV_0, S_2, PV_1, ...:
+//              S_j = Q K_j^T  (SS, M=128 N=64 K=d) into S[j % 2] once PV_{j-2}, the last
+//              reader of that buffer, has completed;
 //              O  += P_j V_j  (TS: P read from TMEM, V from smem as an MN-major operand);
 //   warps 2-5  softmax: thread = TMEM lane = tile row; two passes over S_j in TMEM
-//              (row max, then exp2 / sum / bf16 P written over S_j), bias added and
+//              (row max, then exp2 / sum / bf16 P written over S_j's first 32 columns), bias added and
 //              keys masked only on steps that hold a diagonal or partial chunk; after
 //              the first step a single pass on the running maximum, redone as two
 //              passes only if a row's maximum grows by more than 2^16 (O is then
@@ -36,8 +40,8 @@ namespace {
 
 constexpr int kThreads = 192;
 constexpr int kRows = 128;      // MMA M
-constexpr int kStepKeys = 128;  // keys per step = MMA N of S and K of PV
-constexpr int kNS = 1;          // K / V stages (two CTAs per SM share the SM's shared memory)
+constexpr int kStepKeys = 64;   // keys per step = MMA N of S and K of PV
+constexpr int kNS = 2;          // K / V stages
 constexpr int kNM = 2;          // bias / id stages
 constexpr uint32_t kTmemCols = 256;
 // The running maximum (exp2 domain) is kept until a step's maximum exceeds it by more
@@ -65,18 +69,21 @@ __device__ __forceinline__ float ex2(float x) {
 
 template <int D, int BLK>
 struct Smem {
-    static constexpr int kRegion = kRows * 128;                 // bytes of one 64-column, 128-row swizzled region
+    static constexpr int kRegion = kRows * 128;                 // bytes of one 64-column, 128-row swizzled region (Q)
+    static constexpr int kSRegion = kStepKeys * 128;            // one 64-column region of a K or V stage
     static constexpr int kDh = D / 64;                          // regions per operand
-    static constexpr int kE = kStepKeys / BLK;                  // list entries per step
+    static constexpr int kE = BLK < kStepKeys ? kStepKeys / BLK : 1;   // list entries per step
+    static constexpr int kSub = BLK > kStepKeys ? BLK / kStepKeys : 1; // steps per list entry
+    static constexpr int kRowsE = BLK < kStepKeys ? BLK : kStepKeys;   // keys of one entry in a step
     static constexpr int kQ = 0;
     static constexpr int kK = kQ + kDh * kRegion;
-    static constexpr int kV = kK + kNS * kDh * kRegion;
-    static constexpr int kBias = kV + kNS * kDh * kRegion;      // [kNM][kE * 128] floats (tile_rows <= 128)
+    static constexpr int kV = kK + kNS * kDh * kSRegion;
+    static constexpr int kBias = kV + kNS * kDh * kSRegion;     // [kNM][kE * 128] floats (tile_rows <= 128)
     static constexpr int kIds = kBias + kNM * kE * 128 * 4;     // [kNM][kE] int
     static constexpr int kBars = (kIds + kNM * kE * 4 + 7) & ~7;
     // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], m_full[NM], m_empty[NM],
-    //           s_full, p_full, pv_done, fin
-    static constexpr int kNumBars = 1 + 4 * kNS + 2 * kNM + 3 + 1;
+    //           s_full[2], p_full[2], pv_done[2], fin
+    static constexpr int kNumBars = 1 + 4 * kNS + 2 * kNM + 6 + 1;
     static constexpr int kMisc = kBars + kNumBars * 8;          // tmem base, abort flag, p_min
     static constexpr int kTotal = kMisc + 16 + 8;
 };
@@ -129,7 +136,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
 #pragma unroll
         for (int e = 0; e < Smem<D, BLK>::kE; ++e) ids_pre[e] = e < L.cap ? L.ids[tile_idx * L.cap + e] : 0;
     }
-    const int nsteps = (count + S::kE - 1) / S::kE;
+    const int nsteps = S::kSub > 1 ? count * S::kSub : (count + S::kE - 1) / S::kE;
     const bool test_timeout = (flags & DASH_FLAG_TEST_TIMEOUT) != 0;
     const uint64_t limit_ns = test_timeout ? kWaitNsTest : kWaitNs;
 
@@ -143,9 +150,9 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
     B.m_full = B.v_empty + kNS;
     B.m_empty = B.m_full + kNM;
     B.s_full = B.m_empty + kNM;
-    B.p_full = B.s_full + 1;
-    B.pv_done = B.p_full + 1;
-    B.fin = B.pv_done + 1;
+    B.p_full = B.s_full + 2;
+    B.pv_done = B.p_full + 2;
+    B.fin = B.pv_done + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + S::kMisc);
     volatile int *abort = reinterpret_cast<volatile int *>(sm + S::kMisc + 4);
     long long *p_min_s = reinterpret_cast<long long *>(sm + S::kMisc + 8);
@@ -166,9 +173,11 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
             mbar_init(B.m_full + s, 1);
             mbar_init(B.m_empty + s, 128);
         }
-        mbar_init(B.s_full, 1);
-        mbar_init(B.p_full, 128);
-        mbar_init(B.pv_done, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(B.s_full + s, 1);
+            mbar_init(B.p_full + s, 128);
+            mbar_init(B.pv_done + s, 1);
+        }
         mbar_init(B.fin, 1);
         *abort = 0;
         fence_mbar_init();
@@ -181,8 +190,8 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem;        // S_j, then P_j (bf16) over its first 64 columns
-    const uint32_t tO = tmem + 128;  // O accumulator (D columns)
+    // S_j in columns (j % 2) * 64.., then P_j (bf16) over its first 32; O from column 128
+    const uint32_t tO = tmem + 128;
 
     if (warp == 0) {
         // ------------------------------------------------------------- producer
@@ -199,12 +208,14 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
             const float *bias_g = L.bias + tile_idx * (size_t)L.cap * T;
             int issued_m = 0, issued_k = 0, issued_v = 0;  // steps whose copies were issued
             for (int j = 0; j < nsteps; ++j) {
-                const int e0 = j * S::kE;
-                const int ne = min(S::kE, count - e0);
+                // the step's entries e0.. (ne of them) and its first key within them
+                const int e0 = S::kSub > 1 ? j / S::kSub : j * S::kE;
+                const int ne = S::kSub > 1 ? 1 : min(S::kE, count - e0);
+                const int koff = S::kSub > 1 ? (j % S::kSub) * kStepKeys : 0;
                 const int ms = j % kNM, ks = j % kNS;
                 if (!wait_bar(B.m_empty + ms, ((j / kNM) & 1) ^ 1, limit_ns, abort)) break;
                 int *ids_st = ids_s + ms * S::kE;
-                if (j == 0) {
+                if (e0 == 0) {
 #pragma unroll
                     for (int e = 0; e < S::kE; ++e)
                         if (e < ne) ids_st[e] = ids_pre[e];
@@ -215,18 +226,18 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
                 bulk_load(bias_s + ms * S::kE * 128, bias_g + (size_t)e0 * T, (uint32_t)(ne * T * 4), B.m_full + ms);
                 issued_m = j + 1;
                 if (!wait_bar(B.k_empty + ks, ((j / kNS) & 1) ^ 1, limit_ns, abort)) break;
-                mbar_arrive_expect_tx(B.k_full + ks, (uint32_t)(ne * S::kDh * BLK * 128));
+                mbar_arrive_expect_tx(B.k_full + ks, (uint32_t)(ne * S::kDh * S::kRowsE * 128));
                 for (int e = 0; e < ne; ++e)
                     for (int dh = 0; dh < S::kDh; ++dh)
-                        tma_load_4d(sm + S::kK + (ks * S::kDh + dh) * S::kRegion + e * BLK * 128, &tp.tmK,
-                                    B.k_full + ks, dh * 64, r, ids_st[e] * BLK, (int)b);
+                        tma_load_4d(sm + S::kK + (ks * S::kDh + dh) * S::kSRegion + e * S::kRowsE * 128, &tp.tmK,
+                                    B.k_full + ks, dh * 64, r, ids_st[e] * BLK + koff, (int)b);
                 issued_k = j + 1;
                 if (!wait_bar(B.v_empty + ks, ((j / kNS) & 1) ^ 1, limit_ns, abort)) break;
-                mbar_arrive_expect_tx(B.v_full + ks, (uint32_t)(ne * S::kDh * BLK * 128));
+                mbar_arrive_expect_tx(B.v_full + ks, (uint32_t)(ne * S::kDh * S::kRowsE * 128));
                 for (int e = 0; e < ne; ++e)
                     for (int dh = 0; dh < S::kDh; ++dh)
-                        tma_load_4d(sm + S::kV + (ks * S::kDh + dh) * S::kRegion + e * BLK * 128, &tp.tmV,
-                                    B.v_full + ks, dh * 64, r, ids_st[e] * BLK, (int)b);
+                        tma_load_4d(sm + S::kV + (ks * S::kDh + dh) * S::kSRegion + e * S::kRowsE * 128, &tp.tmV,
+                                    B.v_full + ks, dh * 64, r, ids_st[e] * BLK + koff, (int)b);
                 issued_v = j + 1;
             }
             if (*abort) {
@@ -249,31 +260,39 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
             const uint32_t k_base = smem_u32(sm + S::kK);
             const uint32_t v_base = smem_u32(sm + S::kV);
             bool ok = nsteps == 0 || wait_bar(B.q_full, 0, limit_ns, abort);
-            for (int j = 0; ok && j < nsteps; ++j) {
+            // S_j into S[j % 2]: its K stage, and for j >= 2 the completion of PV_{j-2}
+            auto issue_s = [&](int j) -> bool {
                 const int ks = j % kNS;
-                const int ne = min(S::kE, count - j * S::kE);
-                if (!(ok = wait_bar(B.k_full + ks, (j / kNS) & 1, limit_ns, abort))) break;
-                // the S / P buffer is free once PV_{j-1} has read P_{j-1}
-                if (j > 0 && !(ok = wait_bar(B.pv_done, (j - 1) & 1, limit_ns, abort))) break;
+                if (j >= 2 && !wait_bar(B.pv_done + (j & 1), ((j - 2) >> 1) & 1, limit_ns, abort)) return false;
+                if (!wait_bar(B.k_full + ks, (j / kNS) & 1, limit_ns, abort)) return false;
                 tc_fence_after();
+                const uint32_t tS = tmem + (uint32_t)((j & 1) * kStepKeys);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t qa = q_base + (kk / 4) * S::kRegion + (kk % 4) * 32;
-                    const uint32_t kb = k_base + (ks * S::kDh + kk / 4) * S::kRegion + (kk % 4) * 32;
+                    const uint32_t kb = k_base + (ks * S::kDh + kk / 4) * S::kSRegion + (kk % 4) * 32;
                     mma_ss(tS, smem_desc_sw128(qa, 16, 1024), smem_desc_sw128(kb, 16, 1024), idS, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(B.s_full);
+                mma_commit(B.s_full + (j & 1));
                 mma_commit(B.k_empty + ks);
-                if (!(ok = wait_bar(B.p_full, j & 1, limit_ns, abort))) break;
+                return true;
+            };
+            for (int j = 0; ok && j < min(nsteps, 2); ++j) ok = issue_s(j);
+            for (int j = 0; ok && j < nsteps; ++j) {
+                const int ks = j % kNS;
+                const int ne = S::kSub > 1 ? 1 : min(S::kE, count - j * S::kE);
+                if (!(ok = wait_bar(B.p_full + (j & 1), (j >> 1) & 1, limit_ns, abort))) break;
                 if (!(ok = wait_bar(B.v_full + ks, (j / kNS) & 1, limit_ns, abort))) break;
                 tc_fence_after();
-                const int nks = ne * BLK / 16;
+                const uint32_t tS = tmem + (uint32_t)((j & 1) * kStepKeys);
+                const int nks = ne * S::kRowsE / 16;
                 for (int kk = 0; kk < nks; ++kk) {
-                    const uint32_t vb = v_base + (ks * S::kDh) * S::kRegion + kk * 2048;
-                    mma_ts(tO, tS + kk * 8, smem_desc_sw128(vb, S::kRegion, 1024), idPV, (j > 0 || kk > 0) ? 1u : 0u);
+                    const uint32_t vb = v_base + (ks * S::kDh) * S::kSRegion + kk * 2048;
+                    mma_ts(tO, tS + kk * 8, smem_desc_sw128(vb, S::kSRegion, 1024), idPV, (j > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(B.v_empty + ks);
-                mma_commit(B.pv_done);
+                mma_commit(B.pv_done + (j & 1));
+                if (j + 2 < nsteps) ok = issue_s(j + 2);
             }
             // every MMA this thread issued has completed before TMEM is freed
             mma_commit(B.fin);
@@ -313,7 +332,9 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
         // made uniform across the warp (__any_sync / __all_sync).
         for (int j = 0; j < nsteps; ++j) {
             const int ms = j % kNM;
-            const int ne = min(S::kE, count - j * S::kE);
+            const int ne = S::kSub > 1 ? 1 : min(S::kE, count - j * S::kE);
+            const int koff = S::kSub > 1 ? (j % S::kSub) * kStepKeys : 0;  // first key of the step in its chunk
+            const uint32_t tS = tmem + (uint32_t)((j & 1) * kStepKeys);
             ok = __all_sync(0xffffffffu, wait_bar(B.m_full + ms, (j / kNM) & 1, limit_ns, abort));
             if (!ok) break;
             // per-entry constants of this step: bias (exp2 domain) and, for masking, the
@@ -326,16 +347,16 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
             for (int e = 0; e < S::kE; ++e) {
                 const int id = e < ne ? ids_s[ms * S::kE + e] : 0;
                 bl2[e] = e < ne ? bias_s[ms * S::kE * 128 + e * T + pos] * 1.4426950408889634f : -INFINITY;
-                lim[e] = e < ne ? max(0, min(BLK, vis_end - id * BLK)) : 0;
+                lim[e] = e < ne ? max(0, min(S::kRowsE, vis_end - (id * BLK + koff))) : 0;
                 // a chunk needs per-key masks if it reaches past the sequence or past the
                 // smallest row position of the tile (it is some row's diagonal chunk)
                 if (e < ne) {
-                    const int64_t last_key = (int64_t)id * BLK + BLK - 1;
+                    const int64_t last_key = (int64_t)id * BLK + koff + S::kRowsE - 1;
                     need_mask |= last_key >= G.nk || (G.causal && last_key > p_min);
                 }
             }
             mbar_arrive(B.m_empty + ms);
-            ok = __all_sync(0xffffffffu, wait_bar(B.s_full, j & 1, limit_ns, abort));
+            ok = __all_sync(0xffffffffu, wait_bar(B.s_full + (j & 1), (j >> 1) & 1, limit_ns, abort));
             if (!ok) break;
             tc_fence_after();
             // Single pass on the running maximum of the earlier steps: p = 2^(s * scale +
@@ -348,20 +369,20 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
                 float cbm[S::kE];
 #pragma unroll
                 for (int e = 0; e < S::kE; ++e) cbm[e] = row_ok ? bl2[e] - m_run : -INFINITY;
-                uint32_t pk[64];
+                uint32_t pk[32];
                 float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int qc = 0; qc < 8; ++qc) {
+                for (int qc = 0; qc < 4; ++qc) {
                     uint32_t u[16];
                     tmem_ld16(tS + lane_off + qc * 16, u);
 #pragma unroll
                     for (int x = 0; x < 8; ++x) {
                         const int kc = qc * 16 + 2 * x;
-                        float v0 = fmaf(__uint_as_float(u[2 * x]), sl2, cbm[kc / BLK]);
-                        float v1 = fmaf(__uint_as_float(u[2 * x + 1]), sl2, cbm[(kc + 1) / BLK]);
+                        float v0 = fmaf(__uint_as_float(u[2 * x]), sl2, cbm[kc / S::kRowsE]);
+                        float v1 = fmaf(__uint_as_float(u[2 * x + 1]), sl2, cbm[(kc + 1) / S::kRowsE]);
                         if (need_mask) {  // select before exp2: S outside the list may be any bit pattern
-                            v0 = (kc % BLK) < lim[kc / BLK] ? v0 : -INFINITY;
-                            v1 = ((kc + 1) % BLK) < lim[(kc + 1) / BLK] ? v1 : -INFINITY;
+                            v0 = (kc % S::kRowsE) < lim[kc / S::kRowsE] ? v0 : -INFINITY;
+                            v1 = ((kc + 1) % S::kRowsE) < lim[(kc + 1) / S::kRowsE] ? v1 : -INFINITY;
                         }
                         const float p0 = ex2(v0), p1 = ex2(v1);
                         ps[x & 3] += p0 + p1;
@@ -372,8 +393,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
                 // 2^kRescaleL2 (then so does every p); a sum that overflowed is not finite
                 const float psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
                 if (!__any_sync(0xffffffffu, !(psum <= kRescaleP))) {
-                    tmem_st32(tS + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-                    tmem_st32(tS + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+                    tmem_st32(tS + lane_off, pk);
                     l_run += psum;
                     step_done = true;
                 }
@@ -382,14 +402,15 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
             // pass 1: row maximum of the biased, masked logits (exp2 domain)
             float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int qc = 0; qc < 4; ++qc) {
+            for (int qc = 0; qc < 2; ++qc) {
                 uint32_t u[32];
                 tmem_ld32(tS + lane_off + qc * 32, u);
 #pragma unroll
                 for (int x = 0; x < 32; ++x) {
                     const int kc = qc * 32 + x;
-                    const float v = fmaf(__uint_as_float(u[x]), sl2, bl2[kc / BLK]);
-                    mq[x & 3] = fmaxf(mq[x & 3], (!need_mask || (kc % BLK) < lim[kc / BLK]) ? v : -INFINITY);
+                    const float v = fmaf(__uint_as_float(u[x]), sl2, bl2[kc / S::kRowsE]);
+                    mq[x & 3] = fmaxf(mq[x & 3],
+                                      (!need_mask || (kc % S::kRowsE) < lim[kc / S::kRowsE]) ? v : -INFINITY);
                 }
             }
             float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
@@ -408,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
             }
             if (j > 0 && __any_sync(0xffffffffu, rescale)) {
                 // O must hold every PV up to step j-1 before it is rescaled
-                ok = __all_sync(0xffffffffu, wait_bar(B.pv_done, (j - 1) & 1, limit_ns, abort));
+                ok = __all_sync(0xffffffffu, wait_bar(B.pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, limit_ns, abort));
                 if (!ok) break;
                 tc_fence_after();
 #pragma unroll
@@ -428,18 +449,18 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
             for (int e = 0; e < S::kE; ++e) cbm[e] = live ? bl2[e] - m_run : -INFINITY;
             float pq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int qc = 0; qc < 4; ++qc) {
+            for (int qc = 0; qc < 2; ++qc) {
                 uint32_t u[32];
                 tmem_ld32(tS + lane_off + qc * 32, u);
                 uint32_t pk[16];
 #pragma unroll
                 for (int x = 0; x < 16; ++x) {
                     const int kc = qc * 32 + 2 * x;
-                    float v0 = fmaf(__uint_as_float(u[2 * x]), sl2, cbm[kc / BLK]);
-                    float v1 = fmaf(__uint_as_float(u[2 * x + 1]), sl2, cbm[(kc + 1) / BLK]);
+                    float v0 = fmaf(__uint_as_float(u[2 * x]), sl2, cbm[kc / S::kRowsE]);
+                    float v1 = fmaf(__uint_as_float(u[2 * x + 1]), sl2, cbm[(kc + 1) / S::kRowsE]);
                     if (need_mask) {  // select before exp2: S outside the list may be any bit pattern
-                        v0 = (kc % BLK) < lim[kc / BLK] ? v0 : -INFINITY;
-                        v1 = ((kc + 1) % BLK) < lim[(kc + 1) / BLK] ? v1 : -INFINITY;
+                        v0 = (kc % S::kRowsE) < lim[kc / S::kRowsE] ? v0 : -INFINITY;
+                        v1 = ((kc + 1) % S::kRowsE) < lim[(kc + 1) / S::kRowsE] ? v1 : -INFINITY;
                     }
                     const float p0 = ex2(v0), p1 = ex2(v1);
                     pq[x & 3] += p0 + p1;
@@ -453,13 +474,14 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
             }  // two-pass path
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(B.p_full);
+            mbar_arrive(B.p_full + (j & 1));
         }
         // epilogue: O / l -> bf16
         if (ok && !*abort) {
             bool have = true;
             if (nsteps > 0)
-                have = __all_sync(0xffffffffu, wait_bar(B.pv_done, (nsteps - 1) & 1, limit_ns, abort));
+                have = __all_sync(0xffffffffu, wait_bar(B.pv_done + ((nsteps - 1) & 1), ((nsteps - 1) >> 1) & 1,
+                                                        limit_ns, abort));
             tc_fence_after();
             if (have) {
                 __nv_bfloat16 *op = reinterpret_cast<__nv_bfloat16 *>(const_cast<void *>(O.p)) + b * O.s0 +
@@ -528,8 +550,9 @@ cudaError_t launch_attn_tc(const TView &Q, const TView &K, const TView &V, const
     if (G.nq == 0 || G.b == 0) return cudaSuccess;
     TcParams tp;
     if (!make_map_bf16(&tp.tmQ, Q, G.b, G.nq, G.hq, G.d, G.g, G.tile_rows)) return cudaErrorInvalidValue;
-    if (!make_map_bf16(&tp.tmK, K, G.b, G.nk, G.hkv, G.d, 1, G.B)) return cudaErrorInvalidValue;
-    if (!make_map_bf16(&tp.tmV, V, G.b, G.nk, G.hkv, G.d, 1, G.B)) return cudaErrorInvalidValue;
+    const int box = G.B < kStepKeys ? G.B : kStepKeys;  // rows of one K / V box: a chunk or half of one
+    if (!make_map_bf16(&tp.tmK, K, G.b, G.nk, G.hkv, G.d, 1, box)) return cudaErrorInvalidValue;
+    if (!make_map_bf16(&tp.tmV, V, G.b, G.nk, G.hkv, G.d, 1, box)) return cudaErrorInvalidValue;
 #define DASH_TC_CASE(DD, BB) \
     if (G.d == DD && G.B == BB) return launch_t<DD, BB>(tp, Q, O, G, L, flags, st);
     DASH_TC_CASE(128, 64)
