@@ -92,25 +92,94 @@ struct Bars {
     uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *m_full, *m_empty, *s_full, *p_full, *pv_done, *fin;
 };
 
+// try_wait that lets the hardware suspend the thread for up to hint_ns while the phase
+// is incomplete (it resumes as soon as the phase completes), so that waiting warps do not
+// take issue slots from the softmax warps sharing their scheduler.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+#ifndef DASH_SLEEP_NS
+#define DASH_SLEEP_NS 100000
+#endif
+constexpr uint32_t kSleepNs = DASH_SLEEP_NS;  // longest single suspension of a waiting thread
+
 // Bounded wait.  Gives up after limit_ns (recording a device error and raising
 // the CTA's abort flag) or, when honor_abort is set, as soon as another role
 // has raised it.  Drain waits (copies or MMAs in flight) pass honor_abort = false.
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, uint64_t limit_ns, volatile int *abort,
                                          bool honor_abort = true) {
-    uint64_t t0 = 0;
-    for (uint32_t it = 0;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 0) {
-            const uint64_t now = gtimer();
-            if (it == 0) t0 = now;
-            else if (now - t0 > limit_ns) {
-                report_timeout();
-                *abort = 1;
-                return false;
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = gtimer();
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
+        if (gtimer() - t0 > limit_ns) {
+            report_timeout();
+            *abort = 1;
+            return false;
+        }
+        if (honor_abort && *abort) return false;
+    }
+}
+
+// Packed fp32 pairs (the f32x2 forms of fma / add on sm_100a): one instruction per two values.
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f32x2_split(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// One 64-key step of the single-pass softmax for this thread's row: p = 2^(s * sl2 + cbm)
+// from the step's S columns at taddr, packed to bf16 pairs in pk; returns the row's sum of
+// p.  kMask applies the per-entry key limits (keys past the list or the row's position).
+template <int kE, int kRowsE, bool kMask>
+__device__ __forceinline__ float exp_step(uint32_t taddr, float sl2, const float (&cbm)[kE], const int (&lim)[kE],
+                                          uint32_t (&pk)[32]) {
+    const uint64_t sc2 = f32x2(sl2, sl2);
+    uint64_t acc[2] = {f32x2(0.f, 0.f), f32x2(0.f, 0.f)};
+#pragma unroll
+    for (int qc = 0; qc < 4; ++qc) {
+        uint32_t u[16];
+        tmem_ld16(taddr + qc * 16, u);
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+            const int kc = qc * 16 + 2 * x;  // an entry spans an even number of keys: kc, kc + 1 share it
+            const float cb = cbm[kc / kRowsE];
+            float v0, v1;
+            f32x2_split(fma_f32x2(f32x2(__uint_as_float(u[2 * x]), __uint_as_float(u[2 * x + 1])), sc2, f32x2(cb, cb)),
+                        v0, v1);
+            if (kMask) {  // select before exp2: S outside the list may be any bit pattern
+                v0 = (kc % kRowsE) < lim[kc / kRowsE] ? v0 : -INFINITY;
+                v1 = ((kc + 1) % kRowsE) < lim[kc / kRowsE] ? v1 : -INFINITY;
             }
-            if (honor_abort && *abort) return false;
+            const float p0 = ex2(v0), p1 = ex2(v1);
+            acc[x & 1] = add_f32x2(acc[x & 1], f32x2(p0, p1));
+            pk[qc * 8 + x] = pack_bf16x2(p0, p1);
         }
     }
+    float a, b;
+    f32x2_split(add_f32x2(acc[0], acc[1]), a, b);
+    return a + b;
 }
 
 template <int D, int BLK>
@@ -370,28 +439,10 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
 #pragma unroll
                 for (int e = 0; e < S::kE; ++e) cbm[e] = row_ok ? bl2[e] - m_run : -INFINITY;
                 uint32_t pk[32];
-                float ps[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int qc = 0; qc < 4; ++qc) {
-                    uint32_t u[16];
-                    tmem_ld16(tS + lane_off + qc * 16, u);
-#pragma unroll
-                    for (int x = 0; x < 8; ++x) {
-                        const int kc = qc * 16 + 2 * x;
-                        float v0 = fmaf(__uint_as_float(u[2 * x]), sl2, cbm[kc / S::kRowsE]);
-                        float v1 = fmaf(__uint_as_float(u[2 * x + 1]), sl2, cbm[(kc + 1) / S::kRowsE]);
-                        if (need_mask) {  // select before exp2: S outside the list may be any bit pattern
-                            v0 = (kc % S::kRowsE) < lim[kc / S::kRowsE] ? v0 : -INFINITY;
-                            v1 = ((kc + 1) % S::kRowsE) < lim[(kc + 1) / S::kRowsE] ? v1 : -INFINITY;
-                        }
-                        const float p0 = ex2(v0), p1 = ex2(v1);
-                        ps[x & 3] += p0 + p1;
-                        pk[qc * 8 + x] = pack_bf16x2(p0, p1);
-                    }
-                }
+                const float psum = need_mask ? exp_step<S::kE, S::kRowsE, true>(tS + lane_off, sl2, cbm, lim, pk)
+                                             : exp_step<S::kE, S::kRowsE, false>(tS + lane_off, sl2, cbm, lim, pk);
                 // the step stands while the row's sum of p = 2^(logit - m_run) stays at most
                 // 2^kRescaleL2 (then so does every p); a sum that overflowed is not finite
-                const float psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
                 if (!__any_sync(0xffffffffu, !(psum <= kRescaleP))) {
                     tmem_st32(tS + lane_off, pk);
                     l_run += psum;
@@ -415,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
             }
             float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
             if (!row_ok) mx = -INFINITY;
-            // running maximum: kept unless the step's maximum exceeds it by more than 2^8
+            // running maximum: kept unless the step's maximum exceeds it by more than kRescaleL2
             float f = 1.f;
             const bool rescale = mx > -INFINITY && m_run > -INFINITY && mx > m_run + kRescaleL2;
             if (mx > -INFINITY) {
