@@ -111,6 +111,9 @@ typedef struct {
     const float *kbar;      /* optional precomputed chunk summaries [b][n_chunks][hkv][d] fp32
                                contiguous (from dash_pool_keys, e.g. a decode cache) */
     int flags;              /* DASH_FLAG_* */
+    const dash_tensor_t *qbar; /* optional learned summary queries of Stage 0, see
+                               dash_pool_keys_q; NULL = q̄ = 0 (mean pooling).  Not
+                               together with kbar. */
 } dash_opts_t;
 
 /* Fill *opts with the defaults above.  Returns DASH_OK or DASH_ERR_INVALID_ARG (NULL). */
@@ -133,6 +136,21 @@ DASH_API int dash_attn_fwd_ex(const dash_tensor_t *q, const dash_tensor_t *k, co
  * fp32 contiguous, n_chunks = floor(nk/B) if causal else ceil(nk/B) (a partial
  * chunk is the mean of its real keys).  stream may be NULL. */
 DASH_API int dash_pool_keys(const dash_tensor_t *k, int block_size, int causal, float *kbar, void *stream);
+
+/* Stage 0 with a learned summary query ([Dash] §3.1 Eq. 3, App. G Alg. 1):
+ *   kbar_c^(r) = sum_{t in chunk c} softmax_t(<qbar_c^(r), k_t> / sqrt(d)) k_t,
+ * one online softmax over the chunk's keys, which also serve as the values.
+ *   k     [b, nk, hkv, d] f32 or bf16, as for dash_pool_keys.
+ *   qbar  [1 or b, n_chunks, hkv, d] f32 or bf16 (independent of k's dtype): the
+ *         summary query of every chunk and kv head, with any rotary position
+ *         encoding already applied by the caller (the library applies none).  A
+ *         stride of 0 broadcasts one query over the chunks (and shape[0] == 1 over
+ *         the batch), e.g. a per-head learned query without position encoding.
+ *   kbar  [b][n_chunks][hkv][d] fp32 contiguous output; n_chunks as for dash_pool_keys.
+ * qbar = 0 gives exactly the mean of dash_pool_keys.  Errors as for dash_pool_keys,
+ * plus DASH_ERR_INVALID_ARG when qbar's shape does not match. */
+DASH_API int dash_pool_keys_q(const dash_tensor_t *k, const dash_tensor_t *qbar, int block_size, int causal,
+                              float *kbar, void *stream);
 
 /* Stage 1 alone ([Dash] §3.2 Eq. 4; App. G Alg. 2).  Every output is optional
  * (NULL to skip):

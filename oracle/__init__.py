@@ -50,9 +50,12 @@ def _load():
         lib.dash_oracle_entmax_sort.argtypes = [P, i32, f64, P, P, P]
         lib.dash_oracle_entmax_bisect.argtypes = [P, i32, f64, i32, P, P]
         lib.dash_oracle_pool.argtypes = [P, i64, i32, i32, i32, i32, P]
+        lib.dash_oracle_pool_q.argtypes = [P, P, i64, i32, i32, i32, i32, P]
         lib.dash_oracle_pool.restype = None
         lib.dash_oracle_fwd_rows.argtypes = [P, P, i64, i64, P, P, i64, i32, i32, i32, i32, f64, f64, f64,
                                              i32, i32, P, P, P, P, P, P, P, P]
+        lib.dash_oracle_fwd_rows_q.argtypes = [P, P, i64, i64, P, P, i64, i32, i32, i32, i32, f64, f64, f64, i32,
+                                               i32, P, P, P, P, P, P, P, P, P]
         lib.dash_oracle_dense_attention.argtypes = [P, i64, P, P, i64, i32, i32, i32, i32, P]
         lib.dash_oracle_set_threads.argtypes = [i32]
         lib.dash_oracle_set_threads.restype = None
@@ -119,17 +122,32 @@ def pool(K, block_size: int, n_chunks: int | None = None):
     return out
 
 
+def pool_q(K, Qbar, block_size: int, n_chunks: int | None = None):
+    """Learned-query chunk summaries: K [nk, hkv, d], Qbar [n_chunks, hkv, d] ->
+    [n_chunks, hkv, d] (float64), softmax(<q̄_c, k_t>/sqrt(d)) weights over each chunk."""
+    K = _f32(K)
+    nk, hkv, d = K.shape
+    if n_chunks is None:
+        n_chunks = nk // block_size
+    Qbar = _f32(np.broadcast_to(np.asarray(Qbar, dtype=np.float32), (n_chunks, hkv, d)))
+    out = np.empty((n_chunks, hkv, d), dtype=np.float64)
+    _load().dash_oracle_pool_q(_ptr(K), _ptr(Qbar), nk, hkv, d, int(block_size), int(n_chunks), _ptr(out))
+    return out
+
+
 def n_chunks_for(nk: int, block_size: int, causal: bool) -> int:
     return nk // block_size if causal else -(-nk // block_size)
 
 
 def fwd_rows(Q_rows, rows, nq: int, K, V, block_size: int, alpha: float, *, gamma: float = 1.0,
              sigma: float = 1e8, causal: bool = True, route: int = 0, w_in=None, r_in=None,
-             want=("out", "tau", "w", "routed")):
+             want=("out", "tau", "w", "routed"), qbar=None):
     """Oracle forward for selected query rows of ONE batch element.
 
     Q_rows [nrows, hq, d] are the rows' query vectors, rows [nrows] their
-    indices in [0, nq); K, V are [nk, hkv, d].  Returns a dict with the
+    indices in [0, nq); K, V are [nk, hkv, d].  qbar [n_chunks, hkv, d] (or a
+    shape that broadcasts to it): learned Stage-0 summary queries (None: q̄ = 0,
+    mean pooling).  Returns a dict with the
     requested outputs among out, tau, w, routed, xmt, lambda (see the C file).
     """
     lib = _load()
@@ -151,6 +169,16 @@ def fwd_rows(Q_rows, rows, nq: int, K, V, block_size: int, alpha: float, *, gamm
     if w_in is not None:
         w_in = _f64(w_in).reshape(nrows, hkv, nch)
         r_in = np.ascontiguousarray(r_in, dtype=np.uint8).reshape(nrows, hkv, nch)
+    if qbar is not None:
+        qb = _f32(np.broadcast_to(np.asarray(qbar, dtype=np.float32), (nch, hkv, d)))
+        rc = lib.dash_oracle_fwd_rows_q(_ptr(Q_rows), _ptr(rows), nrows, int(nq), _ptr(K), _ptr(V), nk, hq, hkv,
+                                        d, int(block_size), float(alpha), float(gamma), float(sigma),
+                                        int(bool(causal)), int(route), _ptr(w_in), _ptr(r_in), _ptr(qb),
+                                        _ptr(res["out"]), _ptr(res["tau"]), _ptr(res["w"]), _ptr(res["routed"]),
+                                        _ptr(res["xmt"]), _ptr(res["lambda"]))
+        if rc:
+            raise ValueError("oracle fwd_rows_q rejected its input (rc=%d)" % rc)
+        return {k: v for k, v in res.items() if v is not None}
     rc = lib.dash_oracle_fwd_rows(_ptr(Q_rows), _ptr(rows), nrows, int(nq), _ptr(K), _ptr(V), nk, hq, hkv, d,
                                   int(block_size), float(alpha), float(gamma), float(sigma), int(bool(causal)),
                                   int(route), _ptr(w_in), _ptr(r_in), _ptr(res["out"]), _ptr(res["tau"]),

@@ -14,7 +14,9 @@
  *   - Stage 2 (prior-induced soft.) [Dash §3.3 Eqs. 6-7; §3.4 Eqs. 8-10, Prop. 1]
  *
  * Readings taken where the paper is silent (each is also listed in the design doc):
- *   - the learned summary query is zero, so Stage 0 is the chunk mean  [Dash §3.1]
+ *   - the learned summary query is zero unless one is given, so Stage 0 is the
+ *     chunk mean by default; a given q̄ holds one query per chunk and kv head with
+ *     any position encoding already applied                            [Dash §3.1; App. G Alg. 1]
  *   - causal alignment is bottom-right: query row i sits at key position
  *     p_i = i + nk - nq; its own chunk is c_i = floor(p_i / B); it routes
  *     over the complete chunks c < min(c_i, floor(nk/B))              [Dash App. G Alg. 2]
@@ -233,6 +235,44 @@ ORACLE_API void dash_oracle_pool(const float *K, int64_t nk, int hkv, int d, int
     }
 }
 
+/* k̄_c^{(r)} = sum_{t in C_c} a_t k_t with a_t = exp(<q̄_c^{(r)}, k_t>/sqrt(d)) /
+ * sum_{u in C_c} exp(<q̄_c^{(r)}, k_u>/sqrt(d))  [Dash §3.1 Eq. 3; App. G Alg. 1,
+ * where q̄ carries one query per chunk and kv head].  The largest score is
+ * subtracted before exponentiating; the ratio is unchanged by it.
+ * K: [nk, hkv, d]; Qbar: [n_chunks, hkv, d]; Kbar: [n_chunks, hkv, d]. */
+ORACLE_API void dash_oracle_pool_q(const float *K, const float *Qbar, int64_t nk, int hkv, int d, int B,
+                                   int n_chunks, double *Kbar)
+{
+    const double inv_sqrt_d = 1.0 / sqrt((double)d);
+    for (int c = 0; c < n_chunks; ++c) {
+        int64_t t0 = (int64_t)c * B, t1 = t0 + B;
+        if (t1 > nk) t1 = nk;
+        const int n = (int)(t1 - t0);
+        double *score = (double *)malloc(sizeof(double) * (size_t)n);
+        for (int r = 0; r < hkv; ++r) {
+            const float *qb = Qbar + ((size_t)c * hkv + r) * d;
+            double smax = -INFINITY;
+            for (int j = 0; j < n; ++j) {
+                const float *kt = K + ((size_t)(t0 + j) * hkv + r) * d;
+                double acc = 0.0;
+                for (int e = 0; e < d; ++e) acc += (double)qb[e] * (double)kt[e];
+                score[j] = acc * inv_sqrt_d;
+                if (score[j] > smax) smax = score[j];
+            }
+            double z = 0.0;
+            for (int j = 0; j < n; ++j) z += exp(score[j] - smax);
+            double *out = Kbar + ((size_t)c * hkv + r) * d;
+            for (int e = 0; e < d; ++e) out[e] = 0.0;
+            for (int j = 0; j < n; ++j) {
+                const double a = exp(score[j] - smax) / z;
+                const float *kt = K + ((size_t)(t0 + j) * hkv + r) * d;
+                for (int e = 0; e < d; ++e) out[e] += a * (double)kt[e];
+            }
+        }
+        free(score);
+    }
+}
+
 /* ------------------------------------------------------------------ */
 /* Full forward for selected query rows                                */
 /* ------------------------------------------------------------------ */
@@ -386,12 +426,41 @@ static void stage2_head(const oracle_cfg_t *cf, const float *q, const float *K, 
  *   xmt    [nrows, hq, n_chunks]  x_c - tau per head (NaN outside the visible chunks)
  *   lambda [nrows, hq]            routed-branch mass (route 1 only)
  * n_chunks = floor(nk/B) when causal, ceil(nk/B) otherwise.                */
+static int fwd_rows_impl(const float *Q, const int64_t *rows, int64_t nrows, int64_t nq, const float *K,
+                         const float *V, int64_t nk, int hq, int hkv, int d, int B, double alpha,
+                         double gamma, double sigma, int causal, int route, const double *w_in,
+                         const unsigned char *r_in, const float *Qbar, double *out, double *tau, double *w,
+                         unsigned char *routed, double *xmt, double *lambda);
+
 ORACLE_API int dash_oracle_fwd_rows(const float *Q, const int64_t *rows, int64_t nrows, int64_t nq,
                                     const float *K, const float *V, int64_t nk, int hq, int hkv, int d,
                                     int B, double alpha, double gamma, double sigma, int causal, int route,
                                     const double *w_in, const unsigned char *r_in, double *out,
                                     double *tau, double *w, unsigned char *routed, double *xmt,
                                     double *lambda)
+{
+    return fwd_rows_impl(Q, rows, nrows, nq, K, V, nk, hq, hkv, d, B, alpha, gamma, sigma, causal, route,
+                         w_in, r_in, NULL, out, tau, w, routed, xmt, lambda);
+}
+
+/* As dash_oracle_fwd_rows with Stage 0 taken from the learned summary queries
+ * Qbar [n_chunks, hkv, d] (dash_oracle_pool_q). */
+ORACLE_API int dash_oracle_fwd_rows_q(const float *Q, const int64_t *rows, int64_t nrows, int64_t nq,
+                                      const float *K, const float *V, int64_t nk, int hq, int hkv, int d,
+                                      int B, double alpha, double gamma, double sigma, int causal, int route,
+                                      const double *w_in, const unsigned char *r_in, const float *Qbar,
+                                      double *out, double *tau, double *w, unsigned char *routed,
+                                      double *xmt, double *lambda)
+{
+    return fwd_rows_impl(Q, rows, nrows, nq, K, V, nk, hq, hkv, d, B, alpha, gamma, sigma, causal, route,
+                         w_in, r_in, Qbar, out, tau, w, routed, xmt, lambda);
+}
+
+static int fwd_rows_impl(const float *Q, const int64_t *rows, int64_t nrows, int64_t nq, const float *K,
+                         const float *V, int64_t nk, int hq, int hkv, int d, int B, double alpha,
+                         double gamma, double sigma, int causal, int route, const double *w_in,
+                         const unsigned char *r_in, const float *Qbar, double *out, double *tau, double *w,
+                         unsigned char *routed, double *xmt, double *lambda)
 {
     if (hq % hkv || !(alpha > 1.0) || B <= 0 || d <= 0 || nk <= 0) return -1;
     if (causal && nq > nk) return -1;
@@ -400,7 +469,10 @@ ORACLE_API int dash_oracle_fwd_rows(const float *Q, const int64_t *rows, int64_t
     const int n_chunks = causal ? (int)(nk / B) : (int)((nk + B - 1) / B);
     double *Kbar = (double *)malloc(sizeof(double) * (size_t)(n_chunks ? n_chunks : 1) * hkv * d);
     if (!Kbar) return -2;
-    dash_oracle_pool(K, nk, hkv, d, B, n_chunks, Kbar);
+    if (Qbar)
+        dash_oracle_pool_q(K, Qbar, nk, hkv, d, B, n_chunks, Kbar);
+    else
+        dash_oracle_pool(K, nk, hkv, d, B, n_chunks, Kbar);
     const double kexp = 1.0 / (alpha - 1.0);
     const double zscale = gamma / sqrt((double)d);
     int err = 0;

@@ -10,9 +10,10 @@ Functions mirror the C entry points:
   dash_attn_fwd(q, k, v, out, block_size, alpha, causal, gqa_groups, **opts)
   dash_block_select(q, k, block_size, alpha, causal, gqa_groups, tau=, w=, mask=, lists=, **opts)
   dash_sparse_attn_fwd(q, k, v, out, lists, block_size, causal, gqa_groups, **opts)
-  dash_pool_keys(k, block_size, causal, kbar)
+  dash_pool_keys(k, block_size, causal, kbar, qbar=None)
   make_lists(...), dash_sync_status(), dash_release()
-opts: sigma, gamma, kbar (fp32 tensor), workspace (uint8 tensor), flags, stream.
+opts: sigma, gamma, kbar (fp32 tensor), qbar (Stage-0 summary queries), workspace (uint8
+tensor), flags, stream.
 """
 from __future__ import annotations
 
@@ -60,7 +61,8 @@ class _Lists(ctypes.Structure):
 class _Opts(ctypes.Structure):
     _fields_ = [("sigma", ctypes.c_float), ("gamma", ctypes.c_float), ("stream", ctypes.c_void_p),
                 ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
-                ("kbar", ctypes.c_void_p), ("flags", ctypes.c_int)]
+                ("kbar", ctypes.c_void_p), ("flags", ctypes.c_int),
+                ("qbar", ctypes.POINTER(_Tensor))]
 
 
 _lib = None
@@ -68,7 +70,7 @@ _lib = None
 # every entry point include/dash_attn.h declares
 EXPORTS = ("dash_opts_init", "dash_attn_fwd", "dash_attn_fwd_ex", "dash_pool_keys", "dash_block_select",
            "dash_sparse_attn_fwd", "dash_lists_geometry", "dash_workspace_bytes", "dash_last_error",
-           "dash_sync_status", "dash_release", "dash_version", "dash_attn_fwd_noalloc")
+           "dash_sync_status", "dash_release", "dash_version", "dash_attn_fwd_noalloc", "dash_pool_keys_q")
 
 # size of the library's static scratch area used by dash_attn_fwd_noalloc
 DASH_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -90,6 +92,7 @@ def load_library():
     lib.dash_attn_fwd_ex.argtypes = [T, T, T, T, i32, f32, i32, i32, ctypes.POINTER(_Opts)]
     lib.dash_attn_fwd_noalloc.argtypes = [T, T, T, T, i32, f32, i32, i32, ctypes.POINTER(_Opts)]
     lib.dash_pool_keys.argtypes = [T, i32, i32, P, P]
+    lib.dash_pool_keys_q.argtypes = [T, T, i32, i32, P, P]
     lib.dash_block_select.argtypes = [T, T, i32, f32, i32, i32, P, P, P, ctypes.POINTER(_Lists),
                                       ctypes.POINTER(_Opts)]
     lib.dash_sparse_attn_fwd.argtypes = [T, T, T, T, ctypes.POINTER(_Lists), i32, i32, i32, ctypes.POINTER(_Opts)]
@@ -136,7 +139,7 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _opts(sigma=1e8, gamma=1.0, kbar=None, workspace=None, flags=0, stream=None) -> _Opts:
+def _opts(sigma=1e8, gamma=1.0, kbar=None, workspace=None, flags=0, stream=None, qbar=None) -> _Opts:
     o = _Opts()
     load_library().dash_opts_init(ctypes.byref(o))
     o.sigma = float(sigma)
@@ -151,6 +154,10 @@ def _opts(sigma=1e8, gamma=1.0, kbar=None, workspace=None, flags=0, stream=None)
         if kbar.dtype != torch.float32 or not kbar.is_contiguous():
             raise ValueError("kbar must be a contiguous float32 tensor")
         o.kbar = kbar.data_ptr()
+    if qbar is not None:
+        qd = _desc(qbar)
+        o._qbar_desc = qd  # kept alive with the options
+        o.qbar = ctypes.pointer(qd)
     o.flags = int(flags)
     return o
 
@@ -225,12 +232,20 @@ def dash_attn_fwd_noalloc(q, k, v, out, block_size, alpha, causal=True, gqa_grou
     return out
 
 
-def dash_pool_keys(k, block_size, causal, kbar, stream=None):
+def dash_pool_keys(k, block_size, causal, kbar, stream=None, qbar=None):
+    """Stage 0 into ``kbar`` [b, n_chunks, hkv, d] fp32: the chunk means, or with
+    ``qbar`` [1 or b, n_chunks, hkv, d] (a broadcast view is fine) the learned-query
+    softmax pooling of dash_pool_keys_q."""
     lib = load_library()
     kd = _desc(k)
     s = torch.cuda.current_stream() if stream is None else stream
-    _check(lib.dash_pool_keys(ctypes.byref(kd), int(block_size), int(bool(causal)), _ptr(kbar),
-                              ctypes.c_void_p(s.cuda_stream)))
+    if qbar is None:
+        _check(lib.dash_pool_keys(ctypes.byref(kd), int(block_size), int(bool(causal)), _ptr(kbar),
+                                  ctypes.c_void_p(s.cuda_stream)))
+    else:
+        qd = _desc(qbar)
+        _check(lib.dash_pool_keys_q(ctypes.byref(kd), ctypes.byref(qd), int(block_size), int(bool(causal)),
+                                    _ptr(kbar), ctypes.c_void_p(s.cuda_stream)))
     return kbar
 
 

@@ -239,6 +239,30 @@ int run_stage2(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor
     return DASH_OK;
 }
 
+// Summary queries of Stage 0: [1 or b][n_chunks][hkv][d]; shape[0] == 1 broadcasts over the batch.
+int check_qbar(const dash_tensor_t *qb, const Geom &G, TView *v) {
+    int rc = check_tensor(qb, "qbar");
+    if (rc) return rc;
+    if ((qb->shape[0] != 1 && qb->shape[0] != G.b) || qb->shape[1] != G.n_chunks || qb->shape[2] != G.hkv ||
+        qb->shape[3] != G.d)
+        return fail(DASH_ERR_INVALID_ARG,
+                    "qbar shape [%lld, %lld, %lld, %lld] does not match [1 or %lld, %d chunks, %d kv heads, %d]",
+                    (long long)qb->shape[0], (long long)qb->shape[1], (long long)qb->shape[2],
+                    (long long)qb->shape[3], (long long)G.b, G.n_chunks, G.hkv, G.d);
+    *v = view(qb);
+    if (qb->shape[0] == 1) v->s0 = 0;
+    return DASH_OK;
+}
+
+// Stage 0 into kbar: mean pooling, or the learned-query softmax pooling when qb is given
+// (qb already validated).
+int run_stage0(const dash_tensor_t *k, const dash_tensor_t *qb, const TView &qv, const Geom &G, float *kbar,
+               cudaStream_t st) {
+    cudaError_t e = qb ? launch_pool_keys_q(view(k), k->dtype, qv, qb->dtype, G, kbar, st)
+                       : launch_pool_keys(view(k), k->dtype, G, kbar, st);
+    return e == cudaSuccess ? DASH_OK : cuda_fail(e, "pool_keys");
+}
+
 int validate_qkvo(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v,
                   const dash_tensor_t *out) {
     int rc;
@@ -328,6 +352,21 @@ DASH_API int dash_pool_keys(const dash_tensor_t *k, int block_size, int causal, 
     return DASH_OK;
 }
 
+DASH_API int dash_pool_keys_q(const dash_tensor_t *k, const dash_tensor_t *qbar, int block_size, int causal,
+                              float *kbar, void *stream) {
+    int rc = check_tensor(k, "k");
+    if (rc) return rc;
+    if (!kbar) return fail(DASH_ERR_INVALID_ARG, "kbar is NULL");
+    if (reinterpret_cast<uintptr_t>(kbar) % 16) return fail(DASH_ERR_ALIGNMENT, "kbar not 16-byte aligned");
+    dash_tensor_t q0 = *k;
+    q0.shape[1] = 0;
+    Geom G;
+    if ((rc = make_geom(&q0, k, block_size, causal, 1, &G))) return rc;
+    TView qv;
+    if ((rc = check_qbar(qbar, G, &qv))) return rc;
+    return run_stage0(k, qbar, qv, G, kbar, static_cast<cudaStream_t>(stream));
+}
+
 DASH_API int dash_block_select(const dash_tensor_t *q, const dash_tensor_t *k, int block_size, float alpha,
                                int causal, int gqa_groups, float *tau, float *w, uint32_t *mask,
                                const dash_lists_t *lists, const dash_opts_t *opts) {
@@ -342,6 +381,9 @@ DASH_API int dash_block_select(const dash_tensor_t *q, const dash_tensor_t *k, i
     if (lists && (rc = check_lists(lists, G))) return rc;
     for (const void *p : {(const void *)tau, (const void *)w, (const void *)mask})
         if (reinterpret_cast<uintptr_t>(p) % 16) return fail(DASH_ERR_ALIGNMENT, "outputs must be 16-byte aligned");
+    TView qv{};
+    if (o.qbar && o.kbar) return fail(DASH_ERR_INVALID_ARG, "opts: give kbar or qbar, not both");
+    if (o.qbar && (rc = check_qbar(o.qbar, G, &qv))) return rc;
     if (G.b == 0 || G.nq == 0) return DASH_OK;
     const bool need_kbar = o.kbar == nullptr;
     WsLayout WL = ws_layout(G, need_kbar, true, false);
@@ -351,8 +393,7 @@ DASH_API int dash_block_select(const dash_tensor_t *q, const dash_tensor_t *k, i
     const float *kbar = o.kbar;
     if (need_kbar) {
         float *kb = reinterpret_cast<float *>(ws + WL.kbar);
-        cudaError_t e = launch_pool_keys(view(k), k->dtype, G, kb, st);
-        if (e != cudaSuccess) return cuda_fail(e, "pool_keys");
+        if ((rc = run_stage0(k, o.qbar, qv, G, kb, st))) return rc;
         kbar = kb;
     }
     ListsView LV;
@@ -390,6 +431,9 @@ DASH_API int dash_attn_fwd_ex(const dash_tensor_t *q, const dash_tensor_t *k, co
     Geom G;
     if ((rc = make_geom(q, k, block_size, causal, gqa_groups, &G))) return rc;
     if (o.kbar && reinterpret_cast<uintptr_t>(o.kbar) % 16) return fail(DASH_ERR_ALIGNMENT, "kbar not aligned");
+    TView qv{};
+    if (o.qbar && o.kbar) return fail(DASH_ERR_INVALID_ARG, "opts: give kbar or qbar, not both");
+    if (o.qbar && (rc = check_qbar(o.qbar, G, &qv))) return rc;
     if (G.b == 0 || G.nq == 0) return DASH_OK;
     const bool need_kbar = o.kbar == nullptr;
     const bool dec = attn_decode_supported(G, q->dtype) && !(o.flags & DASH_FLAG_FORCE_SIMT);
@@ -397,11 +441,10 @@ DASH_API int dash_attn_fwd_ex(const dash_tensor_t *q, const dash_tensor_t *k, co
     char *ws = nullptr;
     if ((rc = get_workspace(o, WL.total, &ws))) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(o.stream);
-    cudaError_t e;
     const float *kbar = o.kbar;
     if (need_kbar) {
         float *kb = reinterpret_cast<float *>(ws + WL.kbar);
-        if ((e = launch_pool_keys(view(k), k->dtype, G, kb, st)) != cudaSuccess) return cuda_fail(e, "pool_keys");
+        if ((rc = run_stage0(k, o.qbar, qv, G, kb, st))) return rc;
         kbar = kb;
     }
     const bool regroup = !(o.flags & DASH_FLAG_NO_REGROUP) && G.n_tiles > 1;

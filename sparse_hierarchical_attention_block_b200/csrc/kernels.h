@@ -7,6 +7,9 @@ namespace dash {
 
 // Stage 0 (pool_keys.cu)
 cudaError_t launch_pool_keys(const TView &K, dash_dtype_t dt, const Geom &G, float *kbar, cudaStream_t st);
+// learned summary queries: view [b (stride 0 to broadcast)][n_chunks][hkv][d] of dtype qdt
+cudaError_t launch_pool_keys_q(const TView &K, dash_dtype_t dt, const TView &Qbar, dash_dtype_t qdt, const Geom &G,
+                               float *kbar, cudaStream_t st);
 
 // Stage 1 (block_select.cu)
 struct SelectOut {

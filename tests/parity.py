@@ -33,7 +33,7 @@ def unpack_mask(mask_words: np.ndarray, n_chunks: int) -> np.ndarray:
     return ((w[..., c // 32] >> (c % 32).astype(np.uint32)) & 1).astype(bool)
 
 
-def gpu_stage1(q, k, block_size, alpha, causal, sigma=1e8, gamma=1.0):
+def gpu_stage1(q, k, block_size, alpha, causal, sigma=1e8, gamma=1.0, qbar=None):
     b, nq, hq, _ = q.shape
     hkv = k.shape[2]
     nch = dash.n_chunks(k.shape[1], block_size, causal)
@@ -41,7 +41,9 @@ def gpu_stage1(q, k, block_size, alpha, causal, sigma=1e8, gamma=1.0):
     tau = torch.empty(b, nq, hq, dtype=torch.float32, device=q.device)
     w = torch.empty(b, nq, hkv, nch, dtype=torch.float32, device=q.device) if nch else None
     mask = torch.zeros(b, nq, hkv, max(words, 1), dtype=torch.int32, device=q.device)
-    dash.dash_block_select(q, k, block_size, alpha, causal, tau=tau, w=w, mask=mask, sigma=sigma, gamma=gamma)
+    extra = {} if qbar is None else {"qbar": qbar}
+    dash.dash_block_select(q, k, block_size, alpha, causal, tau=tau, w=w, mask=mask, sigma=sigma, gamma=gamma,
+                           **extra)
     torch.cuda.synchronize()
     return tau, w, mask
 
@@ -51,16 +53,17 @@ def to_np32(t):
 
 
 def check_forward(q, k, v, out, block_size, alpha, causal, sigma=1e8, gamma=1.0, rows=None, batches=None,
-                  label=""):
+                  label="", qbar=None):
     """Compare a GPU forward (``out``) and its Stage 1 with the oracle.
 
-    rows: query indices to check (default all); batches: batch indices (default all).
+    rows: query indices to check (default all); batches: batch indices (default all);
+    qbar: the learned Stage-0 summary queries [1 or b, n_chunks, hkv, d] given to both.
     Returns a dict of statistics.
     """
     b, nq, hq, d = q.shape
     nk, hkv = k.shape[1], k.shape[2]
     nch = dash.n_chunks(nk, block_size, causal)
-    tau_g, w_g, mask_g = gpu_stage1(q, k, block_size, alpha, causal, sigma, gamma)
+    tau_g, w_g, mask_g = gpu_stage1(q, k, block_size, alpha, causal, sigma, gamma, qbar)
     rows = np.arange(nq) if rows is None else np.asarray(rows, dtype=np.int64)
     batches = range(b) if batches is None else batches
     max_tol, mean_tol = OUT_TOL[q.dtype]
@@ -71,8 +74,9 @@ def check_forward(q, k, v, out, block_size, alpha, causal, sigma=1e8, gamma=1.0,
         Qr = to_np32(q[bi].index_select(0, rows_t))
         K = to_np32(k[bi])
         V = to_np32(v[bi])
+        qb = None if qbar is None else to_np32(qbar[bi if qbar.shape[0] > 1 else 0])
         ref = oracle.fwd_rows(Qr, rows, nq, K, V, block_size, alpha, gamma=gamma, sigma=sigma, causal=causal,
-                              want=("out", "tau", "w", "routed", "xmt"))
+                              want=("out", "tau", "w", "routed", "xmt"), qbar=qb)
         tg = tau_g[bi].index_select(0, rows_t).cpu().numpy()
         wg = (w_g[bi].index_select(0, rows_t).cpu().numpy().astype(np.float64) if nch
               else np.zeros((len(rows), hkv, 0)))
@@ -105,7 +109,7 @@ def check_forward(q, k, v, out, block_size, alpha, causal, sigma=1e8, gamma=1.0,
             fr = np.nonzero(frow)[0]
             w_in = np.where(rg[fr], np.maximum(np.maximum(ref["w"][fr], wg[fr]), 1e-300), 0.0)
             re = oracle.fwd_rows(Qr[fr], rows[fr], nq, K, V, block_size, alpha, gamma=gamma, sigma=sigma,
-                                 causal=causal, w_in=w_in, r_in=rg[fr].astype(np.uint8), want=("out",))
+                                 causal=causal, w_in=w_in, r_in=rg[fr].astype(np.uint8), want=("out",), qbar=qb)
             exp_out[fr] = re["out"]
         err = np.abs(og - exp_out)
         stats["rows"] += len(rows)

@@ -80,6 +80,8 @@ FAKE = 1 << 20  # never dereferenced: validation fails first
     ("causal_long_q", dash.DASH_ERR_INVALID_ARG),
     ("null", dash.DASH_ERR_INVALID_ARG),
     ("sigma", dash.DASH_ERR_INVALID_ARG),
+    ("qbar_shape", dash.DASH_ERR_INVALID_ARG),
+    ("qbar_with_kbar", dash.DASH_ERR_INVALID_ARG),
 ])
 def test_validation_rejects(lib, case, code):
     B, alpha, gqa, causal = 64, 1.5, 4, 1
@@ -112,6 +114,13 @@ def test_validation_rejects(lib, case, code):
         q.data = None
     elif case == "sigma":
         opts.sigma = 0.0
+    elif case == "qbar_shape":  # 4 chunks of 64 keys, not 5
+        qb = _t(FAKE, dash.DASH_F32, [1, 5, 2, 128])
+        opts.qbar = ctypes.pointer(qb)
+    elif case == "qbar_with_kbar":
+        qb = _t(FAKE, dash.DASH_F32, [1, 4, 2, 128])
+        opts.qbar = ctypes.pointer(qb)
+        opts.kbar = FAKE
     rc = lib.dash_attn_fwd_ex(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), ctypes.byref(o), B, alpha, causal,
                               gqa, ctypes.byref(opts))
     assert rc == code, lib.dash_last_error()
@@ -122,4 +131,5 @@ def test_opts_defaults(lib):
     o = _Opts()
     assert lib.dash_opts_init(ctypes.byref(o)) == 0
     assert o.sigma == pytest.approx(1e8) and o.gamma == 1.0 and o.flags == 0 and not o.workspace
+    assert not o.qbar and not o.kbar
     assert lib.dash_opts_init(None) == dash.DASH_ERR_INVALID_ARG

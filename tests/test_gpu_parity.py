@@ -79,6 +79,56 @@ def test_simt_path_matches_oracle(case):
     check_forward(q, k, v, out, B, alpha, causal, sigma=sigma, label=f"simt {case}")
 
 
+_DT = {"bf16": torch.bfloat16, "f32": torch.float32}
+
+
+@pytest.mark.parametrize("kdt,qdt,d,B,causal,bcast", [
+    ("bf16", "f32", 128, 64, False, False),   # trailing partial chunk pooled over its real keys
+    ("f32", "bf16", 64, 16, True, True),      # one query per head, broadcast over batch and chunks
+    ("bf16", "bf16", 128, 128, True, False),
+])
+def test_pool_keys_q_matches_oracle(kdt, qdt, d, B, causal, bcast):
+    """Stage 0 with a learned summary query (Eq. 3) against the oracle's pooling."""
+    gen = torch.Generator().manual_seed(41 + d + B)
+    b, nk, hkv = 2, 1000, 2
+    nch = dash.n_chunks(nk, B, causal)
+    k = torch.randn(b, nk, hkv, d, generator=gen).to(_DT[kdt]).cuda()
+    if bcast:
+        qbar = (2 * torch.randn(1, 1, hkv, d, generator=gen)).to(_DT[qdt]).cuda().expand(1, nch, hkv, d)
+    else:
+        qbar = (2 * torch.randn(b, nch, hkv, d, generator=gen)).to(_DT[qdt]).cuda()
+    kbar = torch.empty(b, nch, hkv, d, dtype=torch.float32, device="cuda")
+    dash.dash_pool_keys(k, B, causal, kbar, qbar=qbar)
+    assert dash.dash_sync_status() == 0
+    for bi in range(b):
+        ref = oracle.pool_q(to_np32(k[bi]), to_np32(qbar[bi if qbar.shape[0] > 1 else 0]), B, n_chunks=nch)
+        err = np.abs(to_np32(kbar[bi]).astype(np.float64) - ref).max()
+        assert err <= 5e-5, f"learned pooling error {err}"
+
+
+@pytest.mark.parametrize("case", [CASES[0], CASES[3], CASES[5]], ids=["c0", "c3", "c5"])
+def test_learned_summary_forward(case):
+    """The full forward with learned summary queries against the oracle's forward with the same q̄."""
+    b, nq, nk, hq, hkv, d, B, dt, alpha, causal, sigma = case
+    q, k, v = _planted(b, nq, nk, hq, hkv, d, B, dt, seed=300 + nq, causal=causal)
+    gen = torch.Generator().manual_seed(7 + nq)
+    nch = dash.n_chunks(nk, B, causal)
+    qbar = (0.5 * torch.randn(b, nch, hkv, d, generator=gen)).to(q.dtype).cuda()
+    out = _run(q, k, v, B, alpha, causal, sigma=sigma, qbar=qbar)
+    check_forward(q, k, v, out, B, alpha, causal, sigma=sigma, label=f"learned q̄ {case}", qbar=qbar)
+
+
+def test_learned_summary_arguments_are_checked():
+    q, k, v = _planted(1, 256, 256, 4, 2, 64, 64, "bf16", seed=5)
+    out = torch.empty_like(q)
+    nch = dash.n_chunks(256, 64, True)
+    with pytest.raises(dash.DashError):  # wrong number of chunks
+        dash.dash_attn_fwd(q, k, v, out, 64, 1.5, True, 2, qbar=torch.zeros(1, nch + 1, 2, 64, device="cuda"))
+    kb = torch.zeros(1, nch, 2, 64, device="cuda")
+    with pytest.raises(dash.DashError):  # summaries given twice
+        dash.dash_attn_fwd(q, k, v, out, 64, 1.5, True, 2, kbar=kb, qbar=torch.zeros(1, nch, 2, 64, device="cuda"))
+
+
 @pytest.mark.parametrize("dt,causal", [("bf16", True), ("bf16", False), ("f32", True)])
 def test_uniform_all_chunk_prior_is_dense_attention(dt, causal):
     """Stage 2 alone on lists that route every visible chunk with bias 0 equals

@@ -35,6 +35,12 @@ MUTATIONS = [
      "const double scale = 1.0;\n    /* gather"),
     ("pooling divides by B on a partial chunk", "out[e] /= cnt;", "out[e] /= (double)B;"),
     ("support decided by >= instead of >", "if (s[c] > tau_h) rt[c] = 1;", "if (s[c] >= tau_h - 1e-3) rt[c] = 1;"),
+    ("learned pooling drops 1/sqrt(d)", "score[j] = acc * inv_sqrt_d;", "score[j] = acc;"),
+    ("learned pooling weights not normalised", "const double a = exp(score[j] - smax) / z;",
+     "const double a = exp(score[j] - smax);"),
+    ("learned pooling uses chunk 0's query everywhere", "const float *qb = Qbar + ((size_t)c * hkv + r) * d;",
+     "const float *qb = Qbar + (size_t)r * d;"),
+    ("forward ignores the learned query", "if (Qbar)\n        dash_oracle_pool_q(", "if (0)\n        dash_oracle_pool_q("),
 ]
 
 

@@ -178,6 +178,87 @@ def test_pool_mean_closed_form():
                 assert out[c, r, e] == (r + 1) * (t0 + t1) / 2.0 + e
 
 
+def test_pool_q_zero_query_is_the_mean():
+    """A zero summary query gives uniform weights (Sec. 3.1): the pinned chunk mean."""
+    rng = np.random.default_rng(5)
+    K = rng.normal(size=(200, 3, 16)).astype(np.float32)
+    nch = -(-200 // 64)
+    assert np.abs(oracle.pool_q(K, np.zeros((nch, 3, 16)), 64, n_chunks=nch) -
+                  oracle.pool(K, 64, n_chunks=nch)).max() < 1e-15
+
+
+def test_pool_q_two_keys_is_a_logistic_mix():
+    """For a chunk of two keys Eq. 3 reduces to s(D) k1 + (1 - s(D)) k2 with the logistic
+    s and D = <q, k1 - k2>/sqrt(d); every (chunk, head) has its own query."""
+    from scipy.special import expit
+    rng = np.random.default_rng(6)
+    nk, hkv, d = 12, 3, 8
+    K = rng.normal(size=(nk, hkv, d)).astype(np.float32)
+    Qb = rng.normal(size=(nk // 2, hkv, d)).astype(np.float32)
+    out = oracle.pool_q(K, Qb, 2)
+    for c in range(nk // 2):
+        for r in range(hkv):
+            k1, k2 = K[2 * c, r].astype(np.float64), K[2 * c + 1, r].astype(np.float64)
+            a = expit(float(Qb[c, r].astype(np.float64) @ (k1 - k2)) / np.sqrt(d))
+            assert np.abs(out[c, r] - (a * k1 + (1 - a) * k2)).max() < 1e-14
+
+
+def test_pool_q_large_query_selects_the_best_key():
+    """Scaling q̄ to infinity turns the softmax weights into the indicator of the key
+    with the largest <q̄, k_t> (distinct projections): the summary is that key."""
+    rng = np.random.default_rng(7)
+    nk, hkv, d, B = 96, 2, 16, 32
+    K = rng.normal(size=(nk, hkv, d)).astype(np.float32)
+    u = rng.normal(size=(nk // B, hkv, d))
+    out = oracle.pool_q(K, (1e6 * u).astype(np.float32), B)
+    for c in range(nk // B):
+        for r in range(hkv):
+            u32 = (1e6 * u[c, r]).astype(np.float32).astype(np.float64)
+            best = int(np.argmax(K[c * B:(c + 1) * B, r].astype(np.float64) @ u32))
+            assert np.array_equal(out[c, r], K[c * B + best, r].astype(np.float64))
+
+
+def test_pool_q_invariants():
+    """Identical keys pool to that key; permuting a chunk's keys changes nothing; adding
+    one vector to every key shifts the summary by that vector (the weights are
+    unchanged: every score moves by the same amount)."""
+    rng = np.random.default_rng(8)
+    nk, hkv, d, B = 64, 2, 8, 16
+    K = (rng.integers(-64, 64, size=(nk, hkv, d)) / 16.0).astype(np.float32)
+    Qb = rng.normal(size=(nk // B, hkv, d)).astype(np.float32)
+    base = oracle.pool_q(K, Qb, B)
+    same = np.repeat(K[::B], B, axis=0)
+    assert np.array_equal(oracle.pool_q(same, Qb, B), K[::B].astype(np.float64))
+    perm = np.concatenate([c * B + rng.permutation(B) for c in range(nk // B)])
+    assert np.abs(oracle.pool_q(K[perm], Qb, B) - base).max() < 1e-14
+    shift = (rng.integers(-8, 8, size=(hkv, d)) / 4.0).astype(np.float32)
+    assert np.abs(oracle.pool_q(K + shift, Qb, B) - (base + shift)).max() < 1e-13
+
+
+def test_fwd_uses_the_learned_summaries():
+    """Stage 1 sees only the summaries: with q̄ so large that each chunk's summary is its
+    best-matching key, routing equals mean-pooled routing over keys where every chunk
+    is filled with that key; a zero q̄ reproduces the default forward exactly."""
+    rng = np.random.default_rng(9)
+    nq = nk = 256
+    hq, hkv, d, B = 4, 2, 16, 32
+    Q = rng.normal(size=(nq, hq, d)).astype(np.float32) * 3
+    K = rng.normal(size=(nk, hkv, d)).astype(np.float32)
+    V = rng.normal(size=(nk, hkv, d)).astype(np.float32)
+    u = (1e6 * rng.normal(size=(nk // B, hkv, d))).astype(np.float32)
+    best = oracle.pool_q(K, u, B).astype(np.float32)
+    K_best = np.repeat(best, B, axis=0)
+    a = oracle.fwd(Q, K, V, B, 1.5, sigma=1.0, qbar=u)
+    b = oracle.fwd(Q, K_best, V, B, 1.5, sigma=1.0)
+    assert np.array_equal(a["routed"], b["routed"])
+    assert np.abs(a["w"] - b["w"]).max() < 1e-12
+    assert np.allclose(a["tau"], b["tau"], atol=1e-12, equal_nan=True)
+    z = oracle.fwd(Q, K, V, B, 1.5, sigma=1.0, qbar=np.zeros((nk // B, hkv, d)))
+    ref = oracle.fwd(Q, K, V, B, 1.5, sigma=1.0)
+    for key in ("out", "w", "routed"):
+        assert np.array_equal(z[key], ref[key])
+
+
 # ------------------------------------------------------------ full forward --
 
 def _case(seed, nq, nk, hq, hkv, d, B, planted=True):
