@@ -17,6 +17,15 @@ before every timed step, outside the event pair; warm-up steps untimed.
 Multi-GPU (torchrun): every rank runs an independent replica of the workload
 (the method's (batch, kv-head) units share nothing: no collective); value is
 the work of all ranks over the max-over-ranks time ("scaling": "weak").
+
+    python bench.py --mask-sweep [--sweep-n 16384,32768,65536,98304] [--sweep-s 0.75,0.875,0.9375]
+                    [--sweep-phase prefill,decode]
+
+Controlled-sparsity sweep of Stage 2 (the pages' kernel benchmark: Hq 32, Hkv 2, d 128,
+chunk 64, prefill at batch 1, decoding at batch 24): a random routing mask at block
+sparsity s stands in for the router's, Stage 2 alone is timed on the work lists built
+from it, and torch's dense SDPA on the same inputs is timed beside it for context.  One
+JSON line per (phase, N, s); 1 GPU.
 """
 from __future__ import annotations
 
@@ -309,6 +318,89 @@ def run_ours(args, rank, world, device):
 
 
 # ---------------------------------------------------------------------------
+# controlled-sparsity sweep of Stage 2 (random routing masks)
+# ---------------------------------------------------------------------------
+
+def mask_counts(mask):
+    """|R| per (b, i, r) from bit-packed int32 mask words."""
+    m = mask.to(torch.int64) & 0xFFFFFFFF
+    cnt = torch.zeros(mask.shape[:3], dtype=torch.int64, device=mask.device)
+    for bit in range(32):
+        cnt += (m >> bit).bitwise_and(1).sum(-1)
+    return cnt
+
+
+def run_mask_sweep(args, device):
+    import torch.nn.functional as F
+
+    import sparse_hierarchical_attention_block_b200 as dash
+
+    dash.load_library()
+    peaks = load_peaks()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, n):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        for a, b in ev:
+            flush.fill_(1.0)
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in ev)
+
+    hq, hkv, d, block = 32, 2, 128, 64
+    g = hq // hkv
+    for phase in args.sweep_phase.split(","):
+        for n in (int(x) for x in args.sweep_n.split(",")):
+            b, nq = (1, n) if phase == "prefill" else (24, 1)
+            w = synthetic.Workload(f"mask-sweep-{phase}-{n}", b, nq, n, hq, hkv, d, block, 1.5, True, "bf16", 21,
+                                   False)
+            q, k, v = synthetic.make_inputs(w, device)
+            out = torch.empty_like(q)
+            qt, kt, vt = (x.transpose(1, 2).contiguous() for x in (q, k, v))
+
+            def dense():
+                F.scaled_dot_product_attention(qt, kt, vt, is_causal=phase == "prefill", enable_gqa=True)
+
+            for _ in range(args.warmup):
+                dense()
+            ms_dense = timed(dense, max(3, min(args.steps, 5)))
+            del qt, kt, vt
+            for sp in (float(x) for x in args.sweep_s.split(",")):
+                mask = synthetic.random_block_mask(b, nq, n, hkv, block, sp, seed=31, device=device)
+                lists = dash.lists_from_mask(mask, n, hkv, block, g, causal=True, regroup=True)
+                f2, y, sparsity, exec_f = work_of(w, mask_counts(mask), lists)
+                del mask
+
+                def stage2():
+                    dash.dash_sparse_attn_fwd(q, k, v, out, lists, block, True, g)
+
+                for _ in range(args.warmup):
+                    stage2()
+                if dash.dash_sync_status() != 0:
+                    raise RuntimeError("stage 2 failed")
+                ms2 = timed(stage2, args.steps)
+                if phase == "prefill":
+                    ach, unit, peak = f2 / (ms2 * 1e-3) / 1e12, "TFLOP/s", peaks["bf16_tflops"]
+                else:
+                    ach, unit, peak = y / (ms2 * 1e-3) / 1e9, "GB/s", peaks["hbm_gbs"]
+                print(json.dumps({
+                    "mode": "random-mask Stage 2 sweep", "phase": phase, "n": n, "batch": b,
+                    "target_sparsity": sp, "sparsity": round(sparsity, 4), "hq": hq, "hkv": hkv, "d": d,
+                    "block": block, "stage2_ms": round(ms2, 4), "value": round(ach, 2), "unit": unit,
+                    "roofline_frac": round(ach / peak, 4), "peak_source": peaks["source"],
+                    "union_waste": (round(exec_f / f2, 3) if (exec_f and phase == "prefill") else None),
+                    "dense_sdpa_ms": round(ms_dense, 4), "speedup_vs_dense": round(ms_dense / ms2, 3),
+                    "steps": args.steps, "warmup": args.warmup,
+                    "l2": "flushed (256 MiB write) before every timed call"}), flush=True)
+                del lists
+            del q, k, v, out
+            torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------------------
 # the oracle on the host cores (CPU baseline / reference arm)
 # ---------------------------------------------------------------------------
 
@@ -393,6 +485,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-budget", type=float, default=10.0, help="seconds of oracle work per reference step")
+    ap.add_argument("--mask-sweep", action="store_true", help="controlled-sparsity sweep of Stage 2 (1 GPU)")
+    ap.add_argument("--sweep-n", default="16384,32768,65536,98304")
+    ap.add_argument("--sweep-s", default="0.75,0.875,0.9375")
+    ap.add_argument("--sweep-phase", default="prefill,decode")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -400,6 +496,12 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.warmup < 3:
         args.warmup = 3
+
+    if args.mask_sweep:
+        if rank == 0:
+            torch.cuda.set_device(local)
+            run_mask_sweep(args, torch.device("cuda", local))
+        return 0
 
     if args.impl == "reference":
         if rank != 0:

@@ -165,6 +165,25 @@ DASH_API int dash_block_select(const dash_tensor_t *q, const dash_tensor_t *k, i
                                int causal, int gqa_groups, float *tau, float *w, uint32_t *mask,
                                const dash_lists_t *lists, const dash_opts_t *opts);
 
+/* Stage-2 work lists from a caller's routing mask, e.g. the random block masks of a
+ * controlled-sparsity benchmark ([Dash] §5.2 and App. B.2 inject such a mask at Stage 2)
+ * or an external router.
+ *   mask  [batch][nq][hkv][words] uint32 device memory, words = ceil(n_chunks / 32) with
+ *         n_chunks = floor(nk/B) if causal else ceil(nk/B); bit c % 32 of word c / 32 set
+ *         = chunk c routed for that (query row, kv head).  Only chunks the row may route
+ *         (c < floor(p_i / B) when causal) may be set; other bits make the list longer
+ *         without changing the result.
+ *   Every routed chunk gets bias 0 (a uniform prior over the routed set: the sigma -> inf
+ *   limit of Prop. 1); each row's diagonal chunk is added as in dash_block_select.
+ *   regroup 1 groups rows with similar routed sets into tiles (lists->rows required),
+ *   0 keeps consecutive rows.
+ * lists: caller-owned buffers with the geometry of dash_lists_geometry.  Asynchronous on
+ * stream.  Errors: DASH_ERR_INVALID_ARG (NULL or mismatched buffers, bad sizes),
+ * DASH_ERR_UNSUPPORTED (gqa_groups outside [1, 16] or a block size outside {16, 32, 64, 128}). */
+DASH_API int dash_lists_from_mask(const uint32_t *mask, int64_t batch, int64_t nq, int64_t nk, int hkv,
+                                  int block_size, int gqa_groups, int causal, int regroup, dash_lists_t *lists,
+                                  void *stream);
+
 /* Stage 2 alone ([Dash] §3.3 Eq. 7 in the bias form of Prop. 1; App. G Alg. 3)
  * on caller-supplied lists (for example from dash_block_select, or a random
  * mask).  Returns a dash_status_t. */

@@ -70,7 +70,8 @@ _lib = None
 # every entry point include/dash_attn.h declares
 EXPORTS = ("dash_opts_init", "dash_attn_fwd", "dash_attn_fwd_ex", "dash_pool_keys", "dash_block_select",
            "dash_sparse_attn_fwd", "dash_lists_geometry", "dash_workspace_bytes", "dash_last_error",
-           "dash_sync_status", "dash_release", "dash_version", "dash_attn_fwd_noalloc", "dash_pool_keys_q")
+           "dash_sync_status", "dash_release", "dash_version", "dash_attn_fwd_noalloc", "dash_pool_keys_q",
+           "dash_lists_from_mask")
 
 # size of the library's static scratch area used by dash_attn_fwd_noalloc
 DASH_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -93,6 +94,7 @@ def load_library():
     lib.dash_attn_fwd_noalloc.argtypes = [T, T, T, T, i32, f32, i32, i32, ctypes.POINTER(_Opts)]
     lib.dash_pool_keys.argtypes = [T, i32, i32, P, P]
     lib.dash_pool_keys_q.argtypes = [T, T, i32, i32, P, P]
+    lib.dash_lists_from_mask.argtypes = [P, i64, i64, i64, i32, i32, i32, i32, i32, ctypes.POINTER(_Lists), P]
     lib.dash_block_select.argtypes = [T, T, i32, f32, i32, i32, P, P, P, ctypes.POINTER(_Lists),
                                       ctypes.POINTER(_Opts)]
     lib.dash_sparse_attn_fwd.argtypes = [T, T, T, T, ctypes.POINTER(_Lists), i32, i32, i32, ctypes.POINTER(_Opts)]
@@ -200,6 +202,21 @@ class Lists:
 def make_lists(q, k, block_size, gqa_groups, with_rows=True) -> Lists:
     return Lists(q.shape[0], q.shape[1], k.shape[1], k.shape[2], block_size, gqa_groups, device=q.device,
                  with_rows=with_rows)
+
+
+def lists_from_mask(mask, nk, hkv, block_size, gqa_groups, causal=True, regroup=False, stream=None) -> Lists:
+    """Stage-2 work lists from a routing mask [b, nq, hkv, words] int32 (bit-packed chunks,
+    dash_lists_from_mask): routed chunks get bias 0, each row's diagonal chunk is added."""
+    if not mask.is_cuda or mask.dtype != torch.int32 or not mask.is_contiguous():
+        raise ValueError("mask must be a contiguous int32 CUDA tensor")
+    b, nq = mask.shape[0], mask.shape[1]
+    lists = Lists(b, nq, nk, hkv, block_size, gqa_groups, device=mask.device, with_rows=True)
+    s = torch.cuda.current_stream() if stream is None else stream
+    lc = lists.c()
+    _check(load_library().dash_lists_from_mask(ctypes.c_void_p(mask.data_ptr()), b, nq, nk, hkv, int(block_size),
+                                               int(gqa_groups), int(bool(causal)), int(bool(regroup)),
+                                               ctypes.byref(lc), ctypes.c_void_p(s.cuda_stream)))
+    return lists
 
 
 def dash_attn_fwd(q, k, v, out, block_size, alpha, causal=True, gqa_groups=None, **opts):

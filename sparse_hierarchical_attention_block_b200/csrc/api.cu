@@ -367,6 +367,37 @@ DASH_API int dash_pool_keys_q(const dash_tensor_t *k, const dash_tensor_t *qbar,
     return run_stage0(k, qbar, qv, G, kbar, static_cast<cudaStream_t>(stream));
 }
 
+DASH_API int dash_lists_from_mask(const uint32_t *mask, int64_t batch, int64_t nq, int64_t nk, int hkv,
+                                  int block_size, int gqa_groups, int causal, int regroup, dash_lists_t *lists,
+                                  void *stream) {
+    if (!mask || !lists) return fail(DASH_ERR_INVALID_ARG, "mask or lists is NULL");
+    if (reinterpret_cast<uintptr_t>(mask) % 16) return fail(DASH_ERR_ALIGNMENT, "mask not 16-byte aligned");
+    if (batch < 0 || nq < 0 || hkv <= 0) return fail(DASH_ERR_INVALID_ARG, "bad batch, nq or hkv");
+    if (gqa_groups < 1 || gqa_groups > 16) return fail(DASH_ERR_UNSUPPORTED, "gqa_groups must be in [1, 16]");
+    // the geometry from shapes alone (head dim does not enter the lists)
+    dash_tensor_t q0{}, k0{};
+    q0.dtype = k0.dtype = DASH_BF16;
+    q0.data = k0.data = const_cast<uint32_t *>(mask);
+    q0.shape[0] = k0.shape[0] = batch;
+    q0.shape[1] = nq;
+    k0.shape[1] = nk;
+    q0.shape[2] = (int64_t)hkv * gqa_groups;
+    k0.shape[2] = hkv;
+    q0.shape[3] = k0.shape[3] = 128;
+    Geom G;
+    int rc = make_geom(&q0, &k0, block_size, causal, gqa_groups, &G);
+    if (rc) return rc;
+    if ((rc = check_lists(lists, G))) return rc;
+    if (regroup && !lists->rows) return fail(DASH_ERR_INVALID_ARG, "regroup needs lists->rows");
+    if (G.b == 0 || G.nq == 0) return DASH_OK;
+    const ListsView LV = lists_view(lists);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool rg = regroup && G.n_tiles > 1 && regroup_supported(G);
+    cudaError_t e = rg ? launch_regroup_compact(G, mask, nullptr, nullptr, 1.f, LV, st)
+                       : launch_compact(G, mask, nullptr, nullptr, 1.f, LV, st);
+    return e == cudaSuccess ? DASH_OK : cuda_fail(e, "work-list compaction");
+}
+
 DASH_API int dash_block_select(const dash_tensor_t *q, const dash_tensor_t *k, int block_size, float alpha,
                                int causal, int gqa_groups, float *tau, float *w, uint32_t *mask,
                                const dash_lists_t *lists, const dash_opts_t *opts) {

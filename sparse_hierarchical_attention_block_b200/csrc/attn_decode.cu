@@ -27,7 +27,7 @@ namespace {
 
 constexpr int kDecThreads = 128;
 constexpr int kDecRows = 16;  // mma.sync M
-constexpr int kEntriesPerSplit = 16;
+constexpr int kEntriesPerSplit = 16;  // most list entries one split takes (shared-memory sizing)
 constexpr uint64_t kDecWaitNs = 2000000000ull;
 
 struct DecParams {
@@ -102,7 +102,7 @@ struct DecSmem {
 template <int D, int BLK>
 __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(const __grid_constant__ DecParams dp, TView Q,
                                                                   Geom G, ListsView L, float *__restrict__ part,
-                                                                  int nsplit) {
+                                                                  int nsplit, int eps) {
     using S = DecSmem<D, BLK>;
     extern __shared__ uint8_t dsm_raw[];
     uint8_t *sm = dsm_raw + ((1024 - (smem_u32(dsm_raw) & 1023)) & 1023);
@@ -115,9 +115,9 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(const __grid_c
     const int M = (int)G.nq * g;  // valid rows (nq * g <= 16)
     const size_t tile_idx = ((size_t)b * G.hkv + r) * L.n_tiles;
     const int count = L.count[tile_idx];
-    const int e_begin = split * kEntriesPerSplit;
+    const int e_begin = split * eps;  // eps <= kEntriesPerSplit entries per split
     if (e_begin >= count) return;  // the combine kernel ignores splits past the list
-    const int e_end = min(count, e_begin + kEntriesPerSplit);
+    const int e_end = min(count, e_begin + eps);
     const int n = e_end - e_begin;
     const int32_t *ids = L.ids + tile_idx * L.cap;
     const float *bias = L.bias + tile_idx * (size_t)L.cap * T;
@@ -324,36 +324,50 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(const __grid_c
     }
 }
 
-// One CTA per (kv head, batch): merge the splits of every row.
+// One CTA per (row, kv head, batch), one thread per output column: merge the row's
+// split partials (max, sum, O) in the log2 domain.
 template <int D>
-__global__ void __launch_bounds__(128) combine_kernel(TView O, Geom G, ListsView L, const float *__restrict__ part,
-                                                      int nsplit) {
-    const int r = blockIdx.x;
-    const int64_t b = blockIdx.y;
+__global__ void __launch_bounds__(D) combine_kernel(TView O, Geom G, ListsView L, const float *__restrict__ part,
+                                                    int nsplit, int eps) {
+    const int row = blockIdx.x, r = blockIdx.y;
+    const int64_t b = blockIdx.z;
     const int g = G.g;
-    const int M = (int)G.nq * g;
+    const int col = threadIdx.x;
     const int count = L.count[((size_t)b * G.hkv + r) * L.n_tiles];
-    const int ns = min(nsplit, (count + kEntriesPerSplit - 1) / kEntriesPerSplit);
-    const float *src = part + ((size_t)b * G.hkv + r) * nsplit * kDecRows * (D + 2);
-    for (int idx = threadIdx.x; idx < M * D; idx += blockDim.x) {
-        const int row = idx / D, col = idx % D;
-        float mm = -INFINITY;
-        for (int s = 0; s < ns; ++s) mm = fmaxf(mm, src[((size_t)s * kDecRows + row) * (D + 2)]);
-        float num = 0.f, den = 0.f;
-        for (int s = 0; s < ns; ++s) {
-            const float *p = src + ((size_t)s * kDecRows + row) * (D + 2);
-            const float f = p[0] == -INFINITY ? 0.f : ex2d(p[0] - mm);
-            den += f * p[1];
-            num += f * p[2 + col];
-        }
-        __nv_bfloat16 *op = reinterpret_cast<__nv_bfloat16 *>(const_cast<void *>(O.p)) + b * O.s0 +
-                            tile_row(L, G, ((size_t)b * G.hkv + r) * L.n_tiles, 0, row / g) * O.s1 +
-                            (int64_t)(r * g + row % g) * O.s2;
-        op[col] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
+    const int ns = min(nsplit, (count + eps - 1) / eps);
+    const float *src = part + ((size_t)b * G.hkv + r) * nsplit * kDecRows * (D + 2) + (size_t)row * (D + 2);
+    constexpr size_t kStride = (size_t)kDecRows * (D + 2);  // from one split's partial of this row to the next
+    float mm = -INFINITY;
+#pragma unroll 4
+    for (int s = 0; s < ns; ++s) mm = fmaxf(mm, src[s * kStride]);
+    float num = 0.f, den = 0.f;
+#pragma unroll 4
+    for (int s = 0; s < ns; ++s) {
+        const float *p = src + s * kStride;
+        const float f = p[0] == -INFINITY ? 0.f : ex2d(p[0] - mm);
+        den += f * p[1];
+        num += f * p[2 + col];
     }
+    __nv_bfloat16 *op = reinterpret_cast<__nv_bfloat16 *>(const_cast<void *>(O.p)) + b * O.s0 +
+                        tile_row(L, G, ((size_t)b * G.hkv + r) * L.n_tiles, 0, row / g) * O.s1 +
+                        (int64_t)(r * g + row % g) * O.s2;
+    op[col] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
 }
 
-int n_splits(const Geom &G) { return (G.n_blk + kEntriesPerSplit - 1) / kEntriesPerSplit; }
+// List entries per split: 16, or fewer when the (batch, kv head) units are few, so that
+// the splits a list may need still give every SM several CTAs (16 per SM for lists
+// that route a sixteenth of their chunks).
+int entries_per_split(const Geom &G) {
+    const int64_t units = G.b * (int64_t)G.hkv;
+    for (int eps = kEntriesPerSplit; eps > 4; eps /= 2)
+        if ((int64_t)((G.n_blk + eps - 1) / eps) * units >= 16 * 148) return eps;
+    return 4;
+}
+
+int n_splits(const Geom &G) {
+    const int eps = entries_per_split(G);
+    return (G.n_blk + eps - 1) / eps;
+}
 
 template <int D, int BLK>
 cudaError_t launch_dec(const DecParams &dp, const TView &Q, const TView &O, const Geom &G, const ListsView &L,
@@ -363,11 +377,12 @@ cudaError_t launch_dec(const DecParams &dp, const TView &Q, const TView &O, cons
     cudaError_t e = cudaFuncSetAttribute(attn_decode_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    const int ns = n_splits(G);
+    const int ns = n_splits(G), eps = entries_per_split(G);
     attn_decode_kernel<D, BLK><<<dim3((unsigned)ns, (unsigned)G.hkv, (unsigned)G.b), kDecThreads, smem, st>>>(
-        dp, Q, G, L, part, ns);
+        dp, Q, G, L, part, ns, eps);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    combine_kernel<D><<<dim3((unsigned)G.hkv, (unsigned)G.b), 128, 0, st>>>(O, G, L, part, ns);
+    combine_kernel<D><<<dim3((unsigned)(G.nq * G.g), (unsigned)G.hkv, (unsigned)G.b), D, 0, st>>>(O, G, L, part,
+                                                                                                   ns, eps);
     return cudaGetLastError();
 }
 

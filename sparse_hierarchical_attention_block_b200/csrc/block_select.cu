@@ -418,7 +418,8 @@ __global__ void __launch_bounds__(128) compact_kernel(Geom G, const uint32_t *__
             if (G.causal && c == (int)(row_pos(G, i) / G.B)) {
                 v = 0.f;  // diagonal chunk: bias 0, causal mask in Stage 2
             } else if (c < row_nvis(G, i) && ((mask[rowoff * G.words + c / 32] >> (c % 32)) & 1u)) {
-                v = (logw[logw_index(G, b, r, i, c)] - mu[rowoff]) * inv_sigma;  // d_c = (log w_c - mu) / sigma
+                // d_c = (log w_c - mu) / sigma; 0 for a caller's mask (uniform prior over R)
+                v = logw ? (logw[logw_index(G, b, r, i, c)] - mu[rowoff]) * inv_sigma : 0.f;
             }
         }
         bias[(size_t)e * T + s] = v;
@@ -493,7 +494,7 @@ __global__ void __launch_bounds__(kRegroupThreads) regroup_compact_kernel(Geom G
                 mrow[j * R.ws + w] = m;
                 cnt += __popc(m);
             }
-            murow[j] = mu[(size_t)(b * G.nq + i) * G.hkv + r];
+            murow[j] = mu ? mu[(size_t)(b * G.nq + i) * G.hkv + r] : 0.f;
             k = ((uint32_t)cnt << 16) | (uint32_t)j;
         } else if (j < R.W) {
             for (int w = 0; w < G.words; ++w) mrow[j * R.ws + w] = 0u;
@@ -616,7 +617,8 @@ __global__ void __launch_bounds__(kRegroupThreads) regroup_compact_kernel(Geom G
             if (G.causal && c == (int)(row_pos(G, i) / G.B)) {
                 v = 0.f;
             } else if (c < row_nvis(G, i) && ((mrow[sl * R.ws + c / 32] >> (c % 32)) & 1u)) {
-                v = (logw[logw_index(G, b, r, i, c)] - murow[sl]) * inv_sigma;  // d_c = (log w_c - mu) / sigma
+                // d_c = (log w_c - mu) / sigma; 0 for a caller's mask (uniform prior over R)
+                v = logw ? (logw[logw_index(G, b, r, i, c)] - murow[sl]) * inv_sigma : 0.f;
             }
         }
         bias[(size_t)e * T + j] = v;

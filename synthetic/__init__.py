@@ -157,3 +157,33 @@ def make_inputs(w: Workload, device="cpu", a_max: float | None = None):
     k = parts.k.to(dt)
     v = parts.v.to(dt)
     return q, k, v
+
+
+def random_block_mask(batch: int, nq: int, nk: int, hkv: int, block: int, s: float, seed: int,
+                      causal: bool = True, device="cpu") -> torch.Tensor:
+    """A random routing mask at block sparsity ``s``, the controlled-sparsity input of the
+    Stage-2 benchmark (the pages inject such a mask at Stage 2 in place of the router's).
+
+    Each (batch, query row, kv head) routes round((1 - s) * n_i) of the n_i chunks it may
+    route, uniformly without replacement: n_i = min(floor(p_i / B), floor(nk / B)) with
+    p_i = i + nk - nq when causal, every one of ceil(nk / B) chunks otherwise.  Returns
+    the bit-packed words [batch, nq, hkv, ceil(n_chunks / 32)] as int32 (bit c % 32 of
+    word c // 32 = chunk c), drawn from a generator on ``device`` seeded with ``seed``."""
+    n_chunks = nk // block if causal else -(-nk // block)
+    words = max((n_chunks + 31) // 32, 1)
+    gen = torch.Generator(device=device).manual_seed(seed)
+    if causal:
+        p = torch.arange(nq, device=device, dtype=torch.int64) + (nk - nq)
+        n_vis = torch.clamp(p // block, max=n_chunks)
+    else:
+        n_vis = torch.full((nq,), n_chunks, device=device, dtype=torch.int64)
+    n_sel = torch.round((1.0 - s) * n_vis.to(torch.float64)).to(torch.int64)       # [nq]
+    u = torch.rand(batch, nq, hkv, max(n_chunks, 1), generator=gen, device=device)
+    c = torch.arange(max(n_chunks, 1), device=device)
+    u = torch.where(c.view(1, 1, 1, -1) < n_vis.view(1, -1, 1, 1), u, torch.full_like(u, 2.0))
+    order = torch.argsort(u, dim=-1)                                                  # visible chunks first
+    take = (c.view(1, 1, 1, -1) < n_sel.view(1, -1, 1, 1)).expand_as(order)
+    bits = torch.zeros(batch, nq, hkv, words * 32, dtype=torch.int64, device=device)
+    bits[..., :max(n_chunks, 1)].scatter_(-1, order, take.to(torch.int64))
+    packed = (bits.view(batch, nq, hkv, words, 32) << torch.arange(32, device=device)).sum(-1)
+    return torch.where(packed >= 2 ** 31, packed - 2 ** 32, packed).to(torch.int32)

@@ -129,6 +129,35 @@ def test_learned_summary_arguments_are_checked():
         dash.dash_attn_fwd(q, k, v, out, 64, 1.5, True, 2, kbar=kb, qbar=torch.zeros(1, nch, 2, 64, device="cuda"))
 
 
+@pytest.mark.parametrize("b,nq,nk,hq,hkv,B,s,regroup", [
+    (1, 1024, 1024, 32, 2, 64, 0.75, False),    # the controlled-sparsity benchmark's heads (g = 16)
+    (1, 1024, 1024, 32, 2, 64, 0.9375, True),
+    (2, 700, 1000, 8, 2, 64, 0.5, True),        # ragged, nq < nk
+    (4, 1, 4096, 32, 8, 64, 0.875, False),      # decode (split-KV path)
+])
+def test_random_mask_stage2(b, nq, nk, hq, hkv, B, s, regroup):
+    """Stage 2 on work lists built from a random routing mask (dash_lists_from_mask) against
+    the oracle's Stage 2 given the same routed sets and a uniform prior (bias 0)."""
+    q, k, v = _planted(b, nq, nk, hq, hkv, 128, B, "bf16", seed=500 + nq, planted=False)
+    g = hq // hkv
+    mask = synthetic.random_block_mask(b, nq, nk, hkv, B, s, seed=17, device="cuda")
+    lists = dash.lists_from_mask(mask, nk, hkv, B, g, causal=True, regroup=regroup)
+    out = torch.empty_like(q)
+    dash.dash_sparse_attn_fwd(q, k, v, out, lists, B, True, g)
+    assert dash.dash_sync_status() == 0
+    nch = dash.n_chunks(nk, B, True)
+    bits = ((mask.to(torch.int64) & 0xFFFFFFFF).unsqueeze(-1) >> torch.arange(32, device="cuda")) & 1
+    routed = bits.flatten(-2)[..., :nch].to(torch.uint8).cpu().numpy()
+    max_tol, mean_tol = 2e-2, 2e-3
+    rows = np.arange(nq)
+    for bi in range(b):
+        r_in = routed[bi]
+        ref = oracle.fwd_rows(to_np32(q[bi]), rows, nq, to_np32(k[bi]), to_np32(v[bi]), B, 1.5,
+                              w_in=r_in.astype(np.float64), r_in=r_in, want=("out",))
+        err = np.abs(to_np32(out[bi]).astype(np.float64) - ref["out"])
+        assert err.max() <= max_tol and err.mean() <= mean_tol, (err.max(), err.mean())
+
+
 @pytest.mark.parametrize("dt,causal", [("bf16", True), ("bf16", False), ("f32", True)])
 def test_uniform_all_chunk_prior_is_dense_attention(dt, causal):
     """Stage 2 alone on lists that route every visible chunk with bias 0 equals
