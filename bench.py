@@ -55,8 +55,8 @@ L2_FLUSH_BYTES = 256 << 20
 # (profiles/attn_decode_decode.md).  Workloads without a capture report null.
 TRAFFIC_BYTES = {
     ("prefill8k", 1): 1.4479e8,
-    ("decode", 16): 1.654e9,
-    ("decode", 4): 4.135e8,
+    ("decode", 16): 1.6565e9,
+    ("decode", 4): 4.1412e8,
 }
 
 
