@@ -101,6 +101,9 @@ typedef struct {
                                          arrives at, gives up after a short bound and
                                          reports DASH_ERR_DEVICE_TIMEOUT */
 
+/* Persistent chunk-summary cache for incremental decoding (see dash_summary_cache_create). */
+typedef struct dash_summary_cache dash_summary_cache_t;
+
 /* Optional settings.  Fill with dash_opts_init(). */
 typedef struct {
     float sigma;            /* prior strength sigma > 0; default 1e8 ([Dash] App. F.5 picks 1e8) */
@@ -114,6 +117,9 @@ typedef struct {
     const dash_tensor_t *qbar; /* optional learned summary queries of Stage 0, see
                                dash_pool_keys_q; NULL = q̄ = 0 (mean pooling).  Not
                                together with kbar. */
+    const dash_summary_cache_t *summary_cache; /* optional: Stage 0 and the summaries'
+                               operand form come from this cache, which must hold every
+                               complete chunk of k (causal only; not with kbar or qbar) */
 } dash_opts_t;
 
 /* Fill *opts with the defaults above.  Returns DASH_OK or DASH_ERR_INVALID_ARG (NULL). */
@@ -151,6 +157,33 @@ DASH_API int dash_pool_keys(const dash_tensor_t *k, int block_size, int causal, 
  * plus DASH_ERR_INVALID_ARG when qbar's shape does not match. */
 DASH_API int dash_pool_keys_q(const dash_tensor_t *k, const dash_tensor_t *qbar, int block_size, int causal,
                               float *kbar, void *stream);
+
+/* Persistent chunk-summary cache ([Dash] §3.5: a chunk's summary is written once the
+ * chunk is complete and reused by every later query position and decoding step).  It
+ * holds, in device memory it owns, the fp32 summaries of up to floor(max_nk / block_size)
+ * chunks of `batch` sequences and their bf16 hi + lo split (the operand form of the
+ * tensor-core Stage 1), so that a decoding step pools and splits nothing.
+ * create: allocates on the current device, no chunk pooled.  Errors DASH_ERR_INVALID_ARG
+ *   (sizes, NULL cache), DASH_ERR_UNSUPPORTED (d or block size), DASH_ERR_CUDA (allocation). */
+DASH_API int dash_summary_cache_create(int64_t batch, int64_t max_nk, int hkv, int d, int block_size,
+                                       dash_summary_cache_t **cache);
+/* Pools every chunk completed since the last update: k [batch, nk, hkv, d] (f32 or bf16)
+ * holds the sequences' first nk <= max_nk keys; chunks [pooled, floor(nk/B)) are pooled
+ * (with the learned summary queries qbar [1 or batch, floor(max_nk/B), hkv, d] when not
+ * NULL, as in dash_pool_keys_q) and the split tiles they fall in are rebuilt.  The keys of
+ * pooled chunks must not change afterwards (reset the cache first).  Asynchronous on
+ * stream.  DASH_ERR_INVALID_ARG when k does not match the cache or holds fewer complete
+ * chunks than were pooled. */
+DASH_API int dash_summary_cache_update(dash_summary_cache_t *cache, const dash_tensor_t *k,
+                                       const dash_tensor_t *qbar, void *stream);
+/* Forgets every pooled chunk (new sequences).  Host-side only. */
+DASH_API int dash_summary_cache_reset(dash_summary_cache_t *cache);
+/* Chunks pooled so far; -1 for a NULL cache. */
+DASH_API int64_t dash_summary_cache_chunks(const dash_summary_cache_t *cache);
+/* The fp32 summaries [batch][floor(max_nk/B)][hkv][d] (device memory the cache owns). */
+DASH_API const float *dash_summary_cache_kbar(const dash_summary_cache_t *cache);
+/* Waits for the device, then frees the cache.  NULL is a no-op. */
+DASH_API int dash_summary_cache_destroy(dash_summary_cache_t *cache);
 
 /* Stage 1 alone ([Dash] §3.2 Eq. 4; App. G Alg. 2).  Every output is optional
  * (NULL to skip):

@@ -62,7 +62,7 @@ class _Opts(ctypes.Structure):
     _fields_ = [("sigma", ctypes.c_float), ("gamma", ctypes.c_float), ("stream", ctypes.c_void_p),
                 ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
                 ("kbar", ctypes.c_void_p), ("flags", ctypes.c_int),
-                ("qbar", ctypes.POINTER(_Tensor))]
+                ("qbar", ctypes.POINTER(_Tensor)), ("summary_cache", ctypes.c_void_p)]
 
 
 _lib = None
@@ -71,7 +71,9 @@ _lib = None
 EXPORTS = ("dash_opts_init", "dash_attn_fwd", "dash_attn_fwd_ex", "dash_pool_keys", "dash_block_select",
            "dash_sparse_attn_fwd", "dash_lists_geometry", "dash_workspace_bytes", "dash_last_error",
            "dash_sync_status", "dash_release", "dash_version", "dash_attn_fwd_noalloc", "dash_pool_keys_q",
-           "dash_lists_from_mask")
+           "dash_lists_from_mask", "dash_summary_cache_create", "dash_summary_cache_update",
+           "dash_summary_cache_reset", "dash_summary_cache_chunks", "dash_summary_cache_kbar",
+           "dash_summary_cache_destroy")
 
 # size of the library's static scratch area used by dash_attn_fwd_noalloc
 DASH_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -95,6 +97,14 @@ def load_library():
     lib.dash_pool_keys.argtypes = [T, i32, i32, P, P]
     lib.dash_pool_keys_q.argtypes = [T, T, i32, i32, P, P]
     lib.dash_lists_from_mask.argtypes = [P, i64, i64, i64, i32, i32, i32, i32, i32, ctypes.POINTER(_Lists), P]
+    lib.dash_summary_cache_create.argtypes = [i64, i64, i32, i32, i32, ctypes.POINTER(ctypes.c_void_p)]
+    lib.dash_summary_cache_update.argtypes = [P, T, T, P]
+    lib.dash_summary_cache_reset.argtypes = [P]
+    lib.dash_summary_cache_chunks.argtypes = [P]
+    lib.dash_summary_cache_chunks.restype = i64
+    lib.dash_summary_cache_kbar.argtypes = [P]
+    lib.dash_summary_cache_kbar.restype = P
+    lib.dash_summary_cache_destroy.argtypes = [P]
     lib.dash_block_select.argtypes = [T, T, i32, f32, i32, i32, P, P, P, ctypes.POINTER(_Lists),
                                       ctypes.POINTER(_Opts)]
     lib.dash_sparse_attn_fwd.argtypes = [T, T, T, T, ctypes.POINTER(_Lists), i32, i32, i32, ctypes.POINTER(_Opts)]
@@ -141,7 +151,8 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _opts(sigma=1e8, gamma=1.0, kbar=None, workspace=None, flags=0, stream=None, qbar=None) -> _Opts:
+def _opts(sigma=1e8, gamma=1.0, kbar=None, workspace=None, flags=0, stream=None, qbar=None,
+          summary_cache=None) -> _Opts:
     o = _Opts()
     load_library().dash_opts_init(ctypes.byref(o))
     o.sigma = float(sigma)
@@ -160,8 +171,61 @@ def _opts(sigma=1e8, gamma=1.0, kbar=None, workspace=None, flags=0, stream=None,
         qd = _desc(qbar)
         o._qbar_desc = qd  # kept alive with the options
         o.qbar = ctypes.pointer(qd)
+    if summary_cache is not None:
+        o.summary_cache = summary_cache.handle
     o.flags = int(flags)
     return o
+
+
+class SummaryCache:
+    """Persistent chunk-summary cache for incremental decoding (dash_summary_cache_*):
+    the fp32 summaries of every completed chunk and their split operand form, kept on
+    the device across decoding steps.  update(k) pools the chunks completed since the
+    last update; pass the cache to a forward as ``summary_cache=``."""
+
+    def __init__(self, batch, max_nk, hkv, d, block_size):
+        self._lib = load_library()
+        h = ctypes.c_void_p()
+        _check(self._lib.dash_summary_cache_create(int(batch), int(max_nk), int(hkv), int(d), int(block_size),
+                                                   ctypes.byref(h)))
+        self.handle = h.value
+        self.batch, self.max_nk, self.hkv, self.d, self.block_size = batch, max_nk, hkv, d, block_size
+
+    def update(self, k, qbar=None, stream=None):
+        kd = _desc(k)
+        qd = ctypes.byref(_desc(qbar)) if qbar is not None else None
+        s = torch.cuda.current_stream() if stream is None else stream
+        _check(self._lib.dash_summary_cache_update(self.handle, ctypes.byref(kd), qd, ctypes.c_void_p(s.cuda_stream)))
+        return self
+
+    def reset(self):
+        _check(self._lib.dash_summary_cache_reset(self.handle))
+
+    @property
+    def chunks(self) -> int:
+        return int(self._lib.dash_summary_cache_chunks(self.handle))
+
+    def kbar(self) -> torch.Tensor:
+        """A copy of the cached summaries [batch, max_nk // block_size, hkv, d] (fp32)."""
+        shape = (self.batch, self.max_nk // self.block_size, self.hkv, self.d)
+        ptr = self._lib.dash_summary_cache_kbar(self.handle)
+
+        class _View:  # the cache's own buffer, read through the CUDA array interface
+            __cuda_array_interface__ = {"shape": shape, "typestr": "<f4", "data": (ptr, False), "version": 3,
+                                        "strides": None}
+
+        return torch.as_tensor(_View(), device="cuda").clone()
+
+    def close(self):
+        if self.handle:
+            _check(self._lib.dash_summary_cache_destroy(self.handle))
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def n_chunks(nk: int, block_size: int, causal: bool) -> int:

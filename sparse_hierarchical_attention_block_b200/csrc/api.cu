@@ -19,6 +19,18 @@ int take_device_error_select();
 
 using namespace dash;
 
+// The persistent chunk-summary cache (dash_summary_cache_t in the C header).
+struct dash_summary_cache {
+    int64_t b, max_nk;
+    int hkv, d, B;
+    int cap;       // chunk capacity floor(max_nk / B): the summaries' batch stride
+    int ct_cap;    // 128-chunk tiles of the split form per (batch, kv head)
+    int64_t done;  // chunks pooled so far
+    int dev;
+    float *kbar;     // [b][cap][hkv][d] fp32
+    uint8_t *split;  // [b][hkv][ct_cap] bf16 hi + lo operand tiles
+};
+
 namespace {
 
 thread_local std::string g_last_error;
@@ -87,6 +99,8 @@ int make_geom(const dash_tensor_t *q, const dash_tensor_t *k, int B, int causal,
     G->tile_rows = 128 / gqa;
     G->n_tiles = (nq + G->tile_rows - 1) / G->tile_rows;
     G->words = (G->n_chunks + 31) / 32;
+    G->kbar_cap = G->n_chunks;
+    G->ct_cap = (G->n_chunks + 127) / 128;
     return DASH_OK;
 }
 
@@ -199,7 +213,7 @@ ListsView ws_lists(const Geom &G, char *ws, const WsLayout &WL, bool with_rows) 
 // (and LV->rows, if given, is filled accordingly).
 int run_stage1(const dash_tensor_t *q, const Geom &G, float alpha, const dash_opts_t &o, const float *kbar,
                float *tau, float *w, uint32_t *mask_out, const ListsView *LV, bool regroup, char *ws,
-               const WsLayout &WL, cudaStream_t st) {
+               const WsLayout &WL, cudaStream_t st, const uint8_t *presplit = nullptr) {
     cudaError_t e;
     const bool tile = select_tile_supported(G, q->dtype);
     regroup = regroup && LV && LV->rows && regroup_supported(G);
@@ -208,7 +222,7 @@ int run_stage1(const dash_tensor_t *q, const Geom &G, float alpha, const dash_op
     float *mu = reinterpret_cast<float *>(ws + WL.mu);
     if (tile) {
         e = launch_select_tile(view(q), kbar, G, alpha, o.gamma, tau, w, mask, LV ? logw : nullptr,
-                               LV ? mu : nullptr, ws + WL.split, st);
+                               LV ? mu : nullptr, ws + WL.split, st, presplit);
         if (e != cudaSuccess) return cuda_fail(e, "select_tile");
     } else {
         SelectOut so{tau, w, mask, LV ? logw : nullptr, LV ? mu : nullptr};
@@ -261,6 +275,31 @@ int run_stage0(const dash_tensor_t *k, const dash_tensor_t *qb, const TView &qv,
     cudaError_t e = qb ? launch_pool_keys_q(view(k), k->dtype, qv, qb->dtype, G, kbar, st)
                        : launch_pool_keys(view(k), k->dtype, G, kbar, st);
     return e == cudaSuccess ? DASH_OK : cuda_fail(e, "pool_keys");
+}
+
+// A summary cache given in the options must match the problem and hold every complete chunk.
+int check_cache(const dash_summary_cache *sc, const Geom &G, const dash_opts_t &o) {
+    if (o.kbar || o.qbar) return fail(DASH_ERR_INVALID_ARG, "opts: summary_cache is not used with kbar or qbar");
+    if (!G.causal) return fail(DASH_ERR_INVALID_ARG, "summary_cache needs causal routing");
+    if (sc->b != G.b || sc->hkv != G.hkv || sc->d != G.d || sc->B != G.B)
+        return fail(DASH_ERR_INVALID_ARG, "summary_cache was made for another shape or block size");
+    if (sc->done != G.n_chunks)
+        return fail(DASH_ERR_INVALID_ARG, "summary_cache holds %lld chunks; the keys have %d complete chunks",
+                    (long long)sc->done, G.n_chunks);
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != sc->dev)
+        return fail(DASH_ERR_INVALID_ARG, "summary_cache lives on another device");
+    return DASH_OK;
+}
+
+// The geometry Stage 1 sees with a summary cache: the cache's strides.
+Geom cache_geom(const Geom &G, const dash_summary_cache *sc) {
+    Geom G1 = G;
+    if (sc) {
+        G1.kbar_cap = sc->cap;
+        G1.ct_cap = sc->ct_cap;
+    }
+    return G1;
 }
 
 int validate_qkvo(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v,
@@ -334,6 +373,8 @@ DASH_API size_t dash_workspace_bytes(int64_t batch, int64_t nq, int64_t nk, int 
     G.tile_rows = 128 / G.g;
     G.n_tiles = (nq + G.tile_rows - 1) / G.tile_rows;
     G.words = (G.n_chunks + 31) / 32;
+    G.kbar_cap = G.n_chunks;
+    G.ct_cap = (G.n_chunks + 127) / 128;
     return ws_layout(G, true, true, true).total;
 }
 
@@ -413,15 +454,17 @@ DASH_API int dash_block_select(const dash_tensor_t *q, const dash_tensor_t *k, i
     for (const void *p : {(const void *)tau, (const void *)w, (const void *)mask})
         if (reinterpret_cast<uintptr_t>(p) % 16) return fail(DASH_ERR_ALIGNMENT, "outputs must be 16-byte aligned");
     TView qv{};
+    const dash_summary_cache *sc = o.summary_cache;
+    if (sc && (rc = check_cache(sc, G, o))) return rc;
     if (o.qbar && o.kbar) return fail(DASH_ERR_INVALID_ARG, "opts: give kbar or qbar, not both");
     if (o.qbar && (rc = check_qbar(o.qbar, G, &qv))) return rc;
     if (G.b == 0 || G.nq == 0) return DASH_OK;
-    const bool need_kbar = o.kbar == nullptr;
+    const bool need_kbar = o.kbar == nullptr && !sc;
     WsLayout WL = ws_layout(G, need_kbar, true, false);
     char *ws = nullptr;
     if ((rc = get_workspace(o, WL.total, &ws))) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(o.stream);
-    const float *kbar = o.kbar;
+    const float *kbar = sc ? sc->kbar : o.kbar;
     if (need_kbar) {
         float *kb = reinterpret_cast<float *>(ws + WL.kbar);
         if ((rc = run_stage0(k, o.qbar, qv, G, kb, st))) return rc;
@@ -430,7 +473,8 @@ DASH_API int dash_block_select(const dash_tensor_t *q, const dash_tensor_t *k, i
     ListsView LV;
     if (lists) LV = lists_view(lists);
     const bool regroup = lists && lists->rows && !(o.flags & DASH_FLAG_NO_REGROUP) && G.n_tiles > 1;
-    return run_stage1(q, G, alpha, o, kbar, tau, w, mask, lists ? &LV : nullptr, regroup, ws, WL, st);
+    return run_stage1(q, cache_geom(G, sc), alpha, o, kbar, tau, w, mask, lists ? &LV : nullptr, regroup, ws, WL,
+                      st, sc ? sc->split : nullptr);
 }
 
 DASH_API int dash_sparse_attn_fwd(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v,
@@ -463,16 +507,18 @@ DASH_API int dash_attn_fwd_ex(const dash_tensor_t *q, const dash_tensor_t *k, co
     if ((rc = make_geom(q, k, block_size, causal, gqa_groups, &G))) return rc;
     if (o.kbar && reinterpret_cast<uintptr_t>(o.kbar) % 16) return fail(DASH_ERR_ALIGNMENT, "kbar not aligned");
     TView qv{};
+    const dash_summary_cache *sc = o.summary_cache;
+    if (sc && (rc = check_cache(sc, G, o))) return rc;
     if (o.qbar && o.kbar) return fail(DASH_ERR_INVALID_ARG, "opts: give kbar or qbar, not both");
     if (o.qbar && (rc = check_qbar(o.qbar, G, &qv))) return rc;
     if (G.b == 0 || G.nq == 0) return DASH_OK;
-    const bool need_kbar = o.kbar == nullptr;
+    const bool need_kbar = o.kbar == nullptr && !sc;
     const bool dec = attn_decode_supported(G, q->dtype) && !(o.flags & DASH_FLAG_FORCE_SIMT);
     WsLayout WL = ws_layout(G, need_kbar, true, dec);
     char *ws = nullptr;
     if ((rc = get_workspace(o, WL.total, &ws))) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(o.stream);
-    const float *kbar = o.kbar;
+    const float *kbar = sc ? sc->kbar : o.kbar;
     if (need_kbar) {
         float *kb = reinterpret_cast<float *>(ws + WL.kbar);
         if ((rc = run_stage0(k, o.qbar, qv, G, kb, st))) return rc;
@@ -480,13 +526,106 @@ DASH_API int dash_attn_fwd_ex(const dash_tensor_t *q, const dash_tensor_t *k, co
     }
     const bool regroup = !(o.flags & DASH_FLAG_NO_REGROUP) && G.n_tiles > 1;
     const ListsView LV = ws_lists(G, ws, WL, regroup);
-    if ((rc = run_stage1(q, G, alpha, o, kbar, nullptr, nullptr, nullptr, &LV, regroup, ws, WL, st))) return rc;
+    if ((rc = run_stage1(q, cache_geom(G, sc), alpha, o, kbar, nullptr, nullptr, nullptr, &LV, regroup, ws, WL, st,
+                         sc ? sc->split : nullptr)))
+        return rc;
     return run_stage2(q, k, v, out, G, LV, o, dec ? ws + WL.decode : nullptr, st);
 }
 
 DASH_API int dash_attn_fwd(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v,
                            dash_tensor_t *out, int block_size, float alpha, int causal, int gqa_groups) {
     return dash_attn_fwd_ex(q, k, v, out, block_size, alpha, causal, gqa_groups, nullptr);
+}
+
+DASH_API int dash_summary_cache_create(int64_t batch, int64_t max_nk, int hkv, int d, int block_size,
+                                       dash_summary_cache_t **cache) {
+    if (!cache) return fail(DASH_ERR_INVALID_ARG, "cache is NULL");
+    *cache = nullptr;
+    if (batch < 1 || hkv < 1 || max_nk < block_size || max_nk > (int64_t)1 << 30)
+        return fail(DASH_ERR_INVALID_ARG, "bad batch, hkv or max_nk for a summary cache");
+    if (d != 64 && d != 128) return fail(DASH_ERR_UNSUPPORTED, "head dim %d not in {64, 128}", d);
+    if (block_size != 16 && block_size != 32 && block_size != 64 && block_size != 128)
+        return fail(DASH_ERR_UNSUPPORTED, "block_size %d not in {16, 32, 64, 128}", block_size);
+    auto *c = new dash_summary_cache{};
+    c->b = batch;
+    c->max_nk = max_nk;
+    c->hkv = hkv;
+    c->d = d;
+    c->B = block_size;
+    c->cap = (int)(max_nk / block_size);
+    c->ct_cap = (c->cap + 127) / 128;
+    c->done = 0;
+    cudaError_t e = cudaGetDevice(&c->dev);
+    if (e == cudaSuccess) e = cudaMalloc(&c->kbar, (size_t)batch * c->cap * hkv * d * sizeof(float));
+    if (e == cudaSuccess) {
+        const size_t sb = kbar_split_bytes(batch, hkv, d, c->ct_cap);
+        e = cudaMalloc(&c->split, sb);
+        if (e == cudaSuccess) e = cudaMemset(c->split, 0, sb);
+    }
+    if (e != cudaSuccess) {
+        cudaFree(c->kbar);
+        cudaFree(c->split);
+        delete c;
+        return cuda_fail(e, "summary cache allocation");
+    }
+    *cache = c;
+    return DASH_OK;
+}
+
+DASH_API int dash_summary_cache_update(dash_summary_cache_t *c, const dash_tensor_t *k, const dash_tensor_t *qbar,
+                                       void *stream) {
+    if (!c) return fail(DASH_ERR_INVALID_ARG, "cache is NULL");
+    int rc = check_tensor(k, "k");
+    if (rc) return rc;
+    if (k->shape[0] != c->b || k->shape[2] != c->hkv || k->shape[3] != c->d || k->shape[1] > c->max_nk)
+        return fail(DASH_ERR_INVALID_ARG, "k [%lld, %lld, %lld, %lld] does not fit the summary cache",
+                    (long long)k->shape[0], (long long)k->shape[1], (long long)k->shape[2], (long long)k->shape[3]);
+    dash_tensor_t q0 = *k;
+    q0.shape[1] = 0;
+    Geom G;
+    if ((rc = make_geom(&q0, k, c->B, 1, 1, &G))) return rc;
+    const int c1 = G.n_chunks;
+    if (c1 < c->done)
+        return fail(DASH_ERR_INVALID_ARG, "k has %d complete chunks but the cache pooled %lld (reset it first)", c1,
+                    (long long)c->done);
+    TView qv{};
+    if (qbar) {
+        Geom Gq = G;
+        Gq.n_chunks = c->cap;
+        if ((rc = check_qbar(qbar, Gq, &qv))) return rc;
+    }
+    if (c1 == c->done) return DASH_OK;
+    G.kbar_cap = c->cap;
+    G.ct_cap = c->ct_cap;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int c0 = (int)c->done;
+    cudaError_t e = qbar ? launch_pool_keys_q(view(k), k->dtype, qv, qbar->dtype, G, c->kbar, st, c0, c1)
+                         : launch_pool_keys(view(k), k->dtype, G, c->kbar, st, c0, c1);
+    if (e != cudaSuccess) return cuda_fail(e, "summary cache pooling");
+    // the split tiles the new chunks fall in (chunks past c1 stay zero until they complete)
+    e = launch_kbar_split(c->kbar, G, c->split, c0 / 128, (c1 + 127) / 128, st);
+    if (e != cudaSuccess) return cuda_fail(e, "summary cache split");
+    c->done = c1;
+    return DASH_OK;
+}
+
+DASH_API int dash_summary_cache_reset(dash_summary_cache_t *c) {
+    if (!c) return fail(DASH_ERR_INVALID_ARG, "cache is NULL");
+    c->done = 0;
+    return DASH_OK;
+}
+
+DASH_API int64_t dash_summary_cache_chunks(const dash_summary_cache_t *c) { return c ? c->done : -1; }
+
+DASH_API const float *dash_summary_cache_kbar(const dash_summary_cache_t *c) { return c ? c->kbar : nullptr; }
+
+DASH_API int dash_summary_cache_destroy(dash_summary_cache_t *c) {
+    if (!c) return DASH_OK;
+    cudaError_t e = cudaDeviceSynchronize();
+    cudaFree(c->kbar);
+    cudaFree(c->split);
+    delete c;
+    return e == cudaSuccess ? DASH_OK : cuda_fail(e, "cudaDeviceSynchronize");
 }
 
 DASH_API int dash_sync_status(void *stream) {

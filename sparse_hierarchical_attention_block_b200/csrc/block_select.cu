@@ -279,7 +279,7 @@ __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(TView Q, const
 
     // (1) logits against the chunks visible to the last row of the group
     const int nvis_max = row_nvis(G, i0 + nrows - 1);
-    const float *kb = kbar + ((size_t)b * G.n_chunks * G.hkv + r) * d;
+    const float *kb = kbar + ((size_t)b * G.kbar_cap * G.hkv + r) * d;
     compute_logits<T>(Qs, npairs, kb, (int64_t)G.hkv * d, nvis_max, d, P, P.gamma * rsqrtf((float)d), X, Ks);
 
     // (2) threshold per (row, head) pair

@@ -23,6 +23,9 @@ struct Geom {
     int tile_rows;  // query positions per Stage-2 tile (128 / g)
     int64_t n_tiles;
     int words;      // ceil(n_chunks / 32) mask words per row
+    int kbar_cap;   // chunks per batch element in the chunk-summary buffer (its batch stride;
+                    // n_chunks, or a persistent cache's capacity)
+    int ct_cap;     // 128-chunk tiles per (batch, kv head) in the split-summary buffer
 };
 
 // Strided 4-D tensor view passed by value to kernels (element strides).

@@ -6,10 +6,12 @@
 namespace dash {
 
 // Stage 0 (pool_keys.cu)
-cudaError_t launch_pool_keys(const TView &K, dash_dtype_t dt, const Geom &G, float *kbar, cudaStream_t st);
+// chunks [c0, c1) (c1 < 0: every chunk) into kbar, whose batch stride is G.kbar_cap chunks
+cudaError_t launch_pool_keys(const TView &K, dash_dtype_t dt, const Geom &G, float *kbar, cudaStream_t st, int c0 = 0,
+                             int c1 = -1);
 // learned summary queries: view [b (stride 0 to broadcast)][n_chunks][hkv][d] of dtype qdt
 cudaError_t launch_pool_keys_q(const TView &K, dash_dtype_t dt, const TView &Qbar, dash_dtype_t qdt, const Geom &G,
-                               float *kbar, cudaStream_t st);
+                               float *kbar, cudaStream_t st, int c0 = 0, int c1 = -1);
 
 // Stage 1 (block_select.cu)
 struct SelectOut {
@@ -26,9 +28,15 @@ size_t select_tile_workspace(const Geom &G);
 // Routing of every (row, head) pair on tensor cores (up to 2048 chunks): tau, optional
 // dense w, the bit mask (required), log w of the routed chunks and mu (optional; both
 // are needed to build work lists).  `work` holds select_tile_workspace(G) bytes.
+// presplit: the split summaries already built (a persistent cache, G.ct_cap tiles per
+// (batch, kv head)); null = split kbar into work first
 cudaError_t launch_select_tile(const TView &Q, const float *kbar, const Geom &G, float alpha, float gamma,
                                float *tau, float *w, uint32_t *mask, float *logw, float *mu, void *work,
-                               cudaStream_t st);
+                               cudaStream_t st, const uint8_t *presplit = nullptr);
+// split the summaries of chunk tiles [ct0, ct1) of kbar (batch stride G.kbar_cap chunks) into
+// split (G.ct_cap tiles per (batch, kv head)); chunks >= G.n_chunks are written as zero
+cudaError_t launch_kbar_split(const float *kbar, const Geom &G, uint8_t *split, int ct0, int ct1, cudaStream_t st);
+size_t kbar_split_bytes(int64_t batch, int hkv, int d, int ct_cap);
 // Regroup the query rows of each window of tiles by routed-set size and build the
 // tiles' work lists (with the row permutation) from the per-row masks and biases.
 bool regroup_supported(const Geom &G);

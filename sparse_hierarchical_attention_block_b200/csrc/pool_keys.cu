@@ -15,9 +15,9 @@
 namespace dash {
 
 template <typename T>
-__global__ void __launch_bounds__(256) pool_keys_kernel(TView K, Geom G, float *__restrict__ kbar) {
+__global__ void __launch_bounds__(256) pool_keys_kernel(TView K, Geom G, float *__restrict__ kbar, int c0) {
     constexpr int VEC = 16 / sizeof(T);  // elements per 16-byte load
-    const int c = blockIdx.x;
+    const int c = c0 + (int)blockIdx.x;
     const int64_t b = blockIdx.y;
     const int ncol = G.hkv * G.d / VEC;  // 16-byte column groups of one token row
     const int rs = ncol >= 256 ? 1 : 256 / ncol;
@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(256) pool_keys_kernel(TView K, Geom G, float *
         }
         if (sub == 0 && cg < ncol) {
             const float inv = 1.f / (float)cnt;
-            float *o = kbar + (((size_t)b * G.n_chunks + c) * G.hkv) * G.d + (size_t)cg * VEC;
+            float *o = kbar + (((size_t)b * G.kbar_cap + c) * G.hkv) * G.d + (size_t)cg * VEC;
 #pragma unroll
             for (int e = 0; e < VEC; e += 4)
                 *reinterpret_cast<float4 *>(o + e) =
@@ -71,17 +71,19 @@ __global__ void __launch_bounds__(256) pool_keys_kernel(TView K, Geom G, float *
     }
 }
 
-cudaError_t launch_pool_keys(const TView &K, dash_dtype_t dt, const Geom &G, float *kbar, cudaStream_t st) {
-    if (G.n_chunks == 0 || G.b == 0) return cudaSuccess;
-    dim3 grid((unsigned)G.n_chunks, (unsigned)G.b);
+cudaError_t launch_pool_keys(const TView &K, dash_dtype_t dt, const Geom &G, float *kbar, cudaStream_t st, int c0,
+                             int c1) {
+    if (c1 < 0) c1 = G.n_chunks;
+    if (c1 <= c0 || G.b == 0) return cudaSuccess;
+    dim3 grid((unsigned)(c1 - c0), (unsigned)G.b);
     const int vec = dt == DASH_BF16 ? 8 : 4;
     const int ncol = G.hkv * G.d / vec;
     const int rs = ncol >= 256 ? 1 : 256 / ncol;
     const size_t smem = rs > 1 ? (size_t)rs * ncol * vec * sizeof(float) : 0;
     if (dt == DASH_BF16)
-        pool_keys_kernel<__nv_bfloat16><<<grid, 256, smem, st>>>(K, G, kbar);
+        pool_keys_kernel<__nv_bfloat16><<<grid, 256, smem, st>>>(K, G, kbar, c0);
     else
-        pool_keys_kernel<float><<<grid, 256, smem, st>>>(K, G, kbar);
+        pool_keys_kernel<float><<<grid, 256, smem, st>>>(K, G, kbar, c0);
     return cudaGetLastError();
 }
 
@@ -119,7 +121,8 @@ template <> struct Piece<float, 2> {
 // batch's loads are already in flight, then one online softmax update: m running
 // maximum (exp2 domain), l running sum of 2^(s - m).
 template <typename T, typename TQ, int D>
-__global__ void __launch_bounds__(256) pool_keys_q_kernel(TView K, TView QB, Geom G, float *__restrict__ kbar) {
+__global__ void __launch_bounds__(256) pool_keys_q_kernel(TView K, TView QB, Geom G, float *__restrict__ kbar, int c0,
+                                                          int c1) {
     constexpr int EPL = D / 32;
     using PK = Piece<T, EPL>;
     using PQ = Piece<TQ, EPL>;
@@ -130,8 +133,8 @@ __global__ void __launch_bounds__(256) pool_keys_q_kernel(TView K, TView QB, Geo
     constexpr int kBatch = 16 / kRegsPerKey;
     const int warp = (int)threadIdx.x / 32, lane = (int)threadIdx.x % 32;
     const int64_t unit = (int64_t)blockIdx.x * 8 + warp;
-    if (unit >= (int64_t)G.n_chunks * G.hkv) return;  // whole warps only
-    const int c = (int)(unit / G.hkv), r = (int)(unit % G.hkv);
+    if (unit >= (int64_t)(c1 - c0) * G.hkv) return;  // whole warps only
+    const int c = c0 + (int)(unit / G.hkv), r = (int)(unit % G.hkv);
     const int64_t b = blockIdx.y;
     const int64_t t0 = (int64_t)c * G.B;
     const int64_t t1 = t0 + G.B < G.nk ? t0 + G.B : G.nk;
@@ -198,7 +201,7 @@ __global__ void __launch_bounds__(256) pool_keys_q_kernel(TView K, TView QB, Geo
         m = mn;
     }
     const float inv = 1.f / l;
-    float *o = kbar + (((size_t)b * G.n_chunks + c) * G.hkv + r) * D + lane * EPL;
+    float *o = kbar + (((size_t)b * G.kbar_cap + c) * G.hkv + r) * D + lane * EPL;
     if constexpr (EPL == 4)
         *reinterpret_cast<float4 *>(o) = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
     else
@@ -206,25 +209,27 @@ __global__ void __launch_bounds__(256) pool_keys_q_kernel(TView K, TView QB, Geo
 }
 
 template <typename T, typename TQ>
-cudaError_t launch_pool_q_t(const TView &K, const TView &QB, const Geom &G, float *kbar, cudaStream_t st) {
-    const int64_t units = (int64_t)G.n_chunks * G.hkv;
+cudaError_t launch_pool_q_t(const TView &K, const TView &QB, const Geom &G, float *kbar, cudaStream_t st, int c0,
+                            int c1) {
+    const int64_t units = (int64_t)(c1 - c0) * G.hkv;
     dim3 grid((unsigned)((units + 7) / 8), (unsigned)G.b);
     if (G.d == 128)
-        pool_keys_q_kernel<T, TQ, 128><<<grid, 256, 0, st>>>(K, QB, G, kbar);
+        pool_keys_q_kernel<T, TQ, 128><<<grid, 256, 0, st>>>(K, QB, G, kbar, c0, c1);
     else
-        pool_keys_q_kernel<T, TQ, 64><<<grid, 256, 0, st>>>(K, QB, G, kbar);
+        pool_keys_q_kernel<T, TQ, 64><<<grid, 256, 0, st>>>(K, QB, G, kbar, c0, c1);
     return cudaGetLastError();
 }
 
 cudaError_t launch_pool_keys_q(const TView &K, dash_dtype_t dt, const TView &Qbar, dash_dtype_t qdt, const Geom &G,
-                               float *kbar, cudaStream_t st) {
-    if (G.n_chunks == 0 || G.b == 0) return cudaSuccess;
+                               float *kbar, cudaStream_t st, int c0, int c1) {
+    if (c1 < 0) c1 = G.n_chunks;
+    if (c1 <= c0 || G.b == 0) return cudaSuccess;
     if (G.d != 64 && G.d != 128) return cudaErrorInvalidValue;
     if (dt == DASH_BF16)
-        return qdt == DASH_BF16 ? launch_pool_q_t<__nv_bfloat16, __nv_bfloat16>(K, Qbar, G, kbar, st)
-                                : launch_pool_q_t<__nv_bfloat16, float>(K, Qbar, G, kbar, st);
-    return qdt == DASH_BF16 ? launch_pool_q_t<float, __nv_bfloat16>(K, Qbar, G, kbar, st)
-                            : launch_pool_q_t<float, float>(K, Qbar, G, kbar, st);
+        return qdt == DASH_BF16 ? launch_pool_q_t<__nv_bfloat16, __nv_bfloat16>(K, Qbar, G, kbar, st, c0, c1)
+                                : launch_pool_q_t<__nv_bfloat16, float>(K, Qbar, G, kbar, st, c0, c1);
+    return qdt == DASH_BF16 ? launch_pool_q_t<float, __nv_bfloat16>(K, Qbar, G, kbar, st, c0, c1)
+                            : launch_pool_q_t<float, float>(K, Qbar, G, kbar, st, c0, c1);
 }
 
 }  // namespace dash

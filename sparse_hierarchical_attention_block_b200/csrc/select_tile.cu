@@ -108,18 +108,17 @@ struct TSmem {
 // fetches a chunk tile with two bulk copies.  Chunks past n_chunks are zero.
 template <int D>
 __global__ void __launch_bounds__(256) kbar_split_kernel(const float *__restrict__ kbar, Geom G,
-                                                         uint8_t *__restrict__ split) {
+                                                         uint8_t *__restrict__ split, int ct0) {
     constexpr int kDh = D / 64, kRegion = 128 * 128;
-    const int ct = blockIdx.x, r = blockIdx.y;
+    const int ct = ct0 + (int)blockIdx.x, r = blockIdx.y;
     const int64_t b = blockIdx.z;
-    const int n_ct = gridDim.x;
-    uint8_t *dst = split + ((((size_t)b * G.hkv + r) * n_ct + ct) * 2) * (size_t)(kDh * kRegion);
+    uint8_t *dst = split + ((((size_t)b * G.hkv + r) * G.ct_cap + ct) * 2) * (size_t)(kDh * kRegion);
     for (int u = threadIdx.x; u < 128 * (D / 8); u += 256) {
         const int c = u / (D / 8), j = u % (D / 8);
         const int cg = ct * 128 + c;
         float v[8];
         if (cg < G.n_chunks) {
-            const float *src = kbar + (((size_t)b * G.n_chunks + cg) * G.hkv + r) * D + j * 8;
+            const float *src = kbar + (((size_t)b * G.kbar_cap + cg) * G.hkv + r) * D + j * 8;
             const float4 a = *reinterpret_cast<const float4 *>(src);
             const float4 q = *reinterpret_cast<const float4 *>(src + 4);
             v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = q.x; v[5] = q.y; v[6] = q.z; v[7] = q.w;
@@ -237,8 +236,7 @@ __global__ void __launch_bounds__(128 * CP, 4 / CP) select_tile_kernel(const __g
             for (int dh = 0; dh < S::kDh; ++dh)
                 tma_load_4d(sm + S::kA + dh * S::kAregion + (128 - kNP) * 128, &tmQ, q_full, dh * 64, r * g,
                             (int)(t * npos), (int)b);
-            const int n_ct_all = (G.n_chunks + kChunkTile - 1) / kChunkTile;
-            const uint8_t *ks = ksplit + (((size_t)b * G.hkv + r) * n_ct_all) * 2 * (size_t)(S::kDh * S::kBregion);
+            const uint8_t *ks = ksplit + (((size_t)b * G.hkv + r) * G.ct_cap) * 2 * (size_t)(S::kDh * S::kBregion);
             auto load_b = [&](int k, int s) {
                 const uint8_t *src = ks + (size_t)k * 2 * S::kDh * S::kBregion;
                 mbar_arrive_expect_tx(k_full + s, 2 * S::kDh * S::kBregion);
@@ -592,23 +590,33 @@ bool select_tile_supported(const Geom &G, dash_dtype_t dt) {
 }
 
 size_t select_tile_workspace(const Geom &G) {
-    const size_t n_ct = (G.n_chunks + kChunkTile - 1) / kChunkTile;
-    return (size_t)G.b * G.hkv * n_ct * 2 * (G.d / 64) * 128 * 128;
+    return kbar_split_bytes(G.b, G.hkv, G.d, (G.n_chunks + kChunkTile - 1) / kChunkTile);
+}
+
+cudaError_t launch_kbar_split(const float *kbar, const Geom &G, uint8_t *split, int ct0, int ct1, cudaStream_t st) {
+    if (ct1 <= ct0 || G.b == 0) return cudaSuccess;
+    if (ct1 > G.ct_cap) return cudaErrorInvalidValue;
+    dim3 sg((unsigned)(ct1 - ct0), (unsigned)G.hkv, (unsigned)G.b);
+    if (G.d == 128) kbar_split_kernel<128><<<sg, 256, 0, st>>>(kbar, G, split, ct0);
+    else kbar_split_kernel<64><<<sg, 256, 0, st>>>(kbar, G, split, ct0);
+    return cudaGetLastError();
+}
+
+size_t kbar_split_bytes(int64_t batch, int hkv, int d, int ct_cap) {
+    return (size_t)batch * hkv * ct_cap * 2 * (d / 64) * 128 * 128;
 }
 
 cudaError_t launch_select_tile(const TView &Q, const float *kbar, const Geom &G, float alpha, float gamma,
                                float *tau, float *w, uint32_t *mask, float *logw, float *mu, void *work,
-                               cudaStream_t st) {
+                               cudaStream_t st, const uint8_t *presplit) {
     if (G.nq == 0 || G.b == 0) return cudaSuccess;
     if (!mask) return cudaErrorInvalidValue;
-    uint8_t *ksplit = static_cast<uint8_t *>(work);
-    const int n_ct = (G.n_chunks + kChunkTile - 1) / kChunkTile;
-    if (n_ct > 0) {
-        dim3 sg((unsigned)n_ct, (unsigned)G.hkv, (unsigned)G.b);
-        if (G.d == 128) kbar_split_kernel<128><<<sg, 256, 0, st>>>(kbar, G, ksplit);
-        else kbar_split_kernel<64><<<sg, 256, 0, st>>>(kbar, G, ksplit);
-        cudaError_t e0 = cudaGetLastError();
+    const uint8_t *ksplit = presplit;
+    if (!presplit) {
+        const int n_ct = (G.n_chunks + kChunkTile - 1) / kChunkTile;
+        cudaError_t e0 = launch_kbar_split(kbar, G, static_cast<uint8_t *>(work), 0, n_ct, st);
         if (e0 != cudaSuccess) return e0;
+        ksplit = static_cast<const uint8_t *>(work);
     }
     TileP P;
     P.alpha = alpha;

@@ -133,3 +133,19 @@ def test_opts_defaults(lib):
     assert o.sigma == pytest.approx(1e8) and o.gamma == 1.0 and o.flags == 0 and not o.workspace
     assert not o.qbar and not o.kbar
     assert lib.dash_opts_init(None) == dash.DASH_ERR_INVALID_ARG
+
+
+def test_summary_cache_arguments(lib):
+    """Host-side checks of the summary-cache entry points (no device memory is touched)."""
+    h = ctypes.c_void_p()
+    assert lib.dash_summary_cache_create(1, 10, 1, 128, 64, ctypes.byref(h)) == dash.DASH_ERR_INVALID_ARG
+    assert lib.dash_summary_cache_create(1, 4096, 1, 96, 64, ctypes.byref(h)) == dash.DASH_ERR_UNSUPPORTED
+    assert lib.dash_summary_cache_create(1, 4096, 1, 128, 48, ctypes.byref(h)) == dash.DASH_ERR_UNSUPPORTED
+    assert lib.dash_summary_cache_create(0, 4096, 1, 128, 64, ctypes.byref(h)) == dash.DASH_ERR_INVALID_ARG
+    assert lib.dash_summary_cache_create(1, 4096, 1, 128, 64, None) == dash.DASH_ERR_INVALID_ARG
+    assert lib.dash_summary_cache_chunks(None) == -1
+    assert lib.dash_summary_cache_kbar(None) is None
+    assert lib.dash_summary_cache_destroy(None) == 0
+    assert lib.dash_summary_cache_reset(None) == dash.DASH_ERR_INVALID_ARG
+    k = _t(FAKE, dash.DASH_BF16, [1, 256, 2, 128])
+    assert lib.dash_summary_cache_update(None, ctypes.byref(k), None, None) == dash.DASH_ERR_INVALID_ARG
