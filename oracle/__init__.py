@@ -55,7 +55,7 @@ def _load():
         lib.dash_oracle_fwd_rows.argtypes = [P, P, i64, i64, P, P, i64, i32, i32, i32, i32, f64, f64, f64,
                                              i32, i32, P, P, P, P, P, P, P, P]
         lib.dash_oracle_fwd_rows_q.argtypes = [P, P, i64, i64, P, P, i64, i32, i32, i32, i32, f64, f64, f64, i32,
-                                               i32, P, P, P, P, P, P, P, P, P]
+                                               i32, P, P, P, i32, P, P, P, P, P, P]
         lib.dash_oracle_dense_attention.argtypes = [P, i64, P, P, i64, i32, i32, i32, i32, P]
         lib.dash_oracle_set_threads.argtypes = [i32]
         lib.dash_oracle_set_threads.restype = None
@@ -141,13 +141,14 @@ def n_chunks_for(nk: int, block_size: int, causal: bool) -> int:
 
 def fwd_rows(Q_rows, rows, nq: int, K, V, block_size: int, alpha: float, *, gamma: float = 1.0,
              sigma: float = 1e8, causal: bool = True, route: int = 0, w_in=None, r_in=None,
-             want=("out", "tau", "w", "routed"), qbar=None):
+             want=("out", "tau", "w", "routed"), qbar=None, local: int = 1):
     """Oracle forward for selected query rows of ONE batch element.
 
     Q_rows [nrows, hq, d] are the rows' query vectors, rows [nrows] their
     indices in [0, nq); K, V are [nk, hkv, d].  qbar [n_chunks, hkv, d] (or a
     shape that broadcasts to it): learned Stage-0 summary queries (None: q̄ = 0,
-    mean pooling).  Returns a dict with the
+    mean pooling).  local: chunks of the local window (1: the query's own chunk; 2: it
+    and the one before, App. B.1.1).  Returns a dict with the
     requested outputs among out, tau, w, routed, xmt, lambda (see the C file).
     """
     lib = _load()
@@ -169,11 +170,11 @@ def fwd_rows(Q_rows, rows, nq: int, K, V, block_size: int, alpha: float, *, gamm
     if w_in is not None:
         w_in = _f64(w_in).reshape(nrows, hkv, nch)
         r_in = np.ascontiguousarray(r_in, dtype=np.uint8).reshape(nrows, hkv, nch)
-    if qbar is not None:
-        qb = _f32(np.broadcast_to(np.asarray(qbar, dtype=np.float32), (nch, hkv, d)))
+    if qbar is not None or local != 1:
+        qb = None if qbar is None else _f32(np.broadcast_to(np.asarray(qbar, dtype=np.float32), (nch, hkv, d)))
         rc = lib.dash_oracle_fwd_rows_q(_ptr(Q_rows), _ptr(rows), nrows, int(nq), _ptr(K), _ptr(V), nk, hq, hkv,
                                         d, int(block_size), float(alpha), float(gamma), float(sigma),
-                                        int(bool(causal)), int(route), _ptr(w_in), _ptr(r_in), _ptr(qb),
+                                        int(bool(causal)), int(route), _ptr(w_in), _ptr(r_in), _ptr(qb), int(local),
                                         _ptr(res["out"]), _ptr(res["tau"]), _ptr(res["w"]), _ptr(res["routed"]),
                                         _ptr(res["xmt"]), _ptr(res["lambda"]))
         if rc:

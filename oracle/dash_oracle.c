@@ -20,7 +20,9 @@
  *   - causal alignment is bottom-right: query row i sits at key position
  *     p_i = i + nk - nq; its own chunk is c_i = floor(p_i / B); it routes
  *     over the complete chunks c < min(c_i, floor(nk/B))              [Dash App. G Alg. 2]
- *   - the diagonal branch D_i is { j : c_i*B <= j <= p_i }             [Dash App. G Algs. 2-3]
+ *   - the diagonal branch D_i is { j : c_i*B <= j <= p_i }             [Dash App. G Algs. 2-3];
+ *     with the two-block local window of App. B.1.1 (local = 2) it is
+ *     { j : (c_i - 1)*B <= j <= p_i } and routing covers c < c_i - 1
  *   - non-causal: every chunk (a trailing partial chunk pooled over its
  *     real tokens) is routed, D_i is empty
  *   - the entmax exponent is 1/(alpha-1)                                [Dash Eq. 2, Eq. 13]
@@ -429,8 +431,8 @@ static void stage2_head(const oracle_cfg_t *cf, const float *q, const float *K, 
 static int fwd_rows_impl(const float *Q, const int64_t *rows, int64_t nrows, int64_t nq, const float *K,
                          const float *V, int64_t nk, int hq, int hkv, int d, int B, double alpha,
                          double gamma, double sigma, int causal, int route, const double *w_in,
-                         const unsigned char *r_in, const float *Qbar, double *out, double *tau, double *w,
-                         unsigned char *routed, double *xmt, double *lambda);
+                         const unsigned char *r_in, const float *Qbar, int local, double *out, double *tau,
+                         double *w, unsigned char *routed, double *xmt, double *lambda);
 
 ORACLE_API int dash_oracle_fwd_rows(const float *Q, const int64_t *rows, int64_t nrows, int64_t nq,
                                     const float *K, const float *V, int64_t nk, int hq, int hkv, int d,
@@ -440,27 +442,30 @@ ORACLE_API int dash_oracle_fwd_rows(const float *Q, const int64_t *rows, int64_t
                                     double *lambda)
 {
     return fwd_rows_impl(Q, rows, nrows, nq, K, V, nk, hq, hkv, d, B, alpha, gamma, sigma, causal, route,
-                         w_in, r_in, NULL, out, tau, w, routed, xmt, lambda);
+                         w_in, r_in, NULL, 1, out, tau, w, routed, xmt, lambda);
 }
 
 /* As dash_oracle_fwd_rows with Stage 0 taken from the learned summary queries
- * Qbar [n_chunks, hkv, d] (dash_oracle_pool_q). */
+ * Qbar [n_chunks, hkv, d] (dash_oracle_pool_q; NULL = mean pooling) and a local window
+ * of `local` chunks (1: the query's own chunk, Algs. 2-3; 2: that chunk and the one
+ * before it, App. B.1.1). */
 ORACLE_API int dash_oracle_fwd_rows_q(const float *Q, const int64_t *rows, int64_t nrows, int64_t nq,
                                       const float *K, const float *V, int64_t nk, int hq, int hkv, int d,
                                       int B, double alpha, double gamma, double sigma, int causal, int route,
                                       const double *w_in, const unsigned char *r_in, const float *Qbar,
-                                      double *out, double *tau, double *w, unsigned char *routed,
+                                      int local, double *out, double *tau, double *w, unsigned char *routed,
                                       double *xmt, double *lambda)
 {
+    if (local != 1 && local != 2) return -1;
     return fwd_rows_impl(Q, rows, nrows, nq, K, V, nk, hq, hkv, d, B, alpha, gamma, sigma, causal, route,
-                         w_in, r_in, Qbar, out, tau, w, routed, xmt, lambda);
+                         w_in, r_in, Qbar, local, out, tau, w, routed, xmt, lambda);
 }
 
 static int fwd_rows_impl(const float *Q, const int64_t *rows, int64_t nrows, int64_t nq, const float *K,
                          const float *V, int64_t nk, int hq, int hkv, int d, int B, double alpha,
                          double gamma, double sigma, int causal, int route, const double *w_in,
-                         const unsigned char *r_in, const float *Qbar, double *out, double *tau, double *w,
-                         unsigned char *routed, double *xmt, double *lambda)
+                         const unsigned char *r_in, const float *Qbar, int local, double *out, double *tau,
+                         double *w, unsigned char *routed, double *xmt, double *lambda)
 {
     if (hq % hkv || !(alpha > 1.0) || B <= 0 || d <= 0 || nk <= 0) return -1;
     if (causal && nq > nk) return -1;
@@ -502,8 +507,10 @@ static int fwd_rows_impl(const float *Q, const int64_t *rows, int64_t nrows, int
             int64_t d0 = 0, d1 = -1;
             if (causal) {
                 ci = (int)(p / B);
-                nvis = ci < n_chunks ? ci : n_chunks;
-                d0 = (int64_t)ci * B;
+                /* the local window: the query's own chunk and, for local = 2, the one before */
+                const int first_local = ci - (local - 1) > 0 ? ci - (local - 1) : 0;
+                nvis = first_local < n_chunks ? first_local : n_chunks;
+                d0 = (int64_t)first_local * B;
                 d1 = p;
             } else {
                 ci = -1;

@@ -26,8 +26,8 @@ MUTATIONS = [
      "for (int64_t t = d0; t < d1; ++t) {\n        const float *kt"),
     ("routing bias sign flipped", "(log(w[c]) - mu) / cf->sigma", "(mu - log(w[c])) / cf->sigma"),
     ("routing bias multiplied by sigma", "(log(w[c]) - mu) / cf->sigma", "(log(w[c]) - mu) * cf->sigma"),
-    ("own chunk routed as well", "nvis = ci < n_chunks ? ci : n_chunks;",
-     "nvis = ci + 1 < n_chunks ? ci + 1 : n_chunks;"),
+    ("own chunk routed as well", "nvis = first_local < n_chunks ? first_local : n_chunks;",
+     "nvis = first_local + 1 < n_chunks ? first_local + 1 : n_chunks;"),
     ("group prior not averaged", "wg[c] += ph[c] / g;", "wg[c] += ph[c];"),
     ("Stage-1 scale 1/d instead of 1/sqrt(d)", "const double zscale = gamma / sqrt((double)d);",
      "const double zscale = gamma / (double)d;"),
@@ -40,6 +40,8 @@ MUTATIONS = [
      "const double a = exp(score[j] - smax);"),
     ("learned pooling uses chunk 0's query everywhere", "const float *qb = Qbar + ((size_t)c * hkv + r) * d;",
      "const float *qb = Qbar + (size_t)r * d;"),
+    ("two-block window drops the previous chunk",
+     "const int first_local = ci - (local - 1) > 0 ? ci - (local - 1) : 0;", "const int first_local = ci;"),
     ("forward ignores the learned query", "if (Qbar)\n        dash_oracle_pool_q(", "if (0)\n        dash_oracle_pool_q("),
 ]
 

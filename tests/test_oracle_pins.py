@@ -331,6 +331,28 @@ def test_uniform_all_chunk_prior_is_dense_attention(causal):
     np.testing.assert_allclose(dense, ref.numpy(), atol=1e-12)
 
 
+def test_two_block_window_with_all_chunks_is_dense_attention():
+    """App. B.1.1's local window (the query's chunk and the one before it): with every chunk
+    before the window routed under a uniform prior, Stage 2 covers exactly the keys j <= p_i
+    once each, so it is dense causal attention; rows in the first two chunks route nothing
+    and no row ever routes the chunk just before its own."""
+    nq, nk, hq, hkv, d, B = 70, 100, 4, 2, 16, 16
+    Q, K, V = _case(4, nq, nk, hq, hkv, d, B, planted=False)
+    nch = oracle.n_chunks_for(nk, B, True)
+    rows = np.arange(nq)
+    r_in = np.zeros((nq, hkv, nch), dtype=np.uint8)
+    for i in range(nq):
+        r_in[i, :, :max(0, min((i + nk - nq) // B - 1, nch))] = 1
+    res = oracle.fwd_rows(Q, rows, nq, K, V, B, 1.5, causal=True, w_in=r_in.astype(np.float64), r_in=r_in,
+                          want=("out",), local=2)
+    np.testing.assert_allclose(res["out"], oracle.dense_attention(Q, K, V, causal=True), atol=1e-12)
+    own = oracle.fwd_rows(Q, rows, nq, K, V, B, 1.5, causal=True, want=("out", "tau", "routed"), local=2)
+    c_i = (rows + nk - nq) // B
+    assert np.isnan(own["tau"][c_i <= 1]).all() and not np.isnan(own["tau"][c_i >= 2]).any()
+    for i in range(nq):
+        assert not own["routed"][i, :, max(c_i[i] - 1, 0):].any()
+
+
 def test_group_prior_properties():
     """w sums to 1, its support is the union of the heads' supports, g = 1 gives w = p (Sec. 3.2)."""
     nq, nk, hq, hkv, d, B = 64, 128, 4, 1, 16, 16
