@@ -97,6 +97,10 @@ typedef struct {
 #define DASH_FLAG_FORCE_SIMT 0x1      /* Stage 2 on the CUDA-core path (testing) */
 #define DASH_FLAG_NO_REGROUP 0x2      /* keep consecutive query rows in each tile (no regrouping
                                          of rows by routed-set size) */
+#define DASH_FLAG_LOCAL2 0x4         /* the two-block local window of [Dash] App. B.1.1: the chunk
+                                         before the query's own is attended in full with bias 0
+                                         together with the diagonal chunk, and routing covers the
+                                         chunks before it (causal only) */
 #define DASH_FLAG_TEST_TIMEOUT 0x100  /* testing only: Stage 2 waits on a barrier nothing
                                          arrives at, gives up after a short bound and
                                          reports DASH_ERR_DEVICE_TIMEOUT */

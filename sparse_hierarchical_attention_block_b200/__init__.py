@@ -38,6 +38,7 @@ DASH_BF16 = 1
 
 DASH_FLAG_FORCE_SIMT = 0x1
 DASH_FLAG_NO_REGROUP = 0x2
+DASH_FLAG_LOCAL2 = 0x4  # the two-block local window (the query's chunk and the one before)
 DASH_FLAG_TEST_TIMEOUT = 0x100
 
 

@@ -101,6 +101,17 @@ int make_geom(const dash_tensor_t *q, const dash_tensor_t *k, int B, int causal,
     G->words = (G->n_chunks + 31) / 32;
     G->kbar_cap = G->n_chunks;
     G->ct_cap = (G->n_chunks + 127) / 128;
+    G->local = 1;
+    return DASH_OK;
+}
+
+// The local window the options ask for (App. B.1.1's two blocks with DASH_FLAG_LOCAL2).
+int set_local(const dash_opts_t &o, Geom *G) {
+    G->local = 1;
+    if (o.flags & DASH_FLAG_LOCAL2) {
+        if (!G->causal) return fail(DASH_ERR_INVALID_ARG, "DASH_FLAG_LOCAL2 needs causal attention");
+        G->local = 2;
+    }
     return DASH_OK;
 }
 
@@ -375,6 +386,7 @@ DASH_API size_t dash_workspace_bytes(int64_t batch, int64_t nq, int64_t nk, int 
     G.words = (G.n_chunks + 31) / 32;
     G.kbar_cap = G.n_chunks;
     G.ct_cap = (G.n_chunks + 127) / 128;
+    G.local = 1;
     return ws_layout(G, true, true, true).total;
 }
 
@@ -450,6 +462,7 @@ DASH_API int dash_block_select(const dash_tensor_t *q, const dash_tensor_t *k, i
     if (!(alpha > 1.f) || !isfinite(alpha)) return fail(DASH_ERR_INVALID_ARG, "alpha must be > 1");
     Geom G;
     if ((rc = make_geom(q, k, block_size, causal, gqa_groups, &G))) return rc;
+    if ((rc = set_local(o, &G))) return rc;
     if (lists && (rc = check_lists(lists, G))) return rc;
     for (const void *p : {(const void *)tau, (const void *)w, (const void *)mask})
         if (reinterpret_cast<uintptr_t>(p) % 16) return fail(DASH_ERR_ALIGNMENT, "outputs must be 16-byte aligned");
@@ -505,6 +518,7 @@ DASH_API int dash_attn_fwd_ex(const dash_tensor_t *q, const dash_tensor_t *k, co
     if (!(alpha > 1.f) || !isfinite(alpha)) return fail(DASH_ERR_INVALID_ARG, "alpha must be > 1");
     Geom G;
     if ((rc = make_geom(q, k, block_size, causal, gqa_groups, &G))) return rc;
+    if ((rc = set_local(o, &G))) return rc;
     if (o.kbar && reinterpret_cast<uintptr_t>(o.kbar) % 16) return fail(DASH_ERR_ALIGNMENT, "kbar not aligned");
     TView qv{};
     const dash_summary_cache *sc = o.summary_cache;

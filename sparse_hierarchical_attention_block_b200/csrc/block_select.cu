@@ -368,7 +368,7 @@ __global__ void __launch_bounds__(128) compact_kernel(Geom G, const uint32_t *__
     // diagonal chunk range of the tile's rows (causal)
     int dlo = 0, dhi = -1;
     if (G.causal) {
-        dlo = (int)(row_pos(G, i0) / G.B);
+        dlo = first_local(G, i0);
         dhi = (int)(row_pos(G, i0 + nrows - 1) / G.B);
         if (dhi > G.n_blk - 1) dhi = G.n_blk - 1;
     }
@@ -415,8 +415,8 @@ __global__ void __launch_bounds__(128) compact_kernel(Geom G, const uint32_t *__
         {
             const int64_t i = i0 + s;
             const size_t rowoff = ((size_t)(b * G.nq + i) * G.hkv + r);
-            if (G.causal && c == (int)(row_pos(G, i) / G.B)) {
-                v = 0.f;  // diagonal chunk: bias 0, causal mask in Stage 2
+            if (G.causal && c >= first_local(G, i) && c <= (int)(row_pos(G, i) / G.B)) {
+                v = 0.f;  // local window (diagonal chunk): bias 0, causal mask in Stage 2
             } else if (c < row_nvis(G, i) && ((mask[rowoff * G.words + c / 32] >> (c % 32)) & 1u)) {
                 // d_c = (log w_c - mu) / sigma; 0 for a caller's mask (uniform prior over R)
                 v = logw ? (logw[logw_index(G, b, r, i, c)] - mu[rowoff]) * inv_sigma : 0.f;
@@ -536,11 +536,14 @@ __global__ void __launch_bounds__(kRegroupThreads) regroup_compact_kernel(Geom G
         L.rows[tile_idx * T + j] = slot[j] >= 0 ? (int)(i0 + slot[j]) : -1;
 
     // diagonal chunks of the tile's rows, relative to the window's first chunk
-    const int dbase = G.causal ? (int)(row_pos(G, i0) / G.B) : 0;
+    // (local windows: the diagonal chunk and, with local = 2, the one before it)
+    const int dbase = G.causal ? first_local(G, i0) : 0;
     uint64_t dmask = 0;
     if (G.causal)
         for (int j = lane; j < T; j += 32)
-            if (slot[j] >= 0) dmask |= 1ull << ((int)(row_pos(G, i0 + slot[j]) / G.B) - dbase);
+            if (slot[j] >= 0)
+                for (int c = first_local(G, i0 + slot[j]); c <= (int)(row_pos(G, i0 + slot[j]) / G.B); ++c)
+                    dmask |= 1ull << (c - dbase);
     dmask = ((uint64_t)__reduce_or_sync(0xffffffffu, (uint32_t)(dmask >> 32)) << 32) |
             __reduce_or_sync(0xffffffffu, (uint32_t)dmask);
     const int nd = __popcll(dmask);
@@ -614,7 +617,7 @@ __global__ void __launch_bounds__(kRegroupThreads) regroup_compact_kernel(Geom G
             v = 0.f;  // unused row: never stored
         } else {
             const int64_t i = i0 + sl;
-            if (G.causal && c == (int)(row_pos(G, i) / G.B)) {
+            if (G.causal && c >= first_local(G, i) && c <= (int)(row_pos(G, i) / G.B)) {
                 v = 0.f;
             } else if (c < row_nvis(G, i) && ((mrow[sl * R.ws + c / 32] >> (c % 32)) & 1u)) {
                 // d_c = (log w_c - mu) / sigma; 0 for a caller's mask (uniform prior over R)
@@ -675,8 +678,10 @@ cudaError_t launch_select_rows(const TView &Q, dash_dtype_t dt, const float *kba
 static size_t regroup_smem(const Geom &G) { return RegroupSmem(G, G.tile_rows, G.n_blk).total; }
 
 bool regroup_supported(const Geom &G) {
-    // the tile_rows of a window must fit the sort key's slot field; shared memory is bounded
-    return G.tile_rows * kTilesPerWindow <= 65536 && regroup_smem(G) <= 200 * 1024;
+    // the tile_rows of a window must fit the sort key's slot field; the local-window chunks
+    // a window's rows touch must fit the 64-bit mask; shared memory is bounded
+    const int64_t span = ((int64_t)G.tile_rows * kTilesPerWindow + G.B - 1) / G.B + 1 + (G.local - 1);
+    return G.tile_rows * kTilesPerWindow <= 65536 && span <= 64 && regroup_smem(G) <= 200 * 1024;
 }
 
 cudaError_t launch_regroup_compact(const Geom &G, const uint32_t *mask, const float *logw, const float *mu,

@@ -26,6 +26,7 @@ struct Geom {
     int kbar_cap;   // chunks per batch element in the chunk-summary buffer (its batch stride;
                     // n_chunks, or a persistent cache's capacity)
     int ct_cap;     // 128-chunk tiles per (batch, kv head) in the split-summary buffer
+    int local;      // chunks of the causal local window: 1 (the query's own) or 2 (and the one before)
 };
 
 // Strided 4-D tensor view passed by value to kernels (element strides).
@@ -60,10 +61,16 @@ __host__ __device__ inline size_t logw_index(const Geom &G, int64_t b, int r, in
 
 // Causal geometry of query row i: key position, own chunk, visible chunks.
 __host__ __device__ inline int64_t row_pos(const Geom &G, int64_t i) { return i + G.nk - G.nq; }
+// first chunk of row i's local window (causal): its own chunk, or the one before with local = 2
+__host__ __device__ inline int first_local(const Geom &G, int64_t i) {
+    const int64_t c = row_pos(G, i) / G.B - (G.local - 1);
+    return (int)(c > 0 ? c : 0);
+}
+// chunks row i routes over: every chunk before its local window (all of them when non-causal)
 __host__ __device__ inline int row_nvis(const Geom &G, int64_t i) {
     if (!G.causal) return G.n_chunks;
-    int64_t c = row_pos(G, i) / G.B;
-    return (int)(c < G.n_chunks ? c : G.n_chunks);
+    const int c = first_local(G, i);
+    return c < G.n_chunks ? c : G.n_chunks;
 }
 
 // ---------------------------------------------------------------------------

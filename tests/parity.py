@@ -33,7 +33,7 @@ def unpack_mask(mask_words: np.ndarray, n_chunks: int) -> np.ndarray:
     return ((w[..., c // 32] >> (c % 32).astype(np.uint32)) & 1).astype(bool)
 
 
-def gpu_stage1(q, k, block_size, alpha, causal, sigma=1e8, gamma=1.0, qbar=None):
+def gpu_stage1(q, k, block_size, alpha, causal, sigma=1e8, gamma=1.0, qbar=None, local=1):
     b, nq, hq, _ = q.shape
     hkv = k.shape[2]
     nch = dash.n_chunks(k.shape[1], block_size, causal)
@@ -42,6 +42,8 @@ def gpu_stage1(q, k, block_size, alpha, causal, sigma=1e8, gamma=1.0, qbar=None)
     w = torch.empty(b, nq, hkv, nch, dtype=torch.float32, device=q.device) if nch else None
     mask = torch.zeros(b, nq, hkv, max(words, 1), dtype=torch.int32, device=q.device)
     extra = {} if qbar is None else {"qbar": qbar}
+    if local == 2:
+        extra["flags"] = dash.DASH_FLAG_LOCAL2
     dash.dash_block_select(q, k, block_size, alpha, causal, tau=tau, w=w, mask=mask, sigma=sigma, gamma=gamma,
                            **extra)
     torch.cuda.synchronize()
@@ -53,17 +55,18 @@ def to_np32(t):
 
 
 def check_forward(q, k, v, out, block_size, alpha, causal, sigma=1e8, gamma=1.0, rows=None, batches=None,
-                  label="", qbar=None):
+                  label="", qbar=None, local=1):
     """Compare a GPU forward (``out``) and its Stage 1 with the oracle.
 
     rows: query indices to check (default all); batches: batch indices (default all);
-    qbar: the learned Stage-0 summary queries [1 or b, n_chunks, hkv, d] given to both.
+    qbar: the learned Stage-0 summary queries [1 or b, n_chunks, hkv, d] given to both;
+    local: chunks of the local window (2: DASH_FLAG_LOCAL2 on the GPU).
     Returns a dict of statistics.
     """
     b, nq, hq, d = q.shape
     nk, hkv = k.shape[1], k.shape[2]
     nch = dash.n_chunks(nk, block_size, causal)
-    tau_g, w_g, mask_g = gpu_stage1(q, k, block_size, alpha, causal, sigma, gamma, qbar)
+    tau_g, w_g, mask_g = gpu_stage1(q, k, block_size, alpha, causal, sigma, gamma, qbar, local)
     rows = np.arange(nq) if rows is None else np.asarray(rows, dtype=np.int64)
     batches = range(b) if batches is None else batches
     max_tol, mean_tol = OUT_TOL[q.dtype]
@@ -76,7 +79,7 @@ def check_forward(q, k, v, out, block_size, alpha, causal, sigma=1e8, gamma=1.0,
         V = to_np32(v[bi])
         qb = None if qbar is None else to_np32(qbar[bi if qbar.shape[0] > 1 else 0])
         ref = oracle.fwd_rows(Qr, rows, nq, K, V, block_size, alpha, gamma=gamma, sigma=sigma, causal=causal,
-                              want=("out", "tau", "w", "routed", "xmt"), qbar=qb)
+                              want=("out", "tau", "w", "routed", "xmt"), qbar=qb, local=local)
         tg = tau_g[bi].index_select(0, rows_t).cpu().numpy()
         wg = (w_g[bi].index_select(0, rows_t).cpu().numpy().astype(np.float64) if nch
               else np.zeros((len(rows), hkv, 0)))
@@ -99,7 +102,8 @@ def check_forward(q, k, v, out, block_size, alpha, causal, sigma=1e8, gamma=1.0,
             stats["w_err"] = max(stats["w_err"], float(we))
             assert we <= W_TOL, f"{label}: w error {we}"
         stats["routed"] += int(ro.sum())
-        vis = np.minimum((rows + nk - nq) // block_size, nch) if causal else np.full(len(rows), nch)
+        vis = (np.minimum(np.maximum((rows + nk - nq) // block_size - (local - 1), 0), nch) if causal
+               else np.full(len(rows), nch))
         stats["visible"] += int(vis.sum()) * hkv
         # --- Stage 2 ---
         flagged = diff.any(axis=2)                # [rows, hkv]
@@ -109,7 +113,8 @@ def check_forward(q, k, v, out, block_size, alpha, causal, sigma=1e8, gamma=1.0,
             fr = np.nonzero(frow)[0]
             w_in = np.where(rg[fr], np.maximum(np.maximum(ref["w"][fr], wg[fr]), 1e-300), 0.0)
             re = oracle.fwd_rows(Qr[fr], rows[fr], nq, K, V, block_size, alpha, gamma=gamma, sigma=sigma,
-                                 causal=causal, w_in=w_in, r_in=rg[fr].astype(np.uint8), want=("out",), qbar=qb)
+                                 causal=causal, w_in=w_in, r_in=rg[fr].astype(np.uint8), want=("out",), qbar=qb,
+                                 local=local)
             exp_out[fr] = re["out"]
         err = np.abs(og - exp_out)
         stats["rows"] += len(rows)

@@ -82,6 +82,7 @@ FAKE = 1 << 20  # never dereferenced: validation fails first
     ("sigma", dash.DASH_ERR_INVALID_ARG),
     ("qbar_shape", dash.DASH_ERR_INVALID_ARG),
     ("qbar_with_kbar", dash.DASH_ERR_INVALID_ARG),
+    ("local2_noncausal", dash.DASH_ERR_INVALID_ARG),
 ])
 def test_validation_rejects(lib, case, code):
     B, alpha, gqa, causal = 64, 1.5, 4, 1
@@ -117,6 +118,9 @@ def test_validation_rejects(lib, case, code):
     elif case == "qbar_shape":  # 4 chunks of 64 keys, not 5
         qb = _t(FAKE, dash.DASH_F32, [1, 5, 2, 128])
         opts.qbar = ctypes.pointer(qb)
+    elif case == "local2_noncausal":
+        causal = 0
+        opts.flags = dash.DASH_FLAG_LOCAL2
     elif case == "qbar_with_kbar":
         qb = _t(FAKE, dash.DASH_F32, [1, 4, 2, 128])
         opts.qbar = ctypes.pointer(qb)

@@ -201,6 +201,32 @@ def test_decode_cases(case):
     check_forward(q, k, v, out, B, alpha, True, sigma=sigma, label=f"decode case {case}")
 
 
+@pytest.mark.parametrize("case", [CASES[0], CASES[3], CASES[6], CASES[7]], ids=["c0", "c3", "c6", "c7"])
+def test_two_block_local_window(case):
+    """App. B.1.1's local window (DASH_FLAG_LOCAL2): the chunk before the query's own is
+    attended in full with bias 0 and not routed; against the oracle with the same window."""
+    b, nq, nk, hq, hkv, d, B, dt, alpha, causal, sigma = case
+    q, k, v = _planted(b, nq, nk, hq, hkv, d, B, dt, seed=700 + nq, causal=causal)
+    out = _run(q, k, v, B, alpha, causal, sigma=sigma, flags=dash.DASH_FLAG_LOCAL2)
+    check_forward(q, k, v, out, B, alpha, causal, sigma=sigma, label=f"local2 {case}", local=2)
+
+
+@pytest.mark.parametrize("case", DECODE_CASES[:2], ids=["d0", "d1"])
+def test_two_block_local_window_decode(case):
+    b, nq, nk, hq, hkv, d, B, alpha, sigma = case
+    q, k, v = _planted(b, nq, nk, hq, hkv, d, B, "bf16", seed=800 + nk)
+    out = _run(q, k, v, B, alpha, True, sigma=sigma, flags=dash.DASH_FLAG_LOCAL2)
+    check_forward(q, k, v, out, B, alpha, True, sigma=sigma, label=f"local2 decode {case}", local=2)
+
+
+def test_two_block_local_window_prefill8k_sampled():
+    w = synthetic.WORKLOADS["prefill8k"]
+    q, k, v = synthetic.make_inputs(w, "cuda")
+    out = _run(q, k, v, w.block, w.alpha, True, sigma=1.0, flags=dash.DASH_FLAG_LOCAL2)
+    check_forward(q, k, v, out, w.block, w.alpha, True, sigma=1.0, rows=sample_rows(w.nq, w.block, 512, 3),
+                  label="local2 prefill8k", local=2)
+
+
 def test_decode_with_cached_summaries():
     """A chunk-summary cache from dash_pool_keys (kept across decode steps) gives the same result."""
     b, nq, nk, hq, hkv, d, B = 2, 1, 4096, 8, 2, 128, 64
