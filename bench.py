@@ -54,7 +54,7 @@ L2_FLUSH_BYTES = 256 << 20
 # kernel captured at batch 4 and scaled by the (batch, kv head) units to batch 16
 # (profiles/attn_decode_decode.md).  Workloads without a capture report null.
 TRAFFIC_BYTES = {
-    ("prefill8k", 1): 1.4479e8,
+    ("prefill8k", 1): 1.4460e8,
     ("decode", 16): 1.6565e9,
     ("decode", 4): 4.1412e8,
 }
