@@ -106,10 +106,7 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t pari
         : "memory");
     return ok != 0;
 }
-#ifndef DASH_SLEEP_NS
-#define DASH_SLEEP_NS 100000
-#endif
-constexpr uint32_t kSleepNs = DASH_SLEEP_NS;  // longest single suspension of a waiting thread
+constexpr uint32_t kSleepNs = 100000;  // longest single suspension of a waiting thread
 
 // Bounded wait.  Gives up after limit_ns (recording a device error and raising
 // the CTA's abort flag) or, when honor_abort is set, as soon as another role
