@@ -1,0 +1,68 @@
+"""bench.py's host side on the CPU: the work accounting behind every roofline figure
+(against a brute-force recount) and the reference arm's JSON line."""
+import json
+import subprocess
+import sys
+from pathlib import Path
+
+import numpy as np
+import pytest
+import torch
+
+import bench
+import synthetic
+
+ROOT = Path(__file__).resolve().parents[1]
+
+
+class _Lists:
+    def __init__(self, count):
+        self.count = count
+
+
+def test_work_accounting_matches_a_recount():
+    """F2 = sum_{b,i,h} 4 d (B |R_i| + (p_i mod B) + 1), Y = the K and V bytes of the same
+    keys per kv head, sparsity over the routable chunks, executed = list entries x B x 128 x 4d."""
+    w = synthetic.Workload("acct", 2, 100, 300, 8, 2, 16, 32, 1.5, True, "bf16", 0, False)
+    gen = torch.Generator().manual_seed(1)
+    cnt = torch.zeros(w.batch, w.nq, w.hkv, dtype=torch.int64)
+    for i in range(w.nq):
+        n_vis = min((i + w.nk - w.nq) // w.block, w.nk // w.block)
+        cnt[:, i, :] = torch.randint(0, n_vis + 1, (w.batch, w.hkv), generator=gen)
+    count = torch.randint(1, 9, (w.batch, w.hkv, 13), generator=gen, dtype=torch.int32)
+    f2, y, sparsity, exec_f = bench.work_of(w, cnt, _Lists(count))
+    F2 = Y = routed = visible = 0
+    for b in range(w.batch):
+        for i in range(w.nq):
+            p = i + w.nk - w.nq
+            n_vis = min(p // w.block, w.nk // w.block)
+            for r in range(w.hkv):
+                keys = w.block * int(cnt[b, i, r]) + p % w.block + 1
+                F2 += 4 * w.d * keys * w.g
+                Y += keys * w.d * 2 * 2
+                routed += int(cnt[b, i, r])
+                visible += n_vis
+    assert f2 == F2 and y == Y
+    assert sparsity == pytest.approx(1 - routed / visible)
+    assert exec_f == int(count.sum()) * w.block * 128 * 4 * w.d
+
+
+def test_mask_counts():
+    m = synthetic.random_block_mask(1, 200, 1000, 2, 64, 0.5, seed=3)
+    bits = ((m.to(torch.int64) & 0xFFFFFFFF).unsqueeze(-1) >> torch.arange(32)) & 1
+    assert torch.equal(bench.mask_counts(m), bits.flatten(-2).sum(-1))
+
+
+def test_reference_arm_line():
+    """`--impl reference` prints one JSON line with the oracle timed on the host cores."""
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny", "--steps", "1",
+                        "--warmup", "3", "--ref-budget", "0.2"], cwd=ROOT, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["value"] > 0 and d["steps"] == 1
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+    assert d["config"]["workload"] == "tiny" and np.isfinite(d["ms_per_step"])
