@@ -22,7 +22,12 @@ forward and applying the chain rule step by step, in the forward's order reverse
   Stage-1 scores [Dash §3.2 Eq. 4]: s_c = gamma <q, kbar_c>/sqrt(d):
       dq += gamma sum_c ds_c kbar_c / sqrt(d),  dkbar_c += gamma ds_c q / sqrt(d).
   Stage 0 with the summary query at zero [Dash §3.1 Eq. 3]: kbar_c is the mean of the
-      chunk's keys, so every key of chunk c receives dkbar_c / |C_c|.
+      chunk's keys, so every key of chunk c receives dkbar_c / |C_c|.  With a learned
+      summary query, kbar_c = sum_t a_t k_t with a = softmax_t(<qbar_c, k_t>/sqrt(d)):
+      dk_t += a_t dkbar_c + e_t qbar_c / sqrt(d), dqbar_c = sum_t e_t k_t / sqrt(d), where
+      e_t = a_t (<dkbar_c, k_t> - sum_u a_u <dkbar_c, k_u>).  As sigma grows the prior's
+      gradient, and with it dqbar, falls as 1/sigma: in the limit the summary query gets
+      no gradient at all [Dash App. F.5].
 
 The supports (and R) are piecewise constant in the inputs and carry no gradient.
 Parity pins (tests/test_oracle_backward.py): central finite differences of the C
@@ -46,11 +51,13 @@ def entmax_vjp(p: np.ndarray, dp: np.ndarray, alpha: float) -> np.ndarray:
 
 
 def backward(Q, K, V, dO, block_size: int, alpha: float, *, gamma: float = 1.0, sigma: float = 1e8,
-             causal: bool = True, local: int = 1):
-    """Gradients (dQ, dK, dV) of sum(dO * out) for one batch element.
+             causal: bool = True, local: int = 1, qbar=None):
+    """Gradients (dQ, dK, dV, and dQbar with a learned summary query) of sum(dO * out)
+    for one batch element.
 
-    Q, dO [nq, hq, d]; K, V [nk, hkv, d] (float32 values, as the forward reads them).
-    Returns a dict with out (the forward's output) and dQ, dK, dV in float64."""
+    Q, dO [nq, hq, d]; K, V [nk, hkv, d] (float32 values, as the forward reads them);
+    qbar [n_chunks, hkv, d] or None (q̄ = 0).  Returns a dict with out (the forward's
+    output) and the gradients in float64."""
     Q = np.ascontiguousarray(Q, dtype=np.float32)
     K = np.ascontiguousarray(K, dtype=np.float32)
     V = np.ascontiguousarray(V, dtype=np.float32)
@@ -61,16 +68,28 @@ def backward(Q, K, V, dO, block_size: int, alpha: float, *, gamma: float = 1.0, 
     B = block_size
     nch = n_chunks_for(nk, B, causal)
     rows = np.arange(nq, dtype=np.int64)
+    if qbar is not None:
+        qbar = np.ascontiguousarray(np.broadcast_to(np.asarray(qbar, dtype=np.float32), (nch, hkv, d)))
     ref = fwd_rows(Q, rows, nq, K, V, B, alpha, gamma=gamma, sigma=sigma, causal=causal,
-                   want=("out", "w", "routed", "xmt"), local=local)
+                   want=("out", "w", "routed", "xmt"), local=local, qbar=qbar)
     Qd, Kd, Vd = Q.astype(np.float64), K.astype(np.float64), V.astype(np.float64)
     scale = 1.0 / np.sqrt(d)
     kexp = 1.0 / (alpha - 1.0)
 
-    # chunk summaries (mean of the chunk's real keys) and chunk sizes
+    # chunk summaries and chunk sizes: the mean of the chunk's real keys, or their
+    # softmax-weighted sum under the learned summary query (weights A[c] [size, hkv])
     sizes = np.array([min((c + 1) * B, nk) - c * B for c in range(nch)], dtype=np.float64)
-    Kbar = np.stack([Kd[c * B:c * B + int(sizes[c])].mean(axis=0) for c in range(nch)]) if nch else \
-        np.zeros((0, hkv, d))
+    A = []
+    for c in range(nch):
+        kc = Kd[c * B:c * B + int(sizes[c])]                       # [size, hkv, d]
+        if qbar is None:
+            A.append(np.full(kc.shape[:2], 1.0 / sizes[c]))
+        else:
+            sc = np.einsum("thd,hd->th", kc, qbar[c].astype(np.float64)) * scale
+            a = np.exp(sc - sc.max(axis=0))
+            A.append(a / a.sum(axis=0))
+    Kbar = (np.stack([np.einsum("th,thd->hd", A[c], Kd[c * B:c * B + int(sizes[c])]) for c in range(nch)])
+            if nch else np.zeros((0, hkv, d)))
 
     dQ = np.zeros_like(Qd)
     dK = np.zeros_like(Kd)
@@ -129,7 +148,21 @@ def backward(Q, K, V, dO, block_size: int, alpha: float, *, gamma: float = 1.0, 
                 # s_c = gamma <q, kbar_c> / sqrt(d)
                 dQ[i, h] += gamma * scale * (ds @ Kbar[:nvis, r])
                 dKbar[:nvis, r] += gamma * scale * np.outer(ds, Qd[i, h])
-    # Stage 0: the mean over each chunk's keys
+    # Stage 0: the chunk's keys through the weights A (uniform for the mean)
+    dQbar = np.zeros((nch, hkv, d))
     for c in range(nch):
-        dK[c * B:c * B + int(sizes[c])] += dKbar[c] / sizes[c]
-    return {"out": ref["out"], "dQ": dQ, "dK": dK, "dV": dV}
+        sl = slice(c * B, c * B + int(sizes[c]))
+        kc = Kd[sl]
+        if qbar is None:
+            dK[sl] += dKbar[c] / sizes[c]
+            continue
+        a = A[c]                                                   # [size, hkv]
+        dK[sl] += a[:, :, None] * dKbar[c][None]
+        da = np.einsum("thd,hd->th", kc, dKbar[c])
+        e = a * (da - (a * da).sum(axis=0))
+        dK[sl] += e[:, :, None] * qbar[c].astype(np.float64)[None] * scale
+        dQbar[c] = np.einsum("th,thd->hd", e, kc) * scale
+    res = {"out": ref["out"], "dQ": dQ, "dK": dK, "dV": dV}
+    if qbar is not None:
+        res["dQbar"] = dQbar
+    return res

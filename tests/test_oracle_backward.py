@@ -130,8 +130,7 @@ BACKWARD_MUTATIONS = [
     ("group average not divided by g", "ds = entmax_vjp(p, dw[:nvis] / g, alpha)", "ds = entmax_vjp(p, dw[:nvis], alpha)"),
     ("prior bias gradient not centred by mu", "dlogw = (G - G.mean()) / sigma", "dlogw = G / sigma"),
     ("entmax Jacobian without the threshold's move", "return u * (dp - (u @ dp) / su)", "return u * dp"),
-    ("pooling gradient not divided by the chunk size", "dK[c * B:c * B + int(sizes[c])] += dKbar[c] / sizes[c]",
-     "dK[c * B:c * B + int(sizes[c])] += dKbar[c]"),
+    ("pooling gradient not divided by the chunk size", "dK[sl] += dKbar[c] / sizes[c]", "dK[sl] += dKbar[c]"),
 ]
 
 
@@ -154,3 +153,63 @@ def test_backward_pins_catch_planted_mistakes():
         got = mod.backward(Q, K, V, dO, B, alpha, sigma=sigma)
         worst = max(np.abs(got[n] - fd[n]).max() / max(1.0, np.abs(fd[n]).max()) for n in ("dQ", "dK", "dV"))
         assert worst > 1e-4, "the pins miss: " + name
+
+
+def _fd_qbar(Q, K, V, dO, Qb, B, alpha, sigma):
+    def loss(qb, k):
+        out = oracle.fwd(Q, k, V, B, alpha, sigma=sigma, want=("out",), qbar=qb)["out"]
+        return float((out * dO).sum())
+
+    grads = {}
+    for name, X in (("dQbar", Qb), ("dK", K)):
+        G = np.zeros(X.shape)
+        for idx in np.ndindex(X.shape):
+            Xp, Xm = X.copy(), X.copy()
+            Xp[idx] += STEP
+            Xm[idx] -= STEP
+            if name == "dQbar":
+                G[idx] = (loss(Xp, K) - loss(Xm, K)) / (2 * STEP)
+            else:
+                G[idx] = (loss(Qb, Xp) - loss(Qb, Xm)) / (2 * STEP)
+        grads[name] = G
+    return grads
+
+
+def test_learned_summary_gradients():
+    """With a learned summary query the keys also reach Stage 1 through the pooling softmax,
+    and the query itself gets a gradient (finite differences); that gradient falls as
+    1/sigma (the summary query becomes untrainable as the prior weakens, App. F.5)."""
+    alpha, sigma, B, nq, nk, hq, hkv, d = 1.5, 1.0, 8, 40, 40, 2, 1, 4
+    for Q, K, V, dO in _grid_case(21, nq, nk, hq, hkv, d):
+        Qb = (np.random.default_rng(int(Q[0, 0, 0] * 64) + 300).integers(-96, 96, size=(nk // B, hkv, d)) / 64
+              ).astype(np.float32)
+        x = oracle.fwd(Q, K, V, B, alpha, want=("xmt",), qbar=Qb)["xmt"]
+        if np.nanmin(np.abs(x)) > 1e-3:
+            break
+    got = backward(Q, K, V, dO, B, alpha, sigma=sigma, qbar=Qb)
+    fd = _fd_qbar(Q, K, V, dO, Qb, B, alpha, sigma)
+    for name in ("dQbar", "dK"):
+        err = np.abs(got[name] - fd[name]).max()
+        assert err <= 1e-6 * max(1.0, np.abs(fd[name]).max()), (name, err)
+    assert np.abs(got["dQbar"]).max() > 1e-3
+    a = backward(Q, K, V, dO, B, alpha, sigma=1e5, qbar=Qb)["dQbar"]
+    b = backward(Q, K, V, dO, B, alpha, sigma=1e6, qbar=Qb)["dQbar"]
+    np.testing.assert_allclose(a, 10 * b, rtol=1e-3, atol=1e-12)
+
+
+def test_learned_pooling_backward_pin_catches_a_planted_mistake():
+    import types
+    from pathlib import Path
+
+    src = (Path(oracle.__file__).parent / "backward.py").read_text()
+    orig, mut = "e = a * (da - (a * da).sum(axis=0))", "e = a * da"
+    assert src.count(orig) == 1
+    mod = types.ModuleType("oracle.mutated_backward")
+    mod.__package__ = "oracle"
+    exec(compile(src.replace(orig, mut), "mutated_backward", "exec"), mod.__dict__)
+    alpha, B, nq, nk, hq, hkv, d = 1.5, 8, 40, 40, 2, 1, 4
+    Q, K, V, dO = next(_grid_case(21, nq, nk, hq, hkv, d))
+    Qb = (np.random.default_rng(5).integers(-96, 96, size=(nk // B, hkv, d)) / 64).astype(np.float32)
+    fd = _fd_qbar(Q, K, V, dO, Qb, B, alpha, 1.0)
+    got = mod.backward(Q, K, V, dO, B, alpha, sigma=1.0, qbar=Qb)
+    assert np.abs(got["dQbar"] - fd["dQbar"]).max() > 1e-4
