@@ -125,12 +125,12 @@ class ClockSampler:
 # work accounting (bench-side, from the routing mask the library exports)
 # ---------------------------------------------------------------------------
 
-def routed_counts(dash, q, k, w, alpha, sigma):
+def routed_counts(dash, q, k, w, alpha, sigma, flags=0):
     """|R_i^(r)| per (b, i, r) from dash_block_select's bit-packed mask."""
     nch = dash.n_chunks(w.nk, w.block, True)
     words = max((nch + 31) // 32, 1)
     mask = torch.zeros(w.batch, w.nq, w.hkv, words, dtype=torch.int32, device=q.device)
-    dash.dash_block_select(q, k, w.block, alpha, True, mask=mask, sigma=sigma)
+    dash.dash_block_select(q, k, w.block, alpha, True, mask=mask, sigma=sigma, flags=flags)
     m = mask.to(torch.int64) & 0xFFFFFFFF
     cnt = torch.zeros(w.batch, w.nq, w.hkv, dtype=torch.int64, device=q.device)
     for bit in range(32):
@@ -138,15 +138,17 @@ def routed_counts(dash, q, k, w, alpha, sigma):
     return cnt
 
 
-def work_of(w, cnt, lists):
-    """Selected FLOPs F2, selected K/V bytes Y, sparsity, and the tile-union FLOPs the kernel executes."""
+def work_of(w, cnt, lists, local=1):
+    """Selected FLOPs F2, selected K/V bytes Y, sparsity, and the tile-union FLOPs the kernel
+    executes.  local: chunks of the local window (2: the chunk before the query's own as well)."""
     i = torch.arange(w.nq, device=cnt.device, dtype=torch.int64)
     p = i + w.nk - w.nq
-    diag = (p % w.block + 1).view(1, -1, 1)                        # keys of the diagonal branch
+    first = torch.clamp(p // w.block - (local - 1), min=0)            # first chunk of the local window
+    diag = (p - first * w.block + 1).view(1, -1, 1)                  # keys of the local window
     keys = w.block * cnt + diag                                      # [b, nq, hkv]
     f2 = float((4 * w.d * keys.sum()).item()) * w.g                  # every head of the group
     y = float((keys.sum() * w.d * 2 * 2).item())                     # K and V, bf16, per kv head
-    vis = torch.clamp(p // w.block, max=w.nk // w.block).view(1, -1, 1).expand_as(cnt)
+    vis = torch.clamp(first, max=w.nk // w.block).view(1, -1, 1).expand_as(cnt)
     sparsity = 1.0 - float(cnt.sum().item()) / max(float(vis.sum().item()), 1.0)
     exec_f = None
     if lists is not None:
@@ -188,7 +190,10 @@ def run_ours(args, rank, world, device):
     stream = torch.cuda.current_stream()
 
     cache = None
+    local = 2 if args.local2 else 1
     opts = dict(sigma=sigma)
+    if local == 2:
+        opts["flags"] = dash.DASH_FLAG_LOCAL2
     if decode:
         # the chunk-summary cache persists across decode steps: every complete chunk is
         # pooled (and put in the tensor-core operand form) once, outside the step
@@ -200,8 +205,8 @@ def run_ours(args, rank, world, device):
 
     lists = dash.make_lists(q, k, w.block, w.g)
     dash.dash_block_select(q, k, w.block, alpha, True, lists=lists, **opts)
-    cnt = routed_counts(dash, q, k, w, alpha, sigma)
-    f2, y, sparsity, exec_f = work_of(w, cnt, lists)
+    cnt = routed_counts(dash, q, k, w, alpha, sigma, opts.get("flags", 0))
+    f2, y, sparsity, exec_f = work_of(w, cnt, lists, local)
     torch.cuda.synchronize()
 
     for _ in range(args.warmup):
@@ -302,6 +307,7 @@ def run_ours(args, rank, world, device):
         "config": {"workload": w.name, "batch": w.batch, "nq": w.nq, "nk": w.nk, "hq": w.hq, "hkv": w.hkv,
                    "d": w.d, "block": w.block, "alpha": alpha, "sigma": sigma, "gamma": 1.0, "causal": True,
                    "a_max": synthetic.amax_for(w), "sparsity": round(sparsity, 4),
+                   "local_window_chunks": local,
                    "l2": "flushed (256 MiB write) before every timed step", "parallelism": f"replicas x{world}"},
         "stages_ms": {"total": round(ms, 4), "stage0_1_select": round(ms01, 4), "stage2": round(ms2, 4)},
         "work": {"selected_flops": f2, "selected_kv_bytes": y,
@@ -485,6 +491,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-budget", type=float, default=10.0, help="seconds of oracle work per reference step")
+    ap.add_argument("--local2", action="store_true",
+                    help="two-block local window (the chunk before the query's own attended in full)")
     ap.add_argument("--mask-sweep", action="store_true", help="controlled-sparsity sweep of Stage 2 (1 GPU)")
     ap.add_argument("--sweep-n", default="16384,32768,65536,98304")
     ap.add_argument("--sweep-s", default="0.75,0.875,0.9375")

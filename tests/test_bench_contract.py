@@ -20,24 +20,30 @@ class _Lists:
         self.count = count
 
 
-def test_work_accounting_matches_a_recount():
+@pytest.mark.parametrize("local", [1, 2])
+def test_work_accounting_matches_a_recount(local):
     """F2 = sum_{b,i,h} 4 d (B |R_i| + (p_i mod B) + 1), Y = the K and V bytes of the same
     keys per kv head, sparsity over the routable chunks, executed = list entries x B x 128 x 4d."""
     w = synthetic.Workload("acct", 2, 100, 300, 8, 2, 16, 32, 1.5, True, "bf16", 0, False)
     gen = torch.Generator().manual_seed(1)
+    def window(p):  # first chunk of the local window, and its keys (up to p)
+        first = max(p // w.block - (local - 1), 0)
+        return first, p - first * w.block + 1
+
     cnt = torch.zeros(w.batch, w.nq, w.hkv, dtype=torch.int64)
     for i in range(w.nq):
-        n_vis = min((i + w.nk - w.nq) // w.block, w.nk // w.block)
+        n_vis = min(window(i + w.nk - w.nq)[0], w.nk // w.block)
         cnt[:, i, :] = torch.randint(0, n_vis + 1, (w.batch, w.hkv), generator=gen)
     count = torch.randint(1, 9, (w.batch, w.hkv, 13), generator=gen, dtype=torch.int32)
-    f2, y, sparsity, exec_f = bench.work_of(w, cnt, _Lists(count))
+    f2, y, sparsity, exec_f = bench.work_of(w, cnt, _Lists(count), local)
     F2 = Y = routed = visible = 0
     for b in range(w.batch):
         for i in range(w.nq):
             p = i + w.nk - w.nq
-            n_vis = min(p // w.block, w.nk // w.block)
+            first, local_keys = window(p)
+            n_vis = min(first, w.nk // w.block)
             for r in range(w.hkv):
-                keys = w.block * int(cnt[b, i, r]) + p % w.block + 1
+                keys = w.block * int(cnt[b, i, r]) + local_keys
                 F2 += 4 * w.d * keys * w.g
                 Y += keys * w.d * 2 * 2
                 routed += int(cnt[b, i, r])
