@@ -7,14 +7,16 @@
 // (the split-KV variant the paper's §3.5 describes for incremental decoding)
 // and a second kernel merges the per-split (max, sum, O) partials.
 //
-// attn_decode_kernel: one CTA per (split of the list, kv head, batch), 4 warps.
+// attn_decode_kernel: one CTA per (split of the list, kv head, batch), 4 warps; a split
+//   takes 16 list entries, or 8 or 4 when few (batch, kv head) units would leave SMs idle.
 //   thread 0 streams each listed chunk's K and V (TMA boxes, 128-byte swizzle)
 //   into a ring of stages; each warp takes 16-key groups of the chunk and runs
 //   its own online softmax on the 16-row mma.sync tile (rows = nq*g <= 16):
 //   S = Q K^T, bias + mask, P (bf16) V into fp32 registers.  The warps' states
 //   are merged in shared memory into the split's partial.  HBM-bound: the tensor
 //   work per byte is tiny, the ring keeps ~64 KB per CTA in flight.
-// combine_kernel: O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
+// combine_kernel: one CTA per (row, kv head, batch), a thread per column:
+//   O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
 #include <math.h>
 
 #include "dash_common.cuh"

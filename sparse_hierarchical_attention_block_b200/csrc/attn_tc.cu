@@ -23,11 +23,13 @@
 //   warps 2-5  softmax: thread = TMEM lane = tile row; two passes over S_j in TMEM
 //              (row max, then exp2 / sum / bf16 P written over S_j's first 32 columns), bias added and
 //              keys masked only on steps that hold a diagonal or partial chunk; after
-//              the first step a single pass on the running maximum, redone as two
-//              passes only if a row's maximum grows by more than 2^16 (O is then
-//              rescaled); epilogue O / l -> bf16.
-// Every mbarrier wait is bounded (globaltimer); on expiry the kernel records a
-// device error, drains what it issued, frees TMEM and returns.
+//              the first step a single pass on the running maximum (scale and row sum
+//              on packed f32x2 pairs), redone as two passes only if a row's sum of p
+//              exceeds 2^16 (O is rescaled when the maximum grows by more than 16 in
+//              the exp2 domain); epilogue O / l -> bf16.
+// Every mbarrier wait is bounded (globaltimer); a waiting thread suspends on the
+// barrier rather than polling.  On expiry the kernel records a device error, drains
+// what it issued, frees TMEM and returns.
 #include <math.h>
 
 #include "dash_common.cuh"
