@@ -21,7 +21,9 @@
 //       domain (1/(alpha-1) = 4 at alpha = 1.25 underflows fp32 otherwise), mu,
 //       d, the bit-packed mask and optionally w.
 // compact_kernel: one CTA per (batch, kv head, query tile): union of the tile's
-//   routed chunks, its diagonal chunks first, and the per-row bias table.
+//   routed chunks, its rows' local-window chunks first (the diagonal chunk, and the one
+//   before it with the two-block window of App. B.1.1), and the per-row bias table
+//   (bias 0 on every routed chunk when the mask is a caller's, without log w).
 #include <math.h>
 
 #include "dash_common.cuh"

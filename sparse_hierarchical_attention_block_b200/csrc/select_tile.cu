@@ -5,8 +5,9 @@
 // Eq. 4, App. G Alg. 2):
 //   logits   X = gamma/sqrt(d) * Q K̄^T on tcgen05 into tensor memory: Q is bf16,
 //            the fp32 chunk summaries are split k̄ = hi + lo into two bf16 operands
-//            and both products accumulate in fp32 (relative error ~2^-17, i.e.
-//            fp32-class logits).  TMEM holds 128 lanes x 512 fp32 columns; with LG
+//            (per call, or kept across decoding steps in a summary cache) and both
+//            products accumulate in fp32 (relative error ~2^-17, i.e. fp32-class
+//            logits).  TMEM holds 128 lanes x 512 fp32 columns; with LG
 //            lane groups a CTA routes 128/LG pairs over up to 512*LG chunks: lane
 //            group lg holds chunk tiles lg, lg + LG, ... of its pairs.  The logits
 //            MMA of a tile of lane group lg reads Q through a zero-padded A operand
