@@ -153,3 +153,43 @@ def test_summary_cache_arguments(lib):
     assert lib.dash_summary_cache_reset(None) == dash.DASH_ERR_INVALID_ARG
     k = _t(FAKE, dash.DASH_BF16, [1, 256, 2, 128])
     assert lib.dash_summary_cache_update(None, ctypes.byref(k), None, None) == dash.DASH_ERR_INVALID_ARG
+
+
+def test_lists_from_mask_arguments(lib):
+    """dash_lists_from_mask rejects bad arguments on the host."""
+    nt, cap, tr = dash.lists_geometry(1, 256, 256, 2, 64, 4)
+    good = dash._Lists()
+    good.count = good.ids = good.bias = good.rows = FAKE
+    good.n_tiles, good.cap, good.tile_rows = nt, cap, tr
+    call = lambda mask, lists, **kw: lib.dash_lists_from_mask(  # noqa: E731
+        mask, kw.get("b", 1), kw.get("nq", 256), kw.get("nk", 256), kw.get("hkv", 2), kw.get("B", 64),
+        kw.get("g", 4), 1, kw.get("regroup", 0), ctypes.byref(lists) if lists is not None else None, None)
+    assert call(None, good) == dash.DASH_ERR_INVALID_ARG
+    assert call(FAKE, None) == dash.DASH_ERR_INVALID_ARG
+    assert call(FAKE + 4, good) == dash.DASH_ERR_ALIGNMENT
+    assert call(FAKE, good, g=32) == dash.DASH_ERR_UNSUPPORTED
+    assert call(FAKE, good, B=48) == dash.DASH_ERR_UNSUPPORTED
+    assert call(FAKE, good, nq=512) == dash.DASH_ERR_INVALID_ARG   # lists made for 256 rows
+    no_rows = dash._Lists()
+    no_rows.count = no_rows.ids = no_rows.bias = FAKE
+    no_rows.rows = None
+    no_rows.n_tiles, no_rows.cap, no_rows.tile_rows = nt, cap, tr
+    assert call(FAKE, no_rows, regroup=1) == dash.DASH_ERR_INVALID_ARG
+    assert lib.dash_last_error()
+
+
+def test_pool_keys_q_arguments(lib):
+    """dash_pool_keys_q checks the summary queries' shape against the chunks (every call
+    here is invalid, so nothing reaches the device)."""
+    k = _t(FAKE, dash.DASH_BF16, [2, 1000, 2, 128])  # 1000 // 64 = 15 chunks
+    kbar = FAKE
+    for shape in ([3, 15, 2, 128],    # batch neither 1 nor 2
+                  [1, 16, 2, 128],    # one chunk too many
+                  [1, 15, 1, 128],    # kv heads
+                  [1, 15, 2, 64]):    # head dim
+        qb = _t(FAKE, dash.DASH_F32, shape)
+        rc = lib.dash_pool_keys_q(ctypes.byref(k), ctypes.byref(qb), 64, 1, kbar, None)
+        assert rc == dash.DASH_ERR_INVALID_ARG, (shape, lib.dash_last_error())
+    qb = _t(FAKE, dash.DASH_F32, [1, 15, 2, 128])
+    assert lib.dash_pool_keys_q(ctypes.byref(k), None, 64, 1, kbar, None) == dash.DASH_ERR_INVALID_ARG
+    assert lib.dash_pool_keys_q(ctypes.byref(k), ctypes.byref(qb), 64, 1, None, None) == dash.DASH_ERR_INVALID_ARG
