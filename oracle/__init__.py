@@ -3,7 +3,8 @@
 Only the test-suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  The product library never does, and
 the two share no code: this package wraps ``dash_oracle.c`` (plain C, double
-precision, OpenMP) with ctypes and numpy.
+precision, OpenMP) with ctypes and numpy, and ``backward.py`` differentiates that
+forward (numpy, double precision).
 
 Every function follows "DashAttention: Differentiable and Adaptive Sparse
 Hierarchical Attention" (arXiv 2605.18753); the C file cites the section and
