@@ -1,6 +1,6 @@
 """Benchmark of the DashAttention forward pass on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill8k|prefill32k|prefill128k|decode]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill128k|prefill8k|prefill32k|decode]
                     [--impl ours|reference] [--no-cpu-baseline]
 
 One step = one full forward (Stage 0 pooling, Stage 1 routing + work lists,
@@ -48,13 +48,14 @@ import synthetic  # noqa: E402
 METRIC = "DashAttention fwd ms & TFLOP/s (prefill) / GB/s (decode), % of B200 roofline"
 L2_FLUSH_BYTES = 256 << 20
 
-# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu capture of
-# the current kernel on the workload (the summaries under profiles/ name the command):
-# Stage 2 tensor-core kernel on prefill8k (profiles/attn_tc_prefill8k.md); the decode
-# kernel captured at batch 4 and scaled by the (batch, kv head) units to batch 16
-# (profiles/attn_decode_decode.md).  Workloads without a capture report null.
+# DRAM bytes (read + write) per launch of the dominant kernel, each from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum) of the current kernel: the Stage-2
+# tensor-core kernel on the prefill workloads; the decode kernel captured at batch 4
+# and scaled by the (batch, kv head) units to batch 16.  A workload without a capture
+# of the current kernel reports null.
 TRAFFIC_BYTES = {
-    ("prefill8k", 1): 1.4460e8,
+    ("prefill128k", 1): 6.1389e10,
+    ("prefill8k", 1): 1.4348e8,
     ("decode", 16): 1.6565e9,
     ("decode", 4): 4.1412e8,
 }
@@ -410,30 +411,34 @@ def run_mask_sweep(args, device):
 # the oracle on the host cores (CPU baseline / reference arm)
 # ---------------------------------------------------------------------------
 
-def oracle_sample(w, alpha, sigma, q, k, v, budget_s=15.0, max_rows=None):
-    """Time the fp64 oracle on a bounded row sample of the workload; returns (rows, seconds, flops, bytes, cores)."""
+def oracle_sample(w, alpha, sigma, q, k, v, budget_s=15.0, threads=0, batch_rows=0, max_rows=None, seed=0):
+    """Time the fp64 oracle on a bounded row sample of the workload: batches of random query
+    rows (all heads, batch element 0) until budget_s of oracle time is spent.  threads 0 =
+    every host core.  Returns (rows, seconds, flops, bytes, threads used)."""
     import numpy as np
 
     import oracle
 
-    cores = os.cpu_count() or 1
+    cores = threads or (os.cpu_count() or 1)
     oracle.set_threads(cores)
-    rng = np.random.default_rng(0)
+    rng = np.random.default_rng(seed)
     b = 0
     K = k[b].float().cpu().numpy()
     V = v[b].float().cpu().numpy()
-    rows = np.arange(w.nq) if w.nq <= 16 else np.sort(rng.choice(np.arange(w.nq), min(w.nq, 64), replace=False))
-    t0 = time.perf_counter()
+    # about one second of oracle work per batch: rows cost ~ their visible keys x heads
+    per = batch_rows or max(1, min(256, int(cores * 2e9 / max(w.hq * w.nk * w.d * 4, 1))))
     done = []
+    el = 0.0
     while True:
+        rows = (np.arange(w.nq) if w.nq <= 16 else
+                np.sort(rng.choice(np.arange(w.nq), min(w.nq, per), replace=False)))
         Qr = q[b, torch.from_numpy(rows).to(q.device)].float().cpu().numpy()
+        t0 = time.perf_counter()
         res = oracle.fwd_rows(Qr, rows, w.nq, K, V, w.block, alpha, sigma=sigma, want=("out", "routed"))
+        el += time.perf_counter() - t0
         done.append((rows, res["routed"]))
-        el = time.perf_counter() - t0
         if el > budget_s or (max_rows and sum(len(r) for r, _ in done) >= max_rows) or w.nq <= 16:
             break
-        rows = np.sort(rng.choice(np.arange(w.nq), min(w.nq, 256), replace=False))
-    el = time.perf_counter() - t0
     f2 = 0.0
     y = 0.0
     nrows = 0
@@ -458,7 +463,7 @@ def run_reference(args, device):
     rows = 0
     cores = os.cpu_count() or 1
     for s in range(args.warmup + args.steps):
-        n, el, f2, y, cores = oracle_sample(w, alpha, args.sigma, q, k, v, budget_s=args.ref_budget)
+        n, el, f2, y, cores = oracle_sample(w, alpha, args.sigma, q, k, v, budget_s=args.ref_budget, seed=s)
         if s >= args.warmup:
             per_step.append(el)
             flops += f2
@@ -484,13 +489,13 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="prefill8k", choices=sorted(synthetic.WORKLOADS))
+    ap.add_argument("--workload", default="prefill128k", choices=sorted(synthetic.WORKLOADS))
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (smaller profiling cases)")
     ap.add_argument("--alpha", type=float, default=None)
     ap.add_argument("--sigma", type=float, default=1e8)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ref-budget", type=float, default=10.0, help="seconds of oracle work per reference step")
+    ap.add_argument("--ref-budget", type=float, default=5.0, help="seconds of oracle work per reference step")
     ap.add_argument("--local2", action="store_true",
                     help="two-block local window (the chunk before the query's own attended in full)")
     ap.add_argument("--mask-sweep", action="store_true", help="controlled-sparsity sweep of Stage 2 (1 GPU)")
@@ -528,12 +533,18 @@ def main():
         res, (q, k, v, w, alpha, sigma) = run_ours(args, rank, world, device)
         if rank == 0:
             if not args.no_cpu_baseline and world == 1:
-                n, el, f2, y, cores = oracle_sample(w, alpha, sigma, q, k, v, budget_s=15.0)
                 decode = res["unit"] == "GB/s"
+                n, el, f2, y, cores = oracle_sample(w, alpha, sigma, q, k, v, budget_s=15.0)
                 val = (y / el / 1e9) if decode else (f2 / el / 1e12)
+                # the same oracle on one thread, on a smaller sample
+                n1, el1, f21, y1, _ = oracle_sample(w, alpha, sigma, q, k, v, budget_s=6.0, threads=1, seed=1)
+                val1 = (y1 / el1 / 1e9) if decode else (f21 / el1 / 1e12)
                 res["cpu_baseline"] = {"value": val, "unit": res["unit"], "cores": cores, "kind": "oracle",
-                                       "sample": f"{n} query rows x all heads of batch 0, {el:.1f} s "
-                                                 f"(fp64 oracle, dense masked Stage 2)"}
+                                       "sample": f"{n} random query rows x all heads of batch 0, {el:.1f} s "
+                                                 f"(fp64 oracle, dense masked Stage 2)",
+                                       "single_thread": {"value": val1, "unit": res["unit"], "cores": 1,
+                                                         "sample": f"{n1} random query rows x all heads, "
+                                                                   f"{el1:.1f} s"}}
             print(json.dumps(res))
     finally:
         if world > 1:

@@ -124,6 +124,11 @@ typedef struct {
     const dash_summary_cache_t *summary_cache; /* optional: Stage 0 and the summaries'
                                operand form come from this cache, which must hold every
                                complete chunk of k (causal only; not with kbar or qbar) */
+    float *lse;             /* optional output of the forward passes (dash_attn_fwd_ex,
+                               dash_sparse_attn_fwd): [b][nq][hq] fp32 contiguous, the natural
+                               log-sum-exp of each row's Stage-2 logits z + d over the keys it
+                               attends (the normaliser of Eq. 7's softmax); the backward pass
+                               (dash_attn_bwd) takes it back.  NULL = not written. */
 } dash_opts_t;
 
 /* Fill *opts with the defaults above.  Returns DASH_OK or DASH_ERR_INVALID_ARG (NULL). */
@@ -202,6 +207,33 @@ DASH_API int dash_block_select(const dash_tensor_t *q, const dash_tensor_t *k, i
                                int causal, int gqa_groups, float *tau, float *w, uint32_t *mask,
                                const dash_lists_t *lists, const dash_opts_t *opts);
 
+/* Backward pass of dash_attn_fwd_ex: the gradients of sum(dout * out) with respect to
+ * q, k and v ([Dash] §3.3-3.4 and App. A: the hierarchy is differentiable end to end).
+ * Gradients flow through Stage 2 (softmax attention over the routed and local keys),
+ * through the prior bias d_c = (log w_c - mu)/sigma into the group distribution w, through
+ * each head's alpha-entmax Jacobian into the Stage-1 scores, and through the mean pooling
+ * of Stage 0 into the keys; the routed sets themselves are piecewise constant and carry
+ * no gradient.  Stage 0 and Stage 1 are recomputed (deterministically: the forward's
+ * routing), Stage 2's probabilities are recomputed from lse.
+ *   q, k, v, out, block_size, alpha, causal, gqa_groups and opts (sigma, gamma, flags
+ *     DASH_FLAG_LOCAL2 / NO_REGROUP / FORCE_SIMT, stream, workspace) exactly as given to
+ *     the forward that produced out;
+ *   dout [b, nq, hq, d] the output gradient; lse [b][nq][hq] fp32 from the forward's
+ *     opts->lse;
+ *   dq [b, nq, hq, d], dk, dv [b, nk, hkv, d]: outputs (overwritten), same dtype as q.
+ * Not supported with a summary cache, given summaries or learned summary queries
+ * (DASH_ERR_UNSUPPORTED).  Workspace: dash_bwd_workspace_bytes().  Errors as for
+ * dash_attn_fwd_ex; DASH_ERR_INVALID_ARG when a gradient's shape or dtype does not
+ * match or lse is NULL. */
+DASH_API int dash_attn_bwd(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v,
+                           const dash_tensor_t *out, const dash_tensor_t *dout, const float *lse, dash_tensor_t *dq,
+                           dash_tensor_t *dk, dash_tensor_t *dv, int block_size, float alpha, int causal,
+                           int gqa_groups, const dash_opts_t *opts);
+
+/* Device workspace dash_attn_bwd needs for a problem (bytes, an upper bound). */
+DASH_API size_t dash_bwd_workspace_bytes(int64_t batch, int64_t nq, int64_t nk, int hq, int hkv, int d,
+                                         int block_size, int causal);
+
 /* Stage-2 work lists from a caller's routing mask, e.g. the random block masks of a
  * controlled-sparsity benchmark ([Dash] §5.2 and App. B.2 inject such a mask at Stage 2)
  * or an external router.
@@ -235,7 +267,9 @@ DASH_API int dash_lists_geometry(int64_t batch, int64_t nq, int64_t nk, int hkv,
                                  int64_t *n_tiles, int32_t *cap, int32_t *tile_rows, size_t *count_bytes,
                                  size_t *ids_bytes, size_t *bias_bytes, size_t *rows_bytes);
 
-/* Device workspace dash_attn_fwd_ex needs for a problem (bytes). */
+/* Device workspace dash_attn_fwd_ex needs for a problem (bytes): an upper bound over
+ * every option (it counts the pooled-key area and the split-KV decode partials even
+ * where a summary cache or a prefill shape makes them unnecessary). */
 DASH_API size_t dash_workspace_bytes(int64_t batch, int64_t nq, int64_t nk, int hq, int hkv, int d,
                                      int block_size, int causal);
 
@@ -264,11 +298,14 @@ DASH_API int dash_release(void);
  * to this entry point: it is a deployment variant of dash_attn_fwd_ex.
  *   Arguments and result as dash_attn_fwd_ex; opts may be NULL, and
  *   opts->workspace must be NULL (DASH_ERR_INVALID_ARG otherwise).
- *   A problem whose dash_workspace_bytes() exceeds DASH_NOALLOC_SCRATCH_BYTES is
- *   rejected with DASH_ERR_WORKSPACE before anything is launched.
+ *   A problem whose forward pass needs more scratch than DASH_NOALLOC_SCRATCH_BYTES
+ *   (the workspace dash_attn_fwd_ex would take with the same options, at most
+ *   dash_workspace_bytes()) is rejected with DASH_ERR_WORKSPACE before anything is
+ *   launched.
  *   The first call on a device (with that device current) looks up the array's
  *   device address with cudaGetSymbolAddress; make that first call before any
- *   stream capture.
+ *   stream capture.  The address is kept for the life of the device's primary
+ *   context: do not call this entry point again after a cudaDeviceReset.
  *   All calls share the one array, which keeps the last call's contents (the
  *   forward pass writes every scratch word before reading it).  Calls whose
  *   execution overlaps on the GPU (different streams or host threads) race on

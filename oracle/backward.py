@@ -51,13 +51,17 @@ def entmax_vjp(p: np.ndarray, dp: np.ndarray, alpha: float) -> np.ndarray:
 
 
 def backward(Q, K, V, dO, block_size: int, alpha: float, *, gamma: float = 1.0, sigma: float = 1e8,
-             causal: bool = True, local: int = 1, qbar=None):
+             causal: bool = True, local: int = 1, qbar=None, rows=None):
     """Gradients (dQ, dK, dV, and dQbar with a learned summary query) of sum(dO * out)
     for one batch element.
 
     Q, dO [nq, hq, d]; K, V [nk, hkv, d] (float32 values, as the forward reads them);
     qbar [n_chunks, hkv, d] or None (q̄ = 0).  Returns a dict with out (the forward's
-    output) and the gradients in float64."""
+    output) and the gradients in float64.
+
+    rows: optional query indices.  A row's dQ depends on that row alone (its own Stage 2
+    and its own routing), so with rows given only those rows are differentiated and the
+    result holds dQ of exactly those rows, in the given order (no dK, dV)."""
     Q = np.ascontiguousarray(Q, dtype=np.float32)
     K = np.ascontiguousarray(K, dtype=np.float32)
     V = np.ascontiguousarray(V, dtype=np.float32)
@@ -67,10 +71,10 @@ def backward(Q, K, V, dO, block_size: int, alpha: float, *, gamma: float = 1.0, 
     g = hq // hkv
     B = block_size
     nch = n_chunks_for(nk, B, causal)
-    rows = np.arange(nq, dtype=np.int64)
+    sel = np.arange(nq, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
     if qbar is not None:
         qbar = np.ascontiguousarray(np.broadcast_to(np.asarray(qbar, dtype=np.float32), (nch, hkv, d)))
-    ref = fwd_rows(Q, rows, nq, K, V, B, alpha, gamma=gamma, sigma=sigma, causal=causal,
+    ref = fwd_rows(np.ascontiguousarray(Q[sel]), sel, nq, K, V, B, alpha, gamma=gamma, sigma=sigma, causal=causal,
                    want=("out", "w", "routed", "xmt"), local=local, qbar=qbar)
     Qd, Kd, Vd = Q.astype(np.float64), K.astype(np.float64), V.astype(np.float64)
     scale = 1.0 / np.sqrt(d)
@@ -95,7 +99,7 @@ def backward(Q, K, V, dO, block_size: int, alpha: float, *, gamma: float = 1.0, 
     dK = np.zeros_like(Kd)
     dV = np.zeros_like(Vd)
     dKbar = np.zeros_like(Kbar)
-    for i in range(nq):
+    for n, i in enumerate(sel):
         if causal:
             p_i = i + nk - nq
             c_i = p_i // B
@@ -106,8 +110,8 @@ def backward(Q, K, V, dO, block_size: int, alpha: float, *, gamma: float = 1.0, 
             nvis = nch
             diag = np.arange(0)
         for r in range(hkv):
-            routed = ref["routed"][i, r, :].astype(bool)
-            w = ref["w"][i, r, :]
+            routed = ref["routed"][n, r, :].astype(bool)
+            w = ref["w"][n, r, :]
             Rc = np.nonzero(routed)[0]
             mu = np.log(w[Rc]).mean() if len(Rc) else 0.0
             # tokens attended: routed chunks ascending, then the local window
@@ -142,12 +146,14 @@ def backward(Q, K, V, dO, block_size: int, alpha: float, *, gamma: float = 1.0, 
             dw[Rc] = dlogw / w[Rc]
             for hh in range(g):
                 h = r * g + hh
-                xmt = ref["xmt"][i, h, :nvis]
+                xmt = ref["xmt"][n, h, :nvis]
                 p = np.power(np.maximum(xmt, 0.0), kexp)
                 ds = entmax_vjp(p, dw[:nvis] / g, alpha)
                 # s_c = gamma <q, kbar_c> / sqrt(d)
                 dQ[i, h] += gamma * scale * (ds @ Kbar[:nvis, r])
                 dKbar[:nvis, r] += gamma * scale * np.outer(ds, Qd[i, h])
+    if rows is not None:
+        return {"dQ": dQ[sel], "rows": sel}
     # Stage 0: the chunk's keys through the weights A (uniform for the mean)
     dQbar = np.zeros((nch, hkv, d))
     for c in range(nch):

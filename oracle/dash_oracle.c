@@ -13,7 +13,7 @@
  *   - GQA group aggregation         [Dash §3.2, "average the head-wise probability scores"]
  *   - Stage 2 (prior-induced soft.) [Dash §3.3 Eqs. 6-7; §3.4 Eqs. 8-10, Prop. 1]
  *
- * Readings taken where the paper is silent (each is also listed in the design doc):
+ * Readings taken where the paper is silent:
  *   - the learned summary query is zero unless one is given, so Stage 0 is the
  *     chunk mean by default; a given q̄ holds one query per chunk and kv head with
  *     any position encoding already applied                            [Dash §3.1; App. G Alg. 1]

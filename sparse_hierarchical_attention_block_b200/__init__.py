@@ -63,7 +63,7 @@ class _Opts(ctypes.Structure):
     _fields_ = [("sigma", ctypes.c_float), ("gamma", ctypes.c_float), ("stream", ctypes.c_void_p),
                 ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
                 ("kbar", ctypes.c_void_p), ("flags", ctypes.c_int),
-                ("qbar", ctypes.POINTER(_Tensor)), ("summary_cache", ctypes.c_void_p)]
+                ("qbar", ctypes.POINTER(_Tensor)), ("summary_cache", ctypes.c_void_p), ("lse", ctypes.c_void_p)]
 
 
 _lib = None
@@ -74,7 +74,7 @@ EXPORTS = ("dash_opts_init", "dash_attn_fwd", "dash_attn_fwd_ex", "dash_pool_key
            "dash_sync_status", "dash_release", "dash_version", "dash_attn_fwd_noalloc", "dash_pool_keys_q",
            "dash_lists_from_mask", "dash_summary_cache_create", "dash_summary_cache_update",
            "dash_summary_cache_reset", "dash_summary_cache_chunks", "dash_summary_cache_kbar",
-           "dash_summary_cache_destroy")
+           "dash_summary_cache_destroy", "dash_attn_bwd", "dash_bwd_workspace_bytes")
 
 # size of the library's static scratch area used by dash_attn_fwd_noalloc
 DASH_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -114,6 +114,9 @@ def load_library():
                                         ctypes.POINTER(sz), ctypes.POINTER(sz)]
     lib.dash_workspace_bytes.argtypes = [i64, i64, i64, i32, i32, i32, i32, i32]
     lib.dash_workspace_bytes.restype = sz
+    lib.dash_attn_bwd.argtypes = [T, T, T, T, T, P, T, T, T, i32, f32, i32, i32, ctypes.POINTER(_Opts)]
+    lib.dash_bwd_workspace_bytes.argtypes = [i64, i64, i64, i32, i32, i32, i32, i32]
+    lib.dash_bwd_workspace_bytes.restype = sz
     lib.dash_last_error.restype = ctypes.c_char_p
     lib.dash_sync_status.argtypes = [P]
     lib.dash_version.restype = ctypes.c_char_p
@@ -153,7 +156,7 @@ def _ptr(t):
 
 
 def _opts(sigma=1e8, gamma=1.0, kbar=None, workspace=None, flags=0, stream=None, qbar=None,
-          summary_cache=None) -> _Opts:
+          summary_cache=None, lse=None) -> _Opts:
     o = _Opts()
     load_library().dash_opts_init(ctypes.byref(o))
     o.sigma = float(sigma)
@@ -174,6 +177,10 @@ def _opts(sigma=1e8, gamma=1.0, kbar=None, workspace=None, flags=0, stream=None,
         o.qbar = ctypes.pointer(qd)
     if summary_cache is not None:
         o.summary_cache = summary_cache.handle
+    if lse is not None:
+        if lse.dtype != torch.float32 or not lse.is_contiguous():
+            raise ValueError("lse must be a contiguous float32 tensor [b, nq, hq]")
+        o.lse = lse.data_ptr()
     o.flags = int(flags)
     return o
 
@@ -312,6 +319,28 @@ def dash_attn_fwd_noalloc(q, k, v, out, block_size, alpha, causal=True, gqa_grou
     _check(lib.dash_attn_fwd_noalloc(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.byref(od),
                                      int(block_size), float(alpha), int(bool(causal)), int(g), ctypes.byref(o)))
     return out
+
+
+def dash_attn_bwd(q, k, v, out, dout, lse, dq, dk, dv, block_size, alpha, causal=True, gqa_groups=None, **opts):
+    """Backward pass: writes dq, dk, dv (the gradients of sum(dout * out)) for the forward
+    that produced ``out`` and ``lse`` (pass ``lse=`` to dash_attn_fwd) with the same
+    ``block_size``, ``alpha``, ``causal`` and options (sigma, gamma, flags)."""
+    lib = load_library()
+    g = gqa_groups if gqa_groups is not None else q.shape[2] // k.shape[2]
+    if lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 tensor [b, nq, hq]")
+    ds = [_desc(t) for t in (q, k, v, out, dout, dq, dk, dv)]
+    o = _opts(**opts)
+    _check(lib.dash_attn_bwd(ctypes.byref(ds[0]), ctypes.byref(ds[1]), ctypes.byref(ds[2]), ctypes.byref(ds[3]),
+                             ctypes.byref(ds[4]), ctypes.c_void_p(lse.data_ptr()), ctypes.byref(ds[5]),
+                             ctypes.byref(ds[6]), ctypes.byref(ds[7]), int(block_size), float(alpha),
+                             int(bool(causal)), int(g), ctypes.byref(o)))
+    return dq, dk, dv
+
+
+def dash_bwd_workspace_bytes(batch, nq, nk, hq, hkv, d, block_size, causal=True) -> int:
+    return int(load_library().dash_bwd_workspace_bytes(int(batch), int(nq), int(nk), int(hq), int(hkv), int(d),
+                                                       int(block_size), int(bool(causal))))
 
 
 def dash_pool_keys(k, block_size, causal, kbar, stream=None, qbar=None):

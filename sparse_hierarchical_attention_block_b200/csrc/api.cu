@@ -128,6 +128,7 @@ int check_opts(const dash_opts_t &o) {
     if (!(o.gamma > 0.f) || !isfinite(o.gamma)) return fail(DASH_ERR_INVALID_ARG, "gamma must be > 0");
     if (o.workspace && reinterpret_cast<uintptr_t>(o.workspace) % 256)
         return fail(DASH_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+    if (o.lse && reinterpret_cast<uintptr_t>(o.lse) % 4) return fail(DASH_ERR_ALIGNMENT, "lse not 4-byte aligned");
     return DASH_OK;
 }
 
@@ -252,13 +253,13 @@ int run_stage2(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor
     const dash_dtype_t dt = q->dtype;
     const bool simt = (o.flags & DASH_FLAG_FORCE_SIMT) != 0;
     if (!simt && decode_ws && attn_decode_supported(G, dt)) {
-        e = launch_attn_decode(view(q), view(k), view(v), view(out), G, LV, decode_ws, st);
+        e = launch_attn_decode(view(q), view(k), view(v), view(out), G, LV, decode_ws, st, o.lse);
         if (e != cudaSuccess) return cuda_fail(e, "stage 2 (decode)");
     } else if (!simt && attn_tc_supported(G, dt)) {
-        e = launch_attn_tc(view(q), view(k), view(v), view(out), G, LV, o.flags, st);
+        e = launch_attn_tc(view(q), view(k), view(v), view(out), G, LV, o.flags, st, o.lse);
         if (e != cudaSuccess) return cuda_fail(e, "stage 2 (tensor cores)");
     } else {
-        e = launch_attn_simt(view(q), view(k), view(v), view(out), dt, G, LV, st);
+        e = launch_attn_simt(view(q), view(k), view(v), view(out), dt, G, LV, st, o.lse);
         if (e != cudaSuccess) return cuda_fail(e, "stage 2 (CUDA cores)");
     }
     return DASH_OK;
@@ -328,12 +329,56 @@ int validate_qkvo(const dash_tensor_t *q, const dash_tensor_t *k, const dash_ten
     return DASH_OK;
 }
 
+// Everything dash_attn_fwd_ex decides before it launches: validated geometry, where
+// Stage 0's summaries come from, whether Stage 2 takes the split-KV decode path, and
+// the workspace layout those choices need.
+struct FwdPlan {
+    Geom G;
+    WsLayout WL;
+    TView qv;
+    const dash_summary_cache *sc;
+    bool need_kbar, dec;
+};
+
+int plan_fwd(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v, const dash_tensor_t *out,
+             int block_size, float alpha, int causal, int gqa_groups, const dash_opts_t &o, FwdPlan *P) {
+    int rc;
+    if ((rc = check_opts(o))) return rc;
+    if ((rc = validate_qkvo(q, k, v, out))) return rc;
+    if (!(alpha > 1.f) || !isfinite(alpha)) return fail(DASH_ERR_INVALID_ARG, "alpha must be > 1");
+    Geom &G = P->G;
+    if ((rc = make_geom(q, k, block_size, causal, gqa_groups, &G))) return rc;
+    if ((rc = set_local(o, &G))) return rc;
+    if (o.kbar && reinterpret_cast<uintptr_t>(o.kbar) % 16) return fail(DASH_ERR_ALIGNMENT, "kbar not aligned");
+    P->qv = TView{};
+    P->sc = o.summary_cache;
+    if (P->sc && (rc = check_cache(P->sc, G, o))) return rc;
+    if (o.qbar && o.kbar) return fail(DASH_ERR_INVALID_ARG, "opts: give kbar or qbar, not both");
+    if (o.qbar && (rc = check_qbar(o.qbar, G, &P->qv))) return rc;
+    P->need_kbar = o.kbar == nullptr && !P->sc;
+    P->dec = attn_decode_supported(G, q->dtype) && !(o.flags & DASH_FLAG_FORCE_SIMT);
+    P->WL = (G.b == 0 || G.nq == 0) ? WsLayout{} : ws_layout(G, P->need_kbar, true, P->dec);
+    return DASH_OK;
+}
+
 }  // namespace
 
 namespace dash {
 // Records msg as this thread's last error (dash_last_error) and returns code;
 // for entry points defined in other translation units.
 int report_error(int code, const char *msg) { return fail(code, "%s", msg); }
+
+// The workspace bytes dash_attn_fwd_ex would take for these arguments (validated as it
+// validates them); *need = 0 for an empty problem.
+int fwd_workspace_need(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v,
+                       const dash_tensor_t *out, int block_size, float alpha, int causal, int gqa_groups,
+                       const dash_opts_t *opts, size_t *need) {
+    const dash_opts_t o = opts ? *opts : default_opts();
+    FwdPlan P;
+    const int rc = plan_fwd(q, k, v, out, block_size, alpha, causal, gqa_groups, o, &P);
+    *need = rc ? 0 : P.WL.total;
+    return rc;
+}
 }  // namespace dash
 
 extern "C" {
@@ -512,23 +557,15 @@ DASH_API int dash_attn_fwd_ex(const dash_tensor_t *q, const dash_tensor_t *k, co
                               dash_tensor_t *out, int block_size, float alpha, int causal, int gqa_groups,
                               const dash_opts_t *opts) {
     dash_opts_t o = opts ? *opts : default_opts();
-    int rc;
-    if ((rc = check_opts(o))) return rc;
-    if ((rc = validate_qkvo(q, k, v, out))) return rc;
-    if (!(alpha > 1.f) || !isfinite(alpha)) return fail(DASH_ERR_INVALID_ARG, "alpha must be > 1");
-    Geom G;
-    if ((rc = make_geom(q, k, block_size, causal, gqa_groups, &G))) return rc;
-    if ((rc = set_local(o, &G))) return rc;
-    if (o.kbar && reinterpret_cast<uintptr_t>(o.kbar) % 16) return fail(DASH_ERR_ALIGNMENT, "kbar not aligned");
-    TView qv{};
-    const dash_summary_cache *sc = o.summary_cache;
-    if (sc && (rc = check_cache(sc, G, o))) return rc;
-    if (o.qbar && o.kbar) return fail(DASH_ERR_INVALID_ARG, "opts: give kbar or qbar, not both");
-    if (o.qbar && (rc = check_qbar(o.qbar, G, &qv))) return rc;
+    FwdPlan P;
+    int rc = plan_fwd(q, k, v, out, block_size, alpha, causal, gqa_groups, o, &P);
+    if (rc) return rc;
+    const Geom &G = P.G;
     if (G.b == 0 || G.nq == 0) return DASH_OK;
-    const bool need_kbar = o.kbar == nullptr && !sc;
-    const bool dec = attn_decode_supported(G, q->dtype) && !(o.flags & DASH_FLAG_FORCE_SIMT);
-    WsLayout WL = ws_layout(G, need_kbar, true, dec);
+    const dash_summary_cache *sc = P.sc;
+    const TView qv = P.qv;
+    const bool need_kbar = P.need_kbar, dec = P.dec;
+    const WsLayout &WL = P.WL;
     char *ws = nullptr;
     if ((rc = get_workspace(o, WL.total, &ws))) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(o.stream);
@@ -549,6 +586,169 @@ DASH_API int dash_attn_fwd_ex(const dash_tensor_t *q, const dash_tensor_t *k, co
 DASH_API int dash_attn_fwd(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v,
                            dash_tensor_t *out, int block_size, float alpha, int causal, int gqa_groups) {
     return dash_attn_fwd_ex(q, k, v, out, block_size, alpha, causal, gqa_groups, nullptr);
+}
+
+}  // extern "C"
+
+namespace {
+
+struct BwdLayout {
+    WsLayout F;  // Stage 0-1 state (recomputed) and the work lists
+    size_t tau, drow, gd, dq, dkbar, bitmap, E, ref_off, ref_cnt, refs, qp, dop, lp, dp, total;
+};
+
+BwdLayout bwd_layout(const Geom &G, bool tc) {
+    BwdLayout L{};
+    L.F = ws_layout(G, true, true, false);
+    size_t off = L.F.total;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off += align256(bytes);
+        return o;
+    };
+    const size_t rows = (size_t)G.b * G.nq * G.hq;
+    const size_t bhb = (size_t)G.b * G.hkv * G.n_blk;
+    const int tw = (int)((G.n_tiles + 31) / 32);
+    L.tau = take(rows * 4);
+    L.drow = take(rows * 4);
+    L.gd = take((size_t)G.b * G.nq * G.hkv * (size_t)G.n_chunks * 4);
+    L.dq = take(rows * G.d * 4);
+    L.dkbar = take((size_t)G.b * G.n_chunks * G.hkv * G.d * 4);
+    L.bitmap = take(bhb * tw * 4);
+    L.E = take(bhb * G.n_tiles * 4);
+    L.ref_off = take(bhb * 4);
+    L.ref_cnt = take(bhb * 4);
+    L.refs = take(bhb * G.n_tiles * 8);
+    if (tc) {
+        const size_t tiles = (size_t)G.b * G.hkv * G.n_tiles;
+        L.qp = take(tiles * 128 * G.d * 2);
+        L.dop = take(tiles * 128 * G.d * 2);
+        L.lp = take(tiles * 128 * 4);
+        L.dp = take(tiles * 128 * 4);
+    }
+    L.total = off;
+    return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+DASH_API size_t dash_bwd_workspace_bytes(int64_t batch, int64_t nq, int64_t nk, int hq, int hkv, int d,
+                                         int block_size, int causal) {
+    if (hkv <= 0 || hq % hkv || block_size <= 0 || nk <= 0 || batch < 0 || nq < 0) return 0;
+    Geom G{};
+    G.b = batch;
+    G.nq = nq;
+    G.nk = nk;
+    G.hq = hq;
+    G.hkv = hkv;
+    G.g = hq / hkv;
+    G.d = d;
+    G.B = block_size;
+    G.causal = causal;
+    G.n_chunks = (int)(causal ? nk / block_size : (nk + block_size - 1) / block_size);
+    G.n_blk = (int)((nk + block_size - 1) / block_size);
+    G.tile_rows = 128 / G.g;
+    G.n_tiles = (nq + G.tile_rows - 1) / G.tile_rows;
+    G.words = (G.n_chunks + 31) / 32;
+    G.kbar_cap = G.n_chunks;
+    G.ct_cap = (G.n_chunks + 127) / 128;
+    G.local = 1;
+    return bwd_layout(G, true).total;
+}
+
+DASH_API int dash_attn_bwd(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v,
+                           const dash_tensor_t *out, const dash_tensor_t *dout, const float *lse, dash_tensor_t *dq,
+                           dash_tensor_t *dk, dash_tensor_t *dv, int block_size, float alpha, int causal,
+                           int gqa_groups, const dash_opts_t *opts) {
+    dash_opts_t o = opts ? *opts : default_opts();
+    int rc;
+    if ((rc = check_opts(o))) return rc;
+    if ((rc = validate_qkvo(q, k, v, out))) return rc;
+    if ((rc = check_tensor(dout, "dout")) || (rc = check_tensor(dq, "dq")) || (rc = check_tensor(dk, "dk")) ||
+        (rc = check_tensor(dv, "dv")))
+        return rc;
+    const dash_tensor_t *grads[4] = {dout, dq, dk, dv};
+    for (const dash_tensor_t *t : grads)
+        if (t->dtype != q->dtype) return fail(DASH_ERR_INVALID_ARG, "gradients must share the inputs' dtype");
+    for (int a = 0; a < 4; ++a) {
+        if (dout->shape[a] != q->shape[a] || dq->shape[a] != q->shape[a])
+            return fail(DASH_ERR_INVALID_ARG, "dout and dq must have q's shape");
+        if (dk->shape[a] != k->shape[a] || dv->shape[a] != k->shape[a])
+            return fail(DASH_ERR_INVALID_ARG, "dk and dv must have k's shape");
+    }
+    if (!lse) return fail(DASH_ERR_INVALID_ARG, "lse is NULL (take it from the forward's opts->lse)");
+    if (reinterpret_cast<uintptr_t>(lse) % 4) return fail(DASH_ERR_ALIGNMENT, "lse not 4-byte aligned");
+    if (!(alpha > 1.f) || !isfinite(alpha)) return fail(DASH_ERR_INVALID_ARG, "alpha must be > 1");
+    if (o.kbar || o.qbar || o.summary_cache)
+        return fail(DASH_ERR_UNSUPPORTED, "the backward pass pools the keys itself: no kbar, qbar or summary_cache");
+    Geom G;
+    if ((rc = make_geom(q, k, block_size, causal, gqa_groups, &G))) return rc;
+    if ((rc = set_local(o, &G))) return rc;
+    if (G.b == 0 || G.nq == 0) {
+        // no query rows: every key and value gradient is zero
+        cudaStream_t st = static_cast<cudaStream_t>(o.stream);
+        dash_tensor_t *kv_grads[2] = {dk, dv};
+        for (dash_tensor_t *t : kv_grads) {
+            const size_t bytes = (size_t)t->shape[0] * t->shape[1] * t->shape[2] * t->shape[3] * esize(t->dtype);
+            const bool dense = t->stride[2] == t->shape[3] && t->stride[1] == t->shape[2] * t->shape[3] &&
+                               t->stride[0] == t->shape[1] * t->shape[2] * t->shape[3];
+            if (!dense) return fail(DASH_ERR_UNSUPPORTED, "empty query with strided dk/dv");
+            cudaError_t e = cudaMemsetAsync(t->data, 0, bytes, st);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+        }
+        return DASH_OK;
+    }
+    const bool tc = !(o.flags & DASH_FLAG_FORCE_SIMT) && attn_bwd_tc_supported(G, q->dtype);
+    const BwdLayout BL = bwd_layout(G, tc);
+    char *ws = nullptr;
+    if ((rc = get_workspace(o, BL.total, &ws))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(o.stream);
+    // Stage 0 and Stage 1 again (deterministic: the forward's routing, thresholds and lists)
+    const WsLayout &WL = BL.F;
+    float *kb = reinterpret_cast<float *>(ws + WL.kbar);
+    if ((rc = run_stage0(k, nullptr, TView{}, G, kb, st))) return rc;
+    const bool regroup = !(o.flags & DASH_FLAG_NO_REGROUP) && G.n_tiles > 1;
+    const ListsView LV = ws_lists(G, ws, WL, regroup);
+    float *tau = reinterpret_cast<float *>(ws + BL.tau);
+    uint32_t *mask = reinterpret_cast<uint32_t *>(ws + WL.mask);
+    if ((rc = run_stage1(q, G, alpha, o, kb, tau, nullptr, mask, &LV, regroup, ws, WL, st))) return rc;
+    BwdArgs a;
+    a.G = G;
+    a.L = LV;
+    a.Q = view(q);
+    a.K = view(k);
+    a.V = view(v);
+    a.O = view(out);
+    a.dO = view(dout);
+    a.dQ = view(dq);
+    a.dK = view(dk);
+    a.dV = view(dv);
+    a.lse = lse;
+    a.alpha = alpha;
+    a.gamma = o.gamma;
+    a.sigma = o.sigma;
+    a.kbar = kb;
+    a.tau = tau;
+    a.mask = mask;
+    a.logw = reinterpret_cast<float *>(ws + WL.logw);
+    a.Drow = reinterpret_cast<float *>(ws + BL.drow);
+    a.Gd = reinterpret_cast<float *>(ws + BL.gd);
+    a.dQacc = reinterpret_cast<float *>(ws + BL.dq);
+    a.dKbar = reinterpret_cast<float *>(ws + BL.dkbar);
+    a.bitmap = reinterpret_cast<uint32_t *>(ws + BL.bitmap);
+    a.E = reinterpret_cast<int32_t *>(ws + BL.E);
+    a.ref_off = reinterpret_cast<int32_t *>(ws + BL.ref_off);
+    a.ref_cnt = reinterpret_cast<int32_t *>(ws + BL.ref_cnt);
+    a.refs = reinterpret_cast<int2 *>(ws + BL.refs);
+    a.use_tc = tc;
+    a.Qp = tc ? reinterpret_cast<uint8_t *>(ws + BL.qp) : nullptr;
+    a.dOp = tc ? reinterpret_cast<uint8_t *>(ws + BL.dop) : nullptr;
+    a.Lp = tc ? reinterpret_cast<float *>(ws + BL.lp) : nullptr;
+    a.Dp = tc ? reinterpret_cast<float *>(ws + BL.dp) : nullptr;
+    cudaError_t e = launch_attn_bwd(a, q->dtype, st);
+    return e == cudaSuccess ? DASH_OK : cuda_fail(e, "backward pass");
 }
 
 DASH_API int dash_summary_cache_create(int64_t batch, int64_t max_nk, int hkv, int d, int block_size,

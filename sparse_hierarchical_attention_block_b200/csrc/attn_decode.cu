@@ -330,7 +330,7 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(const __grid_c
 // split partials (max, sum, O) in the log2 domain.
 template <int D>
 __global__ void __launch_bounds__(D) combine_kernel(TView O, Geom G, ListsView L, const float *__restrict__ part,
-                                                    int nsplit, int eps) {
+                                                    int nsplit, int eps, float *lse) {
     const int row = blockIdx.x, r = blockIdx.y;
     const int64_t b = blockIdx.z;
     const int g = G.g;
@@ -350,15 +350,21 @@ __global__ void __launch_bounds__(D) combine_kernel(TView O, Geom G, ListsView L
         den += f * p[1];
         num += f * p[2 + col];
     }
-    __nv_bfloat16 *op = reinterpret_cast<__nv_bfloat16 *>(const_cast<void *>(O.p)) + b * O.s0 +
-                        tile_row(L, G, ((size_t)b * G.hkv + r) * L.n_tiles, 0, row / g) * O.s1 +
+    const int64_t i = tile_row(L, G, ((size_t)b * G.hkv + r) * L.n_tiles, 0, row / g);
+    __nv_bfloat16 *op = reinterpret_cast<__nv_bfloat16 *>(const_cast<void *>(O.p)) + b * O.s0 + i * O.s1 +
                         (int64_t)(r * g + row % g) * O.s2;
     op[col] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
+    if (lse && col == 0)  // natural log of the row's normaliser (log2 domain partials)
+        lse[((size_t)b * G.nq + i) * G.hq + r * g + row % g] =
+            den > 0.f ? (mm + __log2f(den)) * 0.6931471805599453f : -INFINITY;
 }
 
 // List entries per split: 16, or fewer when the (batch, kv head) units are few, so that
 // the splits a list may need still give every SM several CTAs (16 per SM for lists
-// that route a sixteenth of their chunks).
+// that route a sixteenth of their chunks).  The SM count is B200's 148 as a constant,
+// not the current device's: the split count sizes the partials in the workspace, and a
+// fixed count keeps dash_workspace_bytes() independent of the device (on a part with
+// fewer SMs the splits stay correct, only their balance changes).
 int entries_per_split(const Geom &G) {
     const int64_t units = G.b * (int64_t)G.hkv;
     for (int eps = kEntriesPerSplit; eps > 4; eps /= 2)
@@ -373,7 +379,7 @@ int n_splits(const Geom &G) {
 
 template <int D, int BLK>
 cudaError_t launch_dec(const DecParams &dp, const TView &Q, const TView &O, const Geom &G, const ListsView &L,
-                       float *part, cudaStream_t st) {
+                       float *part, cudaStream_t st, float *lse) {
     using S = DecSmem<D, BLK>;
     const size_t smem = S::kTotal + 1024;
     cudaError_t e = cudaFuncSetAttribute(attn_decode_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -384,7 +390,7 @@ cudaError_t launch_dec(const DecParams &dp, const TView &Q, const TView &O, cons
         dp, Q, G, L, part, ns, eps);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     combine_kernel<D><<<dim3((unsigned)(G.nq * G.g), (unsigned)G.hkv, (unsigned)G.b), D, 0, st>>>(O, G, L, part,
-                                                                                                   ns, eps);
+                                                                                                   ns, eps, lse);
     return cudaGetLastError();
 }
 
@@ -402,14 +408,14 @@ size_t attn_decode_workspace(const Geom &G) {
 }
 
 cudaError_t launch_attn_decode(const TView &Q, const TView &K, const TView &V, const TView &O, const Geom &G,
-                               const ListsView &L, void *work, cudaStream_t st) {
+                               const ListsView &L, void *work, cudaStream_t st, float *lse) {
     if (G.nq == 0 || G.b == 0) return cudaSuccess;
     DecParams dp;
     if (!make_map_bf16(&dp.tmK, K, G.b, G.nk, G.hkv, G.d, 1, G.B)) return cudaErrorInvalidValue;
     if (!make_map_bf16(&dp.tmV, V, G.b, G.nk, G.hkv, G.d, 1, G.B)) return cudaErrorInvalidValue;
     float *part = static_cast<float *>(work);
 #define DASH_DEC_CASE(DD, BB) \
-    if (G.d == DD && G.B == BB) return launch_dec<DD, BB>(dp, Q, O, G, L, part, st);
+    if (G.d == DD && G.B == BB) return launch_dec<DD, BB>(dp, Q, O, G, L, part, st, lse);
     DASH_DEC_CASE(128, 64)
     DASH_DEC_CASE(128, 128)
     DASH_DEC_CASE(128, 32)

@@ -24,7 +24,7 @@ constexpr int kSub = 32;  // keys staged per step
 
 template <typename T>
 __global__ void __launch_bounds__(kSimtRows) attn_simt_kernel(TView Q, TView K, TView V, TView O, Geom G,
-                                                              ListsView L) {
+                                                              ListsView L, float *lse) {
     extern __shared__ __align__(16) float sm[];
     const int d = G.d, g = G.g, dp = d + 1;
     float *Qs = sm;                        // [128][d+1]
@@ -109,13 +109,16 @@ __global__ void __launch_bounds__(kSimtRows) attn_simt_kernel(TView Q, TView K, 
         T *ob = reinterpret_cast<T *>(const_cast<void *>(O.p)) + b * O.s0 + i * O.s1 + (int64_t)(r * g + hh) * O.s2;
         const float inv = lrun > 0.f ? 1.f / lrun : 0.f;
         for (int e = 0; e < d; ++e) ob[e] = from_f<T>(Os[m * dp + e] * inv);
+        if (lse)  // natural log of the row's normaliser: (m + log2 l) ln 2
+            lse[((size_t)b * G.nq + i) * G.hq + r * g + hh] =
+                lrun > 0.f ? (mrun + log2f(lrun)) * 0.6931471805599453f : -INFINITY;
     }
 }
 
 }  // namespace
 
 cudaError_t launch_attn_simt(const TView &Q, const TView &K, const TView &V, const TView &O, dash_dtype_t dt,
-                             const Geom &G, const ListsView &L, cudaStream_t st) {
+                             const Geom &G, const ListsView &L, cudaStream_t st, float *lse) {
     if (G.nq == 0 || G.b == 0) return cudaSuccess;
     const size_t smem = (size_t)(2 * kSimtRows + 2 * kSub) * (G.d + 1) * sizeof(float);
     dim3 grid((unsigned)L.n_tiles, (unsigned)G.hkv, (unsigned)G.b);
@@ -124,11 +127,11 @@ cudaError_t launch_attn_simt(const TView &Q, const TView &K, const TView &V, con
         e = cudaFuncSetAttribute(attn_simt_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem);
         if (e != cudaSuccess) return e;
-        attn_simt_kernel<__nv_bfloat16><<<grid, kSimtRows, smem, st>>>(Q, K, V, O, G, L);
+        attn_simt_kernel<__nv_bfloat16><<<grid, kSimtRows, smem, st>>>(Q, K, V, O, G, L, lse);
     } else {
         e = cudaFuncSetAttribute(attn_simt_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        attn_simt_kernel<float><<<grid, kSimtRows, smem, st>>>(Q, K, V, O, G, L);
+        attn_simt_kernel<float><<<grid, kSimtRows, smem, st>>>(Q, K, V, O, G, L, lse);
     }
     return cudaGetLastError();
 }

@@ -57,17 +57,6 @@ struct TcParams {
     CUtensorMap tmQ, tmK, tmV;
 };
 
-__device__ __forceinline__ uint64_t gtimer() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-__device__ __forceinline__ float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
 
 template <int D, int BLK>
 struct Smem {
@@ -94,59 +83,6 @@ struct Bars {
     uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *m_full, *m_empty, *s_full, *p_full, *pv_done, *fin;
 };
 
-// try_wait that lets the hardware suspend the thread for up to hint_ns while the phase
-// is incomplete (it resumes as soon as the phase completes), so that waiting warps do not
-// take issue slots from the softmax warps sharing their scheduler.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
-        : "memory");
-    return ok != 0;
-}
-constexpr uint32_t kSleepNs = 100000;  // longest single suspension of a waiting thread
-
-// Bounded wait.  Gives up after limit_ns (recording a device error and raising
-// the CTA's abort flag) or, when honor_abort is set, as soon as another role
-// has raised it.  Drain waits (copies or MMAs in flight) pass honor_abort = false.
-__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, uint64_t limit_ns, volatile int *abort,
-                                         bool honor_abort = true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = gtimer();
-    for (;;) {
-        if (mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
-        if (gtimer() - t0 > limit_ns) {
-            report_timeout();
-            *abort = 1;
-            return false;
-        }
-        if (honor_abort && *abort) return false;
-    }
-}
-
-// Packed fp32 pairs (the f32x2 forms of fma / add on sm_100a): one instruction per two values.
-__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ void f32x2_split(uint64_t v, float &lo, float &hi) {
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
 
 // One 64-key step of the single-pass softmax for this thread's row: p = 2^(s * sl2 + cbm)
 // from the step's S columns at taddr, packed to bf16 pairs in pk; returns the row's sum of
@@ -183,7 +119,7 @@ __device__ __forceinline__ float exp_step(uint32_t taddr, float sl2, const float
 
 template <int D, int BLK>
 __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_constant__ TcParams tp, TView Qv, TView O,
-                                                              Geom G, ListsView L, int flags) {
+                                                              Geom G, ListsView L, int flags, float *lse) {
     using S = Smem<D, BLK>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -309,14 +245,15 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
                 issued_v = j + 1;
             }
             if (*abort) {
-                // drain: every copy issued must land before the CTA's smem goes away
+                // drain: every copy issued must land before the CTA's smem goes away.  Issued
+                // copies always complete, so each drain wait gets the full bound.
                 for (int j = max(0, issued_k - kNS); j < issued_k; ++j)
-                    wait_bar(B.k_full + j % kNS, (j / kNS) & 1, kWaitNsTest, abort, false);
+                    wait_bar(B.k_full + j % kNS, (j / kNS) & 1, kWaitNs, abort, false);
                 for (int j = max(0, issued_v - kNS); j < issued_v; ++j)
-                    wait_bar(B.v_full + j % kNS, (j / kNS) & 1, kWaitNsTest, abort, false);
+                    wait_bar(B.v_full + j % kNS, (j / kNS) & 1, kWaitNs, abort, false);
                 for (int j = max(0, issued_m - kNM); j < issued_m; ++j)
-                    wait_bar(B.m_full + j % kNM, (j / kNM) & 1, kWaitNsTest, abort, false);
-                if (!gather_q) wait_bar(B.q_full, 0, kWaitNsTest, abort, false);
+                    wait_bar(B.m_full + j % kNM, (j / kNM) & 1, kWaitNs, abort, false);
+                if (!gather_q) wait_bar(B.q_full, 0, kWaitNs, abort, false);
             }
         }
     } else if (warp == 1) {
@@ -364,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
             }
             // every MMA this thread issued has completed before TMEM is freed
             mma_commit(B.fin);
-            wait_bar(B.fin, 0, kWaitNsTest * 50, abort, false);
+            wait_bar(B.fin, 0, kWaitNs, abort, false);
         }
     } else {
         // ------------------------------------------------------------- softmax warpgroup
@@ -537,6 +474,9 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
                 __nv_bfloat16 *op = reinterpret_cast<__nv_bfloat16 *>(const_cast<void *>(O.p)) + b * O.s0 +
                                     i * O.s1 + (int64_t)(r * g + hh) * O.s2;
                 const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+                if (lse && row_ok)  // natural log of the row's normaliser: (m + log2 l) ln 2
+                    lse[((size_t)b * G.nq + i) * G.hq + r * g + hh] =
+                        l_run > 0.f ? (m_run + __log2f(l_run)) * 0.6931471805599453f : -INFINITY;
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t u[32];
@@ -572,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
 
 template <int D, int BLK>
 cudaError_t launch_t(const TcParams &tp, const TView &Q, const TView &O, const Geom &G, const ListsView &L, int flags,
-                     cudaStream_t st) {
+                     cudaStream_t st, float *lse) {
     using S = Smem<D, BLK>;
     const size_t smem = S::kTotal + 1024;
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -580,7 +520,7 @@ cudaError_t launch_t(const TcParams &tp, const TView &Q, const TView &O, const G
     if (e != cudaSuccess) return e;
     const int64_t ctas = L.n_tiles * G.hkv * G.b;
     if (ctas > 0x7fffffff) return cudaErrorInvalidValue;
-    attn_tc_kernel<D, BLK><<<(unsigned)ctas, kThreads, smem, st>>>(tp, Q, O, G, L, flags);
+    attn_tc_kernel<D, BLK><<<(unsigned)ctas, kThreads, smem, st>>>(tp, Q, O, G, L, flags, lse);
     return cudaGetLastError();
 }
 
@@ -596,7 +536,7 @@ bool attn_tc_supported(const Geom &G, dash_dtype_t dt) {
 }
 
 cudaError_t launch_attn_tc(const TView &Q, const TView &K, const TView &V, const TView &O, const Geom &G,
-                           const ListsView &L, int flags, cudaStream_t st) {
+                           const ListsView &L, int flags, cudaStream_t st, float *lse) {
     if (G.nq == 0 || G.b == 0) return cudaSuccess;
     TcParams tp;
     if (!make_map_bf16(&tp.tmQ, Q, G.b, G.nq, G.hq, G.d, G.g, G.tile_rows)) return cudaErrorInvalidValue;
@@ -604,7 +544,7 @@ cudaError_t launch_attn_tc(const TView &Q, const TView &K, const TView &V, const
     if (!make_map_bf16(&tp.tmK, K, G.b, G.nk, G.hkv, G.d, 1, box)) return cudaErrorInvalidValue;
     if (!make_map_bf16(&tp.tmV, V, G.b, G.nk, G.hkv, G.d, 1, box)) return cudaErrorInvalidValue;
 #define DASH_TC_CASE(DD, BB) \
-    if (G.d == DD && G.B == BB) return launch_t<DD, BB>(tp, Q, O, G, L, flags, st);
+    if (G.d == DD && G.B == BB) return launch_t<DD, BB>(tp, Q, O, G, L, flags, st, lse);
     DASH_TC_CASE(128, 64)
     DASH_TC_CASE(128, 128)
     DASH_TC_CASE(128, 32)

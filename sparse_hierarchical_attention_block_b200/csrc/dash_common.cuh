@@ -201,6 +201,72 @@ __device__ __forceinline__ bool mbar_wait_ns(uint64_t *bar, uint32_t parity, uin
 }
 
 // ---------------------------------------------------------------------------
+// Bounded waits of the warp-specialised tensor-core kernels (a CTA-wide abort flag in
+// shared memory lets every role give up once one of them has timed out)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t gtimer() { return global_ns(); }
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// try_wait that lets the hardware suspend the thread for up to hint_ns while the phase
+// is incomplete (it resumes as soon as the phase completes), so that waiting warps do not
+// take issue slots from the warps that share their scheduler.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+constexpr uint32_t kSleepNs = 100000;  // longest single suspension of a waiting thread
+
+// Bounded wait.  Gives up after limit_ns (recording a device error and raising
+// the CTA's abort flag) or, when honor_abort is set, as soon as another role
+// has raised it.  Drain waits (copies or MMAs in flight) pass honor_abort = false.
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, uint64_t limit_ns, volatile int *abort,
+                                         bool honor_abort = true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = gtimer();
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
+        if (gtimer() - t0 > limit_ns) {
+            report_timeout();
+            *abort = 1;
+            return false;
+        }
+        if (honor_abort && *abort) return false;
+    }
+}
+
+// Packed fp32 pairs (the f32x2 forms of fma / add on sm_100a): one instruction per two values.
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f32x2_split(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// ---------------------------------------------------------------------------
 // TMA (tensor maps are built on the host; no multicast anywhere)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *m) {

@@ -46,14 +46,45 @@ cudaError_t launch_compact(const Geom &G, const uint32_t *mask, const float *log
                            const ListsView &L, cudaStream_t st);
 
 // Stage 2 (attn_simt.cu, attn_tc.cu, attn_decode.cu)
+// lse (optional, [b][nq][hq] fp32): natural log-sum-exp of each row's biased logits
 cudaError_t launch_attn_simt(const TView &Q, const TView &K, const TView &V, const TView &O, dash_dtype_t dt,
-                             const Geom &G, const ListsView &L, cudaStream_t st);
+                             const Geom &G, const ListsView &L, cudaStream_t st, float *lse = nullptr);
 bool attn_tc_supported(const Geom &G, dash_dtype_t dt);
 cudaError_t launch_attn_tc(const TView &Q, const TView &K, const TView &V, const TView &O, const Geom &G,
-                           const ListsView &L, int flags, cudaStream_t st);
+                           const ListsView &L, int flags, cudaStream_t st, float *lse = nullptr);
 bool attn_decode_supported(const Geom &G, dash_dtype_t dt);
 size_t attn_decode_workspace(const Geom &G);
 cudaError_t launch_attn_decode(const TView &Q, const TView &K, const TView &V, const TView &O, const Geom &G,
-                               const ListsView &L, void *work, cudaStream_t st);
+                               const ListsView &L, void *work, cudaStream_t st, float *lse = nullptr);
+
+// Backward pass (bwd.cu, attn_bwd_tc.cu).  Everything the kernels need: the forward's
+// inputs and output, the output gradient, the forward's lse, the recomputed Stage 0-1
+// state (summaries, thresholds, masks, log w, work lists) and the workspace areas.
+struct BwdArgs {
+    Geom G;
+    ListsView L;
+    TView Q, K, V, O, dO, dQ, dK, dV;
+    const float *lse;                  // [b][nq][hq] natural log-sum-exp of the forward
+    float alpha, gamma, sigma;
+    const float *kbar;                 // [b][kbar_cap][hkv][d] fp32 chunk summaries
+    const float *tau;                  // [b][nq][hq] Stage-1 thresholds
+    const uint32_t *mask;              // [b][nq][hkv][words] routed chunks
+    const float *logw;                 // log w of the routed chunks (logw_index layout)
+    float *Drow;                       // [b][nq][hq] <dO, O>
+    float *Gd;                         // G per (row, routed chunk), logw_index layout
+    float *dQacc;                      // [b][nq][hq][d] fp32
+    float *dKbar;                      // [b][n_chunks][hkv][d] fp32
+    uint32_t *bitmap;                  // [b][hkv][n_blk][ceil(n_tiles/32)] tiles attending each key block
+    int32_t *E;                        // [b][hkv][n_blk][n_tiles] entry index of the block in the tile's list
+    int32_t *ref_off, *ref_cnt;        // [b][hkv][n_blk] the block's (tile, entry) pairs
+    int2 *refs;                        // [b][hkv][n_tiles * n_blk] pairs
+    bool use_tc;                       // tensor-core Stage-2 kernels (bf16, d = 128, B in {64, 128})
+    uint8_t *Qp, *dOp;                 // tensor-core path: [b][hkv][n_tiles][128][d] bf16 tile rows
+    float *Lp, *Dp;                    // [b][hkv][n_tiles][128] lse (exp2 domain, +inf = empty) and D
+};
+cudaError_t launch_attn_bwd(const BwdArgs &a, dash_dtype_t dt, cudaStream_t st);
+bool attn_bwd_tc_supported(const Geom &G, dash_dtype_t dt);
+cudaError_t launch_attn_bwd_tc_dq(const BwdArgs &a, cudaStream_t st);
+cudaError_t launch_attn_bwd_tc_dkdv(const BwdArgs &a, cudaStream_t st);
 
 }  // namespace dash

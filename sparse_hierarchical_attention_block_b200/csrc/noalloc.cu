@@ -20,11 +20,13 @@
 // life of the process.  In host code its name only stands for the symbol: the
 // device address is looked up with cudaGetSymbolAddress, once per device, on
 // the first call made while that device is current (that first call should come
-// before any stream capture).  All calls share the one area and it keeps the
-// last call's contents; the forward pass writes every scratch word it reads
-// before reading it, so nothing has to be cleared between calls.  Calls whose
-// execution overlaps on the GPU (two streams, or two host threads) race on the
-// area: serialise them.
+// before any stream capture).  The address stays valid for the life of the device's
+// primary context: after cudaDeviceReset the old address must not be used, so this
+// entry point is not to be called again in a process that reset a device.  All
+// calls share the one area and it keeps the last call's contents; the forward pass
+// writes every scratch word it reads before reading it, so nothing has to be
+// cleared between calls.  Calls whose execution overlaps on the GPU (two streams,
+// or two host threads) race on the area: serialise them.
 #include <stdio.h>
 
 #include <mutex>
@@ -34,6 +36,9 @@
 
 namespace dash {
 int report_error(int code, const char *msg);
+int fwd_workspace_need(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v,
+                       const dash_tensor_t *out, int block_size, float alpha, int causal, int gqa_groups,
+                       const dash_opts_t *opts, size_t *need);
 }  // namespace dash
 
 namespace {
@@ -79,21 +84,21 @@ DASH_API int dash_attn_fwd_noalloc(const dash_tensor_t *q, const dash_tensor_t *
     } else {
         dash_opts_init(&o);
     }
-    if (!q || !k) return dash::report_error(DASH_ERR_INVALID_ARG, "q or k is NULL");
-    if (k->shape[2] > 0 && q->shape[2] % k->shape[2] == 0 && block_size > 0 && k->shape[1] > 0) {
-        const size_t need = dash_workspace_bytes(q->shape[0], q->shape[1], k->shape[1], (int)q->shape[2],
-                                                 (int)k->shape[2], (int)q->shape[3], block_size, causal);
-        if (need > (size_t)DASH_NOALLOC_SCRATCH_BYTES) {
-            char msg[256];
-            snprintf(msg, sizeof msg,
-                     "problem needs %zu bytes of scratch; dash_attn_fwd_noalloc holds at most %zu "
-                     "(use dash_attn_fwd_ex with a workspace)",
-                     need, (size_t)DASH_NOALLOC_SCRATCH_BYTES);
-            return dash::report_error(DASH_ERR_WORKSPACE, msg);
-        }
+    // the exact scratch this call's forward pass takes (it depends on the options: a
+    // summary cache or given summaries need no pooled-key area, prefill no split-KV area)
+    size_t need = 0;
+    int rc = dash::fwd_workspace_need(q, k, v, out, block_size, alpha, causal, gqa_groups, &o, &need);
+    if (rc) return rc;
+    if (need > (size_t)DASH_NOALLOC_SCRATCH_BYTES) {
+        char msg[256];
+        snprintf(msg, sizeof msg,
+                 "problem needs %zu bytes of scratch; dash_attn_fwd_noalloc holds at most %zu "
+                 "(use dash_attn_fwd_ex with a workspace)",
+                 need, (size_t)DASH_NOALLOC_SCRATCH_BYTES);
+        return dash::report_error(DASH_ERR_WORKSPACE, msg);
     }
     void *scratch = nullptr;
-    int rc = noalloc_scratch(&scratch);
+    rc = noalloc_scratch(&scratch);
     if (rc) return rc;
     o.workspace = scratch;
     o.workspace_bytes = DASH_NOALLOC_SCRATCH_BYTES;

@@ -111,7 +111,10 @@ def check_forward(q, k, v, out, block_size, alpha, causal, sigma=1e8, gamma=1.0,
         exp_out = ref["out"].copy()
         if frow.any():
             fr = np.nonzero(frow)[0]
-            w_in = np.where(rg[fr], np.maximum(np.maximum(ref["w"][fr], wg[fr]), 1e-300), 0.0)
+            # the oracle's own w on every chunk both select; the GPU's w only on a chunk
+            # that the GPU alone selected (the oracle gave it no mass)
+            both = rg[fr] & ro[fr]
+            w_in = np.where(both, ref["w"][fr], np.where(rg[fr], np.maximum(wg[fr], 1e-300), 0.0))
             re = oracle.fwd_rows(Qr[fr], rows[fr], nq, K, V, block_size, alpha, gamma=gamma, sigma=sigma,
                                  causal=causal, w_in=w_in, r_in=rg[fr].astype(np.uint8), want=("out",), qbar=qb,
                                  local=local)

@@ -46,6 +46,17 @@ def test_tiny_full(sigma):
     check_forward(q, k, v, out, w.block, w.alpha, True, sigma=sigma, label=f"tiny sigma={sigma:g}")
 
 
+@pytest.mark.parametrize("sigma", [1e8, 1.0])
+def test_tiny_planted_full(sigma):
+    """The Tiny shape (fp32, 1 head, 16 chunks) with planted blocks, so that its
+    routing is sparse and the fp32 CUDA-core path routes and masks chunks."""
+    w = synthetic.WORKLOADS["tiny"].with_(planted=True, amax_key="b64", seed=9)
+    q, k, v = synthetic.make_inputs(w, "cuda")
+    out = _run(q, k, v, w.block, w.alpha, True, sigma=sigma)
+    st = check_forward(q, k, v, out, w.block, w.alpha, True, sigma=sigma, label=f"tiny-planted sigma={sigma:g}")
+    assert st["sparsity"] > 0.3
+
+
 CASES = [
     # b, nq, nk, hq, hkv, d, B, dtype, alpha, causal, sigma
     (2, 512, 512, 8, 2, 128, 64, "bf16", 1.5, True, 1.0),
@@ -318,10 +329,11 @@ def test_decode_full():
         check_forward(q, k, v, out, w.block, w.alpha, True, sigma=sigma, label=f"decode sigma={sigma:g}")
 
 
-@pytest.mark.parametrize("alpha", [1.25, 1.5, 2.0])
-def test_prefill128k_sampled(alpha):
+@pytest.mark.parametrize("alpha,sigma", [(1.25, 1.0), (1.5, 1.0), (1.5, 1e8), (2.0, 1.0), (2.0, 1e8)])
+def test_prefill128k_sampled(alpha, sigma):
     w = synthetic.WORKLOADS["prefill128k"]
     q, k, v = synthetic.make_inputs(w, "cuda")
     rows = sample_rows(w.nq, w.block, 512, seed=128)
-    out = _run(q, k, v, w.block, alpha, True, sigma=1.0)
-    check_forward(q, k, v, out, w.block, alpha, True, sigma=1.0, rows=rows, label=f"prefill128k alpha={alpha}")
+    out = _run(q, k, v, w.block, alpha, True, sigma=sigma)
+    check_forward(q, k, v, out, w.block, alpha, True, sigma=sigma, rows=rows,
+                  label=f"prefill128k alpha={alpha} sigma={sigma:g}")
