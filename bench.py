@@ -181,6 +181,8 @@ def run_ours(args, rank, world, device):
     w = synthetic.WORKLOADS[args.workload]
     if args.batch:
         w = w.with_(batch=args.batch)
+    if args.seq and w.nq > 1:
+        w = w.with_(nq=args.seq, nk=args.seq, name=f"{w.name}@{args.seq}")
     alpha = args.alpha or w.alpha
     sigma = args.sigma
     decode = w.nq == 1  # one new query token per sequence
@@ -325,6 +327,81 @@ def run_ours(args, rank, world, device):
 
 
 # ---------------------------------------------------------------------------
+# backward pass (dash_attn_bwd)
+# ---------------------------------------------------------------------------
+
+def run_backward(args, device):
+    """Times dash_attn_bwd on the workload: one step = the whole backward (Stage 0-1
+    recomputed, the Stage-2 gradient on the query and key sides, the routing chain).
+    Algorithmic work: the five products of every (row, attended key) pair
+    (S, dP, dV, dK, dQ: 2 d FLOPs each) = 2.5 x the forward's selected F2."""
+    import sparse_hierarchical_attention_block_b200 as dash
+
+    dash.load_library()
+    w = synthetic.WORKLOADS[args.workload]
+    if args.batch:
+        w = w.with_(batch=args.batch)
+    if args.seq and w.nq > 1:
+        w = w.with_(nq=args.seq, nk=args.seq, name=f"{w.name}@{args.seq}")
+    alpha = args.alpha or w.alpha
+    sigma = args.sigma
+    q, k, v = synthetic.make_inputs(w, device)
+    gen = torch.Generator(device=device).manual_seed(1234)
+    dout = torch.randn(q.shape, generator=gen, device=device).to(q.dtype)
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+    flags = dash.DASH_FLAG_FORCE_SIMT if args.simt else 0
+    dash.dash_attn_fwd(q, k, v, out, w.block, alpha, True, w.g, sigma=sigma, lse=lse, flags=flags)
+    lists = dash.make_lists(q, k, w.block, w.g)
+    dash.dash_block_select(q, k, w.block, alpha, True, lists=lists, sigma=sigma)
+    cnt = routed_counts(dash, q, k, w, alpha, sigma)
+    f2, y, sparsity, exec_f = work_of(w, cnt, lists)
+    f_bwd = 2.5 * f2
+
+    def step():
+        dash.dash_attn_bwd(q, k, v, out, dout, lse, dq, dk, dv, w.block, alpha, True, w.g, sigma=sigma, flags=flags)
+
+    for _ in range(args.warmup):
+        step()
+    if dash.dash_sync_status() != 0:
+        raise RuntimeError("backward warm-up failed")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    smi_id = vis.split(",")[torch.cuda.current_device()] if vis else str(torch.cuda.current_device())
+    with ClockSampler(smi_id) as cs:
+        for a, b in ev:
+            flush.fill_(1.0)
+            a.record(stream)
+            step()
+            b.record(stream)
+        torch.cuda.synchronize()
+    if dash.dash_sync_status() != 0:
+        raise RuntimeError("backward failed")
+    ms = sum(a.elapsed_time(b) for a, b in ev) / len(ev)
+    peaks = load_peaks()
+    ach = f_bwd / (ms * 1e-3) / 1e12
+    return {
+        "mode": "backward", "metric": "DashAttention bwd TFLOP/s on the selected pairs (5 products)",
+        "value": round(ach, 3), "unit": "TFLOP/s", "ms_per_step": round(ms, 4), "steps": args.steps,
+        "warmup": args.warmup, "dtype": "bf16", "data": "synthetic (seeded planted-block generator)",
+        "path": "cuda cores" if args.simt else "tensor cores",
+        "config": {"workload": w.name, "batch": w.batch, "nq": w.nq, "nk": w.nk, "hq": w.hq, "hkv": w.hkv,
+                   "d": w.d, "block": w.block, "alpha": alpha, "sigma": sigma, "sparsity": round(sparsity, 4),
+                   "l2": "flushed (256 MiB write) before every timed step"},
+        "work": {"selected_bwd_flops": f_bwd, "forward_selected_flops": f2,
+                 "union_waste": (round(exec_f / f2, 3) if exec_f else None)},
+        "roofline": {"bound": "tensor", "achieved": round(ach, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(ach / peaks["bf16_tflops"], 4), "traffic": None,
+                     "kernel": "whole dash_attn_bwd call (Stage 0-1 recompute included)",
+                     "peak_source": peaks["source"] + " bf16_tflops (burst)"},
+        "clocks": cs.summary(),
+    }
+
+
+# ---------------------------------------------------------------------------
 # controlled-sparsity sweep of Stage 2 (random routing masks)
 # ---------------------------------------------------------------------------
 
@@ -455,6 +532,8 @@ def run_reference(args, device):
     w = synthetic.WORKLOADS[args.workload]
     if args.batch:
         w = w.with_(batch=args.batch)
+    if args.seq and w.nq > 1:
+        w = w.with_(nq=args.seq, nk=args.seq, name=f"{w.name}@{args.seq}")
     alpha = args.alpha or w.alpha
     q, k, v = synthetic.make_inputs(w, device)
     decode = w.nq == 1
@@ -491,6 +570,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="prefill128k", choices=sorted(synthetic.WORKLOADS))
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (smaller profiling cases)")
+    ap.add_argument("--seq", type=int, default=0,
+                    help="override a prefill workload's sequence length (nq = nk; smaller profiling cases)")
     ap.add_argument("--alpha", type=float, default=None)
     ap.add_argument("--sigma", type=float, default=1e8)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -499,6 +580,8 @@ def main():
     ap.add_argument("--local2", action="store_true",
                     help="two-block local window (the chunk before the query's own attended in full)")
     ap.add_argument("--mask-sweep", action="store_true", help="controlled-sparsity sweep of Stage 2 (1 GPU)")
+    ap.add_argument("--backward", action="store_true", help="time the backward pass dash_attn_bwd (1 GPU)")
+    ap.add_argument("--simt", action="store_true", help="with --backward: the CUDA-core Stage-2 kernels")
     ap.add_argument("--sweep-n", default="16384,32768,65536,98304")
     ap.add_argument("--sweep-s", default="0.75,0.875,0.9375")
     ap.add_argument("--sweep-phase", default="prefill,decode")
@@ -509,6 +592,12 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.warmup < 3:
         args.warmup = 3
+
+    if args.backward:
+        if rank == 0:
+            torch.cuda.set_device(local)
+            print(json.dumps(run_backward(args, torch.device("cuda", local))))
+        return 0
 
     if args.mask_sweep:
         if rank == 0:

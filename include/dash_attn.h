@@ -129,6 +129,18 @@ typedef struct {
                                log-sum-exp of each row's Stage-2 logits z + d over the keys it
                                attends (the normaliser of Eq. 7's softmax); the backward pass
                                (dash_attn_bwd) takes it back.  NULL = not written. */
+    const int64_t *nk_dev;  /* optional, dash_attn_fwd_ex only: DEVICE pointer to the number of
+                               valid keys, read by the kernels when they run, so that one
+                               captured launch sequence (a CUDA graph of a decoding step)
+                               serves every length.  k and v then describe the preallocated
+                               cache (shape[1] = its capacity, at most the summary cache's
+                               max_nk); keys at and past *nk_dev are ignored and the new query
+                               rows sit at the last positions before it.  Needs opts->
+                               summary_cache, which the call itself brings up to date on the
+                               device (up to 16 chunks completed since the previous call;
+                               more: call dash_summary_cache_update first), and the decoding
+                               path: bf16, nq * gqa_groups <= 16, 1 <= *nk_dev <= capacity,
+                               *nk_dev >= nq.  NULL = k's shape[1] is the length. */
 } dash_opts_t;
 
 /* Fill *opts with the defaults above.  Returns DASH_OK or DASH_ERR_INVALID_ARG (NULL). */
@@ -185,9 +197,10 @@ DASH_API int dash_summary_cache_create(int64_t batch, int64_t max_nk, int hkv, i
  * chunks than were pooled. */
 DASH_API int dash_summary_cache_update(dash_summary_cache_t *cache, const dash_tensor_t *k,
                                        const dash_tensor_t *qbar, void *stream);
-/* Forgets every pooled chunk (new sequences).  Host-side only. */
+/* Forgets every pooled chunk (new sequences); waits for the device first. */
 DASH_API int dash_summary_cache_reset(dash_summary_cache_t *cache);
-/* Chunks pooled so far; -1 for a NULL cache. */
+/* Chunks pooled so far by dash_summary_cache_update (catch-up steps of a forward with
+ * opts->nk_dev count on the device only); -1 for a NULL cache. */
 DASH_API int64_t dash_summary_cache_chunks(const dash_summary_cache_t *cache);
 /* The fp32 summaries [batch][floor(max_nk/B)][hkv][d] (device memory the cache owns). */
 DASH_API const float *dash_summary_cache_kbar(const dash_summary_cache_t *cache);

@@ -61,7 +61,11 @@ def backward(Q, K, V, dO, block_size: int, alpha: float, *, gamma: float = 1.0, 
 
     rows: optional query indices.  A row's dQ depends on that row alone (its own Stage 2
     and its own routing), so with rows given only those rows are differentiated and the
-    result holds dQ of exactly those rows, in the given order (no dK, dV)."""
+    result holds dQ of exactly those rows, in the given order (no dK, dV).
+
+    Beside the gradients: G [rows, hkv, n_chunks] the bias gradient of each routed chunk
+    (0 elsewhere), Pmass [rows, hq, n_chunks] each head's Stage-2 probability on each routed
+    chunk, and the forward's out, w, xmt (x - tau per head) and the summaries kbar."""
     Q = np.ascontiguousarray(Q, dtype=np.float32)
     K = np.ascontiguousarray(K, dtype=np.float32)
     V = np.ascontiguousarray(V, dtype=np.float32)
@@ -99,6 +103,8 @@ def backward(Q, K, V, dO, block_size: int, alpha: float, *, gamma: float = 1.0, 
     dK = np.zeros_like(Kd)
     dV = np.zeros_like(Vd)
     dKbar = np.zeros_like(Kbar)
+    Gall = np.zeros((len(sel), hkv, nch))  # the bias gradient G of every routed chunk
+    Pmass = np.zeros((len(sel), hq, nch))  # each head's Stage-2 probability mass on every routed chunk
     for n, i in enumerate(sel):
         if causal:
             p_i = i + nk - nq
@@ -138,8 +144,13 @@ def backward(Q, K, V, dO, block_size: int, alpha: float, *, gamma: float = 1.0, 
                 np.add.at(dK[:, r], toks, np.outer(dl, q) * scale)
                 routed_tok = chunk_of >= 0
                 np.add.at(G, chunk_of[routed_tok], dl[routed_tok])
+                if len(Rc):
+                    pm = np.zeros(len(Rc))
+                    np.add.at(pm, chunk_of[routed_tok], P[routed_tok])
+                    Pmass[n, h, Rc] = pm
             if len(Rc) == 0:
                 continue
+            Gall[n, r, Rc] = G
             # prior bias -> log w -> w -> each head's entmax probabilities
             dlogw = (G - G.mean()) / sigma
             dw = np.zeros(nch)
@@ -153,7 +164,8 @@ def backward(Q, K, V, dO, block_size: int, alpha: float, *, gamma: float = 1.0, 
                 dQ[i, h] += gamma * scale * (ds @ Kbar[:nvis, r])
                 dKbar[:nvis, r] += gamma * scale * np.outer(ds, Qd[i, h])
     if rows is not None:
-        return {"dQ": dQ[sel], "rows": sel}
+        return {"dQ": dQ[sel], "rows": sel, "G": Gall, "Pmass": Pmass, "w": ref["w"], "xmt": ref["xmt"],
+                "kbar": Kbar, "out": ref["out"]}
     # Stage 0: the chunk's keys through the weights A (uniform for the mean)
     dQbar = np.zeros((nch, hkv, d))
     for c in range(nch):
@@ -168,7 +180,8 @@ def backward(Q, K, V, dO, block_size: int, alpha: float, *, gamma: float = 1.0, 
         e = a * (da - (a * da).sum(axis=0))
         dK[sl] += e[:, :, None] * qbar[c].astype(np.float64)[None] * scale
         dQbar[c] = np.einsum("th,thd->hd", e, kc) * scale
-    res = {"out": ref["out"], "dQ": dQ, "dK": dK, "dV": dV}
+    res = {"out": ref["out"], "dQ": dQ, "dK": dK, "dV": dV, "G": Gall, "Pmass": Pmass, "w": ref["w"],
+           "xmt": ref["xmt"], "kbar": Kbar}
     if qbar is not None:
         res["dQbar"] = dQbar
     return res

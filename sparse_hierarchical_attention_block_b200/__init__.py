@@ -63,7 +63,8 @@ class _Opts(ctypes.Structure):
     _fields_ = [("sigma", ctypes.c_float), ("gamma", ctypes.c_float), ("stream", ctypes.c_void_p),
                 ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
                 ("kbar", ctypes.c_void_p), ("flags", ctypes.c_int),
-                ("qbar", ctypes.POINTER(_Tensor)), ("summary_cache", ctypes.c_void_p), ("lse", ctypes.c_void_p)]
+                ("qbar", ctypes.POINTER(_Tensor)), ("summary_cache", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+                ("nk_dev", ctypes.c_void_p)]
 
 
 _lib = None
@@ -156,7 +157,7 @@ def _ptr(t):
 
 
 def _opts(sigma=1e8, gamma=1.0, kbar=None, workspace=None, flags=0, stream=None, qbar=None,
-          summary_cache=None, lse=None) -> _Opts:
+          summary_cache=None, lse=None, nk_dev=None) -> _Opts:
     o = _Opts()
     load_library().dash_opts_init(ctypes.byref(o))
     o.sigma = float(sigma)
@@ -177,6 +178,10 @@ def _opts(sigma=1e8, gamma=1.0, kbar=None, workspace=None, flags=0, stream=None,
         o.qbar = ctypes.pointer(qd)
     if summary_cache is not None:
         o.summary_cache = summary_cache.handle
+    if nk_dev is not None:
+        if nk_dev.dtype != torch.int64 or not nk_dev.is_cuda:
+            raise ValueError("nk_dev must be an int64 tensor on the device (one element)")
+        o.nk_dev = nk_dev.data_ptr()
     if lse is not None:
         if lse.dtype != torch.float32 or not lse.is_contiguous():
             raise ValueError("lse must be a contiguous float32 tensor [b, nq, hq]")

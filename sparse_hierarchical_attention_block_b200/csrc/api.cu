@@ -15,6 +15,7 @@ namespace dash {
 int take_device_error_tc();
 int take_device_error_decode();
 int take_device_error_select();
+int take_device_error_bwd();
 }  // namespace dash
 
 using namespace dash;
@@ -25,10 +26,11 @@ struct dash_summary_cache {
     int hkv, d, B;
     int cap;       // chunk capacity floor(max_nk / B): the summaries' batch stride
     int ct_cap;    // 128-chunk tiles of the split form per (batch, kv head)
-    int64_t done;  // chunks pooled so far
+    int64_t done;  // chunks pooled so far (host-side updates)
     int dev;
     float *kbar;     // [b][cap][hkv][d] fp32
     uint8_t *split;  // [b][hkv][ct_cap] bf16 hi + lo operand tiles
+    int *done_dev;   // chunks pooled so far, in device memory (device-resident key length)
 };
 
 namespace {
@@ -102,6 +104,8 @@ int make_geom(const dash_tensor_t *q, const dash_tensor_t *k, int B, int causal,
     G->kbar_cap = G->n_chunks;
     G->ct_cap = (G->n_chunks + 127) / 128;
     G->local = 1;
+    G->nk_dev = nullptr;
+    G->chunks_dev = nullptr;
     return DASH_OK;
 }
 
@@ -295,9 +299,12 @@ int check_cache(const dash_summary_cache *sc, const Geom &G, const dash_opts_t &
     if (!G.causal) return fail(DASH_ERR_INVALID_ARG, "summary_cache needs causal routing");
     if (sc->b != G.b || sc->hkv != G.hkv || sc->d != G.d || sc->B != G.B)
         return fail(DASH_ERR_INVALID_ARG, "summary_cache was made for another shape or block size");
-    if (sc->done != G.n_chunks)
+    if (!o.nk_dev && sc->done != G.n_chunks)
         return fail(DASH_ERR_INVALID_ARG, "summary_cache holds %lld chunks; the keys have %d complete chunks",
                     (long long)sc->done, G.n_chunks);
+    if (o.nk_dev && G.nk > sc->max_nk)
+        return fail(DASH_ERR_INVALID_ARG, "k's capacity (%lld keys) exceeds the summary cache's max_nk (%lld)",
+                    (long long)G.nk, (long long)sc->max_nk);
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev != sc->dev)
         return fail(DASH_ERR_INVALID_ARG, "summary_cache lives on another device");
@@ -357,6 +364,14 @@ int plan_fwd(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t
     if (o.qbar && (rc = check_qbar(o.qbar, G, &P->qv))) return rc;
     P->need_kbar = o.kbar == nullptr && !P->sc;
     P->dec = attn_decode_supported(G, q->dtype) && !(o.flags & DASH_FLAG_FORCE_SIMT);
+    if (o.nk_dev) {
+        if (!P->sc) return fail(DASH_ERR_INVALID_ARG, "opts->nk_dev needs opts->summary_cache");
+        if (reinterpret_cast<uintptr_t>(o.nk_dev) % 8) return fail(DASH_ERR_ALIGNMENT, "nk_dev not 8-byte aligned");
+        if (!P->dec || !select_tile_supported(G, q->dtype) || G.local != 1)
+            return fail(DASH_ERR_UNSUPPORTED, "opts->nk_dev: decoding only (bf16, nq * gqa_groups <= 16, the "
+                                              "tensor-core Stage 1, the one-block local window)");
+        G.nk_dev = o.nk_dev;
+    }
     P->WL = (G.b == 0 || G.nq == 0) ? WsLayout{} : ws_layout(G, P->need_kbar, true, P->dec);
     return DASH_OK;
 }
@@ -502,6 +517,7 @@ DASH_API int dash_block_select(const dash_tensor_t *q, const dash_tensor_t *k, i
     dash_opts_t o = opts ? *opts : default_opts();
     int rc;
     if ((rc = check_opts(o))) return rc;
+    if (o.nk_dev) return fail(DASH_ERR_UNSUPPORTED, "opts->nk_dev is for dash_attn_fwd_ex");
     if ((rc = check_tensor(q, "q")) || (rc = check_tensor(k, "k"))) return rc;
     if (q->dtype != k->dtype) return fail(DASH_ERR_INVALID_ARG, "q and k must share a dtype");
     if (!(alpha > 1.f) || !isfinite(alpha)) return fail(DASH_ERR_INVALID_ARG, "alpha must be > 1");
@@ -541,6 +557,7 @@ DASH_API int dash_sparse_attn_fwd(const dash_tensor_t *q, const dash_tensor_t *k
     dash_opts_t o = opts ? *opts : default_opts();
     int rc;
     if ((rc = check_opts(o))) return rc;
+    if (o.nk_dev) return fail(DASH_ERR_UNSUPPORTED, "opts->nk_dev is for dash_attn_fwd_ex");
     if ((rc = validate_qkvo(q, k, v, out))) return rc;
     if (!lists) return fail(DASH_ERR_INVALID_ARG, "lists is NULL");
     Geom G;
@@ -569,6 +586,13 @@ DASH_API int dash_attn_fwd_ex(const dash_tensor_t *q, const dash_tensor_t *k, co
     char *ws = nullptr;
     if ((rc = get_workspace(o, WL.total, &ws))) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(o.stream);
+    if (G.nk_dev) {
+        // the cache catches up on the device with the chunks completed since the last step
+        Geom Gc = cache_geom(G, sc);
+        Gc.chunks_dev = sc->done_dev;
+        cudaError_t e = launch_cache_catch_up(view(k), k->dtype, Gc, sc->kbar, sc->split, st);
+        if (e != cudaSuccess) return cuda_fail(e, "summary cache catch-up");
+    }
     const float *kbar = sc ? sc->kbar : o.kbar;
     if (need_kbar) {
         float *kb = reinterpret_cast<float *>(ws + WL.kbar);
@@ -594,7 +618,7 @@ namespace {
 
 struct BwdLayout {
     WsLayout F;  // Stage 0-1 state (recomputed) and the work lists
-    size_t tau, drow, gd, dq, dkbar, bitmap, E, ref_off, ref_cnt, refs, qp, dop, lp, dp, total;
+    size_t tau, drow, gd, dq, dkbar, meang, rho, bitmap, E, ref_off, ref_cnt, refs, qp, dop, lp, dp, total;
 };
 
 BwdLayout bwd_layout(const Geom &G, bool tc) {
@@ -614,6 +638,8 @@ BwdLayout bwd_layout(const Geom &G, bool tc) {
     L.gd = take((size_t)G.b * G.nq * G.hkv * (size_t)G.n_chunks * 4);
     L.dq = take(rows * G.d * 4);
     L.dkbar = take((size_t)G.b * G.n_chunks * G.hkv * G.d * 4);
+    L.meang = take((size_t)G.b * G.nq * G.hkv * 4);
+    L.rho = take(rows * 4);
     L.bitmap = take(bhb * tw * 4);
     L.E = take(bhb * G.n_tiles * 4);
     L.ref_off = take(bhb * 4);
@@ -681,8 +707,9 @@ DASH_API int dash_attn_bwd(const dash_tensor_t *q, const dash_tensor_t *k, const
     if (!lse) return fail(DASH_ERR_INVALID_ARG, "lse is NULL (take it from the forward's opts->lse)");
     if (reinterpret_cast<uintptr_t>(lse) % 4) return fail(DASH_ERR_ALIGNMENT, "lse not 4-byte aligned");
     if (!(alpha > 1.f) || !isfinite(alpha)) return fail(DASH_ERR_INVALID_ARG, "alpha must be > 1");
-    if (o.kbar || o.qbar || o.summary_cache)
-        return fail(DASH_ERR_UNSUPPORTED, "the backward pass pools the keys itself: no kbar, qbar or summary_cache");
+    if (o.kbar || o.qbar || o.summary_cache || o.nk_dev)
+        return fail(DASH_ERR_UNSUPPORTED,
+                    "the backward pass pools the keys itself: no kbar, qbar, summary_cache or nk_dev");
     Geom G;
     if ((rc = make_geom(q, k, block_size, causal, gqa_groups, &G))) return rc;
     if ((rc = set_local(o, &G))) return rc;
@@ -737,6 +764,8 @@ DASH_API int dash_attn_bwd(const dash_tensor_t *q, const dash_tensor_t *k, const
     a.Gd = reinterpret_cast<float *>(ws + BL.gd);
     a.dQacc = reinterpret_cast<float *>(ws + BL.dq);
     a.dKbar = reinterpret_cast<float *>(ws + BL.dkbar);
+    a.meanG = reinterpret_cast<float *>(ws + BL.meang);
+    a.rho = reinterpret_cast<float *>(ws + BL.rho);
     a.bitmap = reinterpret_cast<uint32_t *>(ws + BL.bitmap);
     a.E = reinterpret_cast<int32_t *>(ws + BL.E);
     a.ref_off = reinterpret_cast<int32_t *>(ws + BL.ref_off);
@@ -776,9 +805,13 @@ DASH_API int dash_summary_cache_create(int64_t batch, int64_t max_nk, int hkv, i
         e = cudaMalloc(&c->split, sb);
         if (e == cudaSuccess) e = cudaMemset(c->split, 0, sb);
     }
+    if (e == cudaSuccess) e = cudaMalloc(&c->done_dev, sizeof(int));
+    if (e == cudaSuccess) e = cudaMemset(c->done_dev, 0, sizeof(int));
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) {
         cudaFree(c->kbar);
         cudaFree(c->split);
+        cudaFree(c->done_dev);
         delete c;
         return cuda_fail(e, "summary cache allocation");
     }
@@ -820,11 +853,17 @@ DASH_API int dash_summary_cache_update(dash_summary_cache_t *c, const dash_tenso
     e = launch_kbar_split(c->kbar, G, c->split, c0 / 128, (c1 + 127) / 128, st);
     if (e != cudaSuccess) return cuda_fail(e, "summary cache split");
     c->done = c1;
+    e = launch_set_int(c->done_dev, c1, st);  // the device-side count follows
+    if (e != cudaSuccess) return cuda_fail(e, "summary cache count");
     return DASH_OK;
 }
 
 DASH_API int dash_summary_cache_reset(dash_summary_cache_t *c) {
     if (!c) return fail(DASH_ERR_INVALID_ARG, "cache is NULL");
+    cudaError_t e = cudaDeviceSynchronize();  // no step in flight still counts on the old chunks
+    if (e == cudaSuccess) e = cudaMemset(c->done_dev, 0, sizeof(int));
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "summary cache reset");
     c->done = 0;
     return DASH_OK;
 }
@@ -838,6 +877,7 @@ DASH_API int dash_summary_cache_destroy(dash_summary_cache_t *c) {
     cudaError_t e = cudaDeviceSynchronize();
     cudaFree(c->kbar);
     cudaFree(c->split);
+    cudaFree(c->done_dev);
     delete c;
     return e == cudaSuccess ? DASH_OK : cuda_fail(e, "cudaDeviceSynchronize");
 }
@@ -845,7 +885,8 @@ DASH_API int dash_summary_cache_destroy(dash_summary_cache_t *c) {
 DASH_API int dash_sync_status(void *stream) {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
-    int dev_err = take_device_error_tc() | take_device_error_decode() | take_device_error_select();
+    int dev_err = take_device_error_tc() | take_device_error_decode() | take_device_error_select() |
+                  take_device_error_bwd();
     if (dev_err) return fail(DASH_ERR_DEVICE_TIMEOUT, "a device-side bounded wait ran out");
     return DASH_OK;
 }

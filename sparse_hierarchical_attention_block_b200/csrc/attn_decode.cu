@@ -103,9 +103,11 @@ struct DecSmem {
 
 template <int D, int BLK>
 __global__ void __launch_bounds__(kDecThreads) attn_decode_kernel(const __grid_constant__ DecParams dp, TView Q,
-                                                                  Geom G, ListsView L, float *__restrict__ part,
+                                                                  Geom G0, ListsView L, float *__restrict__ part,
                                                                   int nsplit, int eps) {
     using S = DecSmem<D, BLK>;
+    Geom G = G0;
+    geom_live(G);
     extern __shared__ uint8_t dsm_raw[];
     uint8_t *sm = dsm_raw + ((1024 - (smem_u32(dsm_raw) & 1023)) & 1023);
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + S::kBars);

@@ -7,8 +7,9 @@
 // bias (-inf where the row does not attend the chunk), keys j > p_i masked when
 // causal.  Online softmax in the exp2 domain with fp32 statistics.
 //
-// One CTA per (batch, kv head, query tile of 128/g positions x g heads = 128 rows),
-// the heaviest tiles (latest, causal) of all heads first, two CTAs resident per SM.  A step
+// One CTA per (batch, kv head, query tile of 128/g positions x g heads = 128 rows), the
+// heaviest (latest, causal) tiles first within groups of heads whose K and V fit in L2
+// together (all heads at 8K, one at a time at 128K), two CTAs resident per SM.  A step
 // covers 64 keys (one or more listed chunks, or half of a 128-key chunk); S is
 // double-buffered in tensor memory, so the MMA of step j+1 runs during the softmax of
 // step j.  Warp roles (192 threads):
@@ -119,18 +120,18 @@ __device__ __forceinline__ float exp_step(uint32_t taddr, float sl2, const float
 
 template <int D, int BLK>
 __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_constant__ TcParams tp, TView Qv, TView O,
-                                                              Geom G, ListsView L, int flags, float *lse) {
+                                                              Geom G, ListsView L, int flags, float *lse, int hg) {
     using S = Smem<D, BLK>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    // one CTA per (tile, batch, kv head), launched heaviest (latest, causal) tiles first
-    // across all heads, so that the long tiles do not gather at the end of the grid
-    const int64_t bh = G.b * G.hkv;
-    const int64_t t = (int64_t)L.n_tiles - 1 - (int64_t)blockIdx.x / bh;
-    const int r = (int)(((int64_t)blockIdx.x % bh) % G.hkv);
-    const int64_t b = ((int64_t)blockIdx.x % bh) / G.hkv;
+    // one CTA per (tile, batch, kv head), in the order of tile_order: groups of heads whose
+    // K and V share L2, the heaviest (latest, causal) tiles of a group first
+    const TileOrder to = tile_order(blockIdx.x, L.n_tiles, G.b * G.hkv, hg);
+    const int64_t t = to.t;
+    const int r = (int)(to.bh % G.hkv);
+    const int64_t b = to.bh / G.hkv;
     const int g = G.g, T = L.tile_rows;
     const size_t tile_idx = ((size_t)b * G.hkv + r) * L.n_tiles + t;
     const int count = L.count[tile_idx];
@@ -520,7 +521,8 @@ cudaError_t launch_t(const TcParams &tp, const TView &Q, const TView &O, const G
     if (e != cudaSuccess) return e;
     const int64_t ctas = L.n_tiles * G.hkv * G.b;
     if (ctas > 0x7fffffff) return cudaErrorInvalidValue;
-    attn_tc_kernel<D, BLK><<<(unsigned)ctas, kThreads, smem, st>>>(tp, Q, O, G, L, flags, lse);
+    attn_tc_kernel<D, BLK><<<(unsigned)ctas, kThreads, smem, st>>>(tp, Q, O, G, L, flags, lse,
+                                                                    heads_per_group(G));
     return cudaGetLastError();
 }
 

@@ -351,10 +351,12 @@ __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(TView Q, const
 }
 
 // One CTA per (batch, kv head, query tile).
-__global__ void __launch_bounds__(128) compact_kernel(Geom G, const uint32_t *__restrict__ mask,
+__global__ void __launch_bounds__(128) compact_kernel(Geom G0, const uint32_t *__restrict__ mask,
                                                       const float *__restrict__ logw, const float *__restrict__ mu,
                                                       float inv_sigma, ListsView L) {
     extern __shared__ __align__(16) uint32_t csm[];
+    Geom G = G0;
+    geom_live(G);
     uint32_t *uw = csm;                 // [words] union bits (diagonal range removed)
     int *wofs = reinterpret_cast<int *>(uw + G.words);  // [words + 1] exclusive prefix of popcounts
     const int64_t t = blockIdx.x;

@@ -24,8 +24,10 @@
 //   refs_mark_kernel,     the work lists transposed: for every key block the (tile,
 //   refs_build_kernel     entry) pairs that attend it, tiles ascending (deterministic)
 //   bwd_dkdv_simt_kernel  per key block: dK (Stage 2 + pooling share), dV over its pairs
-//   bwd_route_kernel      per (row, kv head): the prior / entmax / score chain above
-//   bwd_dq_finish_kernel  dQ to the caller's dtype
+//   bwd_route_kernel      per (row, kv head): the prior / entmax / score chain above, added
+//                         to the Stage-2 part of dQ, which it writes in the caller's dtype
+//   bwd_kbar_grad_kernel  per (chunk, kv head): the same chain into the chunk summary
+//   bwd_dq_finish_kernel  dQ to the caller's dtype when no row routes anything
 #include <math.h>
 
 #include "dash_common.cuh"
@@ -342,25 +344,63 @@ __global__ void __launch_bounds__(128) bwd_dkdv_simt_kernel(TView Q, TView K, TV
 // ---------------------------------------------------------------------------
 // Routing gradient on CUDA cores: one warp per (batch, row, kv head).  Lane l holds
 // dimensions l, l + 32, ... of the group's queries.  Three passes over the routed set
-// R_i (mask bits): mean G; per head sum u and sum u dp; then ds, which goes to dQ and
-// (atomically) to dKbar.
+// R_i (mask bits): mean G; per head sum u and sum u dp; then ds, which goes to dQ.  The
+// row's mean G and, per head, <u, dp> / sum u are kept for bwd_kbar_grad_kernel, which
+// forms the summaries' gradient chunk by chunk (no atomics).
 // ---------------------------------------------------------------------------
 constexpr int kMaxG = 16;
+
+// The per-chunk arithmetic both kernels share: for head h's x = xs <q, kbar_c> and
+// threshold th, p = (x - th)^(1/(alpha-1)), u = p^(2-alpha) and u dp with dp = d(log w_c)
+// / (g w_c); false outside the head's own support (u = 0 there).
+__device__ __forceinline__ bool route_terms(float x, float th, float kexp, float uexp, float lw, float dlw, int g,
+                                            float &u, float &ud) {
+    if (!(x > th)) return false;
+    const float lp = kexp * __logf(x - th);        // log p
+    u = __expf(uexp * lp);                          // p^(2 - alpha)
+    ud = __expf(uexp * lp - lw) * dlw / (float)g;   // u dp
+    return true;
+}
+
+// The row's dQ (the Stage-2 part in dQacc plus the routing part dq_route, per head and
+// lane dimension) written in the caller's dtype.
+template <typename T, int DL>
+__device__ __forceinline__ void store_dq(const float *__restrict__ dQacc, TView dQ, const Geom &G, int64_t b,
+                                         int64_t i, int r, int lane, const float (&dq_route)[16][DL], float sc) {
+#pragma unroll
+    for (int h = 0; h < 16; ++h) {
+        if (h >= G.g) break;
+        const float *src = dQacc + (((size_t)b * G.nq + i) * G.hq + r * G.g + h) * G.d;
+        T *dst = reinterpret_cast<T *>(const_cast<void *>(dQ.p)) + b * dQ.s0 + i * dQ.s1 + (int64_t)(r * G.g + h) * dQ.s2;
+#pragma unroll
+        for (int k = 0; k < DL; ++k) dst[lane + 32 * k] = from_f<T>(src[lane + 32 * k] + sc * dq_route[h][k]);
+    }
+}
 
 template <typename T, int DL>  // DL = d / 32 dims per lane
 __global__ void __launch_bounds__(128) bwd_route_kernel(TView Q, const float *__restrict__ kbar, Geom G, float alpha,
                                                         float gamma, float sigma, const float *__restrict__ tau,
                                                         const uint32_t *__restrict__ mask,
                                                         const float *__restrict__ logw, const float *__restrict__ Gd,
-                                                        float *__restrict__ dQacc, float *__restrict__ dKbar) {
+                                                        const float *__restrict__ dQacc, TView dQ,
+                                                        float *__restrict__ meanG_out, float *__restrict__ rho_out) {
     const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
     const int lane = threadIdx.x % 32;
     if (w >= G.b * G.nq * G.hkv) return;
     const int r = (int)(w % G.hkv);
     const int64_t i = (w / G.hkv) % G.nq, b = w / ((int64_t)G.hkv * G.nq);
     const int nvis = row_nvis(G, i);
-    if (nvis <= 0) return;
     const int g = G.g, d = G.d;
+    const float sc = gamma * rsqrtf((float)d);
+    float dq[kMaxG][DL];
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h)
+#pragma unroll
+        for (int k = 0; k < DL; ++k) dq[h][k] = 0.f;
+    if (nvis <= 0) {  // nothing routed: the Stage-2 part alone
+        store_dq<T, DL>(dQacc, dQ, G, b, i, r, lane, dq, sc);
+        return;
+    }
     const uint32_t *mrow = mask + (((size_t)b * G.nq + i) * G.hkv + r) * G.words;
     const int wv = (nvis + 31) / 32;
     // pass 1: mean of G over the routed set
@@ -377,22 +417,23 @@ __global__ void __launch_bounds__(128) bwd_route_kernel(TView Q, const float *__
     }
     sG = warp_sum(sG);
     nR = warp_sum_i(nR);
-    if (nR == 0) return;
+    if (nR == 0) {
+        store_dq<T, DL>(dQacc, dQ, G, b, i, r, lane, dq, sc);
+        return;
+    }
     const float meanG = sG / (float)nR;
+    if (lane == 0) meanG_out[w] = meanG;
     const float inv_sigma = 1.f / sigma;
     const float xs = (alpha - 1.f) * gamma * rsqrtf((float)d);  // x = xs <q, kbar>
     const float kexp = 1.f / (alpha - 1.f), uexp = 2.f - alpha;
-    float q[kMaxG][DL], dq[kMaxG][DL], th[kMaxG], su[kMaxG], sud[kMaxG];
+    float q[kMaxG][DL], th[kMaxG], su[kMaxG], sud[kMaxG];
 #pragma unroll
     for (int h = 0; h < kMaxG; ++h) {
         const bool on = h < g;
         const size_t rid = ((size_t)b * G.nq + i) * G.hq + r * g + (on ? h : 0);
         const T *qp = reinterpret_cast<const T *>(Q.p) + b * Q.s0 + i * Q.s1 + (int64_t)(r * g + (on ? h : 0)) * Q.s2;
 #pragma unroll
-        for (int k = 0; k < DL; ++k) {
-            q[h][k] = on ? to_f<T>(qp[lane + 32 * k]) : 0.f;
-            dq[h][k] = 0.f;
-        }
+        for (int k = 0; k < DL; ++k) q[h][k] = on ? to_f<T>(qp[lane + 32 * k]) : 0.f;
         th[h] = on ? tau[rid] : INFINITY;
         su[h] = 0.f;
         sud[h] = 0.f;
@@ -409,54 +450,106 @@ __global__ void __launch_bounds__(128) bwd_route_kernel(TView Q, const float *__
                 const size_t li = logw_index(G, b, r, i, c);
                 const float dlw = (Gd[li] - meanG) * inv_sigma;
                 const float lw = logw[li];
-                float kv[DL], dkb[DL];
+                float kv[DL];
                 const float *kp = kb_row + (size_t)c * G.hkv * d;
 #pragma unroll
-                for (int k = 0; k < DL; ++k) {
-                    kv[k] = kp[lane + 32 * k];
-                    dkb[k] = 0.f;
-                }
+                for (int k = 0; k < DL; ++k) kv[k] = kp[lane + 32 * k];
 #pragma unroll
                 for (int h = 0; h < kMaxG; ++h) {
                     if (h >= g) break;
                     float dot = 0.f;
 #pragma unroll
                     for (int k = 0; k < DL; ++k) dot = fmaf(q[h][k], kv[k], dot);
-                    const float x = xs * warp_sum(dot);
-                    if (!(x > th[h])) continue;  // outside this head's own support: u = 0
-                    const float lp = kexp * __logf(x - th[h]);       // log p
-                    const float u = __expf(uexp * lp);                 // p^(2 - alpha)
-                    const float ud = __expf(uexp * lp - lw) * dlw / (float)g;  // u dp, dp = dw / g = dlogw / (g w)
+                    float u, ud;
+                    if (!route_terms(xs * warp_sum(dot), th[h], kexp, uexp, lw, dlw, g, u, ud)) continue;
                     if (pass == 0) {
                         su[h] += u;
                         sud[h] += ud;
                     } else {
                         const float ds = ud - u * (sud[h] / su[h]);
 #pragma unroll
-                        for (int k = 0; k < DL; ++k) {
-                            dq[h][k] = fmaf(ds, kv[k], dq[h][k]);
-                            dkb[k] = fmaf(ds, q[h][k], dkb[k]);
-                        }
+                        for (int k = 0; k < DL; ++k) dq[h][k] = fmaf(ds, kv[k], dq[h][k]);
                     }
-                }
-                if (pass == 1) {
-                    const float sc = gamma * rsqrtf((float)d);
-                    float *dst = dKbar + (((size_t)b * G.n_chunks + c) * G.hkv + r) * d;
-#pragma unroll
-                    for (int k = 0; k < DL; ++k)
-                        if (dkb[k] != 0.f) atomicAdd(dst + lane + 32 * k, sc * dkb[k]);
                 }
             }
         }
+        if (pass == 0 && lane == 0) {
+#pragma unroll
+            for (int h = 0; h < kMaxG; ++h)
+                if (h < g) rho_out[((size_t)b * G.nq + i) * G.hq + r * g + h] = su[h] > 0.f ? sud[h] / su[h] : 0.f;
+        }
     }
+    store_dq<T, DL>(dQacc, dQ, G, b, i, r, lane, dq, sc);
+}
+
+// The summaries' gradient, chunk by chunk: one CTA (4 warps) per (routing chunk, kv head,
+// batch) walks the (tile, entry) pairs that list the chunk (the transposed lists) and the
+// tile rows that route it; each (row, head) adds ds q (ds from the row's mean G and
+// <u, dp> / sum u kept by bwd_route_kernel).  Pairs go to the warps round robin and the
+// warps' sums are added in a fixed order: deterministic, no atomics.
+template <typename T, int DL>
+__global__ void __launch_bounds__(128) bwd_kbar_grad_kernel(TView Q, const float *__restrict__ kbar, Geom G,
+                                                            ListsView L, float alpha, float gamma, float sigma,
+                                                            const float *__restrict__ tau,
+                                                            const float *__restrict__ logw,
+                                                            const float *__restrict__ Gd,
+                                                            const float *__restrict__ meanG,
+                                                            const float *__restrict__ rho,
+                                                            const int32_t *__restrict__ ref_off,
+                                                            const int32_t *__restrict__ ref_cnt,
+                                                            const int2 *__restrict__ refs, float *__restrict__ dKbar) {
+    __shared__ float part[4][DL * 32];
+    const int c = blockIdx.x, r = blockIdx.y;
+    const int64_t b = blockIdx.z;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int g = G.g, d = G.d, TR = L.tile_rows;
+    const size_t bh = (size_t)b * G.hkv + r;
+    const int nref = ref_cnt[bh * G.n_blk + c];
+    const int2 *rl = refs + bh * (size_t)L.n_tiles * G.n_blk + ref_off[bh * G.n_blk + c];
+    const float inv_sigma = 1.f / sigma;
+    const float xs = (alpha - 1.f) * gamma * rsqrtf((float)d);
+    const float kexp = 1.f / (alpha - 1.f), uexp = 2.f - alpha;
+    float kv[DL], acc[DL];
+    const float *kp = kbar + (((size_t)b * G.kbar_cap + c) * G.hkv + r) * d;
+#pragma unroll
+    for (int k = 0; k < DL; ++k) {
+        kv[k] = kp[lane + 32 * k];
+        acc[k] = 0.f;
+    }
+    for (int idx = warp; idx < nref * TR; idx += 4) {
+        const int64_t t = rl[idx / TR].x;
+        const int e = rl[idx / TR].y, pos = idx % TR;
+        const size_t tile_lin = bh * L.n_tiles + t;
+        const int64_t i = tile_row(L, G, tile_lin, t, pos);
+        if (i < 0) continue;
+        const float bv = L.bias[tile_lin * (size_t)L.cap * TR + (size_t)e * TR + pos];
+        if (!(bv > -INFINITY) || c >= row_nvis(G, i)) continue;  // the row does not route this chunk
+        const size_t li = logw_index(G, b, r, i, c);
+        const float dlw = (Gd[li] - meanG[((size_t)b * G.nq + i) * G.hkv + r]) * inv_sigma;
+        const float lw = logw[li];
+        for (int h = 0; h < g; ++h) {
+            const size_t rid = ((size_t)b * G.nq + i) * G.hq + r * g + h;
+            const T *qp = reinterpret_cast<const T *>(Q.p) + b * Q.s0 + i * Q.s1 + (int64_t)(r * g + h) * Q.s2;
+            float qv[DL], dot = 0.f;
+#pragma unroll
+            for (int k = 0; k < DL; ++k) {
+                qv[k] = to_f<T>(qp[lane + 32 * k]);
+                dot = fmaf(qv[k], kv[k], dot);
+            }
+            float u, ud;
+            if (!route_terms(xs * warp_sum(dot), tau[rid], kexp, uexp, lw, dlw, g, u, ud)) continue;
+            const float ds = ud - u * rho[rid];
+#pragma unroll
+            for (int k = 0; k < DL; ++k) acc[k] = fmaf(ds, qv[k], acc[k]);
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < DL; ++k) part[warp][lane + 32 * k] = acc[k];
+    __syncthreads();
     const float sc = gamma * rsqrtf((float)d);
-#pragma unroll
-    for (int h = 0; h < kMaxG; ++h) {
-        if (h >= g) break;
-        float *dst = dQacc + (((size_t)b * G.nq + i) * G.hq + r * g + h) * d;
-#pragma unroll
-        for (int k = 0; k < DL; ++k) dst[lane + 32 * k] += sc * dq[h][k];
-    }
+    for (int x = threadIdx.x; x < d; x += 128)
+        dKbar[(((size_t)b * G.n_chunks + c) * G.hkv + r) * d + x] =
+            sc * (((part[0][x] + part[1][x]) + part[2][x]) + part[3][x]);
 }
 
 template <typename T>
@@ -493,19 +586,16 @@ cudaError_t launch_bwd_t(const BwdArgs &a, cudaStream_t st) {
             a.Q, a.K, a.V, a.dO, G, L, a.lse, a.Drow, a.dQacc, a.Gd);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    // the routing chain (prior, group average, entmax, Stage-1 scores)
+    // the routing chain (prior, group average, entmax, Stage-1 scores) into dQ
     if (G.n_chunks > 0) {
-        if ((e = cudaMemsetAsync(a.dKbar, 0, (size_t)G.b * G.n_chunks * G.hkv * G.d * sizeof(float), st)) !=
-            cudaSuccess)
-            return e;
         const int64_t warps = G.b * G.nq * G.hkv;
         const unsigned blocks = (unsigned)((warps * 32 + 127) / 128);
         if (G.d == 128)
             bwd_route_kernel<T, 4><<<blocks, 128, 0, st>>>(a.Q, a.kbar, G, a.alpha, a.gamma, a.sigma, a.tau, a.mask,
-                                                           a.logw, a.Gd, a.dQacc, a.dKbar);
+                                                           a.logw, a.Gd, a.dQacc, a.dQ, a.meanG, a.rho);
         else
             bwd_route_kernel<T, 2><<<blocks, 128, 0, st>>>(a.Q, a.kbar, G, a.alpha, a.gamma, a.sigma, a.tau, a.mask,
-                                                           a.logw, a.Gd, a.dQacc, a.dKbar);
+                                                           a.logw, a.Gd, a.dQacc, a.dQ, a.meanG, a.rho);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     // transposed lists
@@ -518,6 +608,19 @@ cudaError_t launch_bwd_t(const BwdArgs &a, cudaStream_t st) {
     refs_build_kernel<<<dim3((unsigned)G.hkv, (unsigned)G.b), 1024, 0, st>>>(G, L.n_tiles, a.bitmap, a.E, tw,
                                                                             a.ref_off, a.ref_cnt, a.refs);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // the routing chain into the chunk summaries (deterministic, chunk by chunk)
+    if (G.n_chunks > 0) {
+        const dim3 grid((unsigned)G.n_chunks, (unsigned)G.hkv, (unsigned)G.b);
+        if (G.d == 128)
+            bwd_kbar_grad_kernel<T, 4><<<grid, 128, 0, st>>>(a.Q, a.kbar, G, L, a.alpha, a.gamma, a.sigma, a.tau,
+                                                             a.logw, a.Gd, a.meanG, a.rho, a.ref_off, a.ref_cnt,
+                                                             a.refs, a.dKbar);
+        else
+            bwd_kbar_grad_kernel<T, 2><<<grid, 128, 0, st>>>(a.Q, a.kbar, G, L, a.alpha, a.gamma, a.sigma, a.tau,
+                                                             a.logw, a.Gd, a.meanG, a.rho, a.ref_off, a.ref_cnt,
+                                                             a.refs, a.dKbar);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     // Stage 2, key side: dK (with the pooling share), dV
     if (a.use_tc) {
         if ((e = launch_attn_bwd_tc_dkdv(a, st)) != cudaSuccess) return e;
@@ -534,8 +637,10 @@ cudaError_t launch_bwd_t(const BwdArgs &a, cudaStream_t st) {
             a.Q, a.K, a.V, a.dO, a.dK, a.dV, G, L, a.lse, a.Drow, a.ref_off, a.ref_cnt, a.refs, a.dKbar);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    const int64_t n = rows * G.d;
-    bwd_dq_finish_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a.dQacc, a.dQ, G);
+    if (G.n_chunks == 0) {  // no routing at all: dQ is the Stage-2 part
+        const int64_t n = rows * G.d;
+        bwd_dq_finish_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a.dQacc, a.dQ, G);
+    }
     return cudaGetLastError();
 }
 

@@ -27,7 +27,25 @@ struct Geom {
                     // n_chunks, or a persistent cache's capacity)
     int ct_cap;     // 128-chunk tiles per (batch, kv head) in the split-summary buffer
     int local;      // chunks of the causal local window: 1 (the query's own) or 2 (and the one before)
+    // Decoding from a preallocated cache: nk above is the capacity, the number of valid keys
+    // is read from *nk_dev when a kernel runs (null: nk is the length), and *chunks_dev is
+    // the number of chunks a summary cache has pooled (device-side bookkeeping).
+    const int64_t *nk_dev;
+    const int *chunks_dev;
 };
+
+// The geometry a kernel works with: with a device-resident key length, nk is read from
+// device memory (clamped to the capacity the buffers were sized for) and the chunk counts
+// that follow from it are recomputed; every kernel of a step derives the same values.
+__device__ __forceinline__ void geom_live(Geom &G) {
+    if (!G.nk_dev) return;
+    int64_t nk = *G.nk_dev;
+    nk = nk < 0 ? 0 : (nk > G.nk ? G.nk : nk);
+    G.nk = nk;
+    G.n_chunks = (int)(G.causal ? nk / G.B : (nk + G.B - 1) / G.B);
+    G.n_blk = (int)((nk + G.B - 1) / G.B);
+    G.words = (G.n_chunks + 31) / 32;
+}
 
 // Strided 4-D tensor view passed by value to kernels (element strides).
 struct TView {
@@ -71,6 +89,33 @@ __host__ __device__ inline int row_nvis(const Geom &G, int64_t i) {
     if (!G.causal) return G.n_chunks;
     const int c = first_local(G, i);
     return c < G.n_chunks ? c : G.n_chunks;
+}
+
+// ---------------------------------------------------------------------------
+// Order of the query-tile CTAs of a Stage-2 launch.  The (batch, kv head) pairs are
+// taken in groups whose K and V fit in half of the 126 MB L2 together; within a group
+// the CTAs go longest tile (latest, causal) first across the group's pairs, so that
+// the long tiles do not gather at the end of the launch, and the groups follow one
+// another, so that the CTAs in flight read K and V that stay in L2.
+// ---------------------------------------------------------------------------
+struct TileOrder {
+    int64_t t;   // tile index
+    int64_t bh;  // batch * hkv + kv head
+};
+inline int heads_per_group(const Geom &G) {
+    const double per_head = (double)G.nk * G.d * 2.0 * 2.0;  // K and V, bf16
+    int hg = 1;
+    while (hg * 2 <= G.b * G.hkv && (double)(hg * 2) * per_head <= 63.0 * (1 << 20)) hg *= 2;
+    return hg;
+}
+__host__ __device__ inline TileOrder tile_order(int64_t cta, int64_t n_tiles, int64_t bh_total, int hg) {
+    const int64_t per_group = (int64_t)hg * n_tiles;
+    const int64_t gi = cta / per_group, local = cta % per_group;
+    const int64_t hsz = bh_total - gi * hg < hg ? bh_total - gi * hg : hg;  // the last group may be smaller
+    TileOrder o;
+    o.t = n_tiles - 1 - local / hsz;
+    o.bh = gi * hg + local % hsz;
+    return o;
 }
 
 // ---------------------------------------------------------------------------

@@ -13,6 +13,15 @@ cudaError_t launch_pool_keys(const TView &K, dash_dtype_t dt, const Geom &G, flo
 cudaError_t launch_pool_keys_q(const TView &K, dash_dtype_t dt, const TView &Qbar, dash_dtype_t qdt, const Geom &G,
                                float *kbar, cudaStream_t st, int c0 = 0, int c1 = -1);
 
+// Chunks a decoding step may complete since the previous one when the summary cache
+// catches up on the device (a device-resident key length).
+constexpr int kMaxNewChunks = 16;
+// pool the chunks completed since the cache's device count (G.nk_dev, G.chunks_dev set;
+// G.kbar_cap / G.ct_cap the cache's), rebuild their split tiles and advance the count
+cudaError_t launch_cache_catch_up(const TView &K, dash_dtype_t dt, const Geom &G, float *kbar, uint8_t *split,
+                                  cudaStream_t st);
+cudaError_t launch_set_int(int *dst, int v, cudaStream_t st);
+
 // Stage 1 (block_select.cu)
 struct SelectOut {
     float *tau;        // [b][nq][hq] or null
@@ -74,6 +83,8 @@ struct BwdArgs {
     float *Gd;                         // G per (row, routed chunk), logw_index layout
     float *dQacc;                      // [b][nq][hq][d] fp32
     float *dKbar;                      // [b][n_chunks][hkv][d] fp32
+    float *meanG;                      // [b][nq][hkv] mean G over the row's routed chunks
+    float *rho;                        // [b][nq][hq] <u, dp> / sum u of the row's entmax
     uint32_t *bitmap;                  // [b][hkv][n_blk][ceil(n_tiles/32)] tiles attending each key block
     int32_t *E;                        // [b][hkv][n_blk][n_tiles] entry index of the block in the tile's list
     int32_t *ref_off, *ref_cnt;        // [b][hkv][n_blk] the block's (tile, entry) pairs

@@ -14,10 +14,18 @@
 
 namespace dash {
 
+// With a device-resident length (G.chunks_dev set), chunk c0 is counted from the first
+// chunk the cache has not pooled and chunks that are not complete yet are skipped.
 template <typename T>
-__global__ void __launch_bounds__(256) pool_keys_kernel(TView K, Geom G, float *__restrict__ kbar, int c0) {
+__global__ void __launch_bounds__(256) pool_keys_kernel(TView K, Geom G0, float *__restrict__ kbar, int c0) {
     constexpr int VEC = 16 / sizeof(T);  // elements per 16-byte load
-    const int c = c0 + (int)blockIdx.x;
+    Geom G = G0;
+    geom_live(G);
+    int c = c0 + (int)blockIdx.x;
+    if (G.chunks_dev) {
+        c += *G.chunks_dev;
+        if (c >= G.n_chunks) return;
+    }
     const int64_t b = blockIdx.y;
     const int ncol = G.hkv * G.d / VEC;  // 16-byte column groups of one token row
     const int rs = ncol >= 256 ? 1 : 256 / ncol;
@@ -84,6 +92,34 @@ cudaError_t launch_pool_keys(const TView &K, dash_dtype_t dt, const Geom &G, flo
         pool_keys_kernel<__nv_bfloat16><<<grid, 256, smem, st>>>(K, G, kbar, c0);
     else
         pool_keys_kernel<float><<<grid, 256, smem, st>>>(K, G, kbar, c0);
+    return cudaGetLastError();
+}
+
+// After a device-range pooling step: the cache has pooled the chunks up to the live
+// count, or kMaxNewChunks more than before, whichever is fewer.
+__global__ void cache_advance_kernel(Geom G0, int *done, int max_new) {
+    Geom G = G0;
+    geom_live(G);
+    const int d = *done;
+    const int n = min(G.n_chunks, d + max_new);
+    if (n > d) *done = n;
+}
+
+__global__ void set_int_kernel(int *dst, int v) { *dst = v; }
+
+cudaError_t launch_set_int(int *dst, int v, cudaStream_t st) {
+    set_int_kernel<<<1, 1, 0, st>>>(dst, v);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_cache_catch_up(const TView &K, dash_dtype_t dt, const Geom &G, float *kbar, uint8_t *split,
+                                  cudaStream_t st) {
+    if (!G.nk_dev || !G.chunks_dev || G.b == 0) return cudaErrorInvalidValue;
+    cudaError_t e = launch_pool_keys(K, dt, G, kbar, st, 0, kMaxNewChunks);
+    if (e != cudaSuccess) return e;
+    // the new chunks fall in at most two 128-chunk tiles of the split form
+    if ((e = launch_kbar_split(kbar, G, split, 0, kMaxNewChunks / 128 + 2, st)) != cudaSuccess) return e;
+    cache_advance_kernel<<<1, 1, 0, st>>>(G, const_cast<int *>(G.chunks_dev), kMaxNewChunks);
     return cudaGetLastError();
 }
 

@@ -107,11 +107,22 @@ struct TSmem {
 // hi = bf16(k̄), lo = bf16(k̄ - hi), each laid out exactly as the logits MMA reads it
 // (K-major, 64-column regions of 128 rows x 128 bytes, 128-byte swizzle), so a CTA
 // fetches a chunk tile with two bulk copies.  Chunks past n_chunks are zero.
+// With a device-resident length (G.chunks_dev set) the tiles are taken from the first
+// tile holding a chunk the cache has not pooled yet, and only tiles with new chunks run.
 template <int D>
-__global__ void __launch_bounds__(256) kbar_split_kernel(const float *__restrict__ kbar, Geom G,
+__global__ void __launch_bounds__(256) kbar_split_kernel(const float *__restrict__ kbar, Geom G0,
                                                          uint8_t *__restrict__ split, int ct0) {
     constexpr int kDh = D / 64, kRegion = 128 * 128;
-    const int ct = ct0 + (int)blockIdx.x, r = blockIdx.y;
+    Geom G = G0;
+    geom_live(G);
+    int ct = ct0 + (int)blockIdx.x;
+    if (G.chunks_dev) {
+        const int done = *G.chunks_dev;
+        if (done >= G.n_chunks) return;  // nothing new since the last step
+        ct += done / 128;
+        if (ct * 128 >= G.n_chunks) return;
+    }
+    const int r = blockIdx.y;
     const int64_t b = blockIdx.z;
     uint8_t *dst = split + ((((size_t)b * G.hkv + r) * G.ct_cap + ct) * 2) * (size_t)(kDh * kRegion);
     for (int u = threadIdx.x; u < 128 * (D / 8); u += 256) {
@@ -170,9 +181,11 @@ __device__ __forceinline__ void pair_reduce(float *xch, int parity, int slot, in
 
 template <int D, int KINT, int LG, int CP, int NSB>
 __global__ void __launch_bounds__(128 * CP, 4 / CP) select_tile_kernel(const __grid_constant__ CUtensorMap tmQ,
-                                                                      const uint8_t *__restrict__ ksplit, Geom G,
+                                                                      const uint8_t *__restrict__ ksplit, Geom G0,
                                                                       TileP P, TileOut out, uint32_t ncols) {
     using S = TSmem<D, LG, CP, NSB>;
+    Geom G = G0;
+    geom_live(G);
     constexpr int kT = 128 * CP;       // 4 TMEM lane quadrants x CP column parts
     constexpr int kQB = 4 / CP;        // 32-column blocks per chunk tile and thread
     constexpr int kNP = S::kNP;
@@ -596,6 +609,7 @@ size_t select_tile_workspace(const Geom &G) {
 
 cudaError_t launch_kbar_split(const float *kbar, const Geom &G, uint8_t *split, int ct0, int ct1, cudaStream_t st) {
     if (ct1 <= ct0 || G.b == 0) return cudaSuccess;
+    if (G.chunks_dev) ct1 = min(ct1, G.ct_cap);  // device range: tiles past the capacity never run
     if (ct1 > G.ct_cap) return cudaErrorInvalidValue;
     dim3 sg((unsigned)(ct1 - ct0), (unsigned)G.hkv, (unsigned)G.b);
     if (G.d == 128) kbar_split_kernel<128><<<sg, 256, 0, st>>>(kbar, G, split, ct0);

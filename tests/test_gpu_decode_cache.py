@@ -129,3 +129,61 @@ def test_decode_step_replays_from_a_cuda_graph():
         assert torch.equal(out, direct)
     del graph
     cache.close()
+
+
+def test_one_graph_serves_growing_lengths():
+    """Decoding from a preallocated KV cache with a device-resident length (opts nk_dev):
+    one captured step is replayed while the sequences grow one token per step across
+    chunk boundaries (the call itself pools each completed chunk on the device).  Every
+    replay equals, bit for bit, the plain forward on the keys written so far."""
+    b, hq, hkv, d, B, cap = 2, 16, 4, 128, 64, 2048
+    k, v = _kv(b, cap, hkv, d, seed=11)
+    nk0 = 1000
+    cache = dash.SummaryCache(b, cap, hkv, d, B).update(k[:, :nk0])
+    nk_dev = torch.tensor([nk0], dtype=torch.int64, device="cuda")
+    gen = torch.Generator().manual_seed(12)
+    q = torch.empty(b, 1, hq, d, dtype=torch.bfloat16, device="cuda")
+    q.copy_((3 * torch.randn(b, 1, hq, d, generator=gen)).to(torch.bfloat16))
+    out = torch.empty_like(q)
+    ws = torch.empty(dash.dash_workspace_bytes(b, 1, cap, hq, hkv, d, B), dtype=torch.uint8, device="cuda")
+    opts = dict(summary_cache=cache, workspace=ws, nk_dev=nk_dev)
+    dash.dash_attn_fwd(q, k, v, out, B, 1.5, True, hq // hkv, **opts)  # warm-up outside the capture
+    assert dash.dash_sync_status() == 0
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            dash.dash_attn_fwd(q, k, v, out, B, 1.5, True, hq // hkv, stream=side, **opts)
+    torch.cuda.current_stream().wait_stream(side)
+    ref = torch.empty_like(q)
+    # one token per step, then jumps of at most 16 chunks (what one call catches up on)
+    for nk in list(range(nk0 + 1, nk0 + 90)) + [1600, 1601, 1664, 2048]:
+        nk_dev.fill_(nk)
+        q.copy_((3 * torch.randn(b, 1, hq, d, generator=gen)).to(torch.bfloat16))
+        graph.replay()
+        torch.cuda.synchronize()
+        dash.dash_attn_fwd(q, k[:, :nk], v[:, :nk], ref, B, 1.5, True, hq // hkv)
+        assert dash.dash_sync_status() == 0
+        assert torch.equal(out, ref), nk
+    del graph
+    cache.close()
+
+
+def test_device_length_misuse_is_rejected():
+    b, hq, hkv, d, B = 1, 8, 2, 128, 64
+    k, v = _kv(b, 1024, hkv, d, seed=13)
+    q = torch.randn(b, 1, hq, d, device="cuda").to(torch.bfloat16)
+    out = torch.empty_like(q)
+    nk_dev = torch.tensor([700], dtype=torch.int64, device="cuda")
+    with pytest.raises(dash.DashError):  # a device length needs a summary cache
+        dash.dash_attn_fwd(q, k, v, out, B, 1.5, True, 4, nk_dev=nk_dev)
+    small = dash.SummaryCache(b, 512, hkv, d, B)
+    with pytest.raises(dash.DashError):  # the keys' capacity exceeds the cache's
+        dash.dash_attn_fwd(q, k, v, out, B, 1.5, True, 4, nk_dev=nk_dev, summary_cache=small)
+    small.close()
+    cache = dash.SummaryCache(b, 1024, hkv, d, B)
+    with pytest.raises(dash.DashError):  # prefill rows: not the decoding path
+        qq = torch.randn(b, 64, hq, d, device="cuda").to(torch.bfloat16)
+        dash.dash_attn_fwd(qq, k, v, torch.empty_like(qq), B, 1.5, True, 4, nk_dev=nk_dev, summary_cache=cache)
+    cache.close()
