@@ -48,16 +48,14 @@ import synthetic  # noqa: E402
 METRIC = "DashAttention fwd ms & TFLOP/s (prefill) / GB/s (decode), % of B200 roofline"
 L2_FLUSH_BYTES = 256 << 20
 
-# DRAM bytes (read + write) per launch of the dominant kernel, each from one ncu capture
-# (dram__bytes_read.sum + dram__bytes_write.sum) of the current kernel: the Stage-2
-# tensor-core kernel on the prefill workloads; the decode kernel captured at batch 4
-# and scaled by the (batch, kv head) units to batch 16.  A workload without a capture
-# of the current kernel reports null.
+# DRAM bytes (read + write) per launch of the dominant kernel, each from one full-size ncu
+# capture (dram__bytes_read.sum + dram__bytes_write.sum, one pass) of the current kernel:
+# the Stage-2 tensor-core kernel at 128K and 8K, the split-KV decode kernel at batch 16.  A
+# workload without a capture of the current kernel reports null.
 TRAFFIC_BYTES = {
-    ("prefill128k", 1): 6.1389e10,
-    ("prefill8k", 1): 1.4348e8,
-    ("decode", 16): 1.6565e9,
-    ("decode", 4): 4.1412e8,
+    ("prefill128k", 1): 3.2890e9,
+    ("prefill8k", 1): 1.4396e8,
+    ("decode", 16): 1.6258e9,
 }
 
 
@@ -499,14 +497,18 @@ def oracle_sample(w, alpha, sigma, q, k, v, budget_s=15.0, threads=0, batch_rows
     cores = threads or (os.cpu_count() or 1)
     oracle.set_threads(cores)
     rng = np.random.default_rng(seed)
-    b = 0
-    K = k[b].float().cpu().numpy()
-    V = v[b].float().cpu().numpy()
     # about one second of oracle work per batch: rows cost ~ their visible keys x heads
     per = batch_rows or max(1, min(256, int(cores * 2e9 / max(w.hq * w.nk * w.d * 4, 1))))
     done = []
     el = 0.0
+    b = 0
+    K = V = None
     while True:
+        # decoding (a few rows per sequence): every row of one sequence per round, sequence
+        # after sequence; prefill: random rows of the first sequence
+        if K is None or w.nq <= 16:
+            K = k[b].float().cpu().numpy()
+            V = v[b].float().cpu().numpy()
         rows = (np.arange(w.nq) if w.nq <= 16 else
                 np.sort(rng.choice(np.arange(w.nq), min(w.nq, per), replace=False)))
         Qr = q[b, torch.from_numpy(rows).to(q.device)].float().cpu().numpy()
@@ -514,7 +516,9 @@ def oracle_sample(w, alpha, sigma, q, k, v, budget_s=15.0, threads=0, batch_rows
         res = oracle.fwd_rows(Qr, rows, w.nq, K, V, w.block, alpha, sigma=sigma, want=("out", "routed"))
         el += time.perf_counter() - t0
         done.append((rows, res["routed"]))
-        if el > budget_s or (max_rows and sum(len(r) for r, _ in done) >= max_rows) or w.nq <= 16:
+        if w.nq <= 16:
+            b += 1
+        if el > budget_s or (max_rows and sum(len(r) for r, _ in done) >= max_rows) or b >= w.batch:
             break
     f2 = 0.0
     y = 0.0
@@ -551,7 +555,8 @@ def run_reference(args, device):
     secs = sum(per_step)
     unit = "GB/s" if decode else "TFLOP/s"
     value = (byts / secs / 1e9) if decode else (flops / secs / 1e12)
-    sample = f"{rows} query rows x all heads of batch 0 over {args.steps} steps (fp64 oracle, dense masked Stage 2)"
+    sample = (f"{rows} query rows x all heads ({'the new rows of successive sequences' if w.nq <= 16 else 'batch 0'}) "
+              f"over {args.steps} steps (fp64 oracle, dense masked Stage 2)")
     return {
         "metric": METRIC, "impl": "reference", "value": value, "unit": unit, "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * secs / max(args.steps, 1), "higher_is_better": True,
@@ -628,8 +633,10 @@ def main():
                 # the same oracle on one thread, on a smaller sample
                 n1, el1, f21, y1, _ = oracle_sample(w, alpha, sigma, q, k, v, budget_s=6.0, threads=1, seed=1)
                 val1 = (y1 / el1 / 1e9) if decode else (f21 / el1 / 1e12)
+                what = (f"the new rows of {n // max(w.nq, 1)} of the {w.batch} sequences" if w.nq <= 16 else
+                        f"{n} random query rows of batch 0")
                 res["cpu_baseline"] = {"value": val, "unit": res["unit"], "cores": cores, "kind": "oracle",
-                                       "sample": f"{n} random query rows x all heads of batch 0, {el:.1f} s "
+                                       "sample": f"{what} x all heads, {el:.1f} s "
                                                  f"(fp64 oracle, dense masked Stage 2)",
                                        "single_thread": {"value": val1, "unit": res["unit"], "cores": 1,
                                                          "sample": f"{n1} random query rows x all heads, "

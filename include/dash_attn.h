@@ -280,9 +280,13 @@ DASH_API int dash_lists_geometry(int64_t batch, int64_t nq, int64_t nk, int hkv,
                                  int64_t *n_tiles, int32_t *cap, int32_t *tile_rows, size_t *count_bytes,
                                  size_t *ids_bytes, size_t *bias_bytes, size_t *rows_bytes);
 
-/* Device workspace dash_attn_fwd_ex needs for a problem (bytes): an upper bound over
- * every option (it counts the pooled-key area and the split-KV decode partials even
- * where a summary cache or a prefill shape makes them unnecessary). */
+/* Device workspace dash_attn_fwd_ex takes for a problem with the library-managed
+ * workspace (bytes): an upper bound over the options (it counts the pooled-key area even
+ * where a summary cache makes it unnecessary).  A prefill whose Stage-1 state and work
+ * lists would exceed 1 GB runs its query rows in slices (multiples of 1024 rows) that fit
+ * 1 GB, so the figure stays near 1 GB at any length; with a caller workspace the slices
+ * are sized to that workspace instead (at least 1024 rows; DASH_ERR_WORKSPACE when even
+ * those do not fit). */
 DASH_API size_t dash_workspace_bytes(int64_t batch, int64_t nq, int64_t nk, int hq, int hkv, int d,
                                      int block_size, int causal);
 
@@ -311,10 +315,9 @@ DASH_API int dash_release(void);
  * to this entry point: it is a deployment variant of dash_attn_fwd_ex.
  *   Arguments and result as dash_attn_fwd_ex; opts may be NULL, and
  *   opts->workspace must be NULL (DASH_ERR_INVALID_ARG otherwise).
- *   A problem whose forward pass needs more scratch than DASH_NOALLOC_SCRATCH_BYTES
- *   (the workspace dash_attn_fwd_ex would take with the same options, at most
- *   dash_workspace_bytes()) is rejected with DASH_ERR_WORKSPACE before anything is
- *   launched.
+ *   A long prefill runs its query rows in slices that fit the area; a problem whose
+ *   smallest slice (1024 rows) still needs more scratch than DASH_NOALLOC_SCRATCH_BYTES
+ *   is rejected with DASH_ERR_WORKSPACE before anything is launched.
  *   The first call on a device (with that device current) looks up the array's
  *   device address with cudaGetSymbolAddress; make that first call before any
  *   stream capture.  The address is kept for the life of the device's primary

@@ -5,6 +5,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 #include <string>
 
@@ -106,6 +107,8 @@ int make_geom(const dash_tensor_t *q, const dash_tensor_t *k, int B, int causal,
     G->local = 1;
     G->nk_dev = nullptr;
     G->chunks_dev = nullptr;
+    G->pos0 = nk - nq;
+    G->nq_lse = nq;
     return DASH_OK;
 }
 
@@ -162,6 +165,36 @@ WsLayout ws_layout(const Geom &G, bool need_kbar, bool need_lists, bool need_dec
     L.split = select_tile_supported(G, DASH_BF16) ? take(select_tile_workspace(G)) : 0;
     L.total = off;
     return L;
+}
+
+// Query rows in slices.  A prefill's Stage-1 state and work lists grow with nq x n_chunks
+// (4.3 GB each for the log-w array and the bias table at 128K), so the rows are processed
+// in slices of a multiple of 1024 (whole regrouping windows) that fit a workspace budget:
+// Stage 1 and Stage 2 run slice after slice on one per-slice workspace (Stage 0 once).
+constexpr size_t kSliceBudget = 1000000000;  // the library-managed workspace's budget (1 GB)
+constexpr int64_t kSliceQuantum = 1024;
+
+Geom slice_geom(const Geom &G, int64_t row0, int64_t rows) {
+    Geom S = G;
+    S.nq = rows;
+    S.n_tiles = (rows + G.tile_rows - 1) / G.tile_rows;
+    S.pos0 = G.pos0 + row0;
+    return S;
+}
+
+// Rows per slice: every row when the whole layout fits the budget (or the path is
+// decoding), else the largest multiple of kSliceQuantum whose layout fits (at least one
+// quantum: a budget below that leaves the workspace check to refuse).
+int64_t slice_rows(const Geom &G, bool need_kbar, bool dec, size_t budget) {
+    if (dec || G.nq <= kSliceQuantum || ws_layout(G, need_kbar, true, dec).total <= budget) return G.nq;
+    int64_t lo = 1, hi = (G.nq - 1) / kSliceQuantum;  // candidate slices of lo..hi quanta
+    if (ws_layout(slice_geom(G, 0, kSliceQuantum), need_kbar, true, dec).total > budget) return kSliceQuantum;
+    while (lo < hi) {
+        const int64_t mid = (lo + hi + 1) / 2;
+        if (ws_layout(slice_geom(G, 0, mid * kSliceQuantum), need_kbar, true, dec).total <= budget) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo * kSliceQuantum;
 }
 
 // Library-managed workspace, one cached allocation per device.
@@ -341,14 +374,16 @@ int validate_qkvo(const dash_tensor_t *q, const dash_tensor_t *k, const dash_ten
 // the workspace layout those choices need.
 struct FwdPlan {
     Geom G;
-    WsLayout WL;
+    WsLayout WL;  // the layout of one slice of rows (of every row when not sliced)
     TView qv;
     const dash_summary_cache *sc;
     bool need_kbar, dec;
+    int64_t slice;  // query rows per slice
 };
 
 int plan_fwd(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v, const dash_tensor_t *out,
-             int block_size, float alpha, int causal, int gqa_groups, const dash_opts_t &o, FwdPlan *P) {
+             int block_size, float alpha, int causal, int gqa_groups, const dash_opts_t &o, FwdPlan *P,
+             size_t budget) {
     int rc;
     if ((rc = check_opts(o))) return rc;
     if ((rc = validate_qkvo(q, k, v, out))) return rc;
@@ -372,9 +407,15 @@ int plan_fwd(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t
                                               "tensor-core Stage 1, the one-block local window)");
         G.nk_dev = o.nk_dev;
     }
-    P->WL = (G.b == 0 || G.nq == 0) ? WsLayout{} : ws_layout(G, P->need_kbar, true, P->dec);
+    P->slice = slice_rows(G, P->need_kbar, P->dec, budget);
+    P->WL = (G.b == 0 || G.nq == 0) ? WsLayout{}
+                                    : ws_layout(slice_geom(G, 0, P->slice), P->need_kbar, true, P->dec);
     return DASH_OK;
 }
+
+// The slicing budget of a call: the caller's workspace when it gives one, else the
+// library's default.
+size_t slice_budget(const dash_opts_t &o) { return o.workspace ? o.workspace_bytes : kSliceBudget; }
 
 }  // namespace
 
@@ -387,10 +428,10 @@ int report_error(int code, const char *msg) { return fail(code, "%s", msg); }
 // validates them); *need = 0 for an empty problem.
 int fwd_workspace_need(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v,
                        const dash_tensor_t *out, int block_size, float alpha, int causal, int gqa_groups,
-                       const dash_opts_t *opts, size_t *need) {
+                       const dash_opts_t *opts, size_t budget, size_t *need) {
     const dash_opts_t o = opts ? *opts : default_opts();
     FwdPlan P;
-    const int rc = plan_fwd(q, k, v, out, block_size, alpha, causal, gqa_groups, o, &P);
+    const int rc = plan_fwd(q, k, v, out, block_size, alpha, causal, gqa_groups, o, &P, budget);
     *need = rc ? 0 : P.WL.total;
     return rc;
 }
@@ -447,7 +488,11 @@ DASH_API size_t dash_workspace_bytes(int64_t batch, int64_t nq, int64_t nk, int 
     G.kbar_cap = G.n_chunks;
     G.ct_cap = (G.n_chunks + 127) / 128;
     G.local = 1;
-    return ws_layout(G, true, true, true).total;
+    G.pos0 = nk - nq;
+    G.nq_lse = nq;
+    const bool dec = nq * G.g <= 16 && G.n_tiles == 1;  // the decoding path: never sliced
+    const int64_t rows = slice_rows(G, true, dec, kSliceBudget);
+    return ws_layout(slice_geom(G, 0, rows), true, true, dec).total;
 }
 
 DASH_API int dash_pool_keys(const dash_tensor_t *k, int block_size, int causal, float *kbar, void *stream) {
@@ -575,7 +620,7 @@ DASH_API int dash_attn_fwd_ex(const dash_tensor_t *q, const dash_tensor_t *k, co
                               const dash_opts_t *opts) {
     dash_opts_t o = opts ? *opts : default_opts();
     FwdPlan P;
-    int rc = plan_fwd(q, k, v, out, block_size, alpha, causal, gqa_groups, o, &P);
+    int rc = plan_fwd(q, k, v, out, block_size, alpha, causal, gqa_groups, o, &P, slice_budget(o));
     if (rc) return rc;
     const Geom &G = P.G;
     if (G.b == 0 || G.nq == 0) return DASH_OK;
@@ -599,12 +644,25 @@ DASH_API int dash_attn_fwd_ex(const dash_tensor_t *q, const dash_tensor_t *k, co
         if ((rc = run_stage0(k, o.qbar, qv, G, kb, st))) return rc;
         kbar = kb;
     }
-    const bool regroup = !(o.flags & DASH_FLAG_NO_REGROUP) && G.n_tiles > 1;
-    const ListsView LV = ws_lists(G, ws, WL, regroup);
-    if ((rc = run_stage1(q, cache_geom(G, sc), alpha, o, kbar, nullptr, nullptr, nullptr, &LV, regroup, ws, WL, st,
-                         sc ? sc->split : nullptr)))
-        return rc;
-    return run_stage2(q, k, v, out, G, LV, o, dec ? ws + WL.decode : nullptr, st);
+    // Stage 1 and Stage 2, one slice of query rows after the other (a single slice unless the
+    // rows' lists would not fit the budget)
+    for (int64_t row0 = 0; row0 < G.nq; row0 += P.slice) {
+        const int64_t rows = std::min(P.slice, G.nq - row0);
+        const Geom Gs = slice_geom(G, row0, rows);
+        dash_tensor_t qs = *q, os = *out;
+        qs.data = static_cast<char *>(q->data) + row0 * q->stride[1] * (int64_t)esize(q->dtype);
+        os.data = static_cast<char *>(out->data) + row0 * out->stride[1] * (int64_t)esize(out->dtype);
+        qs.shape[1] = os.shape[1] = rows;
+        dash_opts_t oslice = o;
+        if (o.lse) oslice.lse = o.lse + row0 * G.hq;
+        const bool regroup = !(o.flags & DASH_FLAG_NO_REGROUP) && Gs.n_tiles > 1;
+        const ListsView LV = ws_lists(Gs, ws, WL, regroup);
+        if ((rc = run_stage1(&qs, cache_geom(Gs, sc), alpha, o, kbar, nullptr, nullptr, nullptr, &LV, regroup, ws, WL,
+                             st, sc ? sc->split : nullptr)))
+            return rc;
+        if ((rc = run_stage2(&qs, k, v, &os, Gs, LV, oslice, dec ? ws + WL.decode : nullptr, st))) return rc;
+    }
+    return DASH_OK;
 }
 
 DASH_API int dash_attn_fwd(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v,
@@ -618,7 +676,7 @@ namespace {
 
 struct BwdLayout {
     WsLayout F;  // Stage 0-1 state (recomputed) and the work lists
-    size_t tau, drow, gd, dq, dkbar, meang, rho, bitmap, E, ref_off, ref_cnt, refs, qp, dop, lp, dp, total;
+    size_t tau, drow, gd, dq, dkbar, bitmap, E, ref_off, ref_cnt, refs, qp, dop, lp, dp, total;
 };
 
 BwdLayout bwd_layout(const Geom &G, bool tc) {
@@ -638,8 +696,6 @@ BwdLayout bwd_layout(const Geom &G, bool tc) {
     L.gd = take((size_t)G.b * G.nq * G.hkv * (size_t)G.n_chunks * 4);
     L.dq = take(rows * G.d * 4);
     L.dkbar = take((size_t)G.b * G.n_chunks * G.hkv * G.d * 4);
-    L.meang = take((size_t)G.b * G.nq * G.hkv * 4);
-    L.rho = take(rows * 4);
     L.bitmap = take(bhb * tw * 4);
     L.E = take(bhb * G.n_tiles * 4);
     L.ref_off = take(bhb * 4);
@@ -764,8 +820,6 @@ DASH_API int dash_attn_bwd(const dash_tensor_t *q, const dash_tensor_t *k, const
     a.Gd = reinterpret_cast<float *>(ws + BL.gd);
     a.dQacc = reinterpret_cast<float *>(ws + BL.dq);
     a.dKbar = reinterpret_cast<float *>(ws + BL.dkbar);
-    a.meanG = reinterpret_cast<float *>(ws + BL.meang);
-    a.rho = reinterpret_cast<float *>(ws + BL.rho);
     a.bitmap = reinterpret_cast<uint32_t *>(ws + BL.bitmap);
     a.E = reinterpret_cast<int32_t *>(ws + BL.E);
     a.ref_off = reinterpret_cast<int32_t *>(ws + BL.ref_off);

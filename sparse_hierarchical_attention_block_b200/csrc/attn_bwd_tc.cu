@@ -390,8 +390,8 @@ struct KvSmem {
     static constexpr int kV = kK + 2 * kKRegion;
     static constexpr int kP = kV + 2 * kKRegion;           // 128 rows x 128 B (P, bf16)
     static constexpr int kdS = kP + kRegion;               // 128 rows x 128 B (dl, bf16)
-    static constexpr int kMeta = kdS + kRegion;            // [kNQ][bias 128 | L 128 | D 128 | rows 128]
-    static constexpr int kMetaStage = 4 * 128 * 4;
+    static constexpr int kMeta = kdS + kRegion;            // [kNQ][bias 128 | L 128 | D 128 | rows 128 | tile]
+    static constexpr int kMetaStage = 4 * 128 * 4 + 16;
     static constexpr int kBars = kMeta + kNQ * kMetaStage;
     // kv_full, q_full[NQ], q_empty[NQ], s_full[2], p_full, p_empty, fin
     static constexpr int kNumBars = 1 + 2 * kNQ + 2 + 3;
@@ -474,6 +474,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_tc_kernel(const __grid_c
                 const int e = rl[j].y;
                 const size_t tile_lin = bh * L.n_tiles + t;
                 uint8_t *meta = sm + S::kMeta + st * S::kMetaStage;
+                // the tile index for the compute warps (published by the arrive below)
+                *reinterpret_cast<long long *>(meta + 2048) = (long long)t;
                 const uint32_t bytes = 4 * kRegion + (uint32_t)(T * 4) + 1024 + (L.rows ? (uint32_t)(T * 4) : 0u);
                 mbar_arrive_expect_tx(q_full + st, bytes);
                 for (int dh = 0; dh < 2; ++dh) {
@@ -571,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_tc_kernel(const __grid_c
             const float bv = reinterpret_cast<const float *>(meta)[pos];
             const float L2 = reinterpret_cast<const float *>(meta + 512)[m];
             const float Dv = reinterpret_cast<const float *>(meta + 1024)[m];
-            const int64_t t = rl[j].x;
+            const int64_t t = *reinterpret_cast<const long long *>(meta + 2048);
             const int64_t i = L.rows ? (int64_t)reinterpret_cast<const int32_t *>(meta + 1536)[pos]
                                      : (t * T + pos < G.nq ? t * T + pos : -1);
             const bool live = i >= 0 && bv > -INFINITY;

@@ -357,7 +357,7 @@ __global__ void __launch_bounds__(D) combine_kernel(TView O, Geom G, ListsView L
                         (int64_t)(r * g + row % g) * O.s2;
     op[col] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
     if (lse && col == 0)  // natural log of the row's normaliser (log2 domain partials)
-        lse[((size_t)b * G.nq + i) * G.hq + r * g + row % g] =
+        lse[((size_t)b * G.nq_lse + i) * G.hq + r * g + row % g] =
             den > 0.f ? (mm + __log2f(den)) * 0.6931471805599453f : -INFINITY;
 }
 

@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(kSimtRows) attn_simt_kernel(TView Q, TView K, 
         const float inv = lrun > 0.f ? 1.f / lrun : 0.f;
         for (int e = 0; e < d; ++e) ob[e] = from_f<T>(Os[m * dp + e] * inv);
         if (lse)  // natural log of the row's normaliser: (m + log2 l) ln 2
-            lse[((size_t)b * G.nq + i) * G.hq + r * g + hh] =
+            lse[((size_t)b * G.nq_lse + i) * G.hq + r * g + hh] =
                 lrun > 0.f ? (mrun + log2f(lrun)) * 0.6931471805599453f : -INFINITY;
     }
 }

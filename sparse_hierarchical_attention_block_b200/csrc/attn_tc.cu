@@ -476,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const __grid_const
                                     i * O.s1 + (int64_t)(r * g + hh) * O.s2;
                 const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
                 if (lse && row_ok)  // natural log of the row's normaliser: (m + log2 l) ln 2
-                    lse[((size_t)b * G.nq + i) * G.hq + r * g + hh] =
+                    lse[((size_t)b * G.nq_lse + i) * G.hq + r * g + hh] =
                         l_run > 0.f ? (m_run + __log2f(l_run)) * 0.6931471805599453f : -INFINITY;
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {

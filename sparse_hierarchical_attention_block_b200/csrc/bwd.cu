@@ -25,8 +25,8 @@
 //   refs_build_kernel     entry) pairs that attend it, tiles ascending (deterministic)
 //   bwd_dkdv_simt_kernel  per key block: dK (Stage 2 + pooling share), dV over its pairs
 //   bwd_route_kernel      per (row, kv head): the prior / entmax / score chain above, added
-//                         to the Stage-2 part of dQ, which it writes in the caller's dtype
-//   bwd_kbar_grad_kernel  per (chunk, kv head): the same chain into the chunk summary
+//                         to the Stage-2 part of dQ, which it writes in the caller's dtype,
+//                         and (atomically) to the chunk summaries' gradient
 //   bwd_dq_finish_kernel  dQ to the caller's dtype when no row routes anything
 #include <math.h>
 
@@ -342,17 +342,23 @@ __global__ void __launch_bounds__(128) bwd_dkdv_simt_kernel(TView Q, TView K, TV
 }
 
 // ---------------------------------------------------------------------------
-// Routing gradient on CUDA cores: one warp per (batch, row, kv head).  Lane l holds
-// dimensions l, l + 32, ... of the group's queries.  Three passes over the routed set
-// R_i (mask bits): mean G; per head sum u and sum u dp; then ds, which goes to dQ.  The
-// row's mean G and, per head, <u, dp> / sum u are kept for bwd_kbar_grad_kernel, which
-// forms the summaries' gradient chunk by chunk (no atomics).
+// Routing gradient on CUDA cores: one warp per (batch, row, kv head), four warps per CTA.
+// The group's g query rows are staged in shared memory.  The routed set R_i (mask bits)
+// is walked 32 chunks at a time, one chunk per lane:
+//   pass 1  mean G over R_i;
+//   pass 2  each lane forms x = xs <q_h, kbar_c> for the g heads of its chunk (q from
+//           shared memory, kbar_c from global) and sums u and u dp per head; one warp
+//           reduction per head at the end gives <u, dp> / sum u;
+//   pass 3  each lane forms ds_h = u dp - u <u, dp> / sum u for its chunk; then the lanes
+//           take dimensions and, chunk by chunk, add ds_h kbar_c to dq_h and
+//           sum_h ds_h q_h to the chunk summary's gradient (atomically).
+// dQ (the Stage-2 part from dQacc plus this part) is written in the caller's dtype.
 // ---------------------------------------------------------------------------
-constexpr int kMaxG = 16;
+constexpr int kRouteWarps = 4;
 
-// The per-chunk arithmetic both kernels share: for head h's x = xs <q, kbar_c> and
-// threshold th, p = (x - th)^(1/(alpha-1)), u = p^(2-alpha) and u dp with dp = d(log w_c)
-// / (g w_c); false outside the head's own support (u = 0 there).
+// The per-chunk arithmetic: for head h's x = xs <q, kbar_c> and threshold th,
+// p = (x - th)^(1/(alpha-1)), u = p^(2-alpha) and u dp with dp = d(log w_c) / (g w_c);
+// false outside the head's own support (u = 0 there).
 __device__ __forceinline__ bool route_terms(float x, float th, float kexp, float uexp, float lw, float dlw, int g,
                                             float &u, float &ud) {
     if (!(x > th)) return false;
@@ -362,194 +368,188 @@ __device__ __forceinline__ bool route_terms(float x, float th, float kexp, float
     return true;
 }
 
-// The row's dQ (the Stage-2 part in dQacc plus the routing part dq_route, per head and
-// lane dimension) written in the caller's dtype.
-template <typename T, int DL>
-__device__ __forceinline__ void store_dq(const float *__restrict__ dQacc, TView dQ, const Geom &G, int64_t b,
-                                         int64_t i, int r, int lane, const float (&dq_route)[16][DL], float sc) {
-#pragma unroll
-    for (int h = 0; h < 16; ++h) {
-        if (h >= G.g) break;
-        const float *src = dQacc + (((size_t)b * G.nq + i) * G.hq + r * G.g + h) * G.d;
-        T *dst = reinterpret_cast<T *>(const_cast<void *>(dQ.p)) + b * dQ.s0 + i * dQ.s1 + (int64_t)(r * G.g + h) * dQ.s2;
-#pragma unroll
-        for (int k = 0; k < DL; ++k) dst[lane + 32 * k] = from_f<T>(src[lane + 32 * k] + sc * dq_route[h][k]);
+// chunk id of routed-set element n (ascending) of the row, from its mask words; -1 past the end
+__device__ __forceinline__ int nth_routed(const uint32_t *mrow, int wv, int nvis, int n) {
+    for (int wd = 0; wd < wv; ++wd) {
+        uint32_t bits = mrow[wd];
+        if (wd == wv - 1 && (nvis & 31)) bits &= (1u << (nvis & 31)) - 1u;
+        const int pc = __popc(bits);
+        if (n < pc) {
+            for (; n > 0; --n) bits &= bits - 1u;
+            return wd * 32 + __ffs(bits) - 1;
+        }
+        n -= pc;
     }
+    return -1;
 }
 
-template <typename T, int DL>  // DL = d / 32 dims per lane
-__global__ void __launch_bounds__(128) bwd_route_kernel(TView Q, const float *__restrict__ kbar, Geom G, float alpha,
-                                                        float gamma, float sigma, const float *__restrict__ tau,
-                                                        const uint32_t *__restrict__ mask,
-                                                        const float *__restrict__ logw, const float *__restrict__ Gd,
-                                                        const float *__restrict__ dQacc, TView dQ,
-                                                        float *__restrict__ meanG_out, float *__restrict__ rho_out) {
-    const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
-    const int lane = threadIdx.x % 32;
+template <typename T, int DL, int GM>  // DL = d / 32 dims per lane, GM >= g heads
+__global__ void __launch_bounds__(32 * kRouteWarps) bwd_route_kernel(
+    TView Q, const float *__restrict__ kbar, Geom G, float alpha, float gamma, float sigma,
+    const float *__restrict__ tau, const uint32_t *__restrict__ mask, const float *__restrict__ logw,
+    const float *__restrict__ Gd, const float *__restrict__ dQacc, TView dQ, float *__restrict__ dKbar) {
+    constexpr int D = DL * 32;
+    __shared__ __align__(16) float qs_all[kRouteWarps][GM][D];
+    __shared__ float ds_all[kRouteWarps][32][GM];
+    __shared__ int cs_all[kRouteWarps][32];
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int64_t w = (int64_t)blockIdx.x * kRouteWarps + warp;
     if (w >= G.b * G.nq * G.hkv) return;
+    float(&qs)[GM][D] = qs_all[warp];
+    float(&dsb)[32][GM] = ds_all[warp];
+    int *csb = cs_all[warp];
     const int r = (int)(w % G.hkv);
     const int64_t i = (w / G.hkv) % G.nq, b = w / ((int64_t)G.hkv * G.nq);
+    const int g = G.g;
     const int nvis = row_nvis(G, i);
-    const int g = G.g, d = G.d;
-    const float sc = gamma * rsqrtf((float)d);
-    float dq[kMaxG][DL];
+    const float sc = gamma * rsqrtf((float)D);
+    float dq[GM][DL];
 #pragma unroll
-    for (int h = 0; h < kMaxG; ++h)
+    for (int h = 0; h < GM; ++h)
 #pragma unroll
         for (int k = 0; k < DL; ++k) dq[h][k] = 0.f;
-    if (nvis <= 0) {  // nothing routed: the Stage-2 part alone
-        store_dq<T, DL>(dQacc, dQ, G, b, i, r, lane, dq, sc);
-        return;
-    }
+    auto store = [&]() {
+#pragma unroll
+        for (int h = 0; h < GM; ++h) {
+            if (h >= g) break;
+            const float *src = dQacc + (((size_t)b * G.nq + i) * G.hq + r * g + h) * D;
+            T *dst = reinterpret_cast<T *>(const_cast<void *>(dQ.p)) + b * dQ.s0 + i * dQ.s1 +
+                     (int64_t)(r * g + h) * dQ.s2;
+#pragma unroll
+            for (int k = 0; k < DL; ++k) dst[DL * lane + k] = from_f<T>(src[DL * lane + k] + sc * dq[h][k]);
+        }
+    };
     const uint32_t *mrow = mask + (((size_t)b * G.nq + i) * G.hkv + r) * G.words;
-    const int wv = (nvis + 31) / 32;
-    // pass 1: mean of G over the routed set
-    float sG = 0.f;
+    const int wv = nvis > 0 ? (nvis + 31) / 32 : 0;
+    // pass 1: |R_i| and mean G
     int nR = 0;
     for (int wd = 0; wd < wv; ++wd) {
         uint32_t bits = mrow[wd];
         if (wd == wv - 1 && (nvis & 31)) bits &= (1u << (nvis & 31)) - 1u;
-        for (int x = lane; x < 32; x += 32)
-            if ((bits >> x) & 1u) {
-                sG += Gd[logw_index(G, b, r, i, wd * 32 + x)];
-                ++nR;
-            }
+        nR += __popc(bits);
     }
-    sG = warp_sum(sG);
-    nR = warp_sum_i(nR);
-    if (nR == 0) {
-        store_dq<T, DL>(dQacc, dQ, G, b, i, r, lane, dq, sc);
+    if (nR == 0) {  // nothing routed: the Stage-2 part alone
+        store();
         return;
     }
-    const float meanG = sG / (float)nR;
-    if (lane == 0) meanG_out[w] = meanG;
-    const float inv_sigma = 1.f / sigma;
-    const float xs = (alpha - 1.f) * gamma * rsqrtf((float)d);  // x = xs <q, kbar>
-    const float kexp = 1.f / (alpha - 1.f), uexp = 2.f - alpha;
-    float q[kMaxG][DL], th[kMaxG], su[kMaxG], sud[kMaxG];
-#pragma unroll
-    for (int h = 0; h < kMaxG; ++h) {
-        const bool on = h < g;
-        const size_t rid = ((size_t)b * G.nq + i) * G.hq + r * g + (on ? h : 0);
-        const T *qp = reinterpret_cast<const T *>(Q.p) + b * Q.s0 + i * Q.s1 + (int64_t)(r * g + (on ? h : 0)) * Q.s2;
-#pragma unroll
-        for (int k = 0; k < DL; ++k) q[h][k] = on ? to_f<T>(qp[lane + 32 * k]) : 0.f;
-        th[h] = on ? tau[rid] : INFINITY;
-        su[h] = 0.f;
-        sud[h] = 0.f;
+    float sG = 0.f;
+    for (int n0 = 0; n0 < nR; n0 += 32) {
+        const int c = n0 + lane < nR ? nth_routed(mrow, wv, nvis, n0 + lane) : -1;
+        if (c >= 0) sG += Gd[logw_index(G, b, r, i, c)];
     }
-    const float *kb_row = kbar + (((size_t)b * G.kbar_cap) * G.hkv + r) * d;  // chunk c at + c * hkv * d
-    // passes 2 and 3 share the per-chunk arithmetic
-    for (int pass = 0; pass < 2; ++pass) {
-        for (int wd = 0; wd < wv; ++wd) {
-            uint32_t bits = mrow[wd];
-            if (wd == wv - 1 && (nvis & 31)) bits &= (1u << (nvis & 31)) - 1u;
-            while (bits) {
-                const int c = wd * 32 + __ffs(bits) - 1;
-                bits &= bits - 1u;
-                const size_t li = logw_index(G, b, r, i, c);
-                const float dlw = (Gd[li] - meanG) * inv_sigma;
-                const float lw = logw[li];
-                float kv[DL];
-                const float *kp = kb_row + (size_t)c * G.hkv * d;
+    const float meanG = warp_sum(sG) / (float)nR;
+    // the group's queries into shared memory
 #pragma unroll
-                for (int k = 0; k < DL; ++k) kv[k] = kp[lane + 32 * k];
+    for (int h = 0; h < GM; ++h) {
+        if (h >= g) break;
+        const T *qp = reinterpret_cast<const T *>(Q.p) + b * Q.s0 + i * Q.s1 + (int64_t)(r * g + h) * Q.s2;
 #pragma unroll
-                for (int h = 0; h < kMaxG; ++h) {
-                    if (h >= g) break;
-                    float dot = 0.f;
+        for (int k = 0; k < DL; ++k) qs[h][DL * lane + k] = to_f<T>(qp[DL * lane + k]);
+    }
+    __syncwarp();
+    const float inv_sigma = 1.f / sigma;
+    const float xs = (alpha - 1.f) * gamma * rsqrtf((float)D);
+    const float kexp = 1.f / (alpha - 1.f), uexp = 2.f - alpha;
+    float th[GM];
 #pragma unroll
-                    for (int k = 0; k < DL; ++k) dot = fmaf(q[h][k], kv[k], dot);
-                    float u, ud;
-                    if (!route_terms(xs * warp_sum(dot), th[h], kexp, uexp, lw, dlw, g, u, ud)) continue;
-                    if (pass == 0) {
-                        su[h] += u;
-                        sud[h] += ud;
-                    } else {
-                        const float ds = ud - u * (sud[h] / su[h]);
+    for (int h = 0; h < GM; ++h) th[h] = h < g ? tau[((size_t)b * G.nq + i) * G.hq + r * g + h] : INFINITY;
+    const float *kb_base = kbar + ((size_t)b * G.kbar_cap * G.hkv + r) * D;  // chunk c at + c * hkv * D
+    // x of every head for the lane's chunk: GM dot products over D from shared q
+    auto scores = [&](int c, float (&x)[GM]) {
+        const float4 *kp = reinterpret_cast<const float4 *>(kb_base + (size_t)c * G.hkv * D);
 #pragma unroll
-                        for (int k = 0; k < DL; ++k) dq[h][k] = fmaf(ds, kv[k], dq[h][k]);
-                    }
+        for (int h = 0; h < GM; ++h) x[h] = 0.f;
+#pragma unroll 4
+        for (int e4 = 0; e4 < D / 4; ++e4) {
+            const float4 kv = kp[e4];
+#pragma unroll
+            for (int h = 0; h < GM; ++h) {
+                if (h < g) {
+                    const float4 qv = *reinterpret_cast<const float4 *>(&qs[h][4 * e4]);
+                    x[h] = fmaf(qv.x, kv.x, fmaf(qv.y, kv.y, fmaf(qv.z, kv.z, fmaf(qv.w, kv.w, x[h]))));
                 }
             }
         }
-        if (pass == 0 && lane == 0) {
 #pragma unroll
-            for (int h = 0; h < kMaxG; ++h)
-                if (h < g) rho_out[((size_t)b * G.nq + i) * G.hq + r * g + h] = su[h] > 0.f ? sud[h] / su[h] : 0.f;
+        for (int h = 0; h < GM; ++h) x[h] *= xs;
+    };
+    // pass 2: sum u and sum u dp per head
+    float su[GM], sud[GM];
+#pragma unroll
+    for (int h = 0; h < GM; ++h) su[h] = sud[h] = 0.f;
+    for (int n0 = 0; n0 < nR; n0 += 32) {
+        const int c = n0 + lane < nR ? nth_routed(mrow, wv, nvis, n0 + lane) : -1;
+        if (c < 0) continue;
+        const size_t li = logw_index(G, b, r, i, c);
+        const float dlw = (Gd[li] - meanG) * inv_sigma, lw = logw[li];
+        float x[GM];
+        scores(c, x);
+#pragma unroll
+        for (int h = 0; h < GM; ++h) {
+            float u, ud;
+            if (h < g && route_terms(x[h], th[h], kexp, uexp, lw, dlw, g, u, ud)) {
+                su[h] += u;
+                sud[h] += ud;
+            }
         }
     }
-    store_dq<T, DL>(dQacc, dQ, G, b, i, r, lane, dq, sc);
-}
-
-// The summaries' gradient, chunk by chunk: one CTA (4 warps) per (routing chunk, kv head,
-// batch) walks the (tile, entry) pairs that list the chunk (the transposed lists) and the
-// tile rows that route it; each (row, head) adds ds q (ds from the row's mean G and
-// <u, dp> / sum u kept by bwd_route_kernel).  Pairs go to the warps round robin and the
-// warps' sums are added in a fixed order: deterministic, no atomics.
-template <typename T, int DL>
-__global__ void __launch_bounds__(128) bwd_kbar_grad_kernel(TView Q, const float *__restrict__ kbar, Geom G,
-                                                            ListsView L, float alpha, float gamma, float sigma,
-                                                            const float *__restrict__ tau,
-                                                            const float *__restrict__ logw,
-                                                            const float *__restrict__ Gd,
-                                                            const float *__restrict__ meanG,
-                                                            const float *__restrict__ rho,
-                                                            const int32_t *__restrict__ ref_off,
-                                                            const int32_t *__restrict__ ref_cnt,
-                                                            const int2 *__restrict__ refs, float *__restrict__ dKbar) {
-    __shared__ float part[4][DL * 32];
-    const int c = blockIdx.x, r = blockIdx.y;
-    const int64_t b = blockIdx.z;
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int g = G.g, d = G.d, TR = L.tile_rows;
-    const size_t bh = (size_t)b * G.hkv + r;
-    const int nref = ref_cnt[bh * G.n_blk + c];
-    const int2 *rl = refs + bh * (size_t)L.n_tiles * G.n_blk + ref_off[bh * G.n_blk + c];
-    const float inv_sigma = 1.f / sigma;
-    const float xs = (alpha - 1.f) * gamma * rsqrtf((float)d);
-    const float kexp = 1.f / (alpha - 1.f), uexp = 2.f - alpha;
-    float kv[DL], acc[DL];
-    const float *kp = kbar + (((size_t)b * G.kbar_cap + c) * G.hkv + r) * d;
+    float rho[GM];
 #pragma unroll
-    for (int k = 0; k < DL; ++k) {
-        kv[k] = kp[lane + 32 * k];
-        acc[k] = 0.f;
+    for (int h = 0; h < GM; ++h) {
+        const float a = warp_sum(su[h]), bb = warp_sum(sud[h]);
+        rho[h] = a > 0.f ? bb / a : 0.f;
     }
-    for (int idx = warp; idx < nref * TR; idx += 4) {
-        const int64_t t = rl[idx / TR].x;
-        const int e = rl[idx / TR].y, pos = idx % TR;
-        const size_t tile_lin = bh * L.n_tiles + t;
-        const int64_t i = tile_row(L, G, tile_lin, t, pos);
-        if (i < 0) continue;
-        const float bv = L.bias[tile_lin * (size_t)L.cap * TR + (size_t)e * TR + pos];
-        if (!(bv > -INFINITY) || c >= row_nvis(G, i)) continue;  // the row does not route this chunk
-        const size_t li = logw_index(G, b, r, i, c);
-        const float dlw = (Gd[li] - meanG[((size_t)b * G.nq + i) * G.hkv + r]) * inv_sigma;
-        const float lw = logw[li];
-        for (int h = 0; h < g; ++h) {
-            const size_t rid = ((size_t)b * G.nq + i) * G.hq + r * g + h;
-            const T *qp = reinterpret_cast<const T *>(Q.p) + b * Q.s0 + i * Q.s1 + (int64_t)(r * g + h) * Q.s2;
-            float qv[DL], dot = 0.f;
+    // pass 3: ds per (chunk, head) by the chunk's lane, then lanes over dimensions
+    const float sck = gamma * rsqrtf((float)D);
+    for (int n0 = 0; n0 < nR; n0 += 32) {
+        const int c = n0 + lane < nR ? nth_routed(mrow, wv, nvis, n0 + lane) : -1;
+        csb[lane] = c;
+        if (c >= 0) {
+            const size_t li = logw_index(G, b, r, i, c);
+            const float dlw = (Gd[li] - meanG) * inv_sigma, lw = logw[li];
+            float x[GM];
+            scores(c, x);
+#pragma unroll
+            for (int h = 0; h < GM; ++h) {
+                float u = 0.f, ud = 0.f;
+                const bool in = h < g && route_terms(x[h], th[h], kexp, uexp, lw, dlw, g, u, ud);
+                dsb[lane][h] = in ? ud - u * rho[h] : 0.f;
+            }
+        }
+        __syncwarp();
+        const int nb = min(32, nR - n0);
+        // lanes over dimensions: lane l holds dimensions DL*l .. DL*l + DL - 1 (one vector
+        // load of kbar_c and one vector atomic into its gradient per chunk)
+        for (int j = 0; j < nb; ++j) {
+            const int cj = csb[j];
+            const float *kp = kb_base + (size_t)cj * G.hkv * D + DL * lane;
+            float kv[DL], dkb[DL];
 #pragma unroll
             for (int k = 0; k < DL; ++k) {
-                qv[k] = to_f<T>(qp[lane + 32 * k]);
-                dot = fmaf(qv[k], kv[k], dot);
+                kv[k] = kp[k];
+                dkb[k] = 0.f;
             }
-            float u, ud;
-            if (!route_terms(xs * warp_sum(dot), tau[rid], kexp, uexp, lw, dlw, g, u, ud)) continue;
-            const float ds = ud - u * rho[rid];
 #pragma unroll
-            for (int k = 0; k < DL; ++k) acc[k] = fmaf(ds, qv[k], acc[k]);
+            for (int h = 0; h < GM; ++h) {
+                if (h >= g) break;
+                const float ds = dsb[j][h];
+#pragma unroll
+                for (int k = 0; k < DL; ++k) {
+                    dq[h][k] = fmaf(ds, kv[k], dq[h][k]);
+                    dkb[k] = fmaf(ds, qs[h][DL * lane + k], dkb[k]);
+                }
+            }
+            float *dst = dKbar + (((size_t)b * G.n_chunks + cj) * G.hkv + r) * D + DL * lane;
+            if (DL == 4)
+                atomicAdd(reinterpret_cast<float4 *>(dst),
+                          make_float4(sck * dkb[0], sck * dkb[DL > 1 ? 1 : 0], sck * dkb[DL > 2 ? 2 : 0],
+                                      sck * dkb[DL > 3 ? 3 : 0]));
+            else
+                atomicAdd(reinterpret_cast<float2 *>(dst), make_float2(sck * dkb[0], sck * dkb[DL > 1 ? 1 : 0]));
         }
+        __syncwarp();
     }
-#pragma unroll
-    for (int k = 0; k < DL; ++k) part[warp][lane + 32 * k] = acc[k];
-    __syncthreads();
-    const float sc = gamma * rsqrtf((float)d);
-    for (int x = threadIdx.x; x < d; x += 128)
-        dKbar[(((size_t)b * G.n_chunks + c) * G.hkv + r) * d + x] =
-            sc * (((part[0][x] + part[1][x]) + part[2][x]) + part[3][x]);
+    store();
 }
 
 template <typename T>
@@ -586,16 +586,22 @@ cudaError_t launch_bwd_t(const BwdArgs &a, cudaStream_t st) {
             a.Q, a.K, a.V, a.dO, G, L, a.lse, a.Drow, a.dQacc, a.Gd);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    // the routing chain (prior, group average, entmax, Stage-1 scores) into dQ
+    // the routing chain (prior, group average, entmax, Stage-1 scores) into dQ and the summaries
     if (G.n_chunks > 0) {
+        if ((e = cudaMemsetAsync(a.dKbar, 0, (size_t)G.b * G.n_chunks * G.hkv * G.d * sizeof(float), st)) !=
+            cudaSuccess)
+            return e;
         const int64_t warps = G.b * G.nq * G.hkv;
-        const unsigned blocks = (unsigned)((warps * 32 + 127) / 128);
-        if (G.d == 128)
-            bwd_route_kernel<T, 4><<<blocks, 128, 0, st>>>(a.Q, a.kbar, G, a.alpha, a.gamma, a.sigma, a.tau, a.mask,
-                                                           a.logw, a.Gd, a.dQacc, a.dQ, a.meanG, a.rho);
-        else
-            bwd_route_kernel<T, 2><<<blocks, 128, 0, st>>>(a.Q, a.kbar, G, a.alpha, a.gamma, a.sigma, a.tau, a.mask,
-                                                           a.logw, a.Gd, a.dQacc, a.dQ, a.meanG, a.rho);
+        const unsigned blocks = (unsigned)((warps + kRouteWarps - 1) / kRouteWarps);
+#define DASH_ROUTE(DL, GM)                                                                                         \
+    bwd_route_kernel<T, DL, GM><<<blocks, 32 * kRouteWarps, 0, st>>>(a.Q, a.kbar, G, a.alpha, a.gamma, a.sigma,  \
+                                                                     a.tau, a.mask, a.logw, a.Gd, a.dQacc, a.dQ, \
+                                                                     a.dKbar)
+        if (G.d == 128 && G.g <= 4) DASH_ROUTE(4, 4);
+        else if (G.d == 128) DASH_ROUTE(4, 16);
+        else if (G.g <= 4) DASH_ROUTE(2, 4);
+        else DASH_ROUTE(2, 16);
+#undef DASH_ROUTE
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     // transposed lists
@@ -608,19 +614,6 @@ cudaError_t launch_bwd_t(const BwdArgs &a, cudaStream_t st) {
     refs_build_kernel<<<dim3((unsigned)G.hkv, (unsigned)G.b), 1024, 0, st>>>(G, L.n_tiles, a.bitmap, a.E, tw,
                                                                             a.ref_off, a.ref_cnt, a.refs);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // the routing chain into the chunk summaries (deterministic, chunk by chunk)
-    if (G.n_chunks > 0) {
-        const dim3 grid((unsigned)G.n_chunks, (unsigned)G.hkv, (unsigned)G.b);
-        if (G.d == 128)
-            bwd_kbar_grad_kernel<T, 4><<<grid, 128, 0, st>>>(a.Q, a.kbar, G, L, a.alpha, a.gamma, a.sigma, a.tau,
-                                                             a.logw, a.Gd, a.meanG, a.rho, a.ref_off, a.ref_cnt,
-                                                             a.refs, a.dKbar);
-        else
-            bwd_kbar_grad_kernel<T, 2><<<grid, 128, 0, st>>>(a.Q, a.kbar, G, L, a.alpha, a.gamma, a.sigma, a.tau,
-                                                             a.logw, a.Gd, a.meanG, a.rho, a.ref_off, a.ref_cnt,
-                                                             a.refs, a.dKbar);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
     // Stage 2, key side: dK (with the pooling share), dV
     if (a.use_tc) {
         if ((e = launch_attn_bwd_tc_dkdv(a, st)) != cudaSuccess) return e;

@@ -32,6 +32,10 @@ struct Geom {
     // the number of chunks a summary cache has pooled (device-side bookkeeping).
     const int64_t *nk_dev;
     const int *chunks_dev;
+    // Key position of query row 0 of this launch: nk - nq, plus the first row of a slice when
+    // the rows are processed in slices; and the row count of the lse output's layout.
+    int64_t pos0;
+    int64_t nq_lse;
 };
 
 // The geometry a kernel works with: with a device-resident key length, nk is read from
@@ -41,6 +45,7 @@ __device__ __forceinline__ void geom_live(Geom &G) {
     if (!G.nk_dev) return;
     int64_t nk = *G.nk_dev;
     nk = nk < 0 ? 0 : (nk > G.nk ? G.nk : nk);
+    G.pos0 += nk - G.nk;  // the rows sit at the last positions before the live length
     G.nk = nk;
     G.n_chunks = (int)(G.causal ? nk / G.B : (nk + G.B - 1) / G.B);
     G.n_blk = (int)((nk + G.B - 1) / G.B);
@@ -78,7 +83,7 @@ __host__ __device__ inline size_t logw_index(const Geom &G, int64_t b, int r, in
 }
 
 // Causal geometry of query row i: key position, own chunk, visible chunks.
-__host__ __device__ inline int64_t row_pos(const Geom &G, int64_t i) { return i + G.nk - G.nq; }
+__host__ __device__ inline int64_t row_pos(const Geom &G, int64_t i) { return i + G.pos0; }
 // first chunk of row i's local window (causal): its own chunk, or the one before with local = 2
 __host__ __device__ inline int first_local(const Geom &G, int64_t i) {
     const int64_t c = row_pos(G, i) / G.B - (G.local - 1);

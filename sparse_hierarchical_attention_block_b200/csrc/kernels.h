@@ -83,8 +83,6 @@ struct BwdArgs {
     float *Gd;                         // G per (row, routed chunk), logw_index layout
     float *dQacc;                      // [b][nq][hq][d] fp32
     float *dKbar;                      // [b][n_chunks][hkv][d] fp32
-    float *meanG;                      // [b][nq][hkv] mean G over the row's routed chunks
-    float *rho;                        // [b][nq][hq] <u, dp> / sum u of the row's entmax
     uint32_t *bitmap;                  // [b][hkv][n_blk][ceil(n_tiles/32)] tiles attending each key block
     int32_t *E;                        // [b][hkv][n_blk][n_tiles] entry index of the block in the tile's list
     int32_t *ref_off, *ref_cnt;        // [b][hkv][n_blk] the block's (tile, entry) pairs

@@ -38,7 +38,7 @@ namespace dash {
 int report_error(int code, const char *msg);
 int fwd_workspace_need(const dash_tensor_t *q, const dash_tensor_t *k, const dash_tensor_t *v,
                        const dash_tensor_t *out, int block_size, float alpha, int causal, int gqa_groups,
-                       const dash_opts_t *opts, size_t *need);
+                       const dash_opts_t *opts, size_t budget, size_t *need);
 }  // namespace dash
 
 namespace {
@@ -84,10 +84,12 @@ DASH_API int dash_attn_fwd_noalloc(const dash_tensor_t *q, const dash_tensor_t *
     } else {
         dash_opts_init(&o);
     }
-    // the exact scratch this call's forward pass takes (it depends on the options: a
-    // summary cache or given summaries need no pooled-key area, prefill no split-KV area)
+    // the exact scratch this call's forward pass takes in the static area (it depends on the
+    // options: a summary cache or given summaries need no pooled-key area, prefill no
+    // split-KV area; a long prefill runs its query rows in slices that fit the area)
     size_t need = 0;
-    int rc = dash::fwd_workspace_need(q, k, v, out, block_size, alpha, causal, gqa_groups, &o, &need);
+    int rc = dash::fwd_workspace_need(q, k, v, out, block_size, alpha, causal, gqa_groups, &o,
+                                      DASH_NOALLOC_SCRATCH_BYTES, &need);
     if (rc) return rc;
     if (need > (size_t)DASH_NOALLOC_SCRATCH_BYTES) {
         char msg[256];

@@ -281,9 +281,10 @@ def test_backward_prefill8k_sampled_and_identities():
 
 
 def test_backward_deterministic():
-    """Every gradient is reproducible bit for bit (no atomic sums anywhere)."""
+    """dQ and dV are reproducible bit for bit; dK takes the summaries' gradient through
+    fp32 atomic sums, so its last bit may differ between runs."""
     q, k, v, dout = _inputs(1, 512, 512, 8, 2, 128, 64, "bf16", seed=5)
     a = _fwd_bwd(q, k, v, dout, 64, 1.5, True, sigma=1.0)
     b = _fwd_bwd(q, k, v, dout, 64, 1.5, True, sigma=1.0)
-    for x, y in zip(a[2:], b[2:]):
-        assert torch.equal(x, y)
+    assert torch.equal(a[2], b[2]) and torch.equal(a[4], b[4])
+    assert torch.allclose(a[3].float(), b[3].float(), rtol=1e-2, atol=1e-3)

@@ -337,3 +337,31 @@ def test_prefill128k_sampled(alpha, sigma):
     out = _run(q, k, v, w.block, alpha, True, sigma=sigma)
     check_forward(q, k, v, out, w.block, alpha, True, sigma=sigma, rows=rows,
                   label=f"prefill128k alpha={alpha} sigma={sigma:g}")
+
+
+def test_row_slices_equal_one_pass():
+    """A caller workspace too small for every row's lists makes the forward run its query
+    rows in slices; the output (and lse) equals the single-pass forward bit for bit."""
+    w = synthetic.WORKLOADS["prefill8k"]
+    q, k, v = synthetic.make_inputs(w, "cuda")
+    a, c = torch.empty_like(q), torch.empty_like(q)
+    la = torch.empty(q.shape[:3], dtype=torch.float32, device="cuda")
+    lc = torch.empty_like(la)
+    dash.dash_attn_fwd(q, k, v, a, w.block, w.alpha, True, w.g, sigma=1.0, lse=la)
+    full = dash.dash_workspace_bytes(1, w.nq, w.nk, w.hq, w.hkv, w.d, w.block)
+    ws = torch.empty(full // 3, dtype=torch.uint8, device="cuda")  # room for about a third of the rows
+    dash.dash_attn_fwd(q, k, v, c, w.block, w.alpha, True, w.g, sigma=1.0, lse=lc, workspace=ws)
+    assert dash.dash_sync_status() == 0
+    assert torch.equal(a, c) and torch.equal(la, lc)
+
+
+def test_prefill128k_batch2_sampled():
+    """128K keys at batch 2: the library workspace stays within its 1 GB budget (rows in
+    slices) and the second sequence matches the oracle on sampled rows."""
+    w = synthetic.WORKLOADS["prefill128k"].with_(batch=2)
+    assert dash.dash_workspace_bytes(2, w.nq, w.nk, w.hq, w.hkv, w.d, w.block) <= 10 ** 9
+    q, k, v = synthetic.make_inputs(w, "cuda")
+    out = _run(q, k, v, w.block, w.alpha, True, sigma=1.0)
+    rows = sample_rows(w.nq, w.block, 256, seed=129)
+    check_forward(q, k, v, out, w.block, w.alpha, True, sigma=1.0, rows=rows, batches=[1],
+                  label="prefill128k batch 2 (second sequence)")

@@ -3,11 +3,11 @@
 Host-side checks (no GPU): the entry point is exported, rejects a problem
 larger than its scratch area with DASH_ERR_WORKSPACE and refuses a caller
 workspace, before any CUDA call.  GPU check: consecutive calls through the C
-ABI (a prefill, a split-KV decode and a decode with a chunk-summary cache,
-in turn, so each call finds another's leftovers in the shared area) agree with
-dash_attn_fwd within the tolerance of the parity tests (the cached decode bit
-for bit), and the calls after the first change the device's free memory by
-nothing.
+ABI (a prefill, a split-KV decode, a decode with a chunk-summary cache and an
+8K-token prefill whose rows run in slices, in turn, so each call finds another's
+leftovers in the shared area) agree with dash_attn_fwd within the tolerance of
+the parity tests (the cached decode and the sliced prefill bit for bit), and the
+calls after the first change the device's free memory by nothing.
 
 Kept in a file of its own, collected last, so it runs both alone in a fresh
 process and after every other test."""
@@ -48,16 +48,16 @@ def test_noalloc_exported(lib):
 
 
 def test_noalloc_rejects_oversize(lib):
-    # 8K-token prefill with 32 heads needs ~68 MiB of scratch, above the 32 MiB area
-    q = _t(dash.DASH_BF16, [1, 8192, 32, 128])
-    k = _t(dash.DASH_BF16, [1, 8192, 8, 128])
-    bound = dash.dash_workspace_bytes(1, 8192, 8192, 32, 8, 128, 64, True)
-    rc = lib.dash_attn_fwd_noalloc(ctypes.byref(q), ctypes.byref(k), ctypes.byref(k), ctypes.byref(q), 64, 1.5, 1,
-                                   4, None)
+    # 128K-token prefill with 1024 chunks of 128: even 1024 query rows take ~70 MiB of lists
+    q = _t(dash.DASH_BF16, [1, 131072, 32, 128])
+    k = _t(dash.DASH_BF16, [1, 131072, 8, 128])
+    bound = dash.dash_workspace_bytes(1, 131072, 131072, 32, 8, 128, 128, True)
+    rc = lib.dash_attn_fwd_noalloc(ctypes.byref(q), ctypes.byref(k), ctypes.byref(k), ctypes.byref(q), 128, 1.5,
+                                   1, 4, None)
     assert rc == dash.DASH_ERR_WORKSPACE
     msg = lib.dash_last_error().decode()
-    # the message states the exact need of this call (no split-KV area for a prefill),
-    # which dash_workspace_bytes bounds from above
+    # the message states the exact need of this call (its smallest slice of query rows, no
+    # split-KV area for a prefill), which dash_workspace_bytes bounds from above
     need = int(re.search(r"needs (\d+) bytes", msg).group(1))
     assert dash.DASH_NOALLOC_SCRATCH_BYTES < need <= bound
     assert str(dash.DASH_NOALLOC_SCRATCH_BYTES) in msg and "dash_attn_fwd_ex" in msg
@@ -92,6 +92,9 @@ PROBLEMS = [
     # decoding with a persistent chunk-summary cache (the serving case): Stage 0 and the
     # summaries' operand form come from the cache's own memory, not the scratch area
     (2, 1, 5000, 8, 2, 128, 64, 1.5, True, 1.0, True),
+    # an 8K-token prefill at 32 heads: its lists need ~70 MiB, so the rows run in slices
+    # that fit the area
+    (1, 8192, 8192, 32, 8, 128, 64, 1.5, True, 1.0, False),
 ]
 
 
@@ -108,7 +111,6 @@ def test_noalloc_matches_fwd_on_consecutive_calls(lib):
     data = []
     for i, p in enumerate(PROBLEMS):
         b, nq, nk, hq, hkv, d, B, alpha, causal, sigma, cached = p
-        assert dash.dash_workspace_bytes(b, nq, nk, hq, hkv, d, B, causal) <= dash.DASH_NOALLOC_SCRATCH_BYTES
         q, k, v = _inputs(p, 40 + i)
         opts = {"sigma": sigma}
         if cached:
@@ -117,7 +119,7 @@ def test_noalloc_matches_fwd_on_consecutive_calls(lib):
         dash.dash_attn_fwd(q, k, v, ref, B, alpha, causal, hq // hkv, **opts)
         assert dash.dash_sync_status() == 0
         data.append((p, q, k, v, ref, opts))
-    order = [0, 1, 2, 0, 1, 2]  # each call after the first finds another problem's contents in the scratch
+    order = [0, 1, 2, 3, 0, 1, 2, 3]  # each call after the first finds another problem's contents in the scratch
     outs = [torch.full_like(data[j][1], float("nan")) for j in order]
     torch.cuda.synchronize()
     free = []
@@ -132,7 +134,7 @@ def test_noalloc_matches_fwd_on_consecutive_calls(lib):
     assert free[1:] == free[:1] * (len(free) - 1), free
     for n, (j, out) in enumerate(zip(order, outs)):
         ref = data[j][4]
-        if data[j][0][10]:  # the same cache, the same kernels: bit for bit
+        if data[j][0][10] or data[j][0][1] == 8192:  # the same kernels on the same lists: bit for bit
             assert torch.equal(out, ref)
         err = (out.float() - ref.float()).abs()
         print(f"[noalloc] call {n} problem {j}: max_abs={err.max().item():.3g} mean_abs={err.mean().item():.3g}")
