@@ -98,7 +98,8 @@ __host__ __device__ inline int row_nvis(const Geom &G, int64_t i) {
 
 // ---------------------------------------------------------------------------
 // Order of the query-tile CTAs of a Stage-2 launch.  The (batch, kv head) pairs are
-// taken in groups whose K and V fit in half of the 126 MB L2 together; within a group
+// taken in groups whose K and V fit in about three quarters of the 126 MB L2 together
+// (the rest holds the Q rows, biases and lists in flight); within a group
 // the CTAs go longest tile (latest, causal) first across the group's pairs, so that
 // the long tiles do not gather at the end of the launch, and the groups follow one
 // another, so that the CTAs in flight read K and V that stay in L2.
@@ -110,7 +111,7 @@ struct TileOrder {
 inline int heads_per_group(const Geom &G) {
     const double per_head = (double)G.nk * G.d * 2.0 * 2.0;  // K and V, bf16
     int hg = 1;
-    while (hg * 2 <= G.b * G.hkv && (double)(hg * 2) * per_head <= 63.0 * (1 << 20)) hg *= 2;
+    while (hg * 2 <= G.b * G.hkv && (double)(hg * 2) * per_head <= 96.0 * (1 << 20)) hg *= 2;
     return hg;
 }
 __host__ __device__ inline TileOrder tile_order(int64_t cta, int64_t n_tiles, int64_t bh_total, int hg) {
