@@ -234,6 +234,10 @@ DASH_API int dash_block_select(const dash_tensor_t *q, const dash_tensor_t *k, i
  *   dout [b, nq, hq, d] the output gradient; lse [b][nq][hq] fp32 from the forward's
  *     opts->lse;
  *   dq [b, nq, hq, d], dk, dv [b, nk, hkv, d]: outputs (overwritten), same dtype as q.
+ * Reproducibility: dq is identical between runs; dk (whose chunk-summary share, and on
+ * the tensor-core path its Stage-2 share, is summed with fp32 atomics) and, on the
+ * tensor-core path with 128 or more query tiles per (batch, kv head), dv may differ in
+ * their last bits.
  * Not supported with a summary cache, given summaries or learned summary queries
  * (DASH_ERR_UNSUPPORTED).  Workspace: dash_bwd_workspace_bytes().  Errors as for
  * dash_attn_fwd_ex; DASH_ERR_INVALID_ARG when a gradient's shape or dtype does not

@@ -676,7 +676,7 @@ namespace {
 
 struct BwdLayout {
     WsLayout F;  // Stage 0-1 state (recomputed) and the work lists
-    size_t tau, drow, gd, dq, dkbar, bitmap, E, ref_off, ref_cnt, refs, qp, dop, lp, dp, total;
+    size_t tau, drow, gd, dq, dkbar, bitmap, E, ref_off, ref_cnt, refs, qp, dop, lp, dp, dkacc, dvacc, total;
 };
 
 BwdLayout bwd_layout(const Geom &G, bool tc) {
@@ -707,6 +707,8 @@ BwdLayout bwd_layout(const Geom &G, bool tc) {
         L.dop = take(tiles * 128 * G.d * 2);
         L.lp = take(tiles * 128 * 4);
         L.dp = take(tiles * 128 * 4);
+        L.dkacc = take((size_t)G.b * G.nk * G.hkv * G.d * 4);
+        L.dvacc = take((size_t)G.b * G.nk * G.hkv * G.d * 4);
     }
     L.total = off;
     return L;
@@ -830,6 +832,8 @@ DASH_API int dash_attn_bwd(const dash_tensor_t *q, const dash_tensor_t *k, const
     a.dOp = tc ? reinterpret_cast<uint8_t *>(ws + BL.dop) : nullptr;
     a.Lp = tc ? reinterpret_cast<float *>(ws + BL.lp) : nullptr;
     a.Dp = tc ? reinterpret_cast<float *>(ws + BL.dp) : nullptr;
+    a.dKacc = tc ? reinterpret_cast<float *>(ws + BL.dkacc) : nullptr;
+    a.dVacc = tc ? reinterpret_cast<float *>(ws + BL.dvacc) : nullptr;
     cudaError_t e = launch_attn_bwd(a, q->dtype, st);
     return e == cudaSuccess ? DASH_OK : cuda_fail(e, "backward pass");
 }

@@ -26,11 +26,15 @@
 //                      128-byte swizzled row of tile row m), and the MMA thread accumulates
 //                        dV^T += dO^T P  and  dK^T += Q^T dl   (SS, both operands MN-major,
 //                        M = d = 128, N = 64 keys, K = 128 tile rows)
-//                      in TMEM; the epilogue writes dK (with the keys' share of the chunk
-//                      summary's gradient) and dV.
+//                      in TMEM.  A block's pairs are split among up to 8 CTAs (a block
+//                      many tiles attend would otherwise be one long serial chain); each
+//                      adds its share to fp32 accumulators, and bwd_kv_finish_kernel
+//                      adds the chunk summary's share to dK and writes dK, dV in bf16.
 // Every wait is bounded (globaltimer); on expiry a kernel records a device error, drains
 // what it issued, frees TMEM and returns.
 #include <math.h>
+
+#include <algorithm>
 
 #include "dash_common.cuh"
 #include "kernels.h"
@@ -406,22 +410,28 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_tc_kernel(const __grid_c
                                                                   const int32_t *__restrict__ ref_off,
                                                                   const int32_t *__restrict__ ref_cnt,
                                                                   const int2 *__restrict__ refs,
-                                                                  const float *__restrict__ dKbar, TView dK, TView dV,
+                                                                  float *__restrict__ dKacc, float *__restrict__ dVacc,
                                                                   const __nv_bfloat16 *__restrict__ Qp_g,
-                                                                  const __nv_bfloat16 *__restrict__ dOp_g) {
+                                                                  const __nv_bfloat16 *__restrict__ dOp_g,
+                                                                  int nsplit) {
     using S = KvSmem;
     constexpr int kNQ = S::kNQ;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int kb = blockIdx.x, r = blockIdx.y;
+    // CTA (key block kb, split): the block's (tile, entry) pairs split, j, j + nsplit, ...,
+    // among nsplit CTAs, so that a block many tiles attend is not one long serial chain
+    const int kb = blockIdx.x / nsplit, split = blockIdx.x % nsplit, r = blockIdx.y;
     const int64_t b = blockIdx.z;
     const int g = G.g, T = L.tile_rows;
     const int c = (int)((int64_t)kb * kStepKeys / BLK);   // the list entry (chunk / block id) of these keys
     const int64_t key0 = (int64_t)kb * kStepKeys;
     const size_t bh = (size_t)b * G.hkv + r;
-    const int nref = ref_cnt[bh * G.n_blk + c];
-    const int2 *rl = refs + bh * (size_t)L.n_tiles * G.n_blk + ref_off[bh * G.n_blk + c];
+    const int nref_all = ref_cnt[bh * G.n_blk + c];
+    const int nref = nref_all > split ? (nref_all - split + nsplit - 1) / nsplit : 0;
+    const int2 *rl_all = refs + bh * (size_t)L.n_tiles * G.n_blk + ref_off[bh * G.n_blk + c];
+    auto ref_at = [&](int j) -> int2 { return rl_all[split + (int64_t)j * nsplit]; };
+    if (nref == 0) return;  // nothing to add (the accumulators start at zero)
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + S::kBars);
     uint64_t *kv_full = bars, *q_full = kv_full + 1, *q_empty = q_full + kNQ, *s_full = q_empty + kNQ,
@@ -462,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_tc_kernel(const __grid_c
                 tma_load_4d(sm + S::kV + dh * kKRegion, &mp.tmV, kv_full, dh * 64, r, (int)key0, (int)b);
             }
             for (int j = 0; j < min(nref, kPrefetch); ++j) {
-                const size_t tl = bh * L.n_tiles + rl[j].x;
+                const size_t tl = bh * L.n_tiles + ref_at(j).x;
                 l2_prefetch(Qp_g + tl * kTileRows * kD, kTileRows * kD * 2);
                 l2_prefetch(dOp_g + tl * kTileRows * kD, kTileRows * kD * 2);
             }
@@ -470,8 +480,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_tc_kernel(const __grid_c
             for (int j = 0; j < nref; ++j) {
                 const int st = j % kNQ;
                 if (!wait_bar(q_empty + st, ((j / kNQ) & 1) ^ 1, kWaitNs, abort)) break;
-                const int64_t t = rl[j].x;
-                const int e = rl[j].y;
+                const int2 ref = ref_at(j);
+                const int64_t t = ref.x;
+                const int e = ref.y;
                 const size_t tile_lin = bh * L.n_tiles + t;
                 uint8_t *meta = sm + S::kMeta + st * S::kMetaStage;
                 // the tile index for the compute warps (published by the arrive below)
@@ -492,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_tc_kernel(const __grid_c
                 // the tiles of the pair kPrefetch ahead start their way into L2 now, so that
                 // the two-stage ring finds them there
                 if (j + kPrefetch < nref) {
-                    const size_t tl = bh * L.n_tiles + rl[j + kPrefetch].x;
+                    const size_t tl = bh * L.n_tiles + ref_at(j + kPrefetch).x;
                     l2_prefetch(Qp_g + tl * kTileRows * kD, kTileRows * kD * 2);
                     l2_prefetch(dOp_g + tl * kTileRows * kD, kTileRows * kD * 2);
                 }
@@ -535,14 +546,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_tc_kernel(const __grid_c
                 mma_commit(s_full + (j & 1));
                 return true;
             };
-            for (int j = 0; ok && j < min(nref, 2); ++j) ok = issue_sdp(j);
-            for (int j = 0; ok && j < nref; ++j) {
+            // dV^T += dO^T P, dK^T += Q^T dl of pair j over the tile's 128 rows (K steps of 16 rows)
+            auto issue_pv = [&](int j) {
                 const int st = j % kNQ;
-                if (!(ok = wait_bar(p_full, j & 1, kWaitNs, abort))) break;
                 tc_fence_after();
                 const uint32_t q_base = smem_u32(sm + S::kQ + st * 2 * kRegion);
                 const uint32_t do_base = smem_u32(sm + S::kdO + st * 2 * kRegion);
-                // dV^T += dO^T P, dK^T += Q^T dl over the tile's 128 rows (K steps of 16 rows)
 #pragma unroll
                 for (int kk = 0; kk < kTileRows / 16; ++kk) {
                     mma_ss(tdV, smem_desc_sw128(do_base + kk * 2048, kRegion, 1024),
@@ -552,7 +561,32 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_tc_kernel(const __grid_c
                 }
                 mma_commit(p_empty);
                 mma_commit(q_empty + st);
-                if (j + 2 < nref) ok = issue_sdp(j + 2);
+            };
+            for (int j = 0; ok && j < min(nref, 2); ++j) ok = issue_sdp(j);
+            // Whichever product is ready goes first: S, dP of pair next_sdp once its Q / dO
+            // stage has landed (and pv of pair next_sdp - 2, the last reader of its TMEM
+            // buffers' previous contents, has been issued), or dV, dK of pair next_pv once the
+            // softmax warps have written its P and dl.  Waiting on the next pair's tiles no
+            // longer holds back the products of a pair that is ready.
+            int next_sdp = min(nref, 2), next_pv = 0;
+            uint64_t t_last = gtimer();
+            while (ok && next_pv < nref) {
+                if (next_sdp < nref && next_sdp - 2 < next_pv &&
+                    mbar_try_wait(q_full + next_sdp % kNQ, (next_sdp / kNQ) & 1)) {
+                    ok = issue_sdp(next_sdp++);
+                    t_last = gtimer();
+                } else if (next_pv < next_sdp && mbar_try_wait(p_full, next_pv & 1)) {
+                    issue_pv(next_pv++);
+                    t_last = gtimer();
+                } else if (gtimer() - t_last > kWaitNs) {
+                    report_timeout();
+                    *abort = 1;
+                    ok = false;
+                } else if (*abort) {
+                    ok = false;
+                } else {
+                    __nanosleep(64);
+                }
             }
             mma_commit(fin);
             wait_bar(fin, 0, kWaitNs, abort, false);
@@ -617,38 +651,26 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_tc_kernel(const __grid_c
             fence_proxy_async_smem();
             mbar_arrive(p_full);
         }
-        // epilogue: lane m of dV^T / dK^T holds dimension m of the 64 keys
+        // epilogue: lane m of dV^T / dK^T holds dimension m of the 64 keys; this CTA's share
+        // is added to the fp32 accumulators (consecutive lanes: consecutive addresses)
         if (ok && !*abort) {
-            bool have = true;
-            if (nref > 0) have = __all_sync(0xffffffffu, wait_bar(p_empty, (nref - 1) & 1, kWaitNs, abort));
+            const bool have = __all_sync(0xffffffffu, wait_bar(p_empty, (nref - 1) & 1, kWaitNs, abort));
             tc_fence_after();
             if (have) {
                 const float sc = rsqrtf((float)kD);
-                float pool = 0.f;
-                if (c < G.n_chunks) {  // keys of a routing chunk share its summary's gradient
-                    const int64_t size = min((int64_t)G.B, G.nk - (int64_t)c * G.B);
-                    pool = dKbar[(((size_t)b * G.n_chunks + c) * G.hkv + r) * kD + m] / (float)size;
-                }
-                __nv_bfloat16 *dkp = reinterpret_cast<__nv_bfloat16 *>(const_cast<void *>(dK.p)) + b * dK.s0 +
-                                     (int64_t)r * dK.s2 + m;
-                __nv_bfloat16 *dvp = reinterpret_cast<__nv_bfloat16 *>(const_cast<void *>(dV.p)) + b * dV.s0 +
-                                     (int64_t)r * dV.s2 + m;
+                float *dka = dKacc + ((size_t)b * G.nk * G.hkv + r) * kD + m;
+                float *dva = dVacc + ((size_t)b * G.nk * G.hkv + r) * kD + m;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t dvu[32], dku[32];
-                    if (nref > 0) {  // uniform across the CTA
-                        tmem_ld32(tdV + lane_off + half * 32, dvu);
-                        tmem_ld32(tdK + lane_off + half * 32, dku);
-                    } else {
-#pragma unroll
-                        for (int x = 0; x < 32; ++x) dvu[x] = dku[x] = 0u;
-                    }
+                    tmem_ld32(tdV + lane_off + half * 32, dvu);
+                    tmem_ld32(tdK + lane_off + half * 32, dku);
 #pragma unroll
                     for (int x = 0; x < 32; ++x) {
                         const int64_t key = key0 + half * 32 + x;
                         if (key < G.nk) {
-                            dkp[key * dK.s1] = __float2bfloat16_rn(__uint_as_float(dku[x]) * sc + pool);
-                            dvp[key * dV.s1] = __float2bfloat16_rn(__uint_as_float(dvu[x]));
+                            atomicAdd(dka + (size_t)key * G.hkv * kD, __uint_as_float(dku[x]) * sc);
+                            atomicAdd(dva + (size_t)key * G.hkv * kD, __uint_as_float(dvu[x]));
                         }
                     }
                 }
@@ -661,6 +683,36 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_tc_kernel(const __grid_c
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
+}
+
+// dK = the Stage-2 part (accumulated over the split CTAs) + the chunk summary's share,
+// dV; both in bf16.  One thread per four consecutive dimensions.
+__global__ void bwd_kv_finish_kernel(const float4 *__restrict__ dKacc, const float4 *__restrict__ dVacc,
+                                     const float *__restrict__ dKbar, Geom G, TView dK, TView dV) {
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t n = G.b * G.nk * G.hkv * (int64_t)(kD / 4);
+    if (idx >= n) return;
+    const int e4 = (int)(idx % (kD / 4));
+    const int64_t row = idx / (kD / 4);  // (b, key, kv head)
+    const int r = (int)(row % G.hkv);
+    const int64_t key = (row / G.hkv) % G.nk, b = row / ((int64_t)G.hkv * G.nk);
+    float4 k = dKacc[idx];
+    const float4 v = dVacc[idx];
+    const int c = (int)(key / G.B);
+    if (c < G.n_chunks) {  // keys of a routing chunk share its summary's gradient
+        const float inv = 1.f / (float)min((int64_t)G.B, G.nk - (int64_t)c * G.B);
+        const float4 kb = reinterpret_cast<const float4 *>(dKbar + (((size_t)b * G.n_chunks + c) * G.hkv + r) * kD)[e4];
+        k.x += kb.x * inv;
+        k.y += kb.y * inv;
+        k.z += kb.z * inv;
+        k.w += kb.w * inv;
+    }
+    __nv_bfloat16 *dkp = reinterpret_cast<__nv_bfloat16 *>(const_cast<void *>(dK.p)) + b * dK.s0 + key * dK.s1 +
+                         (int64_t)r * dK.s2 + 4 * e4;
+    __nv_bfloat16 *dvp = reinterpret_cast<__nv_bfloat16 *>(const_cast<void *>(dV.p)) + b * dV.s0 + key * dV.s1 +
+                         (int64_t)r * dV.s2 + 4 * e4;
+    *reinterpret_cast<uint2 *>(dkp) = make_uint2(pack_bf16x2(k.x, k.y), pack_bf16x2(k.z, k.w));
+    *reinterpret_cast<uint2 *>(dvp) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
 }
 
 bool make_maps(BwdMaps *mp, const BwdArgs &a) {
@@ -725,20 +777,29 @@ cudaError_t launch_attn_bwd_tc_dkdv(const BwdArgs &a, cudaStream_t st) {
     const int64_t nkb = (G.nk + kStepKeys - 1) / kStepKeys;
     const size_t smem = KvSmem::kTotal + 1024;
     cudaError_t e;
-    dim3 grid((unsigned)nkb, (unsigned)G.hkv, (unsigned)G.b);
+    const size_t acc_bytes = (size_t)G.b * G.nk * G.hkv * kD * sizeof(float);
+    if ((e = cudaMemsetAsync(a.dKacc, 0, acc_bytes, st)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(a.dVacc, 0, acc_bytes, st)) != cudaSuccess) return e;
+    // split the pairs of a block among up to 8 CTAs: one per 64 tiles a block may have
+    const int nsplit = (int)std::min<int64_t>(8, std::max<int64_t>(1, a.L.n_tiles / 64));
+    dim3 grid((unsigned)(nkb * nsplit), (unsigned)G.hkv, (unsigned)G.b);
     if (G.B == 64) {
         if ((e = set_smem(bwd_dkdv_tc_kernel<64>, smem)) != cudaSuccess) return e;
         bwd_dkdv_tc_kernel<64><<<grid, kThreads, smem, st>>>(mp, G, a.L, a.Lp, a.Dp, a.ref_off, a.ref_cnt, a.refs,
-                                                             a.dKbar, a.dK, a.dV,
+                                                             a.dKacc, a.dVacc,
                                                              reinterpret_cast<const __nv_bfloat16 *>(a.Qp),
-                                                             reinterpret_cast<const __nv_bfloat16 *>(a.dOp));
+                                                             reinterpret_cast<const __nv_bfloat16 *>(a.dOp), nsplit);
     } else {
         if ((e = set_smem(bwd_dkdv_tc_kernel<128>, smem)) != cudaSuccess) return e;
         bwd_dkdv_tc_kernel<128><<<grid, kThreads, smem, st>>>(mp, G, a.L, a.Lp, a.Dp, a.ref_off, a.ref_cnt, a.refs,
-                                                              a.dKbar, a.dK, a.dV,
+                                                              a.dKacc, a.dVacc,
                                                               reinterpret_cast<const __nv_bfloat16 *>(a.Qp),
-                                                              reinterpret_cast<const __nv_bfloat16 *>(a.dOp));
+                                                              reinterpret_cast<const __nv_bfloat16 *>(a.dOp), nsplit);
     }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const int64_t n4 = G.b * G.nk * G.hkv * (int64_t)(kD / 4);
+    bwd_kv_finish_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(
+        reinterpret_cast<const float4 *>(a.dKacc), reinterpret_cast<const float4 *>(a.dVacc), a.dKbar, G, a.dK, a.dV);
     return cudaGetLastError();
 }
 

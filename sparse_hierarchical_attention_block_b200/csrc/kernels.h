@@ -89,6 +89,7 @@ struct BwdArgs {
     int2 *refs;                        // [b][hkv][n_tiles * n_blk] pairs
     bool use_tc;                       // tensor-core Stage-2 kernels (bf16, d = 128, B in {64, 128})
     uint8_t *Qp, *dOp;                 // tensor-core path: [b][hkv][n_tiles][128][d] bf16 tile rows
+    float *dKacc, *dVacc;              // tensor-core path: [b][nk][hkv][d] fp32 accumulators
     float *Lp, *Dp;                    // [b][hkv][n_tiles][128] lse (exp2 domain, +inf = empty) and D
 };
 cudaError_t launch_attn_bwd(const BwdArgs &a, dash_dtype_t dt, cudaStream_t st);

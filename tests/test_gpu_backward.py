@@ -281,7 +281,8 @@ def test_backward_prefill8k_sampled_and_identities():
 
 
 def test_backward_deterministic():
-    """dQ and dV are reproducible bit for bit; dK takes the summaries' gradient through
+    """dQ is reproducible bit for bit, and so is dV while each key block's pairs are summed
+    by one CTA (under 128 query tiles, as here); dK takes the summaries' gradient through
     fp32 atomic sums, so its last bit may differ between runs."""
     q, k, v, dout = _inputs(1, 512, 512, 8, 2, 128, 64, "bf16", seed=5)
     a = _fwd_bwd(q, k, v, dout, 64, 1.5, True, sigma=1.0)
