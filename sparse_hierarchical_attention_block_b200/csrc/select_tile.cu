@@ -21,8 +21,9 @@
 //            starting point (AdaSplash-2's initialisation, scanned by the pair's
 //            threads together, each over its own range of bins), then a bracketed
 //            iteration: for alpha = 2 and 1.5 the exact closed form on the current
-//            support (until the support is stable), otherwise Newton, with
-//            bisection as the safeguard; partial sums are combined in a fixed order
+//            support (until the support is stable), for alpha = 1.25 the first root of
+//            the support's quartic (Newton in registers on its power sums), otherwise
+//            Newton on the data, with bisection as the safeguard; partial sums are combined in a fixed order
 //            so every thread of a pair takes the same decisions;
 //   prior    the g heads of a query row sit in g adjacent lanes of one warp; a
 //            reduce-scatter over those lanes gives each lane the g heads' sums for
@@ -44,7 +45,7 @@ namespace {
 
 constexpr int kChunkTile = 128;    // chunks per logits MMA (N)
 constexpr int kMaxTileChunks = 2048;
-constexpr int kXchVals = 5;
+constexpr int kXchVals = 7;  // values a pair exchanges at most at once
 constexpr uint64_t kTileWaitNs = 2000000000ull;
 
 // Lane groups of a row block: its logits fill at most the 512 tensor-memory columns, so
@@ -507,13 +508,21 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_tile_kernel(const __gri
             // bracketed iteration (identical on every thread of the pair: same combined sums)
             float tau = nvis == 1 ? lo : t0;
             bool done = nvis <= 1;
-            constexpr bool kClosed = KINT == 1 || KINT == 2;
+            // a closed form on the current support for alpha = 2 and 1.5; for alpha = 1.25 the
+            // support's quartic, solved from its power sums by Newton in registers
+            constexpr bool kClosed = KINT == 1 || KINT == 2 || KINT == 4;
+            constexpr int kNV = KINT == 4 ? 7 : 5;  // combined values per pass
             int prev_cnt = -1;
             for (int it = 0; it < 40; ++it) {
                 if (!alu_sync_or(!done)) break;
                 // alpha = 2 / 1.5: moments of y = x - mx over the support {x > tau}, its count,
-                // the smallest score inside and the largest outside; otherwise f + 1, -f'/k, count
-                float acc[kXchVals] = {0.f, 0.f, 0.f, INFINITY, -INFINITY};
+                // the smallest score inside and the largest outside; alpha = 1.25: the same with the
+                // first four power sums of z = x - tau (in 0, 1, 5, 6); otherwise f + 1, -f'/k, count
+                float acc[kNV];
+                acc[0] = acc[1] = acc[2] = 0.f;
+                acc[3] = INFINITY;
+                acc[4] = -INFINITY;
+                if (kNV > 5) acc[kNV - 2] = acc[kNV - 1] = 0.f;
                 // a warp whose pairs are all settled skips the pass (the threads of a pair share
                 // their decisions, so the pair's other warps skip it too)
                 if (!__all_sync(0xffffffffu, done)) {
@@ -525,7 +534,14 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_tile_kernel(const __gri
                             const float xv = __uint_as_float(u[x]);
                             const float tt = xv - tau;
                             if (tt > 0.f) {
-                                if (kClosed) {
+                                if (KINT == 4) {
+                                    const float z2 = tt * tt;
+                                    acc[0] += tt;
+                                    acc[1] += z2;
+                                    acc[kNV - 2] = fmaf(z2, tt, acc[kNV - 2]);
+                                    acc[kNV - 1] = fmaf(z2, z2, acc[kNV - 1]);
+                                    acc[3] = fminf(acc[3], xv);
+                                } else if (kClosed) {
                                     const float yv = xv - mx;
                                     acc[0] += yv;
                                     acc[1] = fmaf(yv, yv, acc[1]);
@@ -541,7 +557,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_tile_kernel(const __gri
                         }
                     }
                 }
-                pair_reduce<kXchVals, LG>(xch, parity, slot, p, acc, 1 << 4, 1 << 3);
+                pair_reduce<kNV, LG>(xch, parity, slot, p, acc, 1 << 4, 1 << 3);
                 parity ^= 1;
                 if (done) continue;
                 const int cnt = (int)acc[2];
@@ -549,6 +565,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_tile_kernel(const __gri
                 float f;
                 if (KINT == 1) f = acc[0] - tr * (float)cnt - 1.f;                                    // sum (y - tr) - 1
                 else if (KINT == 2) f = acc[1] - 2.f * tr * acc[0] + tr * tr * (float)cnt - 1.f;     // sum (y - tr)^2 - 1
+                else if (KINT == 4) f = acc[kNV - 1] - 1.f;                                           // sum z^4 - 1
                 else f = acc[0] - 1.f;
                 if (f >= 0.f) lo = tau;
                 else hi = tau;
@@ -559,9 +576,25 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_tile_kernel(const __gri
                     const float m1 = acc[0] / (float)cnt;
                     if (KINT == 1) {
                         nt = mx + (acc[0] - 1.f) / (float)cnt;
-                    } else {
+                    } else if (KINT == 2) {
                         const float var = fmaxf(acc[1] / (float)cnt - m1 * m1, 0.f);
                         nt = mx + m1 - sqrtf(fmaxf(1.f / (float)cnt - var, 0.f));
+                    } else {
+                        // g(dl) = sum_S (z - dl)^4 - 1 = Z4 - 4 Z3 dl + 6 Z2 dl^2 - 4 Z1 dl^3 + Z0 dl^4 - 1 is
+                        // convex and decreasing at dl = 0: Newton from dl = 0 reaches its first root from
+                        // the left (after one step back when g(0) < 0)
+                        const float Z0 = (float)cnt, Z1 = acc[0], Z2 = acc[1], Z3 = acc[kNV - 2], Z4 = acc[kNV - 1];
+                        float dl = 0.f;
+                        for (int k = 0; k < 32; ++k) {
+                            const float gv = (((Z0 * dl - 4.f * Z1) * dl + 6.f * Z2) * dl - 4.f * Z3) * dl + Z4 - 1.f;
+                            const float dg = ((4.f * Z0 * dl - 12.f * Z1) * dl + 12.f * Z2) * dl - 4.f * Z3;
+                            if (!(dg < 0.f)) break;
+                            const float nd = dl - gv / dg;
+                            const bool conv = fabsf(nd - dl) <= 1e-7f * fmaxf(1.f, fabsf(tau));
+                            dl = nd;
+                            if (conv) break;
+                        }
+                        nt = tau + dl;
                     }
                     // (or, with rounding ties, when two closed-form steps in a row saw the same
                     // support: supports {x > tau} are nested, so equal counts mean equal sets)
@@ -985,13 +1018,21 @@ __global__ void __launch_bounds__(128 * CP, 4 / CP) select_tile_pair_kernel(cons
     // bracketed iteration (identical on every thread of the pair: same combined sums)
     float tau = nvis == 1 ? lo : t0;
     bool done = nvis <= 1;
-    constexpr bool kClosed = KINT == 1 || KINT == 2;
+    // a closed form on the current support for alpha = 2 and 1.5; for alpha = 1.25 the
+    // support's quartic, solved from its power sums by Newton in registers
+    constexpr bool kClosed = KINT == 1 || KINT == 2 || KINT == 4;
+    constexpr int kNV = KINT == 4 ? 7 : 5;  // combined values per pass
     int prev_cnt = -1;
     for (int it = 0; it < 40; ++it) {
         if (!__syncthreads_or(!done)) break;
         // alpha = 2 / 1.5: moments of y = x - mx over the support {x > tau}, its count,
-        // the smallest score inside and the largest outside; otherwise f + 1, -f'/k, count
-        float acc[kXchVals] = {0.f, 0.f, 0.f, INFINITY, -INFINITY};
+        // the smallest score inside and the largest outside; alpha = 1.25: the same with the
+        // first four power sums of z = x - tau (in 0, 1, 5, 6); otherwise f + 1, -f'/k, count
+        float acc[kNV];
+        acc[0] = acc[1] = acc[2] = 0.f;
+        acc[3] = INFINITY;
+        acc[4] = -INFINITY;
+        if (kNV > 5) acc[kNV - 2] = acc[kNV - 1] = 0.f;
         // a warp whose pairs are all settled skips the pass (the threads of a pair share
         // their decisions, so the pair's other warps skip it too)
         if (!__all_sync(0xffffffffu, done)) {
@@ -1003,7 +1044,14 @@ __global__ void __launch_bounds__(128 * CP, 4 / CP) select_tile_pair_kernel(cons
                     const float xv = __uint_as_float(u[x]);
                     const float tt = xv - tau;
                     if (tt > 0.f) {
-                        if (kClosed) {
+                        if (KINT == 4) {
+                            const float z2 = tt * tt;
+                            acc[0] += tt;
+                            acc[1] += z2;
+                            acc[kNV - 2] = fmaf(z2, tt, acc[kNV - 2]);
+                            acc[kNV - 1] = fmaf(z2, z2, acc[kNV - 1]);
+                            acc[3] = fminf(acc[3], xv);
+                        } else if (kClosed) {
                             const float yv = xv - mx;
                             acc[0] += yv;
                             acc[1] = fmaf(yv, yv, acc[1]);
@@ -1019,7 +1067,7 @@ __global__ void __launch_bounds__(128 * CP, 4 / CP) select_tile_pair_kernel(cons
                 }
             }
         }
-        pair_reduce_cta<kXchVals, LG, CP>(xch, parity, slot, p, acc, 1 << 4, 1 << 3);
+        pair_reduce_cta<kNV, LG, CP>(xch, parity, slot, p, acc, 1 << 4, 1 << 3);
         parity ^= 1;
         if (done) continue;
         const int cnt = (int)acc[2];
@@ -1027,6 +1075,7 @@ __global__ void __launch_bounds__(128 * CP, 4 / CP) select_tile_pair_kernel(cons
         float f;
         if (KINT == 1) f = acc[0] - tr * (float)cnt - 1.f;                                    // sum (y - tr) - 1
         else if (KINT == 2) f = acc[1] - 2.f * tr * acc[0] + tr * tr * (float)cnt - 1.f;     // sum (y - tr)^2 - 1
+        else if (KINT == 4) f = acc[kNV - 1] - 1.f;                                           // sum z^4 - 1
         else f = acc[0] - 1.f;
         if (f >= 0.f) lo = tau;
         else hi = tau;
@@ -1037,9 +1086,25 @@ __global__ void __launch_bounds__(128 * CP, 4 / CP) select_tile_pair_kernel(cons
             const float m1 = acc[0] / (float)cnt;
             if (KINT == 1) {
                 nt = mx + (acc[0] - 1.f) / (float)cnt;
-            } else {
+            } else if (KINT == 2) {
                 const float var = fmaxf(acc[1] / (float)cnt - m1 * m1, 0.f);
                 nt = mx + m1 - sqrtf(fmaxf(1.f / (float)cnt - var, 0.f));
+            } else {
+                // g(dl) = sum_S (z - dl)^4 - 1 = Z4 - 4 Z3 dl + 6 Z2 dl^2 - 4 Z1 dl^3 + Z0 dl^4 - 1 is
+                // convex and decreasing at dl = 0: Newton from dl = 0 reaches its first root from
+                // the left (after one step back when g(0) < 0)
+                const float Z0 = (float)cnt, Z1 = acc[0], Z2 = acc[1], Z3 = acc[kNV - 2], Z4 = acc[kNV - 1];
+                float dl = 0.f;
+                for (int k = 0; k < 32; ++k) {
+                    const float gv = (((Z0 * dl - 4.f * Z1) * dl + 6.f * Z2) * dl - 4.f * Z3) * dl + Z4 - 1.f;
+                    const float dg = ((4.f * Z0 * dl - 12.f * Z1) * dl + 12.f * Z2) * dl - 4.f * Z3;
+                    if (!(dg < 0.f)) break;
+                    const float nd = dl - gv / dg;
+                    const bool conv = fabsf(nd - dl) <= 1e-7f * fmaxf(1.f, fabsf(tau));
+                    dl = nd;
+                    if (conv) break;
+                }
+                nt = tau + dl;
             }
             // (or, with rounding ties, when two closed-form steps in a row saw the same
             // support: supports {x > tau} are nested, so equal counts mean equal sets)
