@@ -247,6 +247,34 @@ DASH_API int dash_attn_bwd(const dash_tensor_t *q, const dash_tensor_t *k, const
                            dash_tensor_t *dk, dash_tensor_t *dv, int block_size, float alpha, int causal,
                            int gqa_groups, const dash_opts_t *opts);
 
+/* The forward pass of dash_attn_fwd_ex on host-resident q, k, v and out, through device
+ * buffers of the same shapes, with the copies overlapped with the computation: the query
+ * rows are taken in up to n_slices slices of whole multiples of 1024 rows, in order (0 =
+ * automatic: 16 from 16K rows, 4 from 2K, else 1); slice s's rows and the keys they can see (with a causal mask the key prefix up
+ * to the slice's last row position, else all keys) are copied in on one internal stream,
+ * the slice's forward runs on opts->stream once they have landed, and its output rows are
+ * copied out on a second internal stream, so the copies of later slices and the copy back
+ * of earlier ones overlap the computation.  The output is bit-identical to
+ * dash_attn_fwd_ex(q_dev, k_dev, v_dev, out_dev, ...).
+ *   q_host, k_host, v_host, out_host  host memory (page-locked for the copies to be
+ *       asynchronous), [batch, seq, heads, dim] with packed rows: stride = {any >= seq *
+ *       heads * dim, heads * dim, dim, 1};
+ *   q_dev, k_dev, v_dev, out_dev      device buffers, same shapes, dtypes and row packing
+ *       (the caller's; their contents on return are the inputs and the output);
+ *   block_size, alpha, causal, gqa_groups, opts as for dash_attn_fwd_ex, without
+ *       summary_cache, nk_dev, kbar, qbar or lse (DASH_ERR_UNSUPPORTED).
+ * Asynchronous: the call returns once everything is enqueued; the host output is complete
+ * when opts->stream reaches the point of the call (the stream waits for the last copy back).
+ * The inputs must stay unchanged, and the host output untouched, until then.  The device
+ * buffers are not written before the stream's earlier work on them is done.  Not for stream
+ * capture (the internal streams are outside it).  Errors as for dash_attn_fwd_ex; a copy
+ * that fails returns DASH_ERR_CUDA. */
+DASH_API int dash_attn_fwd_host(const dash_tensor_t *q_host, const dash_tensor_t *k_host,
+                                const dash_tensor_t *v_host, dash_tensor_t *out_host, const dash_tensor_t *q_dev,
+                                const dash_tensor_t *k_dev, const dash_tensor_t *v_dev, dash_tensor_t *out_dev,
+                                int block_size, float alpha, int causal, int gqa_groups, int n_slices,
+                                const dash_opts_t *opts);
+
 /* Device workspace dash_attn_bwd needs for a problem (bytes, an upper bound). */
 DASH_API size_t dash_bwd_workspace_bytes(int64_t batch, int64_t nq, int64_t nk, int hq, int hkv, int d,
                                          int block_size, int causal);

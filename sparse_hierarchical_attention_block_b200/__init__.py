@@ -75,7 +75,7 @@ EXPORTS = ("dash_opts_init", "dash_attn_fwd", "dash_attn_fwd_ex", "dash_pool_key
            "dash_sync_status", "dash_release", "dash_version", "dash_attn_fwd_noalloc", "dash_pool_keys_q",
            "dash_lists_from_mask", "dash_summary_cache_create", "dash_summary_cache_update",
            "dash_summary_cache_reset", "dash_summary_cache_chunks", "dash_summary_cache_kbar",
-           "dash_summary_cache_destroy", "dash_attn_bwd", "dash_bwd_workspace_bytes")
+           "dash_summary_cache_destroy", "dash_attn_bwd", "dash_bwd_workspace_bytes", "dash_attn_fwd_host")
 
 # size of the library's static scratch area used by dash_attn_fwd_noalloc
 DASH_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -96,6 +96,7 @@ def load_library():
     lib.dash_attn_fwd.argtypes = [T, T, T, T, i32, f32, i32, i32]
     lib.dash_attn_fwd_ex.argtypes = [T, T, T, T, i32, f32, i32, i32, ctypes.POINTER(_Opts)]
     lib.dash_attn_fwd_noalloc.argtypes = [T, T, T, T, i32, f32, i32, i32, ctypes.POINTER(_Opts)]
+    lib.dash_attn_fwd_host.argtypes = [T, T, T, T, T, T, T, T, i32, f32, i32, i32, i32, ctypes.POINTER(_Opts)]
     lib.dash_pool_keys.argtypes = [T, i32, i32, P, P]
     lib.dash_pool_keys_q.argtypes = [T, T, i32, i32, P, P]
     lib.dash_lists_from_mask.argtypes = [P, i64, i64, i64, i32, i32, i32, i32, i32, ctypes.POINTER(_Lists), P]
@@ -138,10 +139,13 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
-def _desc(t: torch.Tensor) -> _Tensor:
+def _desc(t: torch.Tensor, host: bool = False) -> _Tensor:
     if t.dim() != 4:
         raise ValueError("tensors are [batch, seq, heads, dim]")
-    if not t.is_cuda:
+    if host:
+        if t.is_cuda:
+            raise ValueError("host tensors must be CPU tensors (page-locked for asynchronous copies)")
+    elif not t.is_cuda:
         raise ValueError("tensors must be CUDA tensors (the library has no CPU path)")
     d = _Tensor()
     d.data = t.data_ptr()
@@ -324,6 +328,22 @@ def dash_attn_fwd_noalloc(q, k, v, out, block_size, alpha, causal=True, gqa_grou
     _check(lib.dash_attn_fwd_noalloc(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.byref(od),
                                      int(block_size), float(alpha), int(bool(causal)), int(g), ctypes.byref(o)))
     return out
+
+
+def dash_attn_fwd_host(q_host, k_host, v_host, out_host, q_dev, k_dev, v_dev, out_dev, block_size, alpha,
+                       causal=True, gqa_groups=None, n_slices=0, **opts):
+    """Full forward of host tensors (pinned CPU memory) into ``out_host`` through the device
+    buffers ``*_dev`` (same shapes and dtypes), query rows in ``n_slices`` slices whose
+    copies in and out overlap the computation (0 = automatic).  Asynchronous on ``stream``
+    (default: the current stream): ``out_host`` is complete once that stream has reached
+    this point.  Returns ``out_host``."""
+    lib = load_library()
+    g = gqa_groups if gqa_groups is not None else q_dev.shape[2] // k_dev.shape[2]
+    ds = [_desc(t, host=True) for t in (q_host, k_host, v_host, out_host)] + [_desc(t) for t in (q_dev, k_dev, v_dev, out_dev)]
+    o = _opts(**opts)
+    _check(lib.dash_attn_fwd_host(*[ctypes.byref(d) for d in ds], int(block_size), float(alpha), int(bool(causal)),
+                                  int(g), int(n_slices), ctypes.byref(o)))
+    return out_host
 
 
 def dash_attn_bwd(q, k, v, out, dout, lse, dq, dk, dv, block_size, alpha, causal=True, gqa_groups=None, **opts):

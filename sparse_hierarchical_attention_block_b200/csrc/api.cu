@@ -953,6 +953,7 @@ DASH_API int dash_release(void) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    dash::release_host_staging();
     std::lock_guard<std::mutex> lk(g_ws_mu);
     if (dev >= 0 && dev < 128 && g_ws[dev].p) {
         e = cudaDeviceSynchronize();

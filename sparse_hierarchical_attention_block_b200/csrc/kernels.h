@@ -97,4 +97,7 @@ bool attn_bwd_tc_supported(const Geom &G, dash_dtype_t dt);
 cudaError_t launch_attn_bwd_tc_dq(const BwdArgs &a, cudaStream_t st);
 cudaError_t launch_attn_bwd_tc_dkdv(const BwdArgs &a, cudaStream_t st);
 
+// The host-staged forward's copy streams of the current device (freed by dash_release).
+void release_host_staging();
+
 }  // namespace dash
