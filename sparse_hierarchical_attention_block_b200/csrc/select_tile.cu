@@ -222,7 +222,7 @@ __device__ __forceinline__ void pair_reduce(float *xch, int parity, int slot, in
 // chunk and issues its logits MMAs column block by column block, each as soon as the 16
 // entmax warps have finished the group-prior pass over the block that held it, so the
 // next block's logits are computed while the current block's last pass runs.
-template <int D, int KINT, int LG>
+template <int D, int KINT, int LG, int GQ>
 __global__ void __launch_bounds__(kSelThreads, 1) select_tile_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                                     const uint8_t *__restrict__ ksplit, Geom G0,
                                                                     TileP P, TileOut out, int64_t n_units,
@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_tile_kernel(const __gri
     float *xch = reinterpret_cast<float *>(sm + S::kXch);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int g = G.g;
+    const int g = GQ > 0 ? GQ : G.g;  // the GQA group (a compile-time 4 in the common case)
     const int npos = kNP / g;                 // query positions per row block
     const int64_t nbh = G.b * G.hkv;
     auto unit = [&](int64_t u, int64_t &t, int &r, int64_t &b) {
@@ -726,13 +726,13 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_tile_kernel(const __gri
     }
 }
 
-template <int D, int KINT, int LG>
+template <int D, int KINT, int LG, int GQ>
 cudaError_t launch_sel(const CUtensorMap &tmQ, const uint8_t *ksplit, const Geom &G, const TileP &P,
                        const TileOut &o, cudaStream_t st) {
     using S = TSmem<D, LG>;
     static_assert(S::kTotal + 1024 <= 232448, "shared memory of the Stage-1 kernel");
     const size_t smem = S::kTotal + 1024;
-    cudaError_t e = cudaFuncSetAttribute(select_tile_kernel<D, KINT, LG>,
+    cudaError_t e = cudaFuncSetAttribute(select_tile_kernel<D, KINT, LG, GQ>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int npos = (128 / LG) / G.g;
@@ -742,7 +742,7 @@ cudaError_t launch_sel(const CUtensorMap &tmQ, const uint8_t *ksplit, const Geom
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     const int64_t grid = std::min<int64_t>(n_units, sms);
-    select_tile_kernel<D, KINT, LG><<<(unsigned)grid, kSelThreads, smem, st>>>(tmQ, ksplit, G, P, o, n_units, n_tblk);
+    select_tile_kernel<D, KINT, LG, GQ><<<(unsigned)grid, kSelThreads, smem, st>>>(tmQ, ksplit, G, P, o, n_units, n_tblk);
     return cudaGetLastError();
 }
 
@@ -1241,9 +1241,14 @@ cudaError_t launch_sel_lg(const TView &Q, const uint8_t *ksplit, const Geom &G, 
     CUtensorMap tmQ;
     if (!make_map_bf16(&tmQ, Q, G.b, G.nq, G.hq, G.d, G.g, npos)) return cudaErrorInvalidValue;
     if (G.n_chunks <= 2 * kChunkTile) return launch_sel_pair<D, KINT, 1, 2, 1>(tmQ, ksplit, G, P, o, st);
-    if (LG == 1) return launch_sel<D, KINT, 1>(tmQ, ksplit, G, P, o, st);
-    if (LG == 2) return launch_sel<D, KINT, 2>(tmQ, ksplit, G, P, o, st);
-    return launch_sel<D, KINT, 4>(tmQ, ksplit, G, P, o, st);
+    if (G.g == 4) {
+        if (LG == 1) return launch_sel<D, KINT, 1, 4>(tmQ, ksplit, G, P, o, st);
+        if (LG == 2) return launch_sel<D, KINT, 2, 4>(tmQ, ksplit, G, P, o, st);
+        return launch_sel<D, KINT, 4, 4>(tmQ, ksplit, G, P, o, st);
+    }
+    if (LG == 1) return launch_sel<D, KINT, 1, 0>(tmQ, ksplit, G, P, o, st);
+    if (LG == 2) return launch_sel<D, KINT, 2, 0>(tmQ, ksplit, G, P, o, st);
+    return launch_sel<D, KINT, 4, 0>(tmQ, ksplit, G, P, o, st);
 }
 
 }  // namespace
