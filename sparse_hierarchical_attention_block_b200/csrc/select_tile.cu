@@ -457,7 +457,10 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_tile_kernel(const __gri
 #pragma unroll
                 for (int x = 0; x < 32; ++x) {
                     const float y = __uint_as_float(u[x]) - lo;
-                    if (y >= 0.f) atomicAdd(hist + min(kBins - 1, (int)(y * (float)kBins)) * kNP + p, 1u);
+                    // bin floor(y kBins) as the low bits of y kBins + 2^23 rounded toward zero
+                    // (an FMA instead of a float-to-int conversion)
+                    const int bin = min(kBins - 1, __float_as_int(__fmaf_rz(y, (float)kBins, 8388608.f)) & 0xff);
+                    if (y >= 0.f) atomicAdd(hist + bin * kNP + p, 1u);
                 }
             }
             alu_sync();
@@ -515,7 +518,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_tile_kernel(const __gri
             int prev_cnt = -1;
             for (int it = 0; it < 40; ++it) {
                 if (!alu_sync_or(!done)) break;
-                // alpha = 2 / 1.5: moments of y = x - mx over the support {x > tau}, its count,
+                // alpha = 2 / 1.5: moments of z = x - tau over the support {x > tau}, its count,
                 // the smallest score inside and the largest outside; alpha = 1.25: the same with the
                 // first four power sums of z = x - tau (in 0, 1, 5, 6); otherwise f + 1, -f'/k, count
                 float acc[kNV];
@@ -542,9 +545,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_tile_kernel(const __gri
                                     acc[kNV - 1] = fmaf(z2, z2, acc[kNV - 1]);
                                     acc[3] = fminf(acc[3], xv);
                                 } else if (kClosed) {
-                                    const float yv = xv - mx;
-                                    acc[0] += yv;
-                                    acc[1] = fmaf(yv, yv, acc[1]);
+                                    acc[0] += tt;
+                                    acc[1] = fmaf(tt, tt, acc[1]);
                                     acc[3] = fminf(acc[3], xv);
                                 } else {
                                     acc[0] += rpow<KINT>(tt, P);
@@ -561,10 +563,9 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_tile_kernel(const __gri
                 parity ^= 1;
                 if (done) continue;
                 const int cnt = (int)acc[2];
-                const float tr = tau - mx;  // tau in the y = x - mx frame
                 float f;
-                if (KINT == 1) f = acc[0] - tr * (float)cnt - 1.f;                                    // sum (y - tr) - 1
-                else if (KINT == 2) f = acc[1] - 2.f * tr * acc[0] + tr * tr * (float)cnt - 1.f;     // sum (y - tr)^2 - 1
+                if (KINT == 1) f = acc[0] - 1.f;                                                      // sum z - 1
+                else if (KINT == 2) f = acc[1] - 1.f;                                                 // sum z^2 - 1
                 else if (KINT == 4) f = acc[kNV - 1] - 1.f;                                           // sum z^4 - 1
                 else f = acc[0] - 1.f;
                 if (f >= 0.f) lo = tau;
@@ -575,10 +576,10 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_tile_kernel(const __gri
                     // also {x > nt}: every score of S above nt, every other score at most nt
                     const float m1 = acc[0] / (float)cnt;
                     if (KINT == 1) {
-                        nt = mx + (acc[0] - 1.f) / (float)cnt;
+                        nt = tau + (acc[0] - 1.f) / (float)cnt;
                     } else if (KINT == 2) {
                         const float var = fmaxf(acc[1] / (float)cnt - m1 * m1, 0.f);
-                        nt = mx + m1 - sqrtf(fmaxf(1.f / (float)cnt - var, 0.f));
+                        nt = tau + m1 - sqrtf(fmaxf(1.f / (float)cnt - var, 0.f));
                     } else {
                         // g(dl) = sum_S (z - dl)^4 - 1 = Z4 - 4 Z3 dl + 6 Z2 dl^2 - 4 Z1 dl^3 + Z0 dl^4 - 1 is
                         // convex and decreasing at dl = 0: Newton from dl = 0 reaches its first root from
