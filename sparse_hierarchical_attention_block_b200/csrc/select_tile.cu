@@ -805,7 +805,7 @@ __device__ __forceinline__ void pair_reduce_cta(float *xch, int parity, int slot
     }
 }
 
-template <int D, int KINT, int LG, int CP, int NSB>
+template <int D, int KINT, int LG, int CP, int NSB, int GQ>
 __global__ void __launch_bounds__(128 * CP, 4 / CP) select_tile_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                                       const uint8_t *__restrict__ ksplit, Geom G0,
                                                                       TileP P, TileOut out, uint32_t ncols) {
@@ -830,7 +830,7 @@ __global__ void __launch_bounds__(128 * CP, 4 / CP) select_tile_pair_kernel(cons
     const int L = qd * 32 + lane;             // TMEM lane
     const int lg = L / kNP, p = L % kNP;      // lane group; pair
     const int slot = lg * CP + cp;
-    const int g = G.g;
+    const int g = GQ > 0 ? GQ : G.g;  // the GQA group (a compile-time 4 in the common case)
     const int npos = kNP / g;                 // query positions per CTA
     const int64_t t = (int64_t)gridDim.x - 1 - blockIdx.x;  // latest (longest) rows first
     const int r = blockIdx.y;
@@ -1158,9 +1158,11 @@ __global__ void __launch_bounds__(128 * CP, 4 / CP) select_tile_pair_kernel(cons
         for (int x = 0; x < 32; ++x) tr[lane * 33 + x] = __uint_as_float(u[x]) - tau_r;
         __syncwarp();
         uint32_t word = 0;  // membership bits of this lane's chunks
+#pragma unroll
         for (int x = hh; x < 32; x += g) {
             float v = 0.f;
             bool sel = false;
+#pragma unroll
             for (int h = 0; h < g; ++h) {
                 const float tt = tr[(gbase + h) * 33 + x];
                 if (tt > 0.f) {
@@ -1212,12 +1214,12 @@ __global__ void __launch_bounds__(128 * CP, 4 / CP) select_tile_pair_kernel(cons
     }
 }
 
-template <int D, int KINT, int LG, int CP, int NSB>
+template <int D, int KINT, int LG, int CP, int NSB, int GQ>
 cudaError_t launch_sel_pair(const CUtensorMap &tmQ, const uint8_t *ksplit, const Geom &G, const TileP &P,
                        const TileOut &o, cudaStream_t st) {
     using S = TSmemPair<D, LG, CP, NSB>;
     const size_t smem = S::kTotal + 1024;
-    cudaError_t e = cudaFuncSetAttribute(select_tile_pair_kernel<D, KINT, LG, CP, NSB>,
+    cudaError_t e = cudaFuncSetAttribute(select_tile_pair_kernel<D, KINT, LG, CP, NSB, GQ>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int npos = (128 / LG) / G.g;
@@ -1228,7 +1230,7 @@ cudaError_t launch_sel_pair(const CUtensorMap &tmQ, const uint8_t *ksplit, const
     uint32_t ncols = 32;
     while (ncols < (uint32_t)(((n_ct_all + LG - 1) / LG) * kChunkTile)) ncols *= 2;
     dim3 grid((unsigned)nblk, (unsigned)G.hkv, (unsigned)G.b);
-    select_tile_pair_kernel<D, KINT, LG, CP, NSB><<<grid, 128 * CP, smem, st>>>(tmQ, ksplit, G, P, o, ncols);
+    select_tile_pair_kernel<D, KINT, LG, CP, NSB, GQ><<<grid, 128 * CP, smem, st>>>(tmQ, ksplit, G, P, o, ncols);
     return cudaGetLastError();
 }
 
@@ -1241,7 +1243,9 @@ cudaError_t launch_sel_lg(const TView &Q, const uint8_t *ksplit, const Geom &G, 
     const int npos = (128 / LG) / G.g;
     CUtensorMap tmQ;
     if (!make_map_bf16(&tmQ, Q, G.b, G.nq, G.hq, G.d, G.g, npos)) return cudaErrorInvalidValue;
-    if (G.n_chunks <= 2 * kChunkTile) return launch_sel_pair<D, KINT, 1, 2, 1>(tmQ, ksplit, G, P, o, st);
+    if (G.n_chunks <= 2 * kChunkTile)
+        return G.g == 4 ? launch_sel_pair<D, KINT, 1, 2, 1, 4>(tmQ, ksplit, G, P, o, st)
+                        : launch_sel_pair<D, KINT, 1, 2, 1, 0>(tmQ, ksplit, G, P, o, st);
     if (G.g == 4) {
         if (LG == 1) return launch_sel<D, KINT, 1, 4>(tmQ, ksplit, G, P, o, st);
         if (LG == 2) return launch_sel<D, KINT, 2, 4>(tmQ, ksplit, G, P, o, st);
