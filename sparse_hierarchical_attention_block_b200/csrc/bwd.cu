@@ -552,6 +552,201 @@ __global__ void __launch_bounds__(32 * kRouteWarps) bwd_route_kernel(
     store();
 }
 
+// Sum over the 32 lanes of each of the 32 values P[v], left in lane v (recursive halving:
+// 5 exchange rounds, 31 shuffles).
+__device__ __forceinline__ float reduce_scatter32(float (&P)[32], int lane) {
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) {
+        const bool up = (lane & m) != 0;
+#pragma unroll
+        for (int k = 0; k < m; ++k) {
+            const float keep = up ? P[k + m] : P[k], send = up ? P[k] : P[k + m];
+            P[k] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+    }
+    return P[0];
+}
+
+constexpr int kRouteMaxChunks = 2048;  // routed-list capacity of the batched kernel (per warp)
+
+// The routing chain as bwd_route_kernel computes it, for g <= 4, with the chunk summaries
+// read once per batch of 8 routed chunks by the whole warp (lane l holds dimensions
+// DL*l .. DL*l + DL - 1 of each: one coalesced row per chunk) instead of one lane per chunk
+// streaming its own row.  The scores of the batch (8 chunks x 4 heads) are formed as
+// per-lane partial dot products and summed by a reduce-scatter, which leaves the score of
+// (chunk slot cs, head hs) in lane 4 cs + hs; the entmax terms are that lane's, and the
+// summaries already in registers serve the updates of dQ and of the summaries' gradient.
+template <typename T, int DL>
+__global__ void __launch_bounds__(32 * kRouteWarps) bwd_route8_kernel(
+    TView Q, const float *__restrict__ kbar, Geom G, float alpha, float gamma, float sigma,
+    const float *__restrict__ tau, const uint32_t *__restrict__ mask, const float *__restrict__ logw,
+    const float *__restrict__ Gd, const float *__restrict__ dQacc, TView dQ, float *__restrict__ dKbar) {
+    constexpr int D = DL * 32, GM = 4, NCB = 8;
+    __shared__ int rl_all[kRouteWarps][kRouteMaxChunks];
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int64_t w = (int64_t)blockIdx.x * kRouteWarps + warp;
+    if (w >= G.b * G.nq * G.hkv) return;
+    int *rl = rl_all[warp];
+    const int r = (int)(w % G.hkv);
+    const int64_t i = (w / G.hkv) % G.nq, b = w / ((int64_t)G.hkv * G.nq);
+    const int g = G.g;
+    const int nvis = row_nvis(G, i);
+    const float sc = gamma * rsqrtf((float)D);
+    float dq[GM][DL];
+#pragma unroll
+    for (int h = 0; h < GM; ++h)
+#pragma unroll
+        for (int k = 0; k < DL; ++k) dq[h][k] = 0.f;
+    auto store = [&]() {
+#pragma unroll
+        for (int h = 0; h < GM; ++h) {
+            if (h >= g) break;
+            const float *src = dQacc + (((size_t)b * G.nq + i) * G.hq + r * g + h) * D;
+            T *dst = reinterpret_cast<T *>(const_cast<void *>(dQ.p)) + b * dQ.s0 + i * dQ.s1 +
+                     (int64_t)(r * g + h) * dQ.s2;
+#pragma unroll
+            for (int k = 0; k < DL; ++k) dst[DL * lane + k] = from_f<T>(src[DL * lane + k] + sc * dq[h][k]);
+        }
+    };
+    // pass 1: the routed chunks, ascending, into the warp's list (lanes over mask words)
+    const uint32_t *mrow = mask + (((size_t)b * G.nq + i) * G.hkv + r) * G.words;
+    const int wv = nvis > 0 ? (nvis + 31) / 32 : 0;
+    int nR = 0;
+    for (int w0 = 0; w0 < wv; w0 += 32) {
+        const int wd = w0 + lane;
+        uint32_t bits = wd < wv ? mrow[wd] : 0u;
+        if (wd == wv - 1 && (nvis & 31)) bits &= (1u << (nvis & 31)) - 1u;
+        const int pc = __popc(bits);
+        int incl = pc;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int pos = nR + incl - pc;
+        while (bits) {
+            rl[pos++] = wd * 32 + __ffs(bits) - 1;
+            bits &= bits - 1u;
+        }
+        nR += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    __syncwarp();
+    if (nR == 0) {  // nothing routed: the Stage-2 part alone
+        store();
+        return;
+    }
+    float sG = 0.f;
+    for (int n = lane; n < nR; n += 32) sG += Gd[logw_index(G, b, r, i, rl[n])];
+    const float meanG = warp_sum(sG) / (float)nR;
+    // this lane's dimensions of the group's queries
+    float qv[GM][DL];
+#pragma unroll
+    for (int h = 0; h < GM; ++h) {
+        const T *qp = reinterpret_cast<const T *>(Q.p) + b * Q.s0 + i * Q.s1 + (int64_t)(r * g + (h < g ? h : 0)) * Q.s2;
+#pragma unroll
+        for (int k = 0; k < DL; ++k) qv[h][k] = h < g ? to_f<T>(qp[DL * lane + k]) : 0.f;
+    }
+    const float inv_sigma = 1.f / sigma;
+    const float xs = (alpha - 1.f) * gamma * rsqrtf((float)D);
+    const float kexp = 1.f / (alpha - 1.f), uexp = 2.f - alpha;
+    const int cs = lane / GM, hs = lane % GM;  // this lane's (chunk slot, head) of a batch
+    const float th = hs < g ? tau[((size_t)b * G.nq + i) * G.hq + r * g + hs] : INFINITY;
+    const float *kb_base = kbar + ((size_t)b * G.kbar_cap * G.hkv + r) * D + DL * lane;  // chunk c at + c * hkv * D
+    // batch n0: chunk ids, their summaries (this lane's dimensions) and the lane's score
+    auto batch = [&](int n0, int (&cid)[NCB], float (&kv)[NCB][DL]) -> float {
+        float P[32];
+#pragma unroll
+        for (int k = 0; k < NCB; ++k) {
+            cid[k] = n0 + k < nR ? rl[n0 + k] : -1;
+            if (cid[k] >= 0) {
+                const float *kp = kb_base + (size_t)cid[k] * G.hkv * D;
+                if (DL == 4) {
+                    const float4 t4 = *reinterpret_cast<const float4 *>(kp);
+                    kv[k][0] = t4.x;
+                    kv[k][DL > 1 ? 1 : 0] = t4.y;
+                    kv[k][DL > 2 ? 2 : 0] = t4.z;
+                    kv[k][DL > 3 ? 3 : 0] = t4.w;
+                } else {
+#pragma unroll
+                    for (int j = 0; j < DL; ++j) kv[k][j] = kp[j];
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < DL; ++j) kv[k][j] = 0.f;
+            }
+#pragma unroll
+            for (int h = 0; h < GM; ++h) {
+                float a = 0.f;
+#pragma unroll
+                for (int j = 0; j < DL; ++j) a = fmaf(qv[h][j], kv[k][j], a);
+                P[k * GM + h] = a;
+            }
+        }
+        return reduce_scatter32(P, lane) * xs;
+    };
+    // pass 2: sum u and sum u dp per head (lane (cs, hs) adds its own pair)
+    float su = 0.f, sud = 0.f;
+    for (int n0 = 0; n0 < nR; n0 += NCB) {
+        int cid[NCB];
+        float kv[NCB][DL];
+        const float x = batch(n0, cid, kv);
+        const int c = n0 + cs < nR ? rl[n0 + cs] : -1;  // this lane's chunk
+        if (c >= 0 && hs < g) {
+            const size_t li = logw_index(G, b, r, i, c);
+            float u, ud;
+            if (route_terms(x, th, kexp, uexp, logw[li], (Gd[li] - meanG) * inv_sigma, g, u, ud)) {
+                su += u;
+                sud += ud;
+            }
+        }
+    }
+#pragma unroll
+    for (int o = GM; o < 32; o <<= 1) {  // over the chunk slots of the lane's head
+        su += __shfl_xor_sync(0xffffffffu, su, o);
+        sud += __shfl_xor_sync(0xffffffffu, sud, o);
+    }
+    const float rho = su > 0.f ? sud / su : 0.f;
+    // pass 3: ds per (chunk, head) in its lane, then lanes over dimensions
+    const float sck = gamma * rsqrtf((float)D);
+    for (int n0 = 0; n0 < nR; n0 += NCB) {
+        int cid[NCB];
+        float kv[NCB][DL];
+        const float x = batch(n0, cid, kv);
+        const int c = n0 + cs < nR ? rl[n0 + cs] : -1;  // this lane's chunk
+        float ds = 0.f;
+        if (c >= 0 && hs < g) {
+            const size_t li = logw_index(G, b, r, i, c);
+            float u, ud;
+            if (route_terms(x, th, kexp, uexp, logw[li], (Gd[li] - meanG) * inv_sigma, g, u, ud)) ds = ud - u * rho;
+        }
+#pragma unroll
+        for (int k = 0; k < NCB; ++k) {
+            float dkb[DL];
+#pragma unroll
+            for (int j = 0; j < DL; ++j) dkb[j] = 0.f;
+#pragma unroll
+            for (int h = 0; h < GM; ++h) {
+                const float dsh = __shfl_sync(0xffffffffu, ds, k * GM + h);
+#pragma unroll
+                for (int j = 0; j < DL; ++j) {
+                    dq[h][j] = fmaf(dsh, kv[k][j], dq[h][j]);
+                    dkb[j] = fmaf(dsh, qv[h][j], dkb[j]);
+                }
+            }
+            if (cid[k] >= 0) {
+                float *dst = dKbar + (((size_t)b * G.n_chunks + cid[k]) * G.hkv + r) * D + DL * lane;
+                if (DL == 4)
+                    atomicAdd(reinterpret_cast<float4 *>(dst),
+                              make_float4(sck * dkb[0], sck * dkb[DL > 1 ? 1 : 0], sck * dkb[DL > 2 ? 2 : 0],
+                                          sck * dkb[DL > 3 ? 3 : 0]));
+                else
+                    atomicAdd(reinterpret_cast<float2 *>(dst), make_float2(sck * dkb[0], sck * dkb[DL > 1 ? 1 : 0]));
+            }
+        }
+    }
+    store();
+}
+
 template <typename T>
 __global__ void bwd_dq_finish_kernel(const float *__restrict__ dQacc, TView dQ, Geom G) {
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -597,7 +792,16 @@ cudaError_t launch_bwd_t(const BwdArgs &a, cudaStream_t st) {
     bwd_route_kernel<T, DL, GM><<<blocks, 32 * kRouteWarps, 0, st>>>(a.Q, a.kbar, G, a.alpha, a.gamma, a.sigma,  \
                                                                      a.tau, a.mask, a.logw, a.Gd, a.dQacc, a.dQ, \
                                                                      a.dKbar)
-        if (G.d == 128 && G.g <= 4) DASH_ROUTE(4, 4);
+        if (G.g <= 4 && G.n_chunks <= kRouteMaxChunks) {
+            if (G.d == 128)
+                bwd_route8_kernel<T, 4><<<blocks, 32 * kRouteWarps, 0, st>>>(a.Q, a.kbar, G, a.alpha, a.gamma, a.sigma,
+                                                                            a.tau, a.mask, a.logw, a.Gd, a.dQacc,
+                                                                            a.dQ, a.dKbar);
+            else
+                bwd_route8_kernel<T, 2><<<blocks, 32 * kRouteWarps, 0, st>>>(a.Q, a.kbar, G, a.alpha, a.gamma, a.sigma,
+                                                                            a.tau, a.mask, a.logw, a.Gd, a.dQacc,
+                                                                            a.dQ, a.dKbar);
+        } else if (G.d == 128 && G.g <= 4) DASH_ROUTE(4, 4);
         else if (G.d == 128) DASH_ROUTE(4, 16);
         else if (G.g <= 4) DASH_ROUTE(2, 4);
         else DASH_ROUTE(2, 16);
