@@ -577,7 +577,7 @@ constexpr int kRouteMaxChunks = 2048;  // routed-list capacity of the batched ke
 // (chunk slot cs, head hs) in lane 4 cs + hs; the entmax terms are that lane's, and the
 // summaries already in registers serve the updates of dQ and of the summaries' gradient.
 template <typename T, int DL>
-__global__ void __launch_bounds__(32 * kRouteWarps) bwd_route8_kernel(
+__global__ void __launch_bounds__(32 * kRouteWarps, 4) bwd_route8_kernel(
     TView Q, const float *__restrict__ kbar, Geom G, float alpha, float gamma, float sigma,
     const float *__restrict__ tau, const uint32_t *__restrict__ mask, const float *__restrict__ logw,
     const float *__restrict__ Gd, const float *__restrict__ dQacc, TView dQ, float *__restrict__ dKbar) {
