@@ -339,6 +339,27 @@ def test_prefill128k_sampled(alpha, sigma):
                   label=f"prefill128k alpha={alpha} sigma={sigma:g}")
 
 
+# Shapes that take the persistent Stage-1 kernel (more than 256 routing chunks) outside the
+# benchmark configurations: GQA groups other than 4 (its general code), d = 64, one, two and
+# four lane groups, every alpha with a closed form, nq < nk and a non-causal case.
+PERSISTENT_CASES = [
+    (1, 5000, 5000, 16, 2, 128, 16, 1.5, True, 1.0),   # g = 8, 312 chunks: one lane group
+    (1, 6000, 6000, 4, 2, 64, 16, 1.5, True, 1e8),     # g = 2, d = 64
+    (1, 10000, 10000, 8, 2, 128, 16, 2.0, True, 1.0),  # g = 4, 625 chunks: two lane groups
+    (1, 3000, 20000, 8, 8, 64, 16, 1.25, True, 1.0),   # g = 1, nq < nk, 1250 chunks: four lane groups
+    (1, 2000, 9000, 8, 2, 128, 32, 1.5, False, 1.0),   # non-causal, 282 chunks
+]
+
+
+@pytest.mark.parametrize("case", PERSISTENT_CASES, ids=[f"p{i}" for i in range(len(PERSISTENT_CASES))])
+def test_persistent_stage1_shapes(case):
+    b, nq, nk, hq, hkv, d, B, alpha, causal, sigma = case
+    q, k, v = _planted(b, nq, nk, hq, hkv, d, B, "bf16", seed=nq + hq, causal=causal)
+    rows = sample_rows(nq, B, 192, seed=nk)
+    out = _run(q, k, v, B, alpha, causal, sigma=sigma)
+    check_forward(q, k, v, out, B, alpha, causal, sigma=sigma, rows=rows, label=f"persistent {case}")
+
+
 def test_row_slices_equal_one_pass():
     """A caller workspace too small for every row's lists makes the forward run its query
     rows in slices; the output (and lse) equals the single-pass forward bit for bit."""
