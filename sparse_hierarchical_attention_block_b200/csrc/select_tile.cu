@@ -7,30 +7,35 @@
 //            the fp32 chunk summaries are split k̄ = hi + lo into two bf16 operands
 //            (per call, or kept across decoding steps in a summary cache) and both
 //            products accumulate in fp32 (relative error ~2^-17, i.e. fp32-class
-//            logits).  A row block's logits fill one of two 256-column TMEM buffers:
-//            with LG lane groups a block routes 128/LG pairs over up to 256*LG
-//            chunks, lane group lg holding chunk tiles lg, lg + LG, ... of its
-//            pairs.  The logits MMA of a tile of lane group lg reads Q through a
-//            zero-padded A operand whose only non-zero rows are that group's lanes,
-//            so accumulating the LG groups' products into one column block writes
-//            each group's lanes and adds zero to the others.  A persistent CTA per
-//            SM runs a producer warp (copies and MMAs of the next block into one
-//            buffer) beside 16 entmax warps (the passes below on the other buffer);
-//   tau      4*LG threads per pair walk its TMEM row in 32-column blocks: max, a
-//            128-bin shared-memory histogram over [max x - 1, max x) for the
-//            starting point (AdaSplash-2's initialisation, scanned by the pair's
-//            threads together, each over its own range of bins), then a bracketed
+//            logits).  TMEM holds 128 lanes x 512 fp32 columns; with LG lane groups
+//            a row block routes 128/LG pairs over up to 512*LG chunks, lane group lg
+//            holding chunk tiles lg, lg + LG, ... of its pairs in the same columns.
+//            The logits MMA of a tile of lane group lg reads Q through a zero-padded
+//            A operand whose only non-zero rows are that group's lanes, so
+//            accumulating the LG groups' products into one column block writes each
+//            group's lanes and adds zero to the others.
+//            Above 256 chunks one persistent CTA per SM walks row blocks: tensor
+//            memory is a ring of four 128-column blocks, and a producer warp issues
+//            the next block's logits MMAs column block by column block as the 16
+//            entmax warps release them after their last pass over the current block.
+//            Up to 256 chunks a CTA takes one row block, and two CTAs share an SM;
+//   tau      the threads of a pair walk its TMEM row in 32-column blocks: max, a
+//            32-bin shared-memory histogram over [max x - 1, max x) for the
+//            starting point (AdaSplash-2's initialisation), then a bracketed
 //            iteration: for alpha = 2 and 1.5 the exact closed form on the current
 //            support (until the support is stable), for alpha = 1.25 the first root of
 //            the support's quartic (Newton in registers on its power sums), otherwise
-//            Newton on the data, with bisection as the safeguard; partial sums are combined in a fixed order
-//            so every thread of a pair takes the same decisions;
+//            Newton on the data, with bisection as the safeguard; partial sums are
+//            combined in a fixed order so every thread of a pair takes the same
+//            decisions;
 //   prior    the g heads of a query row sit in g adjacent lanes of one warp; a
-//            reduce-scatter over those lanes gives each lane the g heads' sums for
-//            32/g chunks: w_c = (1/g) sum_h [x_c - tau_h]_+^{1/(alpha-1)}, membership
-//            by comparison, mu = mean log w over the routed chunks
+//            reduce-scatter over those lanes (the persistent kernel) or a
+//            shared-memory transpose (the two-CTA kernel) gives each lane the g heads'
+//            sums for 32/g chunks: w_c = (1/g) sum_h [x_c - tau_h]_+^{1/(alpha-1)},
+//            membership by comparison, mu = mean log w over the routed chunks
 //            (§3.4 Prop. 1); outputs the bit mask, log w of the routed chunks and mu
 //            per row, from which the work lists are built (d = (log w - mu)/sigma).
+// Both kernels are compiled for a GQA group of 4 as a constant and for any group.
 #include <math.h>
 
 #include <algorithm>
