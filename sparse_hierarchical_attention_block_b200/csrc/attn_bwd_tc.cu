@@ -9,8 +9,9 @@
 // chunk (the prior's gradient, taken on by the routing chain in bwd.cu).
 //
 // bwd_tc_prep_kernel   copies each tile's Q and dO rows (the lists' row order) into
-//                      contiguous bf16 tiles and lse (exp2 domain) and D beside them, so
-//                      that both kernels below load whole tiles with TMA.
+//                      contiguous bf16 tiles, with lse (exp2 domain) and D = <dO, O> (formed
+//                      from the same rows) beside them, so that both kernels below load
+//                      whole tiles with TMA.
 // bwd_dq_tc_kernel     one CTA per (batch, kv head, query tile), the latest tiles first
 //                      within groups of heads whose K and V fit in L2 together.  Warp 0 loads the tile once and K, V per 64-key step
 //                      (three-stage rings); warp 1 (one thread) issues
@@ -66,9 +67,8 @@ __device__ __forceinline__ void l2_prefetch(const void *p, uint32_t bytes) {
 }
 
 // ------------------------------------------------------------------ prep
-__global__ void __launch_bounds__(kTileRows) bwd_tc_prep_kernel(TView Q, TView dO, Geom G, ListsView L,
-                                                               const float *__restrict__ lse,
-                                                               const float *__restrict__ Drow, uint4 *__restrict__ Qp,
+__global__ void __launch_bounds__(kTileRows) bwd_tc_prep_kernel(TView Q, TView dO, TView O, Geom G, ListsView L,
+                                                               const float *__restrict__ lse, uint4 *__restrict__ Qp,
                                                                uint4 *__restrict__ dOp, float *__restrict__ Lp,
                                                                float *__restrict__ Dp) {
     const int64_t t = blockIdx.x;
@@ -76,25 +76,41 @@ __global__ void __launch_bounds__(kTileRows) bwd_tc_prep_kernel(TView Q, TView d
     const int64_t b = blockIdx.z;
     const int g = G.g;
     const size_t tile_lin = ((size_t)b * G.hkv + r) * L.n_tiles + t;
-    // 16 threads per row, each one 16-byte piece: 8 rows (2 KB contiguous each way) per pass
+    // 16 threads per row, each one 16-byte piece: 8 rows (2 KB contiguous each way) per pass;
+    // D = <dO, O> of the row from the same pieces (a sum over the row's 16 threads)
     const int piece = threadIdx.x % 16;
     for (int m = threadIdx.x / 16; m < kTileRows; m += kTileRows / 16) {
         const int64_t i = tile_row(L, G, tile_lin, t, m / g);
         const int h = r * g + m % g;
         const size_t row = tile_lin * kTileRows + m;
+        const int64_t ii = i >= 0 ? i : 0;
         const uint4 *qs = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(Q.p) + b * Q.s0 +
-                                                          (i >= 0 ? i : 0) * Q.s1 + (int64_t)h * Q.s2);
+                                                          ii * Q.s1 + (int64_t)h * Q.s2);
         const uint4 *gs = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(dO.p) + b * dO.s0 +
-                                                          (i >= 0 ? i : 0) * dO.s1 + (int64_t)h * dO.s2);
+                                                          ii * dO.s1 + (int64_t)h * dO.s2);
+        const uint4 *os = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(O.p) + b * O.s0 +
+                                                          ii * O.s1 + (int64_t)h * O.s2);
+        const uint4 gv = i >= 0 ? gs[piece] : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 ov = i >= 0 ? os[piece] : make_uint4(0u, 0u, 0u, 0u);
         Qp[row * (kD / 8) + piece] = i >= 0 ? qs[piece] : make_uint4(0u, 0u, 0u, 0u);
-        dOp[row * (kD / 8) + piece] = i >= 0 ? gs[piece] : make_uint4(0u, 0u, 0u, 0u);
+        dOp[row * (kD / 8) + piece] = gv;
+        const __nv_bfloat162 *g2 = reinterpret_cast<const __nv_bfloat162 *>(&gv);
+        const __nv_bfloat162 *o2 = reinterpret_cast<const __nv_bfloat162 *>(&ov);
+        float dsum = 0.f;
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const float2 a2 = __bfloat1622float2(g2[x]), c2 = __bfloat1622float2(o2[x]);
+            dsum = fmaf(a2.x, c2.x, fmaf(a2.y, c2.y, dsum));
+        }
+#pragma unroll
+        for (int o = 8; o >= 1; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
+        if (piece == 0) Dp[row] = dsum;
     }
     const int m = threadIdx.x;
     const int64_t i = tile_row(L, G, tile_lin, t, m / g);
     const size_t row = tile_lin * kTileRows + m;
     const size_t rid = ((size_t)b * G.nq + (i >= 0 ? i : 0)) * G.hq + r * g + m % g;
     Lp[row] = i >= 0 ? lse[rid] * kLog2e : INFINITY;
-    Dp[row] = i >= 0 ? Drow[rid] : 0.f;
 }
 
 // ------------------------------------------------------------------ dQ (query side)
@@ -749,7 +765,7 @@ cudaError_t launch_attn_bwd_tc_dq(const BwdArgs &a, cudaStream_t st) {
     const Geom &G = a.G;
     const ListsView &L = a.L;
     bwd_tc_prep_kernel<<<dim3((unsigned)L.n_tiles, (unsigned)G.hkv, (unsigned)G.b), kTileRows, 0, st>>>(
-        a.Q, a.dO, G, L, a.lse, a.Drow, reinterpret_cast<uint4 *>(a.Qp), reinterpret_cast<uint4 *>(a.dOp), a.Lp, a.Dp);
+        a.Q, a.dO, a.O, G, L, a.lse, reinterpret_cast<uint4 *>(a.Qp), reinterpret_cast<uint4 *>(a.dOp), a.Lp, a.Dp);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     BwdMaps mp;

@@ -766,8 +766,10 @@ cudaError_t launch_bwd_t(const BwdArgs &a, cudaStream_t st) {
     const ListsView &L = a.L;
     cudaError_t e;
     const int64_t rows = G.b * G.nq * G.hq;
-    bwd_rowdot_kernel<T><<<(unsigned)((rows * 32 + 255) / 256), 256, 0, st>>>(a.dO, a.O, G, a.Drow);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (!a.use_tc) {  // the tensor-core path forms D in its tile preparation
+        bwd_rowdot_kernel<T><<<(unsigned)((rows * 32 + 255) / 256), 256, 0, st>>>(a.dO, a.O, G, a.Drow);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     // Stage 2, query side: dQ and the prior's G
     if (a.use_tc) {
         if ((e = launch_attn_bwd_tc_dq(a, st)) != cudaSuccess) return e;
