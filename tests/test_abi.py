@@ -193,3 +193,35 @@ def test_pool_keys_q_arguments(lib):
     qb = _t(FAKE, dash.DASH_F32, [1, 15, 2, 128])
     assert lib.dash_pool_keys_q(ctypes.byref(k), None, 64, 1, kbar, None) == dash.DASH_ERR_INVALID_ARG
     assert lib.dash_pool_keys_q(ctypes.byref(k), ctypes.byref(qb), 64, 1, None, None) == dash.DASH_ERR_INVALID_ARG
+
+
+def test_host_staged_arguments(lib):
+    """dash_attn_fwd_host checks its host / device pairs and options on the host (every call
+    here is invalid, so no copy is enqueued and no device memory is touched)."""
+    shapes = {"q": [1, 256, 8, 128], "k": [1, 256, 2, 128], "v": [1, 256, 2, 128], "o": [1, 256, 8, 128]}
+    host = {n: _t(FAKE, dash.DASH_BF16, s) for n, s in shapes.items()}
+    dev = {n: _t(FAKE, dash.DASH_BF16, s) for n, s in shapes.items()}
+    opts = _Opts()
+    lib.dash_opts_init(ctypes.byref(opts))
+
+    def call(h=host, d=dev, o=opts, n_slices=0, B=64, alpha=1.5):
+        return lib.dash_attn_fwd_host(*[ctypes.byref(h[n]) for n in "qkvo"], *[ctypes.byref(d[n]) for n in "qkvo"],
+                                      B, alpha, 1, 4, n_slices, ctypes.byref(o))
+
+    bad = dict(dev)
+    bad["o"] = _t(FAKE, dash.DASH_BF16, [1, 128, 8, 128])  # not the host output's shape
+    assert call(d=bad) == dash.DASH_ERR_INVALID_ARG
+    bad = dict(host)
+    bad["k"] = _t(FAKE, dash.DASH_F32, shapes["k"])  # another dtype than its device buffer
+    assert call(h=bad) == dash.DASH_ERR_INVALID_ARG
+    bad = dict(host)
+    bad["q"] = _t(FAKE, dash.DASH_BF16, shapes["q"], stride=[256 * 8 * 128, 8 * 128 + 64, 128, 1])  # rows not packed
+    assert call(h=bad) == dash.DASH_ERR_UNSUPPORTED
+    assert call(n_slices=-1) == dash.DASH_ERR_INVALID_ARG
+    with_lse = _Opts()
+    lib.dash_opts_init(ctypes.byref(with_lse))
+    with_lse.lse = FAKE
+    assert call(o=with_lse) == dash.DASH_ERR_UNSUPPORTED
+    assert call(B=48) == dash.DASH_ERR_UNSUPPORTED  # the forward's own validation, before any copy
+    assert call(alpha=1.0) == dash.DASH_ERR_INVALID_ARG
+    assert lib.dash_last_error()
