@@ -155,6 +155,23 @@ def work_of(w, cnt, lists, local=1):
     return f2, y, sparsity, exec_f
 
 
+def count_launches(fn, fallback):
+    """Library kernels one call of fn launches, counted by the CUDA profiler on an extra,
+    untimed call (long prefills run in several row slices, so the count depends on the
+    size); `fallback` (the per-slice count) if the profiler is unavailable."""
+    try:
+        from torch.profiler import ProfilerActivity, profile
+        torch.cuda.synchronize()
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            fn()
+            torch.cuda.synchronize()
+        n = sum(1 for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA
+                and "dash::" in e.name and "kernel" in e.name)
+        return (n, "counted") if n > 0 else (fallback, "per-slice count (profiler saw no kernel)")
+    except Exception as exc:  # noqa: BLE001
+        return fallback, f"per-slice count (profiler unavailable: {type(exc).__name__})"
+
+
 def max_over_ranks(values, world, device):
     """Element-wise maximum of per-rank timings (every rank takes this collective step)."""
     t = torch.tensor(values, dtype=torch.float64, device=device)
@@ -280,6 +297,7 @@ def run_ours(args, rank, world, device):
     h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
     d2h = oh.numel() * oh.element_size()
 
+    launches_per_step, launches_src = count_launches(step, 4 if decode else 5)
     ms, ms2, ms01, ms_e2e = max_over_ranks([ms, ms2, ms01, ms_e2e], world, device)
 
     peaks = load_peaks()
@@ -327,9 +345,11 @@ def run_ours(args, rank, world, device):
                 "path": ("dash_attn_fwd_host: query-row slices, copies in and out on two streams beside the compute"
                          if not decode else "new token's q, k, v in; summary cache update; forward; output out"),
                 "ms_per_step": round(ms_e2e, 4)},
-        # per step: prefill pool_keys, kbar_split, select_tile, regroup_compact, attn_tc;
-        # decode (summaries and their operand form cached) select_tile, compact, attn_decode, combine
-        "gpu_launches": args.steps * (4 if decode else 5),
+        # per step, per row slice: prefill pool_keys, kbar_split (once), select_tile,
+        # regroup_compact, attn_tc; decode (summaries and their operand form cached)
+        # select_tile, compact, attn_decode, combine
+        "gpu_launches": args.steps * launches_per_step,
+        "gpu_launches_source": launches_src,
         "clocks": cs.summary(),
     }
     return res, (q, k, v, w, alpha, sigma)
