@@ -72,3 +72,10 @@ def test_reference_arm_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
     assert d["config"]["workload"] == "tiny" and np.isfinite(d["ms_per_step"])
+
+
+def test_launch_count_falls_back_without_a_profiler_view():
+    """gpu_launches comes from the CUDA profiler on an extra call; where the profiler sees no
+    library kernel (here: no GPU at all) the bench reports the per-slice count and says so."""
+    n, src = bench.count_launches(lambda: None, 5)
+    assert n == 5 and src.startswith("per-slice count")
