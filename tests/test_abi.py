@@ -225,3 +225,14 @@ def test_host_staged_arguments(lib):
     assert call(B=48) == dash.DASH_ERR_UNSUPPORTED  # the forward's own validation, before any copy
     assert call(alpha=1.0) == dash.DASH_ERR_INVALID_ARG
     assert lib.dash_last_error()
+
+
+def test_workspace_stays_within_the_slicing_budget(lib):
+    """Long prefills run in row slices whose work lists fit about 1 GB of library workspace
+    (host-side arithmetic only): 128K keys at batch 1 and 2, block 128 and 64."""
+    for b, B in ((1, 128), (2, 128), (1, 64)):
+        need = dash.dash_workspace_bytes(b, 131072, 131072, 32, 8, 128, B)
+        assert 0 < need <= 10 ** 9, (b, B, need)
+    # a short prefill takes the single-slice layout, which is smaller still
+    assert dash.dash_workspace_bytes(1, 8192, 8192, 32, 8, 128, 64) < dash.dash_workspace_bytes(1, 131072, 131072,
+                                                                                                 32, 8, 128, 128)
