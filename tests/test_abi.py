@@ -236,3 +236,29 @@ def test_workspace_stays_within_the_slicing_budget(lib):
     # a short prefill takes the single-slice layout, which is smaller still
     assert dash.dash_workspace_bytes(1, 8192, 8192, 32, 8, 128, 64) < dash.dash_workspace_bytes(1, 131072, 131072,
                                                                                                  32, 8, 128, 128)
+
+
+def test_backward_arguments(lib):
+    """dash_attn_bwd rejects a missing lse and gradients of the wrong shape or dtype on the
+    host (every call here is invalid, so nothing reaches the device)."""
+    shp = {"q": [1, 256, 8, 128], "k": [1, 256, 2, 128]}
+    t = {n: _t(FAKE, dash.DASH_BF16, shp["q" if n in ("q", "o", "do", "dq") else "k"])
+         for n in ("q", "k", "v", "o", "do", "dq", "dk", "dv")}
+    opts = _Opts()
+    lib.dash_opts_init(ctypes.byref(opts))
+
+    def call(lse=FAKE, **kw):
+        a = dict(t)
+        a.update(kw)
+        return lib.dash_attn_bwd(ctypes.byref(a["q"]), ctypes.byref(a["k"]), ctypes.byref(a["v"]),
+                                 ctypes.byref(a["o"]), ctypes.byref(a["do"]), lse, ctypes.byref(a["dq"]),
+                                 ctypes.byref(a["dk"]), ctypes.byref(a["dv"]), 64, 1.5, 1, 4, ctypes.byref(opts))
+
+    assert call(lse=None) == dash.DASH_ERR_INVALID_ARG
+    assert call(dq=_t(FAKE, dash.DASH_BF16, [1, 128, 8, 128])) == dash.DASH_ERR_INVALID_ARG
+    assert call(do=_t(FAKE, dash.DASH_BF16, [1, 256, 4, 128])) == dash.DASH_ERR_INVALID_ARG
+    assert call(dk=_t(FAKE, dash.DASH_F32, shp["k"])) == dash.DASH_ERR_INVALID_ARG
+    assert lib.dash_last_error()
+    # the backward keeps the forward's Stage 0-1 state plus its own (transposed lists, tiles)
+    assert dash.dash_bwd_workspace_bytes(1, 8192, 8192, 32, 8, 128, 64) > dash.dash_workspace_bytes(
+        1, 8192, 8192, 32, 8, 128, 64)
